@@ -1,0 +1,150 @@
+/*
+ * nc.h — C ABI of the B200 KV-cache Transformer inference engine.
+ *
+ * The engine runs the forward pass of the nanochat-style dense Transformer
+ * (launch Q&A of "Karpathy再放大招：8000行代碼復現ChatGPT全棧..." : Llama-like,
+ * RoPE and no positional embedding, QK norm, untied embedding/unembedding, a
+ * norm after the token embedding, relu^2 MLP, RMSNorm without parameters, no
+ * biases, multi-query attention, logit softcap) as the two operations the
+ * same page names for its inference Engine: prefill and single-token decode
+ * against a per-sequence KV cache ("高效推理": KV-cache engine with simple
+ * prefill/decode). Forking a prefilled cache to N samples serves the RL
+ * rollouts the page lists ("RL ... GRPO on GSM8K").
+ *
+ * Conventions for every call:
+ *  - Pointers named d_* are DEVICE pointers (CUDA global memory on the
+ *    model's device) owned by the caller; other pointers are host pointers.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Work is
+ *    enqueued on it and the call returns without waiting; outputs are valid
+ *    once the stream has been synchronised.
+ *  - Return value: NC_OK (0) or an NC_E* code; nc_last_error() gives a
+ *    message for the last failing call on this thread. Argument errors are
+ *    detected on the host before anything is enqueued, so a failing call has
+ *    changed nothing. Conditions only visible on the device (a token id out
+ *    of range, a decode position that is not the sequence's current length)
+ *    never fault: the kernels clamp/skip and set a bit in the model's device
+ *    status word, read with nc_device_status().
+ *  - The library owns the weights, KV caches and workspaces it allocates;
+ *    calls on one model/cache must not overlap on different streams.
+ *  - Only one GPU is used: the device current when the model is created.
+ */
+#ifndef NC_H
+#define NC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define NC_OK 0
+#define NC_EINVAL 1   /* null pointer, bad shape, config/blob mismatch */
+#define NC_ERANGE 2   /* batch or length beyond what the cache was created for */
+#define NC_ENOMEM 3   /* device allocation failed */
+#define NC_ECUDA 4    /* a CUDA runtime call failed (message has the CUDA error) */
+#define NC_EUNSUP 5   /* valid config that this build has no kernel for */
+
+/* Device status bits (nc_device_status). */
+#define NC_DEV_BAD_TOKEN 1u     /* a token id was outside [0, vocab): clamped */
+#define NC_DEV_BAD_POSITION 2u  /* decode position != current length or >= max_seq: sequence skipped */
+#define NC_DEV_TIMEOUT 4u       /* a bounded in-kernel wait ran out (pipeline error) */
+
+/* Storage type of weights, activations and KV cache. Accumulation is fp32. */
+#define NC_F32 0
+#define NC_BF16 1
+
+/* Model shape. Fields follow the feature list above; n_kv_head = 1 is the
+ * page's multi-query attention. Constants the pages leave open are inputs:
+ * rope_base (10000), softcap (15), norm_eps (1e-6, inside the sqrt of every
+ * RMSNorm). */
+typedef struct {
+  int depth;       /* number of Transformer blocks (>= 0) */
+  int d_model;     /* residual width d */
+  int n_head;      /* query heads H; n_head * head_dim == d_model */
+  int n_kv_head;   /* KV heads; must divide n_head (this build: 1) */
+  int head_dim;    /* hd, even */
+  int mlp_hidden;  /* F (4*d in the presets) */
+  int vocab;       /* V */
+  float rope_base;
+  float softcap;
+  float norm_eps;
+  int dtype;       /* NC_F32 or NC_BF16 */
+} nc_config;
+
+typedef struct nc_model nc_model;
+typedef struct nc_kv nc_kv;
+
+/* Create a model on the current CUDA device from a host weight blob.
+ * Blob: tensors back to back, row-major [out, in], element type cfg->dtype
+ * (fp32, or bf16 bit patterns), in this order: wte[V,d]; for each layer
+ * Wq[H*hd,d], Wk[Hkv*hd,d], Wv[Hkv*hd,d], Wo[d,H*hd], Wfc[F,d], Wproj[d,F];
+ * then the untied lm_head Wlm[V,d]. blob_bytes must match exactly. The blob
+ * is copied to the device before the call returns; the caller keeps
+ * ownership of it. Errors: NC_EINVAL (null, inconsistent config, size
+ * mismatch), NC_EUNSUP, NC_ENOMEM, NC_ECUDA. */
+int nc_model_create(const nc_config *cfg, const void *host_blob, size_t blob_bytes, nc_model **out);
+
+/* Free the model (waits for the device to finish). NULL is ignored. */
+void nc_model_destroy(nc_model *model);
+
+/* Read and clear the model's device status word (NC_DEV_* bits) raised by
+ * kernels since the last call. Synchronises the device. */
+int nc_device_status(nc_model *model, uint32_t *out_bits);
+
+/* Create a KV cache for up to max_batch sequences of up to max_seq tokens,
+ * plus the workspace prefill/decode need (sized for max_batch*max_seq
+ * prefill rows). Layout per layer: K and V [max_batch][max_seq][Hkv*hd] of
+ * the model's dtype, K stored after RoPE and QK norm. All lengths start at
+ * 0. Errors: NC_EINVAL, NC_ENOMEM, NC_ECUDA. */
+int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out);
+
+/* Free a cache (waits for the device). NULL is ignored. */
+void nc_kv_destroy(nc_kv *kv);
+
+/* Copy the current lengths of sequences 0..n-1 to host memory out[n].
+ * Synchronises the device. Errors: NC_EINVAL, NC_ERANGE (n > max_batch). */
+int nc_kv_lengths(const nc_kv *kv, int n, int32_t *out);
+
+/* Prefill: run the prompts d_tokens[B,T] (int32, row-major) from position 0
+ * into sequences 0..B-1 of `kv`, replacing whatever they held; afterwards
+ * each has length T. Outputs (each may be NULL):
+ *   d_logits  fp32 softcapped logits: [B,V] for the last position when
+ *             logits_mode == 0, or [B,T,V] for every position when 1;
+ *   d_next    int32 [B]: argmax over the vocabulary of the last position's
+ *             logits (+ d_noise[b,:] if given), lowest index on ties;
+ *   d_noise   fp32 [B,V] additive noise for d_next (e.g. Gumbel), or NULL.
+ * Errors: NC_EINVAL (null kv/model/tokens, B or T < 1, bad logits_mode),
+ * NC_ERANGE (B > max_batch, T > max_seq), NC_ECUDA. */
+int nc_prefill(nc_model *model, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode,
+               float *d_logits, int32_t *d_next, const float *d_noise, void *stream);
+
+/* Decode one token for each of sequences 0..B-1: d_tokens[B] are fed at
+ * d_positions[B] (int32, device). positions[b] must equal sequence b's
+ * current length (< max_seq); the token's K/V are appended there and the
+ * length becomes positions[b]+1. Positions may differ between sequences.
+ * Outputs as in nc_prefill: d_logits fp32 [B,V], d_next int32 [B] (argmax of
+ * logits + d_noise[b,:] when d_noise is non-NULL). A sequence whose position
+ * is wrong is skipped (outputs untouched, cache unchanged) and
+ * NC_DEV_BAD_POSITION is raised. Errors: NC_EINVAL, NC_ERANGE (B >
+ * max_batch), NC_ECUDA. */
+int nc_decode_step(nc_model *model, nc_kv *kv, const int32_t *d_tokens, const int32_t *d_positions, int B,
+                   const float *d_noise, float *d_logits, int32_t *d_next, void *stream);
+
+/* Fork: copy sequence src_seq of `src` (its first len tokens, every layer,
+ * K and V) into sequences dst_first .. dst_first+n-1 of `dst` and set their
+ * lengths to len. src and dst may be the same cache (the source must not be
+ * among the destinations). Both caches must belong to the same model.
+ * Errors: NC_EINVAL, NC_ERANGE (indices out of range, len > dst max_seq),
+ * NC_ECUDA. */
+int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream);
+
+/* Message for the last failing nc_* call on this thread ("" if none). */
+const char *nc_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NC_H */

@@ -1,0 +1,316 @@
+// nc_api.cu — the C ABI (include/nc.h): objects, argument checks, and the
+// prefill / decode / fork call sequences over the engine's kernels.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "nc_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+#define NC_CUDA_TRY(expr)                                                                       \
+  do {                                                                                          \
+    cudaError_t e_ = (expr);                                                                    \
+    if (e_ != cudaSuccess) return fail(NC_ECUDA, "%s: %s", #expr, cudaGetErrorString(e_));     \
+  } while (0)
+
+int check_config(const nc_config *c) {
+  if (!c) return fail(NC_EINVAL, "config is NULL");
+  if (c->depth < 0 || c->d_model <= 0 || c->n_head <= 0 || c->n_kv_head <= 0 || c->head_dim <= 0 ||
+      c->mlp_hidden <= 0 || c->vocab <= 0)
+    return fail(NC_EINVAL, "config has a non-positive size");
+  if (c->head_dim % 2) return fail(NC_EINVAL, "head_dim must be even (RoPE pairs)");
+  if (c->n_head * c->head_dim != c->d_model) return fail(NC_EINVAL, "n_head * head_dim != d_model");
+  if (c->n_head % c->n_kv_head) return fail(NC_EINVAL, "n_kv_head must divide n_head");
+  if (c->dtype != NC_F32 && c->dtype != NC_BF16) return fail(NC_EINVAL, "dtype must be NC_F32 or NC_BF16");
+  if (!(c->softcap > 0.f) || !(c->rope_base > 0.f) || !(c->norm_eps >= 0.f))
+    return fail(NC_EINVAL, "softcap and rope_base must be > 0, norm_eps >= 0");
+  return NC_OK;
+}
+
+size_t blob_elems(const nc_config &c) {
+  size_t d = c.d_model, qd = (size_t)c.n_head * c.head_dim, kd = (size_t)c.n_kv_head * c.head_dim;
+  size_t F = c.mlp_hidden, V = c.vocab;
+  size_t per_layer = qd * d + 2 * kd * d + d * qd + F * d + d * F;
+  return 2 * V * d + per_layer * (size_t)c.depth;
+}
+
+inline cudaStream_t as_stream(void *s) { return (cudaStream_t)s; }
+
+inline void *layer_ptr(const nc_kv *kv, void *base, int l) {
+  return (char *)base + (size_t)l * kv->layer_elems * kv->model->elem;
+}
+
+// The transformer blocks for M rows already embedded into kv->x.
+int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  int d = c.d_model, H = c.n_head, Hkv = c.n_kv_head, hd = c.head_dim, F = c.mlp_hidden;
+  int qkv_w = (H + 2 * Hkv) * hd;
+  const uint8_t *valid = kv->valid;
+  for (int l = 0; l < c.depth; l++) {
+    const nc_layer_w &w = m->layers[l];
+    void *kc = layer_ptr(kv, kv->k, l), *vc = layer_ptr(kv, kv->v, l);
+    nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
+    nc::k_gemm_generic(c.dtype, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s);
+    nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, H, Hkv, hd, kv->rope, kv->q, kc, vc, kv->max_seq, valid,
+                             c.norm_eps, s);
+    nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, H, Hkv, hd, kv->max_seq, kv->y, s);
+    nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s);
+    nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
+    nc::k_gemm_generic(c.dtype, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s);
+    nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s);
+  }
+  return NC_OK;
+}
+
+// Final norm of `rows` rows of x (row r taken from x row r*stride + offset),
+// lm_head with softcap into logits (row-major, ldo = V), argmax into next.
+void run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, float *logits, const uint8_t *valid,
+              cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  nc::k_rmsnorm_rows(c.dtype, kv->x, rows, c.d_model, stride, offset, c.norm_eps, kv->h, s);
+  nc::k_gemm_generic(c.dtype, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab,
+                     c.softcap, valid, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *nc_last_error(void) { return g_err.c_str(); }
+
+int nc_model_create(const nc_config *cfg, const void *host_blob, size_t blob_bytes, nc_model **out) {
+  if (!out) return fail(NC_EINVAL, "out is NULL");
+  *out = nullptr;
+  int rc = check_config(cfg);
+  if (rc) return rc;
+  if (!host_blob) return fail(NC_EINVAL, "blob is NULL");
+  size_t elem = cfg->dtype == NC_F32 ? 4 : 2;
+  size_t want = blob_elems(*cfg) * elem;
+  if (blob_bytes != want)
+    return fail(NC_EINVAL, "blob has %zu bytes, config needs %zu", blob_bytes, want);
+  nc_model *m = new nc_model();
+  m->cfg = *cfg;
+  m->elem = elem;
+  m->blob_bytes = blob_bytes;
+  cudaError_t e = cudaGetDevice(&m->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&m->num_sms, cudaDevAttrMultiProcessorCount, m->device);
+  if (e == cudaSuccess) e = cudaMalloc(&m->blob, blob_bytes);
+  if (e == cudaSuccess) e = cudaMemcpy(m->blob, host_blob, blob_bytes, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMalloc(&m->status, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(m->status, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) {
+    int code = (e == cudaErrorMemoryAllocation) ? NC_ENOMEM : NC_ECUDA;
+    nc_model_destroy(m);
+    cudaGetLastError();
+    return fail(code, "model allocation/copy failed: %s", cudaGetErrorString(e));
+  }
+  const nc_config &c = *cfg;
+  size_t d = c.d_model, qd = (size_t)c.n_head * c.head_dim, kd = (size_t)c.n_kv_head * c.head_dim;
+  size_t F = c.mlp_hidden, V = c.vocab;
+  char *p = (char *)m->blob;
+  m->wte = p;
+  p += V * d * elem;
+  m->layers.resize(c.depth);
+  for (int l = 0; l < c.depth; l++) {
+    nc_layer_w &w = m->layers[l];
+    w.wqkv = p;
+    p += (qd + 2 * kd) * d * elem;
+    w.wo = p;
+    p += d * qd * elem;
+    w.wfc = p;
+    p += F * d * elem;
+    w.wproj = p;
+    p += d * F * elem;
+  }
+  m->wlm = p;
+  *out = m;
+  return NC_OK;
+}
+
+void nc_model_destroy(nc_model *m) {
+  if (!m) return;
+  cudaDeviceSynchronize();
+  cudaFree(m->blob);
+  cudaFree(m->status);
+  delete m;
+}
+
+int nc_device_status(nc_model *m, uint32_t *out_bits) {
+  if (!m || !out_bits) return fail(NC_EINVAL, "null argument");
+  NC_CUDA_TRY(cudaDeviceSynchronize());
+  NC_CUDA_TRY(cudaMemcpy(out_bits, m->status, sizeof(uint32_t), cudaMemcpyDeviceToHost));
+  NC_CUDA_TRY(cudaMemset(m->status, 0, sizeof(uint32_t)));
+  return NC_OK;
+}
+
+int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out) {
+  if (!out) return fail(NC_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (!model) return fail(NC_EINVAL, "model is NULL");
+  if (max_batch <= 0 || max_seq <= 0) return fail(NC_EINVAL, "max_batch and max_seq must be positive");
+  const nc_config &c = model->cfg;
+  nc_kv *kv = new nc_kv();
+  kv->model = const_cast<nc_model *>(model);
+  kv->max_batch = max_batch;
+  kv->max_seq = max_seq;
+  size_t kd = (size_t)c.n_kv_head * c.head_dim, elem = model->elem;
+  kv->layer_elems = (size_t)max_batch * max_seq * kd;
+  kv->max_rows = (size_t)max_batch * max_seq;
+  size_t rows = kv->max_rows, d = c.d_model, qd = (size_t)c.n_head * c.head_dim;
+  size_t qkv_w = qd + 2 * kd, F = c.mlp_hidden, half = c.head_dim / 2;
+  size_t cache_bytes = kv->layer_elems * elem * (size_t)(c.depth > 0 ? c.depth : 1);
+  cudaError_t e = cudaSuccess;
+  auto alloc = [&](void **p, size_t bytes) {
+    if (e == cudaSuccess) e = cudaMalloc(p, bytes ? bytes : 16);
+  };
+  alloc(&kv->k, cache_bytes);
+  alloc(&kv->v, cache_bytes);
+  alloc((void **)&kv->len, sizeof(int32_t) * max_batch);
+  alloc((void **)&kv->valid, max_batch);
+  alloc((void **)&kv->rope, sizeof(float2) * max_seq * half);
+  alloc((void **)&kv->x, sizeof(float) * rows * d);
+  alloc(&kv->h, elem * rows * (d > qd ? d : qd));
+  alloc(&kv->qkv, elem * rows * qkv_w);
+  alloc(&kv->q, elem * rows * qd);
+  alloc(&kv->y, elem * rows * qd);
+  alloc(&kv->f, elem * rows * F);
+  alloc((void **)&kv->logits, sizeof(float) * (size_t)max_batch * c.vocab);
+  if (e == cudaSuccess) e = cudaMemset(kv->len, 0, sizeof(int32_t) * max_batch);
+  if (e == cudaSuccess) e = cudaMemset(kv->valid, 0, max_batch);
+  if (e == cudaSuccess) {
+    // RoPE table: angle pos * base^(-2i/hd) in double, stored as (cos, sin).
+    float2 *tab = (float2 *)malloc(sizeof(float2) * max_seq * half);
+    if (!tab) {
+      e = cudaErrorMemoryAllocation;
+    } else {
+      for (int p = 0; p < max_seq; p++)
+        for (size_t i = 0; i < half; i++) {
+          double theta = pow((double)c.rope_base, -2.0 * (double)i / (double)c.head_dim);
+          double a = (double)p * theta;
+          tab[p * half + i] = make_float2((float)cos(a), (float)sin(a));
+        }
+      e = cudaMemcpy(kv->rope, tab, sizeof(float2) * max_seq * half, cudaMemcpyHostToDevice);
+      free(tab);
+    }
+  }
+  if (e != cudaSuccess) {
+    int code = (e == cudaErrorMemoryAllocation) ? NC_ENOMEM : NC_ECUDA;
+    nc_kv_destroy(kv);
+    cudaGetLastError();
+    return fail(code, "kv allocation failed: %s", cudaGetErrorString(e));
+  }
+  *out = kv;
+  return NC_OK;
+}
+
+void nc_kv_destroy(nc_kv *kv) {
+  if (!kv) return;
+  cudaDeviceSynchronize();
+  void *ps[] = {kv->k, kv->v, kv->len, kv->valid, kv->rope, kv->x, kv->h, kv->qkv, kv->q, kv->y, kv->f, kv->logits};
+  for (void *p : ps) cudaFree(p);
+  delete kv;
+}
+
+int nc_kv_lengths(const nc_kv *kv, int n, int32_t *out) {
+  if (!kv || !out || n < 0) return fail(NC_EINVAL, "bad argument");
+  if (n > kv->max_batch) return fail(NC_ERANGE, "n=%d > max_batch=%d", n, kv->max_batch);
+  NC_CUDA_TRY(cudaDeviceSynchronize());
+  NC_CUDA_TRY(cudaMemcpy(out, kv->len, sizeof(int32_t) * n, cudaMemcpyDeviceToHost));
+  return NC_OK;
+}
+
+int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode, float *d_logits,
+               int32_t *d_next, const float *d_noise, void *stream) {
+  if (!m || !kv || !d_tokens) return fail(NC_EINVAL, "null model, kv or tokens");
+  if (kv->model != m) return fail(NC_EINVAL, "kv belongs to another model");
+  if (B < 1 || T < 1) return fail(NC_EINVAL, "B and T must be >= 1");
+  if (logits_mode != 0 && logits_mode != 1) return fail(NC_EINVAL, "logits_mode must be 0 (last) or 1 (all)");
+  if (B > kv->max_batch) return fail(NC_ERANGE, "B=%d > max_batch=%d", B, kv->max_batch);
+  if (T > kv->max_seq) return fail(NC_ERANGE, "T=%d > max_seq=%d", T, kv->max_seq);
+  const nc_config &c = m->cfg;
+  cudaStream_t s = as_stream(stream);
+  int M = B * T;
+  nc::k_prefill_begin(kv->len, kv->valid, B, T, s);
+  nc::k_embed_norm(c.dtype, d_tokens, M, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
+  nc::RowMap rm{T, nullptr};
+  run_blocks(m, kv, M, rm, s);
+  float *logits;
+  long long last_off, row_stride;
+  if (logits_mode == 1) {
+    if (d_logits) {
+      run_head(m, kv, M, 1, 0, d_logits, nullptr, s);
+      logits = d_logits;
+      last_off = (long long)(T - 1) * c.vocab;
+      row_stride = (long long)T * c.vocab;
+    } else {
+      run_head(m, kv, B, T, T - 1, kv->logits, nullptr, s);
+      logits = kv->logits;
+      last_off = 0;
+      row_stride = c.vocab;
+    }
+  } else {
+    logits = d_logits ? d_logits : kv->logits;
+    run_head(m, kv, B, T, T - 1, logits, nullptr, s);
+    last_off = 0;
+    row_stride = c.vocab;
+  }
+  if (d_next) nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_t *d_positions, int B,
+                   const float *d_noise, float *d_logits, int32_t *d_next, void *stream) {
+  if (!m || !kv || !d_tokens || !d_positions) return fail(NC_EINVAL, "null model, kv, tokens or positions");
+  if (kv->model != m) return fail(NC_EINVAL, "kv belongs to another model");
+  if (B < 1) return fail(NC_EINVAL, "B must be >= 1");
+  if (B > kv->max_batch) return fail(NC_ERANGE, "B=%d > max_batch=%d", B, kv->max_batch);
+  const nc_config &c = m->cfg;
+  cudaStream_t s = as_stream(stream);
+  nc::k_decode_begin(d_positions, kv->len, kv->valid, B, kv->max_seq, m->status, s);
+  nc::k_embed_norm(c.dtype, d_tokens, B, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
+  nc::RowMap rm{1, d_positions};
+  run_blocks(m, kv, B, rm, s);
+  float *logits = d_logits ? d_logits : kv->logits;
+  run_head(m, kv, B, 1, 0, logits, kv->valid, s);
+  if (d_next) nc::k_argmax_rows(logits, B, c.vocab, c.vocab, d_noise, d_next, kv->valid, s);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream) {
+  if (!src || !dst) return fail(NC_EINVAL, "null cache");
+  if (src->model != dst->model) return fail(NC_EINVAL, "caches belong to different models");
+  if (n < 1) return fail(NC_EINVAL, "n must be >= 1");
+  if (src_seq < 0 || src_seq >= src->max_batch) return fail(NC_ERANGE, "src_seq out of range");
+  if (dst_first < 0 || dst_first + n > dst->max_batch) return fail(NC_ERANGE, "destinations out of range");
+  if (dst->max_seq < src->max_seq)
+    return fail(NC_ERANGE, "destination max_seq %d < source max_seq %d", dst->max_seq, src->max_seq);
+  if (src == dst && src_seq >= dst_first && src_seq < dst_first + n)
+    return fail(NC_EINVAL, "source sequence is among the destinations");
+  const nc_config &c = src->model->cfg;
+  nc::k_kv_fork((int)src->model->elem, src->k, src->v, src->layer_elems, src->max_seq, src_seq, src->len, dst->k,
+                dst->v, dst->layer_elems, dst->max_seq, dst_first, n, dst->len, c.depth, c.n_kv_head * c.head_dim,
+                src->model->status, as_stream(stream));
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// nc_internal.h — engine objects and kernel launchers (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "nc.h"
+#include "nc_common.cuh"
+
+struct nc_layer_w {
+  const void *wqkv;   // [(H + 2*Hkv)*hd, d]: Wq, Wk, Wv are adjacent in the blob
+  const void *wo;     // [d, H*hd]
+  const void *wfc;    // [F, d]
+  const void *wproj;  // [d, F]
+};
+
+struct nc_model {
+  nc_config cfg;
+  int device = 0;
+  int num_sms = 0;
+  size_t elem = 4;             // bytes per stored element
+  void *blob = nullptr;        // device copy of the whole weight blob
+  size_t blob_bytes = 0;
+  const void *wte = nullptr;   // [V, d]
+  const void *wlm = nullptr;   // [V, d]
+  std::vector<nc_layer_w> layers;
+  uint32_t *status = nullptr;  // device status word (NC_DEV_* bits)
+  bool fast = false;           // bf16 + shapes the sm_100a kernels cover
+};
+
+struct nc_kv {
+  nc_model *model = nullptr;
+  int max_batch = 0, max_seq = 0;
+  size_t layer_elems = 0;      // max_batch * max_seq * Hkv * hd
+  void *k = nullptr, *v = nullptr;  // [depth][max_batch][max_seq][Hkv*hd]
+  int32_t *len = nullptr;      // device [max_batch]
+  uint8_t *valid = nullptr;    // device [max_batch]: row takes part in this decode step
+  float2 *rope = nullptr;      // device [max_seq][hd/2] (cos, sin), angles in double on the host
+  // workspace sized for max_rows = max_batch * max_seq activation rows
+  size_t max_rows = 0;
+  float *x = nullptr;          // [rows, d] fp32 residual stream
+  void *h = nullptr;           // [rows, max(d, H*hd)] normed activations (storage type)
+  void *qkv = nullptr;         // [rows, (H + 2*Hkv)*hd]
+  void *q = nullptr;           // [rows, H*hd] rotated + normed queries
+  void *y = nullptr;           // [rows, H*hd] attention output
+  void *f = nullptr;           // [rows, F] relu^2 hidden
+  float *logits = nullptr;     // [max_batch, V] when the caller passes no logits buffer
+};
+
+namespace nc {
+
+enum Epi { EPI_STORE = 0, EPI_RELU2 = 1, EPI_RESID = 2, EPI_SOFTCAP = 3 };
+
+// ---- generic kernels (any even head_dim; fp32 or bf16 storage) ----
+void k_prefill_begin(int32_t *len, uint8_t *valid, int B, int T, cudaStream_t s);
+void k_decode_begin(const int32_t *positions, int32_t *len, uint8_t *valid, int B, int max_seq,
+                    uint32_t *status, cudaStream_t s);
+void k_embed_norm(int dtype, const int32_t *tokens, int M, const void *wte, int d, int vocab, float eps,
+                  float *x, uint32_t *status, cudaStream_t s);
+void k_rmsnorm_rows(int dtype, const float *x, int rows, int d, int src_stride, int src_offset, float eps,
+                    void *out, cudaStream_t s);
+void k_gemm_generic(int dtype, int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out,
+                    int ldo, float cap, const uint8_t *valid_rows, cudaStream_t s);
+void k_rope_qknorm_append(int dtype, const void *qkv, RowMap rm, int M, int H, int Hkv, int hd,
+                          const float2 *rope, void *q_out, void *kc, void *vc, int max_seq,
+                          const uint8_t *valid, float eps, cudaStream_t s);
+void k_attention_generic(int dtype, const void *q, const void *kc, const void *vc, RowMap rm, int M, int H,
+                         int Hkv, int hd, int max_seq, void *y, cudaStream_t s);
+void k_argmax_rows(const float *logits, int rows, int V, long long row_stride, const float *noise,
+                   int32_t *next, const uint8_t *valid, cudaStream_t s);
+void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_layer_elems, int src_max_seq,
+               int src_seq, const int32_t *src_len, void *dst_k, void *dst_v, size_t dst_layer_elems,
+               int dst_max_seq, int dst_first, int n, int32_t *dst_len, int depth, int kd, uint32_t *status,
+               cudaStream_t s);
+
+}  // namespace nc
