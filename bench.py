@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the KV-cache Transformer engine on B200.
+
+Metric: d20 bf16 prefill tok/s and decode tok/s (B=32), with the fraction of
+the tensor-core / HBM roofline.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+One timed step = one nc_prefill of the d20 prefill workload (8 prompts x 2048
+Zipf tokens, N(0,0.02) bf16 weights): embedding + norm, 20 blocks (QKV, RoPE +
+QK norm + KV append, causal MQA, O-proj, relu^2 MLP), final norm, lm_head with
+softcap and the argmax token pick, all on the device. The decode workload (32
+sequences prefilled to 2048 tokens, then 128 greedy decode steps at
+positions 2048..2175) is timed as a whole loop and reported under "decode".
+Inputs are synthetic; weights stream from HBM every step (1.0 GB > 126 MB L2).
+
+With --gpus N > 1 (under torchrun) every rank runs the same workload on its own
+GPU as an independent replica (the engine has no cross-GPU step); the timed
+region is bracketed by barriers and the time is the max over ranks.
+
+--impl reference times the CPU oracle (plain C, double precision) on a
+bounded sample of the same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "d20 bf16 prefill tok/s & decode tok/s (B=32); % of HBM / tensor-core roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------ accounting
+def linear_params(cfg) -> int:
+    """Weights of the per-layer linears (QKV, O, fc, proj), all layers."""
+    d, hd, H, Hkv, F = cfg.d_model, cfg.head_dim, cfg.n_head, cfg.n_kv_head, cfg.mlp_hidden
+    return cfg.depth * (d * (H + 2 * Hkv) * hd + H * hd * d + 2 * d * F)
+
+
+def prefill_flops(cfg, B: int, T: int) -> dict:
+    """Algorithmic FLOPs of one prefill with last-position logits."""
+    lin = 2 * B * T * linear_params(cfg)
+    attn = cfg.depth * B * 4 * cfg.n_head * cfg.head_dim * T * (T + 1) // 2
+    head = 2 * B * cfg.d_model * cfg.vocab
+    return {"gemm": lin, "attn": attn, "head": head, "total": lin + attn + head}
+
+
+def decode_bytes(cfg, B: int, ctx_avg: float) -> dict:
+    """Algorithmic HBM bytes of one decode step (bf16 weights and cache, fp32 logits)."""
+    kd = cfg.n_kv_head * cfg.head_dim
+    w_lin = 2 * linear_params(cfg)
+    w_head = 2 * cfg.vocab * cfg.d_model
+    kv_read = cfg.depth * B * ctx_avg * kd * 2 * 2
+    kv_write = cfg.depth * B * kd * 2 * 2
+    logits = 4 * B * cfg.vocab
+    total = w_lin + w_head + kv_read + kv_write + logits
+    return {"weights_linear": w_lin, "weights_head": w_head, "kv_read": kv_read, "kv_write": kv_write,
+            "logits": logits, "total": total}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d["bf16_tflops_sustained"])}, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+                power.append(float(parts[3].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_prefill_sample(cfg, blob, prompts, n_tokens: int):
+    """Time the oracle's prefill of the first n_tokens of prompt 0; -> (tok/s, seconds, threads)."""
+    import oracle as orc
+    om = orc.OracleModel(cfg, blob)
+    t0 = time.perf_counter()
+    om.forward_full(prompts[0, :n_tokens], all_positions=False)
+    dt = time.perf_counter() - t0
+    return n_tokens / dt, dt, orc.num_threads()
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import nc_synth as syn
+    import oracle as orc
+    w = syn.WORKLOADS["d20_prefill"]
+    cfg = w.model
+    blob = syn.make_blob(cfg, w.weight_seed)
+    prompts = syn.prompt_tokens(w)
+    om = orc.OracleModel(cfg, blob)
+    n_tok = args.ref_tokens
+    for _ in range(args.warmup):
+        om.forward_full(prompts[0, :n_tok], all_positions=False)
+    times = []
+    for s in range(args.steps):
+        seq = prompts[s % w.batch, :n_tok]
+        t0 = time.perf_counter()
+        om.forward_full(seq, all_positions=False)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps * n_tok / total
+    sample = (f"oracle prefill of the first {n_tok} tokens of one d20 prompt per step "
+              f"(the workload is 8 x 2048 tokens)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "d20_prefill: 8 x 2048 Zipf(1.1) tokens, d20 bf16 N(0,0.02) weights",
+                   "batch": w.batch, "seq_len": w.prompt_len, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": orc.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+
+    import kv_cache_transformer_b200 as nc
+    import nc_synth as syn
+    from kv_cache_transformer_b200 import build as ncbuild
+    if rank == 0:
+        ncbuild.build()
+    barrier(world)
+
+    peaks, peaks_src = load_peaks()
+    wp, wd = syn.WORKLOADS["d20_prefill"], syn.WORKLOADS["d20_decode"]
+    cfg = wp.model
+    blob = syn.make_blob(cfg, wp.weight_seed)
+    model = nc.Model(cfg, blob)
+    max_seq = wd.prompt_len + wd.decode_steps
+    kv = model.kv(max(wp.batch, wd.batch), max_seq)
+    stream = torch.cuda.current_stream()
+    B, T, V = wp.batch, wp.prompt_len, cfg.vocab
+
+    prompts_np = syn.prompt_tokens(wp)
+    tokens = torch.from_numpy(prompts_np).cuda()
+    logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
+    nxt = torch.empty((B,), dtype=torch.int32, device="cuda")
+
+    # ---------------- prefill: device-resident inputs
+    for _ in range(args.warmup):
+        model.prefill(kv, tokens, 0, logits, nxt)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    model.profile(True)
+    model.profile_read()
+    n0 = nc.nc_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        model.prefill(kv, tokens, 0, logits, nxt)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = nc.nc_launch_count() - n0
+    kms, kn = model.profile_read()
+    model.profile(False)
+    clk = clocks.stop()
+    barrier(world)
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_step = t_ms / args.steps
+    value = world * args.steps * B * T / (t_ms / 1e3)
+
+    fl = prefill_flops(cfg, B, T)
+    gemm_ms = kms[nc.NC_K_GEMM] / args.steps  # GEMM time per step
+    gemm_launch_per_step = kn[nc.NC_K_GEMM] / args.steps
+    gemm_tflops = fl["gemm"] / (gemm_ms / 1e3) / 1e12
+    peak_tc = peaks["bf16_tflops_sustained"]
+    roofline = {
+        "bound": "tensor", "kernel": "prefill linear-layer GEMMs (QKV, O, fc relu^2, proj)",
+        "achieved": gemm_tflops, "peak": peak_tc, "unit": "TFLOP/s", "frac": gemm_tflops / peak_tc,
+        "traffic": None, "peak_source": f"{peaks_src} bf16_tflops_sustained",
+        "flops_per_launch": fl["gemm"] / max(gemm_launch_per_step, 1),
+        "ms_per_launch": gemm_ms / max(gemm_launch_per_step, 1),
+        "launches_per_step": gemm_launch_per_step,
+    }
+    step_tflops = fl["total"] / (ms_step / 1e3) / 1e12
+    kernel_share = {nc.K_CLASS_NAMES[i]: round(float(kms[i] / max(kms.sum(), 1e-9)), 4) for i in range(nc.NC_K_COUNT)}
+
+    # ---------------- prefill end to end: pinned host tokens in, logits + tokens out
+    tok_host = torch.from_numpy(prompts_np).pin_memory()
+    logits_host = torch.empty((B, V), dtype=torch.float32).pin_memory()
+    nxt_host = torch.empty((B,), dtype=torch.int32).pin_memory()
+    tok_dev = torch.empty_like(tokens)
+    for _ in range(args.warmup):
+        tok_dev.copy_(tok_host, non_blocking=True)
+        model.prefill(kv, tok_dev, 0, logits, nxt)
+        logits_host.copy_(logits, non_blocking=True)
+        nxt_host.copy_(nxt, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(args.steps):
+        tok_dev.copy_(tok_host, non_blocking=True)
+        model.prefill(kv, tok_dev, 0, logits, nxt)
+        logits_host.copy_(logits, non_blocking=True)
+        nxt_host.copy_(nxt, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    te_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    e2e = {"value": world * args.steps * B * T / (te_ms / 1e3), "unit": "tok/s",
+           "h2d_bytes_per_step": tok_host.numel() * 4,
+           "d2h_bytes_per_step": logits_host.numel() * 4 + nxt_host.numel() * 4}
+
+    # ---------------- decode: 32 sequences at 2048 tokens, 128 greedy steps
+    decode = None
+    if not args.no_decode:
+        decode = run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local)
+
+    # ---------------- CPU oracle on a bounded sample (rank 0, N = 1)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tps, secs, thr = oracle_prefill_sample(cfg, blob, prompts_np, args.ref_tokens)
+        cpu = {"value": tps, "unit": "tok/s", "cores": thr, "kind": "oracle",
+               "sample": f"oracle prefill of the first {args.ref_tokens} tokens of prompt 0 "
+                         f"({secs:.1f} s on {thr} threads)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "d20_prefill: 8 x 2048 Zipf(1.1) tokens, d20 bf16 N(0,0.02) weights, "
+                               "last-position logits + argmax", "batch": B, "seq_len": T,
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (1.0 GB of weights streamed per step)"},
+        "roofline": roofline,
+        "step_tflops": step_tflops, "step_frac_of_peak": step_tflops / peak_tc,
+        "kernel_time_share": kernel_share,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clk,
+        "decode": decode,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    kv.close()
+    model.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local):
+    import torch
+    import kv_cache_transformer_b200 as nc
+    import nc_synth as syn
+    B, T, S, V = wd.batch, wd.prompt_len, args.decode_steps, cfg.vocab
+    prompts = torch.from_numpy(syn.prompt_tokens(wd)).cuda()
+    logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
+    cur = torch.empty((B,), dtype=torch.int32, device="cuda")
+    nxt = torch.empty((B,), dtype=torch.int32, device="cuda")
+    positions = [torch.full((B,), T + s, dtype=torch.int32, device="cuda") for s in range(S)]
+    stream = torch.cuda.current_stream()
+    # warm-up: a prefill and a few steps, then a fresh prefill for the timed loop
+    model.prefill(kv, prompts, 0, logits, cur)
+    for s in range(min(args.warmup, S)):
+        model.decode_step(kv, cur, positions[s], None, logits, nxt)
+        cur, nxt = nxt, cur
+    model.prefill(kv, prompts, 0, logits, cur)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    clocks = ClockSampler(local)
+    barrier(world)
+    clocks.start()
+    model.profile(True)
+    model.profile_read()
+    n0 = nc.nc_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(S):
+        model.decode_step(kv, cur, positions[s], None, logits, nxt)
+        cur, nxt = nxt, cur
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = nc.nc_launch_count() - n0
+    kms, kn = model.profile_read()
+    model.profile(False)
+    clk = clocks.stop()
+    assert model.status() == 0
+    barrier(world)
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_step = t_ms / S
+    by = decode_bytes(cfg, B, T + (S + 1) / 2.0)
+    gbs = by["total"] / (ms_step / 1e3) / 1e9
+    gemm_ms = kms[nc.NC_K_GEMM] / S
+    gemm_gbs = by["weights_linear"] / (gemm_ms / 1e3) / 1e9
+    return {
+        "value": world * B * S / (t_ms / 1e3), "unit": "tok/s", "ms_per_step": ms_step, "steps": S,
+        "config": {"workload": "d20_decode: 32 sequences prefilled to 2048 Zipf tokens, 128 greedy steps "
+                               "(positions 2048..2175)", "batch": B, "ctx": [T, T + S]},
+        "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "bytes_per_step": by["total"], "peak_source": f"{peaks_src} hbm_gbs"},
+        "gemm_roofline": {"bound": "hbm", "kernel": "decode linear layers (weight streaming)",
+                          "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": gemm_gbs / peaks["hbm_gbs"], "bytes_per_step": by["weights_linear"]},
+        "kernel_time_share": {nc.K_CLASS_NAMES[i]: round(float(kms[i] / max(kms.sum(), 1e-9)), 4)
+                              for i in range(nc.NC_K_COUNT)},
+        "gpu_launches": int(launches), "clocks": clk,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=128,
+                    help="tokens of one prompt the CPU oracle runs per sample")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

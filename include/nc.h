@@ -140,6 +140,29 @@ int nc_decode_step(nc_model *model, nc_kv *kv, const int32_t *d_tokens, const in
  * NC_ECUDA. */
 int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream);
 
+/* ---- tracing ----
+ * Kernel classes for nc_profile_read. */
+#define NC_K_GEMM 0   /* linear layers: QKV, O-proj, MLP fc, MLP proj */
+#define NC_K_ATTN 1   /* attention, prefill or decode (with any split combine) */
+#define NC_K_HEAD 2   /* final norm, lm_head with softcap, token pick */
+#define NC_K_MISC 3   /* embedding, norms, RoPE/QK norm/KV append, bookkeeping, fork */
+#define NC_K_COUNT 4
+
+/* Turn per-class device timing on (1) or off (0) for calls on this model.
+ * When on, every launch (or fused group of launches) is bracketed by CUDA
+ * events on the call's stream; the events add no work on the device. */
+int nc_profile_enable(nc_model *model, int on);
+
+/* Sum of event-timed durations in ms (ms[NC_K_COUNT]) and kernel launch
+ * counts (launches[NC_K_COUNT]) per class since profiling was enabled or
+ * last read; then resets them. Synchronises the device. Either output may be
+ * NULL. */
+int nc_profile_read(nc_model *model, double *ms, long long *launches);
+
+/* Number of kernels this library has launched in this process so far
+ * (a CUDA graph replay counts each of its kernel nodes). */
+unsigned long long nc_launch_count(void);
+
 /* Message for the last failing nc_* call on this thread ("" if none). */
 const char *nc_last_error(void);
 

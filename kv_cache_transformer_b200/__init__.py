@@ -33,7 +33,10 @@ NC_F32, NC_BF16 = 0, 1
 EXPORTS = (
     "nc_model_create", "nc_model_destroy", "nc_device_status", "nc_kv_create", "nc_kv_destroy",
     "nc_kv_lengths", "nc_prefill", "nc_decode_step", "nc_kv_fork", "nc_last_error",
+    "nc_profile_enable", "nc_profile_read", "nc_launch_count",
 )
+NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_COUNT = 0, 1, 2, 3, 4
+K_CLASS_NAMES = ("gemm", "attn", "head", "misc")
 
 
 class NcError(RuntimeError):
@@ -74,8 +77,12 @@ def lib() -> ctypes.CDLL:
             L.nc_kv_fork.argtypes = [vp, i, vp, i, i, vp]
             L.nc_last_error.restype = ctypes.c_char_p
             L.nc_last_error.argtypes = []
+            L.nc_profile_enable.argtypes = [vp, i]
+            L.nc_profile_read.argtypes = [vp, vp, vp]
+            L.nc_launch_count.argtypes = []
+            L.nc_launch_count.restype = ctypes.c_ulonglong
             for name in EXPORTS:
-                if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error"):
+                if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error", "nc_launch_count"):
                     getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -186,6 +193,22 @@ def nc_kv_fork(src_h, src_seq: int, dst_h, dst_first: int, n: int, stream=None):
     _check(lib().nc_kv_fork(src_h, int(src_seq), dst_h, int(dst_first), int(n), _stream(stream)))
 
 
+def nc_profile_enable(model_h, on: bool = True):
+    _check(lib().nc_profile_enable(model_h, 1 if on else 0))
+
+
+def nc_profile_read(model_h):
+    """-> (ms[NC_K_COUNT], launches[NC_K_COUNT]) per kernel class since the last read."""
+    ms = np.zeros(NC_K_COUNT, dtype=np.float64)
+    n = np.zeros(NC_K_COUNT, dtype=np.int64)
+    _check(lib().nc_profile_read(model_h, ctypes.c_void_p(ms.ctypes.data), ctypes.c_void_p(n.ctypes.data)))
+    return ms, n
+
+
+def nc_launch_count() -> int:
+    return int(lib().nc_launch_count())
+
+
 # ----------------------------------------------------------------- wrappers
 class Model:
     """A model on the current CUDA device (weights copied from a host blob)."""
@@ -212,6 +235,12 @@ class Model:
 
     def status(self) -> int:
         return nc_device_status(self._h)
+
+    def profile(self, on: bool = True):
+        nc_profile_enable(self._h, on)
+
+    def profile_read(self):
+        return nc_profile_read(self._h)
 
     def kv(self, max_batch: int, max_seq: int) -> "KVCache":
         return KVCache(self, max_batch, max_seq)

@@ -53,6 +53,40 @@ size_t blob_elems(const nc_config &c) {
 
 inline cudaStream_t as_stream(void *s) { return (cudaStream_t)s; }
 
+cudaEvent_t take_event(nc_model *m) {
+  if (!m->event_pool.empty()) {
+    cudaEvent_t e = m->event_pool.back();
+    m->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets the launches issued in its lifetime with CUDA events when the
+// model's profiling is on (nc_profile_enable); a no-op otherwise.
+struct ProfScope {
+  nc_model *m;
+  int cls;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  unsigned long long n0 = 0;
+  ProfScope(nc_model *m_, int cls_, cudaStream_t s_) : m(m_), cls(cls_), s(s_) {
+    if (m->prof) {
+      a = take_event(m);
+      n0 = nc::g_launches.load();
+      cudaEventRecord(a, s);
+    }
+  }
+  ~ProfScope() {
+    if (!a) return;
+    cudaEvent_t b = take_event(m);
+    cudaEventRecord(b, s);
+    m->prof_recs.push_back({cls, (long long)(nc::g_launches.load() - n0), a, b});
+  }
+};
+
 inline void *layer_ptr(const nc_kv *kv, void *base, int l) {
   return (char *)base + (size_t)l * kv->layer_elems * kv->model->elem;
 }
@@ -66,15 +100,36 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
   for (int l = 0; l < c.depth; l++) {
     const nc_layer_w &w = m->layers[l];
     void *kc = layer_ptr(kv, kv->k, l), *vc = layer_ptr(kv, kv->v, l);
-    nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
-    nc::k_gemm_generic(c.dtype, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s);
-    nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, H, Hkv, hd, kv->rope, kv->q, kc, vc, kv->max_seq, valid,
-                             c.norm_eps, s);
-    nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, H, Hkv, hd, kv->max_seq, kv->y, s);
-    nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s);
-    nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
-    nc::k_gemm_generic(c.dtype, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s);
-    nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s);
+    {
+      ProfScope p(m, NC_K_MISC, s);
+      nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
+    }
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      nc::k_gemm_generic(c.dtype, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s);
+    }
+    {
+      ProfScope p(m, NC_K_MISC, s);
+      nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, H, Hkv, hd, kv->rope, kv->q, kc, vc, kv->max_seq, valid,
+                               c.norm_eps, s);
+    }
+    {
+      ProfScope p(m, NC_K_ATTN, s);
+      nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, H, Hkv, hd, kv->max_seq, kv->y, s);
+    }
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s);
+    }
+    {
+      ProfScope p(m, NC_K_MISC, s);
+      nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
+    }
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      nc::k_gemm_generic(c.dtype, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s);
+      nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s);
+    }
   }
   return NC_OK;
 }
@@ -84,6 +139,7 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
 void run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, float *logits, const uint8_t *valid,
               cudaStream_t s) {
   const nc_config &c = m->cfg;
+  ProfScope p(m, NC_K_HEAD, s);
   nc::k_rmsnorm_rows(c.dtype, kv->x, rows, c.d_model, stride, offset, c.norm_eps, kv->h, s);
   nc::k_gemm_generic(c.dtype, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab,
                      c.softcap, valid, s);
@@ -147,6 +203,11 @@ int nc_model_create(const nc_config *cfg, const void *host_blob, size_t blob_byt
 void nc_model_destroy(nc_model *m) {
   if (!m) return;
   cudaDeviceSynchronize();
+  for (auto &r : m->prof_recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (cudaEvent_t e : m->event_pool) cudaEventDestroy(e);
   cudaFree(m->blob);
   cudaFree(m->status);
   delete m;
@@ -247,8 +308,11 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
   const nc_config &c = m->cfg;
   cudaStream_t s = as_stream(stream);
   int M = B * T;
-  nc::k_prefill_begin(kv->len, kv->valid, B, T, s);
-  nc::k_embed_norm(c.dtype, d_tokens, M, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
+  {
+    ProfScope p(m, NC_K_MISC, s);
+    nc::k_prefill_begin(kv->len, kv->valid, B, T, s);
+    nc::k_embed_norm(c.dtype, d_tokens, M, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
+  }
   nc::RowMap rm{T, nullptr};
   run_blocks(m, kv, M, rm, s);
   float *logits;
@@ -271,7 +335,10 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
     last_off = 0;
     row_stride = c.vocab;
   }
-  if (d_next) nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
+  if (d_next) {
+    ProfScope p(m, NC_K_HEAD, s);
+    nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -284,13 +351,19 @@ int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_
   if (B > kv->max_batch) return fail(NC_ERANGE, "B=%d > max_batch=%d", B, kv->max_batch);
   const nc_config &c = m->cfg;
   cudaStream_t s = as_stream(stream);
-  nc::k_decode_begin(d_positions, kv->len, kv->valid, B, kv->max_seq, m->status, s);
-  nc::k_embed_norm(c.dtype, d_tokens, B, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
+  {
+    ProfScope p(m, NC_K_MISC, s);
+    nc::k_decode_begin(d_positions, kv->len, kv->valid, B, kv->max_seq, m->status, s);
+    nc::k_embed_norm(c.dtype, d_tokens, B, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
+  }
   nc::RowMap rm{1, d_positions};
   run_blocks(m, kv, B, rm, s);
   float *logits = d_logits ? d_logits : kv->logits;
   run_head(m, kv, B, 1, 0, logits, kv->valid, s);
-  if (d_next) nc::k_argmax_rows(logits, B, c.vocab, c.vocab, d_noise, d_next, kv->valid, s);
+  if (d_next) {
+    ProfScope p(m, NC_K_HEAD, s);
+    nc::k_argmax_rows(logits, B, c.vocab, c.vocab, d_noise, d_next, kv->valid, s);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -306,11 +379,41 @@ int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *
   if (src == dst && src_seq >= dst_first && src_seq < dst_first + n)
     return fail(NC_EINVAL, "source sequence is among the destinations");
   const nc_config &c = src->model->cfg;
+  ProfScope p(src->model, NC_K_MISC, as_stream(stream));
   nc::k_kv_fork((int)src->model->elem, src->k, src->v, src->layer_elems, src->max_seq, src_seq, src->len, dst->k,
                 dst->v, dst->layer_elems, dst->max_seq, dst_first, n, dst->len, c.depth, c.n_kv_head * c.head_dim,
                 src->model->status, as_stream(stream));
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
+
+int nc_profile_enable(nc_model *m, int on) {
+  if (!m) return fail(NC_EINVAL, "model is NULL");
+  m->prof = on != 0;
+  return NC_OK;
+}
+
+int nc_profile_read(nc_model *m, double *ms, long long *launches) {
+  if (!m) return fail(NC_EINVAL, "model is NULL");
+  NC_CUDA_TRY(cudaDeviceSynchronize());
+  double t[NC_K_COUNT] = {0};
+  long long n[NC_K_COUNT] = {0};
+  for (auto &r : m->prof_recs) {
+    float e = 0.f;
+    if (cudaEventElapsedTime(&e, r.a, r.b) == cudaSuccess) t[r.cls] += e;
+    n[r.cls] += r.launches;
+    m->event_pool.push_back(r.a);
+    m->event_pool.push_back(r.b);
+  }
+  m->prof_recs.clear();
+  cudaGetLastError();
+  for (int i = 0; i < NC_K_COUNT; i++) {
+    if (ms) ms[i] = t[i];
+    if (launches) launches[i] = n[i];
+  }
+  return NC_OK;
+}
+
+unsigned long long nc_launch_count(void) { return nc::g_launches.load(); }
 
 }  // extern "C"

@@ -15,6 +15,8 @@
 
 namespace nc {
 
+std::atomic<unsigned long long> g_launches{0};
+
 // --------------------------------------------------------------- sequences
 __global__ void prefill_begin_kernel(int32_t *len, uint8_t *valid, int B, int T) {
   int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -25,6 +27,7 @@ __global__ void prefill_begin_kernel(int32_t *len, uint8_t *valid, int B, int T)
 }
 
 void k_prefill_begin(int32_t *len, uint8_t *valid, int B, int T, cudaStream_t s) {
+  count_launch();
   prefill_begin_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, valid, B, T);
 }
 
@@ -43,6 +46,7 @@ __global__ void decode_begin_kernel(const int32_t *positions, int32_t *len, uint
 
 void k_decode_begin(const int32_t *positions, int32_t *len, uint8_t *valid, int B, int max_seq,
                     uint32_t *status, cudaStream_t s) {
+  count_launch();
   decode_begin_kernel<<<(B + 127) / 128, 128, 0, s>>>(positions, len, valid, B, max_seq, status);
 }
 
@@ -71,6 +75,7 @@ __global__ void embed_norm_kernel(const int32_t *tokens, const T *wte, int d, in
 void k_embed_norm(int dtype, const int32_t *tokens, int M, const void *wte, int d, int vocab, float eps,
                   float *x, uint32_t *status, cudaStream_t s) {
   if (M <= 0) return;
+  count_launch();
   if (dtype == NC_F32)
     embed_norm_kernel<float><<<M, 256, 0, s>>>(tokens, (const float *)wte, d, vocab, eps, x, status);
   else
@@ -94,6 +99,7 @@ __global__ void rmsnorm_rows_kernel(const float *x, int d, int src_stride, int s
 void k_rmsnorm_rows(int dtype, const float *x, int rows, int d, int src_stride, int src_offset, float eps,
                     void *out, cudaStream_t s) {
   if (rows <= 0) return;
+  count_launch();
   if (dtype == NC_F32)
     rmsnorm_rows_kernel<float><<<rows, 256, 0, s>>>(x, d, src_stride, src_offset, eps, (float *)out);
   else
@@ -168,10 +174,10 @@ static void gemm_generic_t(int epi, const void *A, int lda, const void *W, int M
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   const T *a = (const T *)A, *w = (const T *)W;
   switch (epi) {
-    case EPI_STORE: gemm_generic_kernel<T, EPI_STORE><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
-    case EPI_RELU2: gemm_generic_kernel<T, EPI_RELU2><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
-    case EPI_RESID: gemm_generic_kernel<T, EPI_RESID><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
-    default: gemm_generic_kernel<T, EPI_SOFTCAP><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
+    case EPI_STORE: count_launch(); gemm_generic_kernel<T, EPI_STORE><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
+    case EPI_RELU2: count_launch(); gemm_generic_kernel<T, EPI_RELU2><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
+    case EPI_RESID: count_launch(); gemm_generic_kernel<T, EPI_RESID><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
+    default: count_launch(); gemm_generic_kernel<T, EPI_SOFTCAP><<<grid, 256, 0, s>>>(a, lda, w, M, N, K, out, ldo, cap, valid); break;
   }
 }
 
@@ -230,6 +236,7 @@ void k_rope_qknorm_append(int dtype, const void *qkv, RowMap rm, int M, int H, i
                           const uint8_t *valid, float eps, cudaStream_t s) {
   if (M <= 0) return;
   size_t smem = sizeof(float) * ((size_t)(H + 2 * Hkv) * hd + H + Hkv);
+  count_launch();
   if (dtype == NC_F32)
     rope_qknorm_kernel<float><<<M, 128, smem, s>>>((const float *)qkv, rm, H, Hkv, hd, rope, (float *)q_out,
                                                    (float *)kc, (float *)vc, max_seq, valid, eps);
@@ -286,11 +293,13 @@ void k_attention_generic(int dtype, const void *q, const void *kc, const void *v
   if (dtype == NC_F32) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    count_launch();
     attn_generic_kernel<float><<<grid, 128, smem, s>>>((const float *)q, (const float *)kc, (const float *)vc, rm,
                                                        H, Hkv, hd, max_seq, (float *)y);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_generic_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    count_launch();
     attn_generic_kernel<bf16><<<grid, 128, smem, s>>>((const bf16 *)q, (const bf16 *)kc, (const bf16 *)vc, rm, H,
                                                       Hkv, hd, max_seq, (bf16 *)y);
   }
@@ -326,6 +335,7 @@ __global__ void argmax_rows_kernel(const float *logits, int V, long long row_str
 void k_argmax_rows(const float *logits, int rows, int V, long long row_stride, const float *noise,
                    int32_t *next, const uint8_t *valid, cudaStream_t s) {
   if (rows <= 0) return;
+  count_launch();
   argmax_rows_kernel<<<rows, 512, 0, s>>>(logits, V, row_stride, noise, next, valid);
 }
 
@@ -366,6 +376,7 @@ void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_
     // no layers: only the lengths change
     grid.y = 1;
   }
+  count_launch();
   kv_fork_kernel<<<grid, 256, 0, s>>>((const uint32_t *)src_k, (const uint32_t *)src_v, src_layer_words,
                                       src_seq_words, (size_t)src_seq * src_seq_words, src_len + src_seq,
                                       (uint32_t *)dst_k, (uint32_t *)dst_v, dst_layer_words, dst_seq_words,

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <vector>
 
 #include "nc.h"
@@ -28,6 +29,15 @@ struct nc_model {
   std::vector<nc_layer_w> layers;
   uint32_t *status = nullptr;  // device status word (NC_DEV_* bits)
   bool fast = false;           // bf16 + shapes the sm_100a kernels cover
+  // tracing (nc_profile_*)
+  bool prof = false;
+  struct ProfRec {
+    int cls;
+    long long launches;
+    cudaEvent_t a, b;
+  };
+  std::vector<ProfRec> prof_recs;
+  std::vector<cudaEvent_t> event_pool;
 };
 
 struct nc_kv {
@@ -50,6 +60,10 @@ struct nc_kv {
 };
 
 namespace nc {
+
+// Kernels launched by this library (nc_launch_count).
+extern std::atomic<unsigned long long> g_launches;
+inline void count_launch(unsigned long long n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 enum Epi { EPI_STORE = 0, EPI_RELU2 = 1, EPI_RESID = 2, EPI_SOFTCAP = 3 };
 
