@@ -1,0 +1,40 @@
+/*
+ * nc_kernels.h — kernel-level entry points of the B200 engine library.
+ *
+ * These expose single building blocks of the forward pass for callers that
+ * assemble their own pipeline (and for unit tests of the kernels). Same
+ * conventions as nc.h: d_* are device pointers owned by the caller, work is
+ * enqueued on `stream` (a cudaStream_t, NULL = legacy default stream),
+ * return NC_OK or an NC_E* code with nc_last_error() set.
+ */
+#ifndef NC_KERNELS_H
+#define NC_KERNELS_H
+
+#include "nc.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogues of nc_gemm_bf16. */
+#define NC_EPI_STORE 0    /* d_out bf16 [M, ldo]: acc */
+#define NC_EPI_RELU2 1    /* d_out bf16 [M, ldo]: relu(acc)^2 (the MLP activation) */
+#define NC_EPI_RESID 2    /* d_out fp32 [M, ldo]: d_out += acc (residual add) */
+#define NC_EPI_SOFTCAP 3  /* d_out fp32 [M, ldo]: cap * tanh(acc / cap) (logit softcap) */
+
+/* Linear layer without bias (feature list: "no bias in the linear layers"):
+ * acc[m, n] = sum_k A[m, k] * W[n, k], A bf16 [M, K] with row pitch lda
+ * elements, W bf16 [N, K] row-major (a weight stored [out, in]), fp32
+ * accumulation; the epilogue writes d_out. Runs on the tcgen05 tensor-core
+ * kernel when M >= 128, K % 64 == 0, N % 32 == 0 and lda % 8 == 0 (16-byte
+ * rows for TMA), otherwise on the generic kernel. Device pointers must be
+ * 16-byte aligned. Errors: NC_EINVAL (null pointer, non-positive size,
+ * lda < K, ldo < N, unknown epilogue), NC_ECUDA. */
+int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K, int epi, void *d_out, int ldo,
+                 float cap, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NC_KERNELS_H */

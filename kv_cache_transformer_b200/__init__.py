@@ -33,8 +33,9 @@ NC_F32, NC_BF16 = 0, 1
 EXPORTS = (
     "nc_model_create", "nc_model_destroy", "nc_device_status", "nc_kv_create", "nc_kv_destroy",
     "nc_kv_lengths", "nc_prefill", "nc_decode_step", "nc_kv_fork", "nc_last_error",
-    "nc_profile_enable", "nc_profile_read", "nc_launch_count",
+    "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
 )
+NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_COUNT = 0, 1, 2, 3, 4
 K_CLASS_NAMES = ("gemm", "attn", "head", "misc")
 
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
             L.nc_profile_read.argtypes = [vp, vp, vp]
             L.nc_launch_count.argtypes = []
             L.nc_launch_count.restype = ctypes.c_ulonglong
+            L.nc_gemm_bf16.argtypes = [vp, i, vp, i, i, i, i, vp, i, ctypes.c_float, vp]
             for name in EXPORTS:
                 if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error", "nc_launch_count"):
                     getattr(L, name).restype = ctypes.c_int
@@ -207,6 +209,19 @@ def nc_profile_read(model_h):
 
 def nc_launch_count() -> int:
     return int(lib().nc_launch_count())
+
+
+def nc_gemm_bf16(A, W, out, epi: int = NC_EPI_STORE, cap: float = 15.0, stream=None):
+    """out (epi) A @ W.T for bf16 CUDA tensors A [M, K] (row pitch A.stride(0)) and W [N, K]."""
+    import torch
+    M, K = A.shape
+    N = W.shape[0]
+    if A.dtype != torch.bfloat16 or W.dtype != torch.bfloat16 or A.stride(1) != 1 or not W.is_contiguous():
+        raise TypeError("A and W must be bf16 with unit inner stride (W contiguous)")
+    if W.shape[1] != K or out.shape[0] < M or out.stride(1) != 1:
+        raise ValueError("shape mismatch")
+    _check(lib().nc_gemm_bf16(ctypes.c_void_p(A.data_ptr()), A.stride(0), ctypes.c_void_p(W.data_ptr()), M, N, K,
+                              int(epi), ctypes.c_void_p(out.data_ptr()), out.stride(0), float(cap), _stream(stream)))
 
 
 # ----------------------------------------------------------------- wrappers

@@ -8,6 +8,7 @@
 #include <string>
 
 #include "nc_internal.h"
+#include "nc_kernels.h"
 
 namespace {
 
@@ -91,6 +92,17 @@ inline void *layer_ptr(const nc_kv *kv, void *base, int l) {
   return (char *)base + (size_t)l * kv->layer_elems * kv->model->elem;
 }
 
+// Linear layer out (epi) A[M,K] * W[N,K]^T: tcgen05 kernel for bf16 models
+// once there is at least one full 128-row tile, the generic kernel otherwise.
+void linear(nc_model *m, int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
+            float cap, const uint8_t *valid, cudaStream_t s) {
+  if (m->fast && M >= 128 && !valid && nc::gemm_tc_supported(M, N, K, lda)) {
+    if (nc::k_gemm_tc(epi, A, lda, W, M, N, K, out, ldo, cap, m->status, m->num_sms, s) == cudaSuccess) return;
+    cudaGetLastError();
+  }
+  nc::k_gemm_generic(m->cfg.dtype, epi, A, lda, W, M, N, K, out, ldo, cap, valid, s);
+}
+
 // The transformer blocks for M rows already embedded into kv->x.
 int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
@@ -106,7 +118,7 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
-      nc::k_gemm_generic(c.dtype, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s);
+      linear(m, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s);
     }
     {
       ProfScope p(m, NC_K_MISC, s);
@@ -119,7 +131,7 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
-      nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s);
+      linear(m, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s);
     }
     {
       ProfScope p(m, NC_K_MISC, s);
@@ -127,8 +139,8 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
-      nc::k_gemm_generic(c.dtype, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s);
-      nc::k_gemm_generic(c.dtype, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s);
+      linear(m, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s);
+      linear(m, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s);
     }
   }
   return NC_OK;
@@ -141,8 +153,7 @@ void run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, float *l
   const nc_config &c = m->cfg;
   ProfScope p(m, NC_K_HEAD, s);
   nc::k_rmsnorm_rows(c.dtype, kv->x, rows, c.d_model, stride, offset, c.norm_eps, kv->h, s);
-  nc::k_gemm_generic(c.dtype, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab,
-                     c.softcap, valid, s);
+  linear(m, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab, c.softcap, valid, s);
 }
 
 }  // namespace
@@ -196,6 +207,7 @@ int nc_model_create(const nc_config *cfg, const void *host_blob, size_t blob_byt
     p += d * F * elem;
   }
   m->wlm = p;
+  m->fast = c.dtype == NC_BF16;
   *out = m;
   return NC_OK;
 }
@@ -415,5 +427,29 @@ int nc_profile_read(nc_model *m, double *ms, long long *launches) {
 }
 
 unsigned long long nc_launch_count(void) { return nc::g_launches.load(); }
+
+int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K, int epi, void *d_out, int ldo,
+                 float cap, void *stream) {
+  if (!d_A || !d_W || !d_out) return fail(NC_EINVAL, "null pointer");
+  if (M <= 0 || N <= 0 || K <= 0 || lda < K || ldo < N) return fail(NC_EINVAL, "bad GEMM shape");
+  if (epi < NC_EPI_STORE || epi > NC_EPI_SOFTCAP) return fail(NC_EINVAL, "unknown epilogue %d", epi);
+  static uint32_t *status = nullptr;
+  static int sms = 0;
+  if (!status) {
+    int dev = 0;
+    NC_CUDA_TRY(cudaGetDevice(&dev));
+    NC_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    NC_CUDA_TRY(cudaMalloc(&status, sizeof(uint32_t)));
+    NC_CUDA_TRY(cudaMemset(status, 0, sizeof(uint32_t)));
+  }
+  cudaStream_t s = as_stream(stream);
+  if (M >= 128 && nc::gemm_tc_supported(M, N, K, lda) &&
+      nc::k_gemm_tc(epi, d_A, lda, d_W, M, N, K, d_out, ldo, cap, status, sms, s) == cudaSuccess)
+    return NC_OK;
+  cudaGetLastError();
+  nc::k_gemm_generic(NC_BF16, epi, d_A, lda, d_W, M, N, K, d_out, ldo, cap, nullptr, s);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
 
 }  // extern "C"

@@ -1,0 +1,327 @@
+// nc_attn_tc.cu — causal multi-query prefill attention on tcgen05.
+//
+// With one KV head, the H query heads of a position all read the same keys
+// and values (the feature list's multi-query attention). The queries of a
+// sequence, stored [T, H, hd], are therefore one [T*H, hd] matrix whose row
+// r = t*H + h belongs to position t. A CTA takes 128 consecutive rows
+// (about 128/H positions, every head) and streams the sequence's K/V tiles
+// once for all of them:
+//   S  = Q K^T          (tcgen05, M=128 rows, N=128 keys, K=hd=128) -> TMEM
+//   P  = exp(S*scale - m) with the causal mask key <= t(row), online max/sum
+//   O += P V            (tcgen05, A = P from shared memory, B = V read
+//                        MN-major straight from the cache layout)  -> TMEM
+// and finally y = O / l in bf16.
+// Warp roles (192 threads): warp 0 TMA producer (Q once, K/V tiles through a
+// 2-stage ring), warp 1 TMEM allocator + MMA issuer (S_{j+1} overlaps the
+// softmax of tile j), warps 2-5 softmax / O rescale / epilogue, one thread
+// per row. Waits are bounded as in the GEMM.
+#include "nc_internal.h"
+#include "nc_sm100.cuh"
+
+namespace nc {
+using namespace sm100;
+
+bool make_map_bf16_k64(CUtensorMap *map, const void *ptr, int rows, int cols, int ld, int box_rows);
+
+namespace {
+
+constexpr int HD = 128;           // head dim handled here
+constexpr int BR = 128;           // rows (position, head) per CTA
+constexpr int BKV = 128;          // keys per tile
+constexpr int ST = 2;             // K/V stages
+constexpr int SUB = 128 * 64 * 2; // one 128-row x 64-column swizzled box: 16 KB
+constexpr int TILE = 2 * SUB;     // 128 x 128 bf16: 32 KB
+constexpr int OFF_Q = 0;
+constexpr int OFF_P = TILE;
+constexpr int OFF_K = 2 * TILE;              // ST tiles
+constexpr int OFF_V = 2 * TILE + ST * TILE;  // ST tiles
+constexpr int OFF_BAR = 2 * TILE + 2 * ST * TILE;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;  // O: cols 0..127, S buffers: 128..255, 256..383
+
+struct AttnArgs {
+  int T, H, max_seq;
+  int rows_per_seq;  // T*H
+  float scale_log2;  // log2(e) / sqrt(hd)
+  bf16 *y;           // [B*T*H, 128]
+  uint32_t *status;
+};
+
+// Shared-memory descriptor for an MN-major operand (V: keys x dims, dims
+// contiguous) written by TMA with 128-byte swizzle as two boxes of 64 dims:
+// 8-key groups 1024 B apart (stride byte offset), the second 64-dim box 16 KB
+// further (leading byte offset).
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)(SUB >> 4) << 16;   // leading byte offset: next 64-element MN chunk
+  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: next 8-row K group
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+      "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+      "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                           const __grid_constant__ CUtensorMap mapV, AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint32_t raw = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  uint64_t *q_full = bar;             // 1
+  uint64_t *k_full = bar + 1;         // ST
+  uint64_t *v_full = k_full + ST;     // ST
+  uint64_t *kv_empty = v_full + ST;   // ST
+  uint64_t *s_full = kv_empty + ST;   // 2
+  uint64_t *p_full = s_full + 2;      // 1 (128 arrivals)
+  uint64_t *o_done = p_full + 1;      // 1
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_rt = (a.rows_per_seq + BR - 1) / BR;
+  const int rt = n_rt - 1 - blockIdx.x;  // heaviest tiles first
+  const int b = blockIdx.y;
+  const int row0 = rt * BR;              // first row inside the sequence
+  int t_max = (row0 + BR - 1) / a.H;
+  if (t_max > a.T - 1) t_max = a.T - 1;
+  const int n_kv = t_max / BKV + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < ST; s++) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tO = tmem, tS = tmem + 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int qrow = b * a.rows_per_seq + row0;
+      const int krow = b * a.max_seq;
+      mbar_arrive_expect_tx(q_full, TILE);
+      tma_load_2d(smem + OFF_Q, &mapQ, 0, qrow, q_full);
+      tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, qrow, q_full);
+      for (int j = 0; j < n_kv; j++) {
+        const int s = j % ST;
+        const uint32_t ph = (j / ST) & 1;
+        if (!mbar_wait(&kv_empty[s], ph ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(&k_full[s], TILE);
+        tma_load_2d(smem + OFF_K + s * TILE, &mapK, 0, krow + j * BKV, &k_full[s]);
+        tma_load_2d(smem + OFF_K + s * TILE + SUB, &mapK, 64, krow + j * BKV, &k_full[s]);
+        mbar_arrive_expect_tx(&v_full[s], TILE);
+        tma_load_2d(smem + OFF_V + s * TILE, &mapV, 0, krow + j * BKV, &v_full[s]);
+        tma_load_2d(smem + OFF_V + s * TILE + SUB, &mapV, 64, krow + j * BKV, &v_full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(BR, BKV);
+      const uint32_t id_o = idesc_bf16_f32(BR, HD) | (1u << 16);  // B (V) is MN-major
+      const uint32_t q0 = smem_u32(smem + OFF_Q), p0 = smem_u32(smem + OFF_P);
+      bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
+      // S_j = Q K_j^T into S buffer j % 2
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % ST;
+        if (!mbar_wait(&k_full[s], (j / ST) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t k0 = smem_u32(smem + OFF_K + s * TILE);
+        const uint32_t d = tS + (j & 1) * 128;
+#pragma unroll
+        for (int k = 0; k < HD / 16; k++) {
+          const uint32_t off = (k >> 2) * SUB + (k & 3) * 32;
+          mma_bf16(d, desc_k_sw128(q0 + off), desc_k_sw128(k0 + off), id_s, k != 0);
+        }
+        mma_commit(&s_full[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < n_kv && ok; j++) {
+        if (j + 1 < n_kv && !issue_s(j + 1)) break;
+        if (!mbar_wait(p_full, j & 1, abort_flag, a.status)) break;
+        const int s = j % ST;
+        if (!mbar_wait(&v_full[s], (j / ST) & 1, abort_flag, a.status)) break;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(smem + OFF_V + s * TILE);
+#pragma unroll
+        for (int k = 0; k < BKV / 16; k++) {
+          const uint32_t poff = (k >> 2) * SUB + (k & 3) * 32;
+          mma_bf16(tO, desc_k_sw128(p0 + poff), desc_mn_sw128(v0 + k * 2048), id_o, (j | k) != 0);
+        }
+        mma_commit(o_done);
+        mma_commit(&kv_empty[s]);
+      }
+    }
+  } else {
+    // softmax / correction / epilogue: thread <-> row
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int row = row0 + r;                  // row inside the sequence
+    const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    uint8_t *prow = smem + OFF_P + r * 128;    // row r of both 64-key boxes
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv && ok; j++) {
+      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sbase = tS + (j & 1) * 128 + lane_off;
+      const int kbase = j * BKV;
+      // pass 1: row max of the masked, scaled scores
+      float tmax = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < BKV; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(sbase + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; i++)
+          if (kbase + c + i <= t_row) tmax = fmaxf(tmax, __uint_as_float(v[i]) * a.scale_log2);
+      }
+      const float m_new = fmaxf(m, tmax);
+      const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+      // the previous P.V must be finished before O or the P buffer change
+      if (j > 0 && !mbar_wait(o_done, (j - 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      tc_fence_after();
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + c, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + lane_off + c, o);
+        }
+        tmem_st_wait();
+      }
+      // pass 2: p = exp2(s*scale_log2 - m_new), bf16 into the swizzled P tile
+      float sum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BKV; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(sbase + c, v);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float p0 = (kbase + c + i <= t_row) ? exp2f(__uint_as_float(v[i]) * a.scale_log2 - m_new) : 0.f;
+          float p1 = (kbase + c + i + 1 <= t_row) ? exp2f(__uint_as_float(v[i + 1]) * a.scale_log2 - m_new) : 0.f;
+          sum += p0 + p1;
+          pk[i / 2] = pack2(p0, p1);
+        }
+        // 32 keys = four 16-byte chunks; chunk index XOR (row & 7) (128-byte swizzle)
+        const int box = c >> 6;
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+          const int chunk = ((c & 63) >> 3) + q;
+          uint4 *dst = reinterpret_cast<uint4 *>(prow + box * SUB + ((chunk ^ (r & 7)) << 4));
+          *dst = make_uint4(pk[q * 4 + 0], pk[q * 4 + 1], pk[q * 4 + 2], pk[q * 4 + 3]);
+        }
+      }
+      l = l * alpha + sum;
+      m = m_new;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, a.status)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      bf16 *dst = a.y + ((size_t)b * a.rows_per_seq + row) * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + lane_off + c, o);
+        tmem_ld_wait();
+        if (row < a.rows_per_seq) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+#pragma unroll
+          for (int q = 0; q < 4; q++) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) f[i] = __uint_as_float(o[q * 8 + i]) * inv;
+            d4[q] = make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
+          }
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+bool attn_prefill_tc_supported(int H, int Hkv, int hd) { return hd == HD && Hkv == 1 && H >= 1; }
+
+// q: [B*T*H, 128] bf16 (rotated + normed), kc/vc: layer cache [max_batch*max_seq, 128],
+// y: [B*T*H, 128] bf16.
+cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int max_batch,
+                              int max_seq, void *y, uint32_t *status, cudaStream_t s) {
+  CUtensorMap mq, mk, mv;
+  const int rows = T * H;
+  if (!make_map_bf16_k64(&mq, q, B * rows, HD, HD, BR) ||
+      !make_map_bf16_k64(&mk, kc, max_batch * max_seq, HD, HD, BKV) ||
+      !make_map_bf16_k64(&mv, vc, max_batch * max_seq, HD, HD, BKV))
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  AttnArgs a;
+  a.T = T;
+  a.H = H;
+  a.max_seq = max_seq;
+  a.rows_per_seq = rows;
+  a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  a.y = (bf16 *)y;
+  a.status = status;
+  dim3 grid((rows + BR - 1) / BR, B);
+  count_launch();
+  attn_prefill_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace nc

@@ -89,4 +89,10 @@ void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_
                int dst_max_seq, int dst_first, int n, int32_t *dst_len, int depth, int kd, uint32_t *status,
                cudaStream_t s);
 
+
+// ---- sm_100a tensor-core GEMM (nc_gemm_tc.cu) ----
+bool gemm_tc_supported(int M, int N, int K, int lda);
+cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
+                      float cap, uint32_t *status, int num_sms, cudaStream_t s);
+
 }  // namespace nc

@@ -1,0 +1,79 @@
+"""Kernel-level parity: the tcgen05 GEMM entry point (nc_gemm_bf16) against a
+float64 CPU matmul of the same bf16 operands, for every epilogue, ragged and
+full-size shapes; rows outside M must stay untouched."""
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+
+def _ref(A, W, rows=None):
+    import torch
+    a = A.cpu().double() if rows is None else A.cpu().double()[rows]
+    return a @ W.cpu().double().T
+
+
+def _apply(epi, acc, prev, cap=15.0):
+    import kv_cache_transformer_b200 as nc
+    if epi == nc.NC_EPI_STORE:
+        return acc
+    if epi == nc.NC_EPI_RELU2:
+        return np.maximum(acc, 0) ** 2
+    if epi == nc.NC_EPI_RESID:
+        return prev + acc
+    return cap * np.tanh(acc / cap)
+
+
+def _tol(epi, want, K):
+    # bf16 outputs carry one rounding (relative 2^-8); fp32 outputs only the
+    # accumulation error of K fp32 partial sums, which grows like sqrt(K)
+    if epi in (0, 1):
+        return 2.0 ** -8 * np.abs(want) + 1e-4
+    return 3e-6 * np.sqrt(K) * (1 + np.abs(want))
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 256, 64),      # one tile, one k-block
+    (300, 1536, 1280),   # ragged M, d20 QKV width
+    (257, 1920, 1664),   # ragged M and N (d26 QKV), K not a multiple of 128
+    (1000, 5120, 1280),  # d20 MLP fc
+    (640, 1280, 5120),   # d20 MLP proj (long K)
+    (96, 512, 128),      # M < 128: generic kernel
+])
+@pytest.mark.parametrize("epi", [0, 1, 2, 3])
+def test_gemm_bf16_matches_float64(M, N, K, epi):
+    import torch
+    import kv_cache_transformer_b200 as nc
+    g = torch.Generator().manual_seed(M * 7 + N + K + epi)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    out_dtype = torch.bfloat16 if epi in (0, 1) else torch.float32
+    pad = 3
+    prev = torch.randn(M + pad, N, generator=g).to(out_dtype)
+    out = prev.clone().cuda()
+    nc.nc_gemm_bf16(A.cuda(), W.cuda(), out, epi)
+    torch.cuda.synchronize()
+    got = out.cpu().double().numpy()
+    acc = _ref(A, W).numpy()
+    want = _apply(epi, acc, prev[:M].double().numpy())
+    err = np.abs(got[:M] - want)
+    assert np.all(err <= _tol(epi, want, K)), f"max err {err.max():.3g}"
+    assert torch.equal(out[M:].cpu(), prev[M:]), "rows beyond M were written"
+
+
+def test_gemm_bf16_full_size_sampled_rows():
+    # d20 prefill MLP fc at full size (M = 8 x 2048): sampled rows only
+    import torch
+    import kv_cache_transformer_b200 as nc
+    M, N, K = 16384, 5120, 1280
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    nc.nc_gemm_bf16(A.cuda(), W.cuda(), out, nc.NC_EPI_RELU2)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(0).choice(M, 96, replace=False))
+    rows[-1] = M - 1
+    want = np.maximum(_ref(A, W, torch.from_numpy(rows)).numpy(), 0) ** 2
+    got = out.cpu()[torch.from_numpy(rows)].double().numpy()
+    assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-4)
