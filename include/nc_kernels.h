@@ -33,6 +33,17 @@ extern "C" {
 int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K, int epi, void *d_out, int ldo,
                  float cap, void *stream);
 
+/* Causal multi-query attention (one KV head shared by all H query heads;
+ * feature list: "multi-query attention") for B sequences of T positions:
+ *   y[b,t,h,:] = sum_{j<=t} softmax_j(q[b,t,h,:] . k[b,j,:] / sqrt(hd)) v[b,j,:]
+ * d_q, d_y bf16 [B, T, H, hd] (queries after RoPE and QK norm); d_k, d_v bf16
+ * [B, max_seq, hd] (keys after RoPE and QK norm; rows 0..T-1 of each sequence
+ * are used, rows T..max_seq-1 must hold finite values). Runs on the tcgen05
+ * kernel when hd == 128, else on the generic kernel. Errors: NC_EINVAL,
+ * NC_ECUDA. */
+int nc_attention_prefill_bf16(const void *d_q, const void *d_k, const void *d_v, int B, int T, int H, int hd,
+                              int max_seq, void *d_y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

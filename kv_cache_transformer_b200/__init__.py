@@ -34,6 +34,7 @@ EXPORTS = (
     "nc_model_create", "nc_model_destroy", "nc_device_status", "nc_kv_create", "nc_kv_destroy",
     "nc_kv_lengths", "nc_prefill", "nc_decode_step", "nc_kv_fork", "nc_last_error",
     "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
+    "nc_attention_prefill_bf16",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_COUNT = 0, 1, 2, 3, 4
@@ -83,6 +84,7 @@ def lib() -> ctypes.CDLL:
             L.nc_launch_count.argtypes = []
             L.nc_launch_count.restype = ctypes.c_ulonglong
             L.nc_gemm_bf16.argtypes = [vp, i, vp, i, i, i, i, vp, i, ctypes.c_float, vp]
+            L.nc_attention_prefill_bf16.argtypes = [vp, vp, vp, i, i, i, i, i, vp, vp]
             for name in EXPORTS:
                 if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error", "nc_launch_count"):
                     getattr(L, name).restype = ctypes.c_int
@@ -222,6 +224,18 @@ def nc_gemm_bf16(A, W, out, epi: int = NC_EPI_STORE, cap: float = 15.0, stream=N
         raise ValueError("shape mismatch")
     _check(lib().nc_gemm_bf16(ctypes.c_void_p(A.data_ptr()), A.stride(0), ctypes.c_void_p(W.data_ptr()), M, N, K,
                               int(epi), ctypes.c_void_p(out.data_ptr()), out.stride(0), float(cap), _stream(stream)))
+
+
+def nc_attention_prefill_bf16(q, k, v, y, stream=None):
+    """Causal MQA: q, y bf16 [B, T, H, hd]; k, v bf16 [B, max_seq, hd] (CUDA, contiguous)."""
+    import torch
+    B, T, H, hd = q.shape
+    if k.shape[0] != B or k.shape[2] != hd or k.shape != v.shape or y.shape != q.shape:
+        raise ValueError("shape mismatch")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (y, "y")):
+        _dptr(t, torch.bfloat16, name=n)
+    _check(lib().nc_attention_prefill_bf16(_dptr(q), _dptr(k), _dptr(v), B, T, H, hd, k.shape[1], _dptr(y),
+                                           _stream(stream)))
 
 
 # ----------------------------------------------------------------- wrappers

@@ -103,6 +103,18 @@ void linear(nc_model *m, int epi, const void *A, int lda, const void *W, int M, 
   nc::k_gemm_generic(m->cfg.dtype, epi, A, lda, W, M, N, K, out, ldo, cap, valid, s);
 }
 
+// Causal MQA attention of the M rows in kv->q against layer cache kc/vc.
+void attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  if (m->fast && !rm.pos && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim)) {
+    if (nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, kv->max_batch, kv->max_seq, kv->y, m->status,
+                              s) == cudaSuccess)
+      return;
+    cudaGetLastError();
+  }
+  nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->max_seq, kv->y, s);
+}
+
 // The transformer blocks for M rows already embedded into kv->x.
 int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
@@ -127,7 +139,7 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
     }
     {
       ProfScope p(m, NC_K_ATTN, s);
-      nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, H, Hkv, hd, kv->max_seq, kv->y, s);
+      attention(m, kv, kc, vc, M, rm, s);
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
@@ -265,6 +277,9 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   alloc(&kv->y, elem * rows * qd);
   alloc(&kv->f, elem * rows * F);
   alloc((void **)&kv->logits, sizeof(float) * (size_t)max_batch * c.vocab);
+  // zeroed caches: attention may read (and mask) slots past a sequence's length
+  if (e == cudaSuccess) e = cudaMemset(kv->k, 0, cache_bytes);
+  if (e == cudaSuccess) e = cudaMemset(kv->v, 0, cache_bytes);
   if (e == cudaSuccess) e = cudaMemset(kv->len, 0, sizeof(int32_t) * max_batch);
   if (e == cudaSuccess) e = cudaMemset(kv->valid, 0, max_batch);
   if (e == cudaSuccess) {
@@ -428,20 +443,49 @@ int nc_profile_read(nc_model *m, double *ms, long long *launches) {
 
 unsigned long long nc_launch_count(void) { return nc::g_launches.load(); }
 
+static int kernel_status_init(uint32_t **status, int *sms) {
+  static uint32_t *st = nullptr;
+  static int n = 0;
+  if (!st) {
+    int dev = 0;
+    NC_CUDA_TRY(cudaGetDevice(&dev));
+    NC_CUDA_TRY(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev));
+    NC_CUDA_TRY(cudaMalloc(&st, sizeof(uint32_t)));
+    NC_CUDA_TRY(cudaMemset(st, 0, sizeof(uint32_t)));
+  }
+  *status = st;
+  *sms = n;
+  return NC_OK;
+}
+
+int nc_attention_prefill_bf16(const void *d_q, const void *d_k, const void *d_v, int B, int T, int H, int hd,
+                              int max_seq, void *d_y, void *stream) {
+  if (!d_q || !d_k || !d_v || !d_y) return fail(NC_EINVAL, "null pointer");
+  if (B <= 0 || T <= 0 || H <= 0 || hd <= 0 || (hd & 1) || max_seq < T) return fail(NC_EINVAL, "bad attention shape");
+  uint32_t *status;
+  int sms;
+  int rc = kernel_status_init(&status, &sms);
+  if (rc) return rc;
+  cudaStream_t s = as_stream(stream);
+  if (nc::attn_prefill_tc_supported(H, 1, hd) &&
+      nc::k_attn_prefill_tc(d_q, d_k, d_v, B, T, H, B, max_seq, d_y, status, s) == cudaSuccess)
+    return NC_OK;
+  cudaGetLastError();
+  nc::RowMap rm{T, nullptr};
+  nc::k_attention_generic(NC_BF16, d_q, d_k, d_v, rm, B * T, H, 1, hd, max_seq, d_y, s);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
 int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K, int epi, void *d_out, int ldo,
                  float cap, void *stream) {
   if (!d_A || !d_W || !d_out) return fail(NC_EINVAL, "null pointer");
   if (M <= 0 || N <= 0 || K <= 0 || lda < K || ldo < N) return fail(NC_EINVAL, "bad GEMM shape");
   if (epi < NC_EPI_STORE || epi > NC_EPI_SOFTCAP) return fail(NC_EINVAL, "unknown epilogue %d", epi);
-  static uint32_t *status = nullptr;
-  static int sms = 0;
-  if (!status) {
-    int dev = 0;
-    NC_CUDA_TRY(cudaGetDevice(&dev));
-    NC_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    NC_CUDA_TRY(cudaMalloc(&status, sizeof(uint32_t)));
-    NC_CUDA_TRY(cudaMemset(status, 0, sizeof(uint32_t)));
-  }
+  uint32_t *status;
+  int sms;
+  int rc = kernel_status_init(&status, &sms);
+  if (rc) return rc;
   cudaStream_t s = as_stream(stream);
   if (M >= 128 && nc::gemm_tc_supported(M, N, K, lda) &&
       nc::k_gemm_tc(epi, d_A, lda, d_W, M, N, K, d_out, ldo, cap, status, sms, s) == cudaSuccess)

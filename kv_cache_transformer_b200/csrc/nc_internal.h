@@ -95,4 +95,10 @@ bool gemm_tc_supported(int M, int N, int K, int lda);
 cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
                       float cap, uint32_t *status, int num_sms, cudaStream_t s);
 
+
+// ---- sm_100a causal MQA prefill attention (nc_attn_tc.cu) ----
+bool attn_prefill_tc_supported(int H, int Hkv, int hd);
+cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int max_batch,
+                              int max_seq, void *y, uint32_t *status, cudaStream_t s);
+
 }  // namespace nc

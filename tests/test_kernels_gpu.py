@@ -77,3 +77,41 @@ def test_gemm_bf16_full_size_sampled_rows():
     want = np.maximum(_ref(A, W, torch.from_numpy(rows)).numpy(), 0) ** 2
     got = out.cpu()[torch.from_numpy(rows)].double().numpy()
     assert np.all(np.abs(got - want) <= 2.0 ** -8 * np.abs(want) + 1e-4)
+
+
+def _attn_ref(q, k, v, T):
+    """Causal MQA in float64: q [B,T,H,hd], k/v [B,S,hd] (first T rows used)."""
+    import torch
+    qd = q.double().permute(0, 2, 1, 3)                  # B,H,T,hd
+    kd, vd = k.double()[:, :T], v.double()[:, :T]        # B,T,hd
+    s = torch.einsum("bhtd,bjd->bhtj", qd, kd) / np.sqrt(q.shape[-1])
+    mask = torch.ones(T, T, dtype=torch.bool).triu(1)
+    s = s.masked_fill(mask, float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    return torch.einsum("bhtj,bjd->bhtd", p, vd).permute(0, 2, 1, 3)
+
+
+@pytest.mark.parametrize("B,T,H,hd,extra", [
+    (1, 1, 10, 128, 0),      # one position: y = v0
+    (2, 130, 10, 128, 6),    # two key tiles, ragged, cache longer than T
+    (1, 2048, 10, 128, 0),   # d20 prompt length: 16 key tiles, 160 row tiles
+    (2, 300, 13, 128, 20),   # d26 heads: rows per tile span partial positions
+    (3, 77, 15, 128, 3),     # d30 heads, last row tile partial
+    (2, 50, 2, 64, 0),       # head_dim 64: generic kernel
+])
+def test_attention_prefill_matches_float64(B, T, H, hd, extra):
+    import torch
+    import kv_cache_transformer_b200 as nc
+    g = torch.Generator().manual_seed(B * 1000 + T + H)
+    S = T + extra
+    q = torch.randn(B, T, H, hd, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, S, hd, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, S, hd, generator=g).to(torch.bfloat16)
+    y = torch.full((B, T, H, hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nc.nc_attention_prefill_bf16(q.cuda(), k.cuda(), v.cuda(), y)
+    torch.cuda.synchronize()
+    want = _attn_ref(q, k, v, T).numpy()
+    got = y.cpu().double().numpy()
+    err = np.abs(got - want)
+    assert np.all(np.isfinite(got))
+    assert np.all(err <= 1e-2 + 2.0 ** -8 * np.abs(want)), f"max err {err.max():.3g}"
