@@ -168,6 +168,103 @@ void run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, float *l
   linear(m, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab, c.softcap, valid, s);
 }
 
+// The decode step on the sm_100a decode kernels (bf16, head_dim 128, B <= 32).
+cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *positions, int B,
+                                 const float *noise, float *logits, int32_t *next, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  const int d = c.d_model, H = c.n_head, F = c.mlp_hidden, V = c.vocab, sms = m->num_sms;
+  const float eps = c.norm_eps;
+  cudaError_t e;
+  {
+    ProfScope p(m, NC_K_MISC, s);
+    e = nc::k_dec_embed(tokens, positions, kv->len, kv->pos_ws, kv->valid, B, kv->max_seq, m->wte, d, V, eps, kv->x,
+                        kv->ss, 32, m->status, s);
+    if (e != cudaSuccess) return e;
+  }
+  for (int l = 0; l < c.depth; l++) {
+    const nc_layer_w &w = m->layers[l];
+    void *kc = layer_ptr(kv, kv->k, l), *vc = layer_ptr(kv, kv->v, l);
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      e = nc::k_dec_linear(0 /*norm*/, 0 /*qkv*/, w.wqkv, (H + 2) * 128, d, B, kv->x, kv->ss, 32, eps, nullptr,
+                           kv->part, kv->counters, nullptr, nullptr, kv->q, kc, vc, kv->max_seq, H, kv->pos_ws,
+                           kv->valid, kv->rope, nullptr, nullptr, 0.f, nullptr, nullptr, nullptr, m->status, sms, s);
+      if (e != cudaSuccess) return e;
+    }
+    {
+      ProfScope p(m, NC_K_ATTN, s);
+      e = nc::k_dec_attn(kv->q, kc, vc, kv->pos_ws, kv->valid, B, H, kv->max_seq, kv->attn_chunk, kv->attn_splits,
+                         kv->part, kv->counters, kv->y, s);
+      if (e != cudaSuccess) return e;
+    }
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      e = nc::k_dec_linear(1 /*bf16*/, 1 /*resid*/, w.wo, d, H * 128, B, nullptr, nullptr, 32, eps, kv->y, kv->part,
+                           kv->counters, kv->x, kv->ss, nullptr, nullptr, nullptr, kv->max_seq, H, kv->pos_ws,
+                           kv->valid, kv->rope, nullptr, nullptr, 0.f, nullptr, nullptr, nullptr, m->status, sms, s);
+      if (e != cudaSuccess) return e;
+      e = nc::k_dec_linear(0 /*norm*/, 2 /*relu2*/, w.wfc, F, d, B, kv->x, kv->ss, 32, eps, nullptr, kv->part,
+                           kv->counters, nullptr, nullptr, kv->f, nullptr, nullptr, kv->max_seq, H, kv->pos_ws,
+                           kv->valid, kv->rope, nullptr, nullptr, 0.f, nullptr, nullptr, nullptr, m->status, sms, s);
+      if (e != cudaSuccess) return e;
+      e = nc::k_dec_linear(1 /*bf16*/, 1 /*resid*/, w.wproj, d, F, B, nullptr, nullptr, 32, eps, kv->f, kv->part,
+                           kv->counters, kv->x, kv->ss, nullptr, nullptr, nullptr, kv->max_seq, H, kv->pos_ws,
+                           kv->valid, kv->rope, nullptr, nullptr, 0.f, nullptr, nullptr, nullptr, m->status, sms, s);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  ProfScope p(m, NC_K_HEAD, s);
+  return nc::k_dec_linear(0 /*norm*/, 3 /*lmhead*/, m->wlm, V, d, B, kv->x, kv->ss, 32, eps, nullptr, kv->part,
+                          kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq, H, kv->pos_ws,
+                          kv->valid, kv->rope, logits, noise, c.softcap, kv->cand_v, kv->cand_i, next, m->status, sms,
+                          s);
+}
+
+// Replay the cached graph of the decode step when the call matches the last
+// captured one; otherwise capture a new graph (on the cache's own stream) and
+// launch it. Profiling runs the launches directly so that events can bracket
+// them.
+int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *positions, int B, const float *noise,
+                float *logits, int32_t *next, cudaStream_t s) {
+  if (m->prof) {
+    cudaError_t e = decode_fast_launches(m, kv, tokens, positions, B, noise, logits, next, s);
+    if (e != cudaSuccess) return fail(NC_ECUDA, "decode launch failed: %s", cudaGetErrorString(e));
+    return NC_OK;
+  }
+  nc_kv::GraphKey key{tokens, positions, noise, logits, next, B};
+  bool hit = kv->graph && memcmp(&key, &kv->graph_key, sizeof key) == 0;
+  if (!hit) {
+    if (kv->graph) {
+      cudaGraphExecDestroy(kv->graph);
+      kv->graph = nullptr;
+    }
+    unsigned long long n0 = nc::g_launches.load();
+    NC_CUDA_TRY(cudaStreamBeginCapture(kv->cap_stream, cudaStreamCaptureModeThreadLocal));
+    cudaError_t e = decode_fast_launches(m, kv, tokens, positions, B, noise, logits, next, kv->cap_stream);
+    cudaGraph_t g = nullptr;
+    cudaError_t e2 = cudaStreamEndCapture(kv->cap_stream, &g);
+    if (e != cudaSuccess || e2 != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      cudaGetLastError();
+      return fail(NC_ECUDA, "decode graph capture failed: %s",
+                  cudaGetErrorString(e != cudaSuccess ? e : e2));
+    }
+    cudaError_t e3 = cudaGraphInstantiate(&kv->graph, g, 0);
+    cudaGraphDestroy(g);
+    if (e3 != cudaSuccess) {
+      kv->graph = nullptr;
+      cudaGetLastError();
+      return fail(NC_ECUDA, "decode graph instantiate failed: %s", cudaGetErrorString(e3));
+    }
+    kv->graph_kernels = nc::g_launches.load() - n0;
+    nc::g_launches.fetch_sub(kv->graph_kernels);  // counted when the graph runs
+    kv->graph_key = key;
+  }
+  NC_CUDA_TRY(cudaGraphLaunch(kv->graph, s));
+  nc::count_launch(kv->graph_kernels);
+  return NC_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -277,6 +374,19 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   alloc(&kv->y, elem * rows * qd);
   alloc(&kv->f, elem * rows * F);
   alloc((void **)&kv->logits, sizeof(float) * (size_t)max_batch * c.vocab);
+  alloc((void **)&kv->pos_ws, sizeof(int32_t) * max_batch);
+  kv->dec_fast = nc::decode_fast_supported(c, 1);
+  if (kv->dec_fast) {
+    int nb = max_batch < 32 ? max_batch : 32;
+    kv->part_floats = nc::decode_part_floats(c, nb, max_seq, model->num_sms, &kv->attn_splits, &kv->attn_chunk);
+    alloc((void **)&kv->ss, sizeof(float) * (size_t)(c.d_model / 128) * 32);
+    alloc((void **)&kv->part, sizeof(float) * kv->part_floats);
+    alloc((void **)&kv->counters, sizeof(unsigned) * 1024);
+    alloc((void **)&kv->cand_v, sizeof(float) * (size_t)(c.vocab / 128) * 32);
+    alloc((void **)&kv->cand_i, sizeof(int) * (size_t)(c.vocab / 128) * 32);
+    if (e == cudaSuccess) e = cudaMemset(kv->counters, 0, sizeof(unsigned) * 1024);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&kv->cap_stream, cudaStreamNonBlocking);
+  }
   // zeroed caches: attention may read (and mask) slots past a sequence's length
   if (e == cudaSuccess) e = cudaMemset(kv->k, 0, cache_bytes);
   if (e == cudaSuccess) e = cudaMemset(kv->v, 0, cache_bytes);
@@ -311,7 +421,11 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
 void nc_kv_destroy(nc_kv *kv) {
   if (!kv) return;
   cudaDeviceSynchronize();
-  void *ps[] = {kv->k, kv->v, kv->len, kv->valid, kv->rope, kv->x, kv->h, kv->qkv, kv->q, kv->y, kv->f, kv->logits};
+  if (kv->graph) cudaGraphExecDestroy(kv->graph);
+  if (kv->cap_stream) cudaStreamDestroy(kv->cap_stream);
+  void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
+                kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
+                kv->part,   kv->counters, kv->cand_v, kv->cand_i};
   for (void *p : ps) cudaFree(p);
   delete kv;
 }
@@ -372,12 +486,20 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
 
 int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_t *d_positions, int B,
                    const float *d_noise, float *d_logits, int32_t *d_next, void *stream) {
-  if (!m || !kv || !d_tokens || !d_positions) return fail(NC_EINVAL, "null model, kv, tokens or positions");
+  if (!m || !kv || !d_tokens) return fail(NC_EINVAL, "null model, kv or tokens");
   if (kv->model != m) return fail(NC_EINVAL, "kv belongs to another model");
   if (B < 1) return fail(NC_EINVAL, "B must be >= 1");
   if (B > kv->max_batch) return fail(NC_ERANGE, "B=%d > max_batch=%d", B, kv->max_batch);
   const nc_config &c = m->cfg;
   cudaStream_t s = as_stream(stream);
+  float *logits = d_logits ? d_logits : kv->logits;
+  if (kv->dec_fast && nc::decode_fast_supported(c, B))
+    return decode_fast(m, kv, d_tokens, d_positions, B, d_noise, logits, d_next, s);
+  if (!d_positions) {
+    // positions default to the current lengths
+    NC_CUDA_TRY(cudaMemcpyAsync(kv->pos_ws, kv->len, sizeof(int32_t) * B, cudaMemcpyDeviceToDevice, s));
+    d_positions = kv->pos_ws;
+  }
   {
     ProfScope p(m, NC_K_MISC, s);
     nc::k_decode_begin(d_positions, kv->len, kv->valid, B, kv->max_seq, m->status, s);
@@ -385,7 +507,6 @@ int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_
   }
   nc::RowMap rm{1, d_positions};
   run_blocks(m, kv, B, rm, s);
-  float *logits = d_logits ? d_logits : kv->logits;
   run_head(m, kv, B, 1, 0, logits, kv->valid, s);
   if (d_next) {
     ProfScope p(m, NC_K_HEAD, s);

@@ -57,6 +57,25 @@ struct nc_kv {
   void *y = nullptr;           // [rows, H*hd] attention output
   void *f = nullptr;           // [rows, F] relu^2 hidden
   float *logits = nullptr;     // [max_batch, V] when the caller passes no logits buffer
+  // decode fast path (bf16, head_dim 128, one KV head, B <= 32)
+  bool dec_fast = false;
+  int32_t *pos_ws = nullptr;   // [max_batch] positions of the current step
+  float *ss = nullptr;         // [d/128][32] partial sums of squares of x rows
+  float *part = nullptr;       // split-K / split-KV partials
+  size_t part_floats = 0;
+  unsigned *counters = nullptr;  // [1024], zero between launches
+  float *cand_v = nullptr;     // [V/128][32] per-tile argmax winners
+  int *cand_i = nullptr;
+  int attn_chunk = 0, attn_splits = 0;
+  // CUDA graph of the last decode step's launches, replayed while the call's
+  // pointers and batch stay the same
+  cudaStream_t cap_stream = nullptr;
+  cudaGraphExec_t graph = nullptr;
+  struct GraphKey {
+    const void *tokens, *positions, *noise, *logits, *next;
+    int B;
+  } graph_key = {};
+  unsigned long long graph_kernels = 0;
 };
 
 namespace nc {
@@ -100,5 +119,22 @@ cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int
 bool attn_prefill_tc_supported(int H, int Hkv, int hd);
 cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int max_batch,
                               int max_seq, void *y, uint32_t *status, cudaStream_t s);
+
+
+// ---- decode step kernels (nc_decode.cu) ----
+bool decode_fast_supported(const nc_config &c, int B);
+size_t decode_part_floats(const nc_config &c, int max_batch, int max_seq, int num_sms, int *attn_splits,
+                          int *attn_chunk);
+cudaError_t k_dec_embed(const int32_t *tokens, const int32_t *positions, int32_t *len, int32_t *pos_ws,
+                        uint8_t *valid, int B, int max_seq, const void *wte, int d, int vocab, float eps, float *x,
+                        float *ss, int ssb, uint32_t *status, cudaStream_t s);
+cudaError_t k_dec_linear(int src, int epi, const void *W, int N, int K, int B, const float *x, const float *ss, int ssb,
+                         float eps, const void *act, float *part, unsigned *counters, float *xres, float *ss_out,
+                         void *out, void *kc, void *vc, int max_seq, int H, const int32_t *pos, const uint8_t *valid,
+                         const float2 *rope, float *logits, const float *noise, float cap, float *cand_v, int *cand_i,
+                         int32_t *next, uint32_t *status, int num_sms, cudaStream_t s);
+cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int32_t *pos, const uint8_t *valid, int B,
+                       int H, int max_seq, int chunk, int splits, float *part, unsigned *counters, void *y,
+                       cudaStream_t s);
 
 }  // namespace nc
