@@ -231,9 +231,28 @@ int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *po
     if (e != cudaSuccess) return fail(NC_ECUDA, "decode launch failed: %s", cudaGetErrorString(e));
     return NC_OK;
   }
-  nc_kv::GraphKey key{tokens, positions, noise, logits, next, B};
-  bool hit = kv->graph && memcmp(&key, &kv->graph_key, sizeof key) == 0;
-  if (!hit) {
+  nc_kv::GraphKey key;
+  memset(&key, 0, sizeof key);  // compared bytewise, padding included
+  key.tokens = tokens;
+  key.positions = positions;
+  key.noise = noise;
+  key.logits = logits;
+  key.next = next;
+  key.B = B;
+  const bool same = memcmp(&key, &kv->graph_key, sizeof key) == 0;
+  if (!same || !kv->graph_ready) {
+    // a new call shape runs directly; the graph is captured once it repeats
+    if (kv->graph) {
+      cudaGraphExecDestroy(kv->graph);
+      kv->graph = nullptr;
+    }
+    kv->graph_key = key;
+    kv->graph_ready = true;
+    cudaError_t e = decode_fast_launches(m, kv, tokens, positions, B, noise, logits, next, s);
+    if (e != cudaSuccess) return fail(NC_ECUDA, "decode launch failed: %s", cudaGetErrorString(e));
+    return NC_OK;
+  }
+  if (!kv->graph) {
     if (kv->graph) {
       cudaGraphExecDestroy(kv->graph);
       kv->graph = nullptr;
@@ -258,7 +277,6 @@ int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *po
     }
     kv->graph_kernels = nc::g_launches.load() - n0;
     nc::g_launches.fetch_sub(kv->graph_kernels);  // counted when the graph runs
-    kv->graph_key = key;
   }
   NC_CUDA_TRY(cudaGraphLaunch(kv->graph, s));
   nc::count_launch(kv->graph_kernels);

@@ -75,6 +75,7 @@ struct nc_kv {
     const void *tokens, *positions, *noise, *logits, *next;
     int B;
   } graph_key = {};
+  bool graph_ready = false;    // graph_key has run once directly
   unsigned long long graph_kernels = 0;
 };
 
