@@ -238,6 +238,14 @@ def run_ours(args):
     logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
     nxt = torch.empty((B,), dtype=torch.int32, device="cuda")
 
+    if args.only == "decode":
+        dec = run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "only": "decode", "decode": dec}), flush=True)
+        kv.close()
+        model.close()
+        return
+
     # ---------------- prefill: device-resident inputs
     for _ in range(args.warmup):
         model.prefill(kv, tokens, 0, logits, nxt)
@@ -433,6 +441,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", choices=("all", "decode"), default="all",
+                    help="decode: skip the prefill timing (for profiling the decode kernels)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=128,
                     help="tokens of one prompt the CPU oracle runs per sample")
