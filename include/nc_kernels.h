@@ -44,6 +44,21 @@ int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K,
 int nc_attention_prefill_bf16(const void *d_q, const void *d_k, const void *d_v, int B, int T, int H, int hd,
                               int max_seq, void *d_y, void *stream);
 
+/* Single-token (decode) multi-query attention for B sequences, head_dim 128,
+ * H <= 16 query heads sharing one KV head:
+ *   y[b,h,:] = sum_{j<=pos[b]} softmax_j(q[b,h,:] . k[b,j,:] / sqrt(128)) v[b,j,:]
+ * split over the keys (flash decoding) with a merge of the partial softmax
+ * states. d_q, d_y bf16 [B, H, 128]; d_k, d_v bf16 [B, max_seq, 128];
+ * d_pos int32 [B], each in [0, max_seq) (clamped on the device otherwise).
+ * d_workspace: device scratch of nc_attention_decode_workspace_bytes(B,
+ * max_seq) bytes, zero-filled before its first use; the call leaves it ready
+ * for the next one. Calls sharing a workspace must not overlap on the GPU.
+ * Errors: NC_EINVAL (null pointer, bad shape, H > 16, workspace too small),
+ * NC_ECUDA. */
+size_t nc_attention_decode_workspace_bytes(int B, int max_seq);
+int nc_attention_decode_bf16(const void *d_q, const void *d_k, const void *d_v, const int32_t *d_pos, int B, int H,
+                             int max_seq, void *d_y, void *d_workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -616,6 +616,39 @@ int nc_attention_prefill_bf16(const void *d_q, const void *d_k, const void *d_v,
   return NC_OK;
 }
 
+static int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
+size_t nc_attention_decode_workspace_bytes(int B, int max_seq) {
+  if (B <= 0 || max_seq <= 0) return 0;
+  int sms = device_sms(), chunk, splits;
+  if (sms <= 0) sms = 148;
+  nc::attn_decode_plan(B, max_seq, sms, &chunk, &splits);
+  return nc::attn_decode_partial_floats(B, splits) * sizeof(float) + sizeof(unsigned) * (size_t)B;
+}
+
+int nc_attention_decode_bf16(const void *d_q, const void *d_k, const void *d_v, const int32_t *d_pos, int B, int H,
+                             int max_seq, void *d_y, void *d_workspace, size_t workspace_bytes, void *stream) {
+  if (!d_q || !d_k || !d_v || !d_pos || !d_y || !d_workspace) return fail(NC_EINVAL, "null pointer");
+  if (B <= 0 || H <= 0 || H > 16 || max_seq <= 0) return fail(NC_EINVAL, "bad decode attention shape");
+  int sms = device_sms(), chunk, splits;
+  if (sms <= 0) return fail(NC_ECUDA, "no CUDA device");
+  nc::attn_decode_plan(B, max_seq, sms, &chunk, &splits);
+  const size_t part = nc::attn_decode_partial_floats(B, splits);
+  if (workspace_bytes < part * sizeof(float) + sizeof(unsigned) * (size_t)B)
+    return fail(NC_EINVAL, "workspace of %zu bytes is too small", workspace_bytes);
+  float *pf = (float *)d_workspace;
+  unsigned *counters = (unsigned *)(pf + part);
+  cudaError_t e = nc::k_dec_attn(d_q, d_k, d_v, d_pos, nullptr, B, H, max_seq, chunk, splits, pf, counters, d_y,
+                                 as_stream(stream));
+  if (e != cudaSuccess) return fail(NC_ECUDA, "decode attention launch: %s", cudaGetErrorString(e));
+  return NC_OK;
+}
+
 int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K, int epi, void *d_out, int ldo,
                  float cap, void *stream) {
   if (!d_A || !d_W || !d_out) return fail(NC_EINVAL, "null pointer");

@@ -434,7 +434,7 @@ struct DecAttnArgs {
   const bf16 *q;        // [B][H][128]
   const bf16 *kc, *vc;  // [max_batch][max_seq][128]
   const int32_t *pos;
-  const uint8_t *valid;
+  const uint8_t *valid;  // null: every sequence takes part
   int H, max_seq, chunk, splits;
   float scale_log2;
   float *part;          // [B][splits][16][130]: m, l, O[128] per head row
@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(ATHREADS) dec_attn_kernel(DecAttnArgs a) {
   const int g = lane >> 2, t4 = lane & 3;
   pdl_wait();
   int pos = a.pos[b];
-  const bool ok = a.valid[b] != 0;
+  const bool ok = a.valid ? a.valid[b] != 0 : true;
   pos = pos < 0 ? 0 : (pos >= a.max_seq ? a.max_seq - 1 : pos);
   const int n_keys = pos + 1;
   const int k_begin = split * a.chunk;
@@ -767,6 +767,19 @@ size_t decode_part_floats(const nc_config &c, int max_batch, int max_seq, int nu
   size_t fa = (size_t)max_batch * (*attn_splits) * 16 * 130;
   return need > fa ? need : fa;
 }
+
+// Split-KV plan for the kernel-level decode attention entry points: keys in
+// chunks of a multiple of 64, about two CTAs per SM over the batch, at most
+// 16 splits per sequence.
+void attn_decode_plan(int B, int max_seq, int num_sms, int *chunk, int *splits) {
+  int c = AKT;
+  while (((max_seq + c - 1) / c) * B > 2 * num_sms && c < max_seq) c += AKT;
+  while ((max_seq + c - 1) / c > 16) c += AKT;
+  *chunk = c;
+  *splits = (max_seq + c - 1) / c;
+}
+
+size_t attn_decode_partial_floats(int B, int splits) { return (size_t)B * splits * 16 * 130; }
 
 cudaError_t k_dec_embed(const int32_t *tokens, const int32_t *positions, int32_t *len, int32_t *pos_ws,
                         uint8_t *valid, int B, int max_seq, const void *wte, int d, int vocab, float eps, float *x,

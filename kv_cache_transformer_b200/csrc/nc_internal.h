@@ -134,6 +134,8 @@ cudaError_t k_dec_linear(int src, int epi, const void *W, int N, int K, int B, c
                          void *out, void *kc, void *vc, int max_seq, int H, const int32_t *pos, const uint8_t *valid,
                          const float2 *rope, float *logits, const float *noise, float cap, float *cand_v, int *cand_i,
                          int32_t *next, uint32_t *status, int num_sms, cudaStream_t s);
+void attn_decode_plan(int B, int max_seq, int num_sms, int *chunk, int *splits);
+size_t attn_decode_partial_floats(int B, int splits);
 cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int32_t *pos, const uint8_t *valid, int B,
                        int H, int max_seq, int chunk, int splits, float *part, unsigned *counters, void *y,
                        cudaStream_t s);

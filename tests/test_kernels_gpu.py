@@ -115,3 +115,37 @@ def test_attention_prefill_matches_float64(B, T, H, hd, extra):
     err = np.abs(got - want)
     assert np.all(np.isfinite(got))
     assert np.all(err <= 1e-2 + 2.0 ** -8 * np.abs(want)), f"max err {err.max():.3g}"
+
+
+def _decode_ref(q, k, v, pos):
+    import torch
+    out = torch.zeros(q.shape, dtype=torch.float64)
+    for b in range(q.shape[0]):
+        n = int(pos[b]) + 1
+        s = q[b].double() @ k[b, :n].double().T / np.sqrt(128.0)
+        out[b] = torch.softmax(s, dim=-1) @ v[b, :n].double()
+    return out
+
+
+@pytest.mark.parametrize("B,H,max_seq", [(1, 13, 1536), (7, 10, 300), (32, 10, 2176), (5, 15, 64)])
+def test_attention_decode_matches_float64(B, H, max_seq):
+    import torch
+    import kv_cache_transformer_b200 as nc
+    g = torch.Generator().manual_seed(B * 31 + H + max_seq)
+    q = torch.randn(B, H, 128, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, max_seq, 128, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, max_seq, 128, generator=g).to(torch.bfloat16)
+    pos = torch.randint(0, max_seq, (B,), generator=g, dtype=torch.int32)
+    pos[0] = max_seq - 1
+    if B > 1:
+        pos[1] = 0
+    ws = torch.zeros(nc.nc_attention_decode_workspace_bytes(B, max_seq), dtype=torch.uint8, device="cuda")
+    y = torch.full((B, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):  # the workspace is reusable as the call leaves it
+        nc.nc_attention_decode_bf16(q.cuda(), k.cuda(), v.cuda(), pos.cuda(), y, ws)
+        torch.cuda.synchronize()
+        want = _decode_ref(q, k, v, pos).numpy()
+        got = y.cpu().double().numpy()
+        err = np.abs(got - want)
+        assert np.all(np.isfinite(got))
+        assert np.all(err <= 1e-2 + 2.0 ** -8 * np.abs(want)), f"max err {err.max():.3g}"
