@@ -59,6 +59,23 @@ size_t nc_attention_decode_workspace_bytes(int B, int max_seq);
 int nc_attention_decode_bf16(const void *d_q, const void *d_k, const void *d_v, const int32_t *d_pos, int B, int H,
                              int max_seq, void *d_y, void *d_workspace, size_t workspace_bytes, void *stream);
 
+/* nc_attention_decode_bf16 without a workspace argument, for callers that
+ * cannot allocate device memory (a serving runtime whose allocator owns all
+ * of it, a plugin host without a workspace hook, a fixed-footprint
+ * deployment). The pages have no counterpart: this is a packaging variant of
+ * the decode attention above, with the same inputs, outputs and results.
+ * Its scratch is a static array inside the library (about 4.3 MB, held on
+ * every GPU that loads the library until the process exits); no call
+ * allocates or frees device memory. Limits: B <= 32, H <= 16, and max_seq
+ * small enough for 16 key splits (the split rule grows the chunk to fit).
+ * The first call on each device looks up the array's device address, so
+ * make that first call before any stream capture. All calls share the one
+ * array: calls that overlap on the GPU (other streams, other threads) race
+ * and must be serialised by the caller. Errors: NC_EINVAL (null pointer, bad
+ * shape, B or max_seq beyond the limits), NC_ECUDA. */
+int nc_attention_decode_bf16_static(const void *d_q, const void *d_k, const void *d_v, const int32_t *d_pos, int B,
+                                    int H, int max_seq, void *d_y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

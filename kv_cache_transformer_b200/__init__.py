@@ -35,6 +35,7 @@ EXPORTS = (
     "nc_kv_lengths", "nc_prefill", "nc_decode_step", "nc_kv_fork", "nc_last_error",
     "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
     "nc_attention_prefill_bf16", "nc_attention_decode_workspace_bytes", "nc_attention_decode_bf16",
+    "nc_attention_decode_bf16_static",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_COUNT = 0, 1, 2, 3, 4
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
             L.nc_attention_decode_workspace_bytes.argtypes = [i, i]
             L.nc_attention_decode_workspace_bytes.restype = ctypes.c_size_t
             L.nc_attention_decode_bf16.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp, sz, vp]
+            L.nc_attention_decode_bf16_static.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp]
             for name in EXPORTS:
                 if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error", "nc_launch_count",
                                 "nc_attention_decode_workspace_bytes"):
@@ -258,6 +260,18 @@ def nc_attention_decode_bf16(q, k, v, pos, y, workspace, stream=None):
     _check(lib().nc_attention_decode_bf16(_dptr(q), _dptr(k), _dptr(v), _dptr(pos, torch.int32, B, "pos"), B, H,
                                           k.shape[1], _dptr(y), _dptr(workspace), workspace.numel() *
                                           workspace.element_size(), _stream(stream)))
+
+
+def nc_attention_decode_bf16_static(q, k, v, pos, y, stream=None):
+    """nc_attention_decode_bf16 using the library's static scratch (no workspace, no allocation)."""
+    import torch
+    B, H, hd = q.shape
+    if hd != 128 or k.shape[0] != B or k.shape[2] != 128 or k.shape != v.shape or y.shape != q.shape:
+        raise ValueError("shape mismatch")
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (y, "y")):
+        _dptr(t, torch.bfloat16, name=n)
+    _check(lib().nc_attention_decode_bf16_static(_dptr(q), _dptr(k), _dptr(v), _dptr(pos, torch.int32, B, "pos"), B,
+                                                 H, k.shape[1], _dptr(y), _stream(stream)))
 
 
 # ----------------------------------------------------------------- wrappers

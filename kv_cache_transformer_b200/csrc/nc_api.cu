@@ -285,6 +285,11 @@ int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *po
 
 }  // namespace
 
+namespace nc {
+// Record a message for nc_last_error() from other translation units.
+int set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace nc
+
 extern "C" {
 
 const char *nc_last_error(void) { return g_err.c_str(); }

@@ -81,6 +81,9 @@ struct nc_kv {
 
 namespace nc {
 
+// Set the message returned by nc_last_error(); returns code.
+int set_error(int code, const char *msg);
+
 // Kernels launched by this library (nc_launch_count).
 extern std::atomic<unsigned long long> g_launches;
 inline void count_launch(unsigned long long n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
