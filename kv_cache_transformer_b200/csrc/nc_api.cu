@@ -103,6 +103,27 @@ void linear(nc_model *m, int epi, const void *A, int lda, const void *W, int M, 
   nc::k_gemm_generic(m->cfg.dtype, epi, A, lda, W, M, N, K, out, ldo, cap, valid, s);
 }
 
+// h = bf16/fp32 rmsnorm of the M rows of x.
+void norm_rows(nc_model *m, nc_kv *kv, int M, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  if (nc::rowops_supported(c) && nc::k_rows_norm_bf16(kv->x, M, c.d_model, c.norm_eps, kv->h, s) == cudaSuccess)
+    return;
+  cudaGetLastError();
+  nc::k_rmsnorm_rows(c.dtype, kv->x, M, c.d_model, 1, 0, c.norm_eps, kv->h, s);
+}
+
+// RoPE + QK norm of the M rows of kv->qkv, q out, K/V appended to the cache.
+void rope_append(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  if (!rm.pos && nc::rowops_supported(c) &&
+      nc::k_rope_qk_bf16(kv->qkv, M, rm.T, c.n_head, kv->rope, kv->q, kc, vc, kv->max_seq, c.norm_eps, s) ==
+          cudaSuccess)
+    return;
+  cudaGetLastError();
+  nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->rope, kv->q, kc, vc,
+                           kv->max_seq, kv->valid, c.norm_eps, s);
+}
+
 // Causal MQA attention of the M rows in kv->q against layer cache kc/vc.
 void attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
@@ -120,13 +141,12 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
   int d = c.d_model, H = c.n_head, Hkv = c.n_kv_head, hd = c.head_dim, F = c.mlp_hidden;
   int qkv_w = (H + 2 * Hkv) * hd;
-  const uint8_t *valid = kv->valid;
   for (int l = 0; l < c.depth; l++) {
     const nc_layer_w &w = m->layers[l];
     void *kc = layer_ptr(kv, kv->k, l), *vc = layer_ptr(kv, kv->v, l);
     {
       ProfScope p(m, NC_K_MISC, s);
-      nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
+      norm_rows(m, kv, M, s);
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
@@ -134,8 +154,7 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
     }
     {
       ProfScope p(m, NC_K_MISC, s);
-      nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, H, Hkv, hd, kv->rope, kv->q, kc, vc, kv->max_seq, valid,
-                               c.norm_eps, s);
+      rope_append(m, kv, kc, vc, M, rm, s);
     }
     {
       ProfScope p(m, NC_K_ATTN, s);
@@ -147,7 +166,7 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
     }
     {
       ProfScope p(m, NC_K_MISC, s);
-      nc::k_rmsnorm_rows(c.dtype, kv->x, M, d, 1, 0, c.norm_eps, kv->h, s);
+      norm_rows(m, kv, M, s);
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
@@ -407,6 +426,7 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
     alloc((void **)&kv->counters, sizeof(unsigned) * 1024);
     alloc((void **)&kv->cand_v, sizeof(float) * (size_t)(c.vocab / 128) * 32);
     alloc((void **)&kv->cand_i, sizeof(int) * (size_t)(c.vocab / 128) * 32);
+    alloc((void **)&kv->xl, sizeof(float) * (size_t)32 * c.d_model);
     if (e == cudaSuccess) e = cudaMemset(kv->counters, 0, sizeof(unsigned) * 1024);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&kv->cap_stream, cudaStreamNonBlocking);
   }
@@ -448,7 +468,7 @@ void nc_kv_destroy(nc_kv *kv) {
   if (kv->cap_stream) cudaStreamDestroy(kv->cap_stream);
   void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
                 kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
-                kv->part,   kv->counters, kv->cand_v, kv->cand_i};
+                kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl};
   for (void *p : ps) cudaFree(p);
   delete kv;
 }
@@ -495,6 +515,18 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
     }
   } else {
     logits = d_logits ? d_logits : kv->logits;
+    if (kv->dec_fast && nc::decode_fast_supported(c, B)) {
+      // last rows -> fused norm + lm_head + softcap + argmax (the decode head kernel)
+      ProfScope p(m, NC_K_HEAD, s);
+      cudaError_t e = nc::k_gather_rows_ss(kv->x, B, c.d_model, T, T - 1, kv->xl, kv->ss, 32, s);
+      if (e == cudaSuccess)
+        e = nc::k_dec_linear(0 /*norm*/, 3 /*lmhead*/, m->wlm, c.vocab, c.d_model, B, kv->xl, kv->ss, 32, c.norm_eps,
+                             nullptr, kv->part, kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq,
+                             c.n_head, kv->pos_ws, kv->valid, kv->rope, logits, d_noise, c.softcap, kv->cand_v,
+                             kv->cand_i, d_next, m->status, m->num_sms, s);
+      if (e != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(e));
+      return NC_OK;
+    }
     run_head(m, kv, B, T, T - 1, logits, nullptr, s);
     last_off = 0;
     row_stride = c.vocab;

@@ -66,6 +66,7 @@ struct nc_kv {
   unsigned *counters = nullptr;  // [1024], zero between launches
   float *cand_v = nullptr;     // [V/128][32] per-tile argmax winners
   int *cand_i = nullptr;
+  float *xl = nullptr;         // [32][d] last-position rows of a prefill, for the fused lm_head
   int attn_chunk = 0, attn_splits = 0;
   // CUDA graph of the last decode step's launches, replayed while the call's
   // pointers and batch stay the same
@@ -124,6 +125,14 @@ bool attn_prefill_tc_supported(int H, int Hkv, int hd);
 cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int max_batch,
                               int max_seq, void *y, uint32_t *status, cudaStream_t s);
 
+
+// ---- row-wise prefill kernels for bf16 head_dim-128 models (nc_rowops.cu) ----
+bool rowops_supported(const nc_config &c);
+cudaError_t k_rows_norm_bf16(const float *x, int rows, int d, float eps, void *h, cudaStream_t s);
+cudaError_t k_rope_qk_bf16(const void *qkv, int M, int T, int H, const float2 *rope, void *q_out, void *kc, void *vc,
+                           int max_seq, float eps, cudaStream_t s);
+cudaError_t k_gather_rows_ss(const float *x, int rows, int d, int stride, int offset, float *xl, float *ss, int ssb,
+                             cudaStream_t s);
 
 // ---- decode step kernels (nc_decode.cu) ----
 bool decode_fast_supported(const nc_config &c, int B);
