@@ -146,7 +146,8 @@ int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *
 #define NC_K_ATTN 1   /* attention, prefill or decode (with any split combine) */
 #define NC_K_HEAD 2   /* final norm, lm_head with softcap, token pick */
 #define NC_K_MISC 3   /* embedding, norms, RoPE/QK norm/KV append, bookkeeping, fork */
-#define NC_K_COUNT 4
+#define NC_K_STEP 4   /* a whole decode step run as one persistent kernel */
+#define NC_K_COUNT 5
 
 /* Turn per-class device timing on (1) or off (0) for calls on this model.
  * When on, every launch (or fused group of launches) is bracketed by CUDA

@@ -38,8 +38,8 @@ EXPORTS = (
     "nc_attention_decode_bf16_static",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
-NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_COUNT = 0, 1, 2, 3, 4
-K_CLASS_NAMES = ("gemm", "attn", "head", "misc")
+NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_STEP, NC_K_COUNT = 0, 1, 2, 3, 4, 5
+K_CLASS_NAMES = ("gemm", "attn", "head", "misc", "step")
 
 
 class NcError(RuntimeError):

@@ -194,6 +194,12 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
   const int d = c.d_model, H = c.n_head, F = c.mlp_hidden, V = c.vocab, sms = m->num_sms;
   const float eps = c.norm_eps;
   cudaError_t e;
+  if (kv->step_grid > 0 && nc::decode_step_supported(c, B)) {
+    ProfScope p(m, NC_K_STEP, s);
+    return nc::k_decode_step(m, B, kv->max_batch, kv->max_seq, kv->step_maps, tokens, positions, kv->len, kv->x,
+                             kv->xl, kv->step_ss, kv->q, kv->y, kv->f, kv->k, kv->v, kv->rope, logits, noise, next,
+                             kv->cand_v, kv->cand_i, kv->step_bar, kv->step_grid, s);
+  }
   {
     ProfScope p(m, NC_K_MISC, s);
     e = nc::k_dec_embed(tokens, positions, kv->len, kv->pos_ws, kv->valid, B, kv->max_seq, m->wte, d, V, eps, kv->x,
@@ -429,6 +435,19 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
     alloc((void **)&kv->xl, sizeof(float) * (size_t)32 * c.d_model);
     if (e == cudaSuccess) e = cudaMemset(kv->counters, 0, sizeof(unsigned) * 1024);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&kv->cap_stream, cudaStreamNonBlocking);
+    // whole-step kernel: tensor maps of the weights and of this cache
+    if (e == cudaSuccess && nc::decode_step_supported(c, 1)) {
+      const int nmaps = nc::decode_step_maps_count(c);
+      std::vector<CUtensorMap> maps(nmaps);
+      alloc((void **)&kv->step_maps, sizeof(CUtensorMap) * nmaps);
+      alloc((void **)&kv->step_bar, sizeof(unsigned long long));
+      alloc((void **)&kv->step_ss, sizeof(float) * (size_t)(2 * c.depth + 1) * 32);
+      if (e == cudaSuccess) e = cudaMemset(kv->step_bar, 0, sizeof(unsigned long long));
+      if (e == cudaSuccess && nc::decode_step_build_maps(model, kv->k, kv->v, max_batch, max_seq, maps.data())) {
+        e = cudaMemcpy(kv->step_maps, maps.data(), sizeof(CUtensorMap) * nmaps, cudaMemcpyHostToDevice);
+        if (e == cudaSuccess) kv->step_grid = nc::decode_step_grid(model->num_sms);
+      }
+    }
   }
   // zeroed caches: attention may read (and mask) slots past a sequence's length
   if (e == cudaSuccess) e = cudaMemset(kv->k, 0, cache_bytes);
@@ -468,7 +487,8 @@ void nc_kv_destroy(nc_kv *kv) {
   if (kv->cap_stream) cudaStreamDestroy(kv->cap_stream);
   void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
                 kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
-                kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl};
+                kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl,     kv->step_maps, kv->step_bar,
+                kv->step_ss};
   for (void *p : ps) cudaFree(p);
   delete kv;
 }

@@ -9,6 +9,7 @@
 
 #include "nc.h"
 #include "nc_common.cuh"
+#include <cuda.h>
 
 struct nc_layer_w {
   const void *wqkv;   // [(H + 2*Hkv)*hd, d]: Wq, Wk, Wv are adjacent in the blob
@@ -67,6 +68,11 @@ struct nc_kv {
   float *cand_v = nullptr;     // [V/128][32] per-tile argmax winners
   int *cand_i = nullptr;
   float *xl = nullptr;         // [32][d] last-position rows of a prefill, for the fused lm_head
+  // whole-step decode kernel (nc_step.cu)
+  int step_grid = 0;           // CTAs of the step kernel, 0 = not available
+  CUtensorMap *step_maps = nullptr;  // device copy of the step kernel's tensor maps
+  unsigned long long *step_bar = nullptr;  // its grid-barrier counter
+  float *step_ss = nullptr;    // [2*depth+1][32]
   int attn_chunk = 0, attn_splits = 0;
   // CUDA graph of the last decode step's launches, replayed while the call's
   // pointers and batch stay the same
@@ -151,5 +157,18 @@ size_t attn_decode_partial_floats(int B, int splits);
 cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int32_t *pos, const uint8_t *valid, int B,
                        int H, int max_seq, int chunk, int splits, float *part, unsigned *counters, void *y,
                        cudaStream_t s);
+
+
+// ---- whole decode step in one persistent kernel (nc_step.cu) ----
+bool decode_step_supported(const nc_config &c, int B);
+int decode_step_maps_count(const nc_config &c);
+bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *vcache, int max_batch, int max_seq,
+                            CUtensorMap *out);
+int decode_step_grid(int num_sms);
+cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, const CUtensorMap *maps_dev,
+                          const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
+                          float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
+                          const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
+                          int grid, cudaStream_t s);
 
 }  // namespace nc
