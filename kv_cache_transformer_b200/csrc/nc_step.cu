@@ -445,14 +445,16 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
 }
 
 // LM head tile (full K, no reduction): softcap, logits, per-tile argmax.
-__device__ void head_epilogue(const StepArgs &a, const Smem &s, int nt, const uint32_t (&r)[NB], float *tl, int e) {
+// r holds tile row n (this thread's TMEM lane) for every batch column.
+__device__ void head_epilogue(const StepArgs &a, const Smem &s, int nt, const uint32_t (&r)[NB], float *tl, int n,
+                              int e) {
   const int lane = e & 31, w = e >> 5;
-  const int col = nt * 128 + e;
+  const int col = nt * 128 + n;
   const float inv = 1.0f / a.cap;
   for (int b = 0; b < a.B; b++) {
     const float z = a.cap * tanhf(__uint_as_float(r[b]) * inv);
     if (s.valid[b]) a.logits[(size_t)b * a.V + col] = z;
-    tl[e * (NB + 1) + b] = z + (a.noise ? a.noise[(size_t)b * a.V + col] : 0.f);
+    tl[n * (NB + 1) + b] = z + (a.noise ? a.noise[(size_t)b * a.V + col] : 0.f);
   }
   epi_sync();
   for (int b = w; b < a.B; b += 4) {
@@ -725,7 +727,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     const int quarter = warp & 3;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int n = quarter * 32 + lane;  // TMEM lane of this thread
-    uint32_t t = 0;                     // ring slots consumed by the attention
+    uint32_t t = 0;                     // ring slot counter, in the producer's order
     uint32_t xf = 0, units = 0, rounds = 0;
     bool x_pending = false;             // a staged X is waiting for x_free
     const int P = n_phases(a);
@@ -817,6 +819,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
             if (g.nkb == 0) break;
           }
           if (!ok) break;
+          t += g.nkb;  // the unit's weight tiles went through the ring (consumed by the MMA warp)
           if (!mbar_wait(s.acc_full, units & 1, s.abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
           uint32_t r[NB];
@@ -827,7 +830,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           if (g.nkb == 0)
             for (int j = 0; j < NB; j++) r[j] = 0u;  // this rank holds no k-blocks
           if (type == P_HEAD) {
-            head_epilogue(a, s, nt, r, tl, e);
+            head_epilogue(a, s, nt, r, tl, n, e);
             continue;
           }
           // cluster reduction over the K split: each CTA finishes NB/CL columns
@@ -968,6 +971,9 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
   a.cand_i = cand_i;
   a.bar = bar;
   a.status = m->status;
+  // grid-barrier counter from zero for every step
+  cudaError_t e = cudaMemsetAsync(bar, 0, sizeof(unsigned long long), s);
+  if (e != cudaSuccess) return e;
   count_launch();
   decode_step_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(a);
   return cudaGetLastError();
