@@ -53,6 +53,7 @@ constexpr int SLOT = 16384;
 constexpr int XKB = 20;                // X staging capacity, 64-column blocks
 constexpr int THREADS = 192;
 constexpr int KT = 64;                 // keys per attention tile
+constexpr int NACC = 4;                // TMEM accumulators the K loop rotates over
 
 constexpr int OFF_RING = 0;
 constexpr int OFF_X = OFF_RING + RING * SLOT;          // XKB * NB * 128 bytes
@@ -310,9 +311,14 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
             t++;
             tc_fence_after();
             const uint32_t w0 = smem_u32(ring + slot * SLOT), x0 = smem_u32(xs + kb * NB * 128);
+            // consecutive k-blocks accumulate into different TMEM accumulators, so
+            // their MMAs do not wait on one another; the epilogue adds them up
+            const int kg = c0 + kb;
+            const uint32_t acc = tmem + (uint32_t)(kg % NACC) * NB;
+            const bool fresh = kg < NACC;
 #pragma unroll
             for (int k = 0; k < 4; k++)
-              mma_bf16(tmem, desc_k_sw128(w0 + 32 * k), desc_k_sw128(x0 + 32 * k), idesc, first ? (k != 0) : 1);
+              mma_bf16(acc, desc_k_sw128(w0 + 32 * k), desc_k_sw128(x0 + 32 * k), idesc, (fresh && k == 0) ? 0 : 1);
             first = false;
             mma_commit(&s.empty[slot]);
           }
@@ -335,27 +341,57 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
 
 // ------------------------------------------------- compute-side helpers
 // X staging: X[b][kb*64 + c] for this pass, NB rows, 128-byte swizzled.
+// Loads are issued in batches of U per thread before any is consumed, so a
+// pass costs a few L2 round trips instead of one per item.
 __device__ void stage_x(const StepArgs &a, const Smem &s, uint8_t *xs, int type, int kb_begin, int nkb, int e) {
+  constexpr int U = 16;
   const bool norm = (type == P_QKV || type == P_FC || type == P_HEAD);
   const float *xsrc = (type == P_FC) ? a.x1 : a.x0;
   const bf16 *act = (type == P_OPROJ) ? a.y : a.f;
   const int K = (type == P_PROJ) ? a.F : a.d;
-  for (int idx = e; idx < nkb * NB * 8; idx += 128) {
-    const int c = idx & 7, b = (idx >> 3) % NB, kbl = idx / (8 * NB);
-    const int k = (kb_begin + kbl) * 64 + c * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (b < a.B) {
-      if (norm) {
-        const float4 *src = reinterpret_cast<const float4 *>(xsrc + (size_t)b * a.d + k);
-        const float4 p = src[0], q = src[1];
+  const int total = nkb * NB * 8;
+  for (int base = e; base < total; base += 128 * U) {
+    if (norm) {
+      float4 p[U], q[U];
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int idx = base + u * 128;
+        const int c = idx & 7, b = (idx >> 3) % NB, kbl = idx / (8 * NB);
+        p[u] = q[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < total && b < a.B) {
+          const float4 *src = reinterpret_cast<const float4 *>(xsrc + (size_t)b * a.d + (kb_begin + kbl) * 64 + c * 8);
+          p[u] = src[0];
+          q[u] = src[1];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int idx = base + u * 128;
+        if (idx >= total) break;
+        const int c = idx & 7, b = (idx >> 3) % NB, kbl = idx / (8 * NB);
         const float r = s.inv[b];
-        v = make_uint4(pack_bf(p.x * r, p.y * r), pack_bf(p.z * r, p.w * r), pack_bf(q.x * r, q.y * r),
-                       pack_bf(q.z * r, q.w * r));
-      } else {
-        v = *reinterpret_cast<const uint4 *>(act + (size_t)b * K + k);
+        const uint4 v = make_uint4(pack_bf(p[u].x * r, p[u].y * r), pack_bf(p[u].z * r, p[u].w * r),
+                                   pack_bf(q[u].x * r, q[u].y * r), pack_bf(q[u].z * r, q[u].w * r));
+        *reinterpret_cast<uint4 *>(xs + kbl * NB * 128 + b * 128 + ((c ^ (b & 7)) << 4)) = v;
+      }
+    } else {
+      uint4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int idx = base + u * 128;
+        const int c = idx & 7, b = (idx >> 3) % NB, kbl = idx / (8 * NB);
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (idx < total && b < a.B)
+          v[u] = *reinterpret_cast<const uint4 *>(act + (size_t)b * K + (kb_begin + kbl) * 64 + c * 8);
+      }
+#pragma unroll
+      for (int u = 0; u < U; u++) {
+        const int idx = base + u * 128;
+        if (idx >= total) break;
+        const int c = idx & 7, b = (idx >> 3) % NB, kbl = idx / (8 * NB);
+        *reinterpret_cast<uint4 *>(xs + kbl * NB * 128 + b * 128 + ((c ^ (b & 7)) << 4)) = v[u];
       }
     }
-    *reinterpret_cast<uint4 *>(xs + kbl * NB * 128 + b * 128 + ((c ^ (b & 7)) << 4)) = v;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -368,23 +404,54 @@ __device__ void load_inv(const StepArgs &a, const Smem &s, const float *ss, int 
 
 // Epilogue of one reduced 128-row tile for the batch columns b in [b0, b1):
 // tl[n * (NB+1) + j] holds row n (thread e = n), column b0 + j.
+// Global operands of the epilogue, loaded before the cluster exchange so that
+// their latency overlaps it.
+struct EpiPre {
+  float xv[NB / CL];   // residual inputs (OPROJ / PROJ)
+  float2 cs[NB / CL];  // RoPE (cos, sin) of the row's pair at each column's position (QKV)
+};
+
+__device__ __forceinline__ void epi_preload(const StepArgs &a, const Smem &s, int type, int nt, int b0, int b1, int e,
+                                            EpiPre &pre) {
+  const int nb = b1 - b0, col = nt * 128 + e;
+  if (type == P_OPROJ || type == P_PROJ) {
+    const float *xin = type == P_OPROJ ? a.x0 : a.x1;
+#pragma unroll
+    for (int j = 0; j < NB / CL; j++) pre.xv[j] = j < nb ? xin[(size_t)(b0 + j) * a.d + col] : 0.f;
+  } else if (type == P_QKV && nt <= a.H) {
+#pragma unroll
+    for (int j = 0; j < NB / CL; j++) {
+      pre.cs[j] = make_float2(1.f, 0.f);
+      if (j < nb) {
+        const int p = min(max(s.pos[b0 + j], 0), a.max_seq - 1);
+        pre.cs[j] = a.rope[(size_t)p * 64 + (e & 63)];
+      }
+    }
+  }
+}
+
 __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int layer, int nt, float *tl, int b0,
-                              int b1, int e) {
+                              int b1, int e, const EpiPre &pre) {
   const int lane = e & 31, w = e >> 5, nb = b1 - b0;
   const int col = nt * 128 + e;
   if (type == P_FC) {
-    for (int j = 0; j < nb; j++) {
-      const float v = fmaxf(tl[e * (NB + 1) + j], 0.f);
-      a.f[(size_t)(b0 + j) * a.F + col] = __float2bfloat16_rn(v * v);
+#pragma unroll
+    for (int j = 0; j < NB / CL; j++) {
+      if (j < nb) {
+        const float v = fmaxf(tl[e * (NB + 1) + j], 0.f);
+        a.f[(size_t)(b0 + j) * a.F + col] = __float2bfloat16_rn(v * v);
+      }
     }
   } else if (type == P_OPROJ || type == P_PROJ) {
-    const float *xin = type == P_OPROJ ? a.x0 : a.x1;
     float *xout = type == P_OPROJ ? a.x1 : a.x0;
     float *ss = a.ss + (size_t)(type == P_OPROJ ? 2 * layer + 1 : 2 * layer + 2) * 32;
-    for (int j = 0; j < nb; j++) {
-      const float v = xin[(size_t)(b0 + j) * a.d + col] + tl[e * (NB + 1) + j];
-      xout[(size_t)(b0 + j) * a.d + col] = v;
-      tl[e * (NB + 1) + j] = v * v;
+#pragma unroll
+    for (int j = 0; j < NB / CL; j++) {
+      if (j < nb) {
+        const float v = pre.xv[j] + tl[e * (NB + 1) + j];
+        xout[(size_t)(b0 + j) * a.d + col] = v;
+        tl[e * (NB + 1) + j] = v * v;
+      }
     }
     epi_sync();
     for (int j = w; j < nb; j += 4) {
@@ -400,13 +467,11 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
       // RoPE on split-half pairs (e, e^64), then RMS norm over the head
       constexpr int MJ = NB / CL;
       float rot[MJ];
-      const int i = e & 63;
 #pragma unroll
       for (int j = 0; j < MJ; j++) {
         rot[j] = 0.f;
         if (j < nb) {
-          const int p = min(max(s.pos[b0 + j], 0), a.max_seq - 1);
-          const float2 cs = a.rope[(size_t)p * 64 + i];
+          const float2 cs = pre.cs[j];
           const float v = tl[e * (NB + 1) + j], u = tl[(e ^ 64) * (NB + 1) + j];
           rot[j] = e < 64 ? v * cs.x - u * cs.y : u * cs.y + v * cs.x;
         }
@@ -451,10 +516,16 @@ __device__ void head_epilogue(const StepArgs &a, const Smem &s, int nt, const ui
   const int lane = e & 31, w = e >> 5;
   const int col = nt * 128 + n;
   const float inv = 1.0f / a.cap;
-  for (int b = 0; b < a.B; b++) {
-    const float z = a.cap * tanhf(__uint_as_float(r[b]) * inv);
-    if (s.valid[b]) a.logits[(size_t)b * a.V + col] = z;
-    tl[n * (NB + 1) + b] = z + (a.noise ? a.noise[(size_t)b * a.V + col] : 0.f);
+  float nz[NB];
+#pragma unroll
+  for (int b = 0; b < NB; b++) nz[b] = (a.noise && b < a.B) ? a.noise[(size_t)b * a.V + col] : 0.f;
+#pragma unroll
+  for (int b = 0; b < NB; b++) {
+    if (b < a.B) {
+      const float z = a.cap * tanhf(__uint_as_float(r[b]) * inv);
+      if (s.valid[b]) a.logits[(size_t)b * a.V + col] = z;
+      tl[n * (NB + 1) + b] = z + nz[b];
+    }
   }
   epi_sync();
   for (int b = w; b < a.B; b += 4) {
@@ -711,7 +782,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     s.pos[b] = ok ? p : 0;
     s.valid[b] = ok;
   }
-  if (warp == 1) tmem_alloc(s.tmem_slot, NB);
+  if (warp == 1) tmem_alloc(s.tmem_slot, NB * NACC);
   tc_fence_before();
   __syncthreads();
   cluster.sync();  // peers' barriers are initialised before any remote arrive
@@ -823,8 +894,18 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           if (!mbar_wait(s.acc_full, units & 1, s.abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
           uint32_t r[NB];
-          tmem_ld32(tmem + lane_off, r);
-          tmem_ld_wait();
+          {
+            const int nacc = min(NACC, g.nkb);
+            tmem_ld32(tmem + lane_off, r);
+            for (int q = 1; q < nacc; q++) {
+              uint32_t r2[NB];
+              tmem_ld32(tmem + lane_off + (uint32_t)q * NB, r2);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < NB; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
+            }
+            tmem_ld_wait();
+          }
           tc_fence_before();
           mbar_arrive(s.acc_empty);
           if (g.nkb == 0)
@@ -839,18 +920,37 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           for (int j = 0; j < NB; j++) red[n * NB + j] = __uint_as_float(r[j]);
           epi_sync();
           if (e < CL) mbar_arrive_remote(s.red_full, e);
-          if (!mbar_wait_cluster(s.red_full, rounds & 1, s.abort_flag, a.status)) { ok = false; break; }
           const int b0 = rank * (NB / CL), b1 = min(a.B, b0 + NB / CL);
-          for (int j = 0; j < NB / CL; j++) {
-            float sum = 0.f;
+          EpiPre pre;
+          epi_preload(a, s, type, nt, b0, b1, e, pre);
+          if (!mbar_wait_cluster(s.red_full, rounds & 1, s.abort_flag, a.status)) { ok = false; break; }
+          {
+            float pv[CL][NB / CL];
 #pragma unroll
-            for (int q = 0; q < CL; q++) sum += cluster.map_shared_rank(red, q)[e * NB + rank * (NB / CL) + j];
-            tl[e * (NB + 1) + j] = sum;
+            for (int q = 0; q < CL; q++) {
+              const float4 *src =
+                  reinterpret_cast<const float4 *>(cluster.map_shared_rank(red, q) + e * NB + rank * (NB / CL));
+#pragma unroll
+              for (int j4 = 0; j4 < NB / CL / 4; j4++) {
+                const float4 v4 = src[j4];
+                pv[q][4 * j4 + 0] = v4.x;
+                pv[q][4 * j4 + 1] = v4.y;
+                pv[q][4 * j4 + 2] = v4.z;
+                pv[q][4 * j4 + 3] = v4.w;
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < NB / CL; j++) {
+              float sum = 0.f;
+#pragma unroll
+              for (int q = 0; q < CL; q++) sum += pv[q][j];
+              tl[e * (NB + 1) + j] = sum;
+            }
           }
           epi_sync();
           if (e < CL) mbar_arrive_remote(s.red_free, e);
           rounds++;
-          if (b1 > b0) gemm_epilogue(a, s, type, layer, nt, tl, b0, b1, e);
+          if (b1 > b0) gemm_epilogue(a, s, type, layer, nt, tl, b0, b1, e, pre);
           epi_sync();
         }
       }
@@ -865,7 +965,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, NB);
+    tmem_dealloc(tmem, NB * NACC);
   }
 }
 
