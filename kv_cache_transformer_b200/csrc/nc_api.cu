@@ -441,7 +441,7 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
       std::vector<CUtensorMap> maps(nmaps);
       alloc((void **)&kv->step_maps, sizeof(CUtensorMap) * nmaps);
       alloc((void **)&kv->step_bar, sizeof(unsigned long long));
-      alloc((void **)&kv->step_ss, sizeof(float) * (size_t)(2 * c.depth + 1) * 32);
+      alloc((void **)&kv->step_ss, sizeof(float) * (size_t)(2 * c.depth + 1) * 16 * 32);
       if (e == cudaSuccess) e = cudaMemset(kv->step_bar, 0, sizeof(unsigned long long));
       if (e == cudaSuccess && nc::decode_step_build_maps(model, kv->k, kv->v, max_batch, max_seq, maps.data())) {
         e = cudaMemcpy(kv->step_maps, maps.data(), sizeof(CUtensorMap) * nmaps, cudaMemcpyHostToDevice);

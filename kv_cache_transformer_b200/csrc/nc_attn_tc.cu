@@ -12,9 +12,12 @@
 //                        MN-major straight from the cache layout)  -> TMEM
 // and finally y = O / l in bf16.
 // Warp roles (192 threads): warp 0 TMA producer (Q once, K/V tiles through a
-// 2-stage ring), warp 1 TMEM allocator + MMA issuer (S_{j+1} overlaps the
-// softmax of tile j), warps 2-5 softmax / O rescale / epilogue, one thread
-// per row. Waits are bounded as in the GEMM.
+// 2-stage ring), warp 1 TMEM allocator + MMA issuer (S_{j+1} is issued before
+// P_j is consumed), warps 2-5 softmax / O rescale / epilogue, one thread per
+// row. P is double-buffered, so the softmax of tile j+1 overlaps P_j V_j, and
+// O is rescaled only when a row's running max grows by more than 2^8 (the
+// probabilities of a tile are then at most 256, exact in fp32 and bf16).
+// Waits are bounded as in the GEMM.
 #include "nc_internal.h"
 #include "nc_sm100.cuh"
 
@@ -32,10 +35,11 @@ constexpr int ST = 2;             // K/V stages
 constexpr int SUB = 128 * 64 * 2; // one 128-row x 64-column swizzled box: 16 KB
 constexpr int TILE = 2 * SUB;     // 128 x 128 bf16: 32 KB
 constexpr int OFF_Q = 0;
-constexpr int OFF_P = TILE;
-constexpr int OFF_K = 2 * TILE;              // ST tiles
-constexpr int OFF_V = 2 * TILE + ST * TILE;  // ST tiles
-constexpr int OFF_BAR = 2 * TILE + 2 * ST * TILE;
+constexpr int OFF_P = TILE;                  // 2 tiles (double-buffered P)
+constexpr int OFF_K = 3 * TILE;              // ST tiles
+constexpr int OFF_V = 3 * TILE + ST * TILE;  // ST tiles
+constexpr int OFF_BAR = 3 * TILE + 2 * ST * TILE;
+constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when the max grows by more than 2^8
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr int THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;  // O: cols 0..127, S buffers: 128..255, 256..383
@@ -92,9 +96,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *v_full = k_full + ST;     // ST
   uint64_t *kv_empty = v_full + ST;   // ST
   uint64_t *s_full = kv_empty + ST;   // 2
-  uint64_t *p_full = s_full + 2;      // 1 (128 arrivals)
-  uint64_t *o_done = p_full + 1;      // 1
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 1);
+  uint64_t *p_full = s_full + 2;      // 2 (128 arrivals), one per P buffer
+  uint64_t *o_done = p_full + 2;      // 2, one per P buffer
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -113,10 +117,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&mapQ);
@@ -173,17 +178,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) ok = issue_s(0);
       for (int j = 0; j < n_kv && ok; j++) {
         if (j + 1 < n_kv && !issue_s(j + 1)) break;
-        if (!mbar_wait(p_full, j & 1, abort_flag, a.status)) break;
+        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) break;
         const int s = j % ST;
         if (!mbar_wait(&v_full[s], (j / ST) & 1, abort_flag, a.status)) break;
         tc_fence_after();
-        const uint32_t v0 = smem_u32(smem + OFF_V + s * TILE);
+        const uint32_t v0 = smem_u32(smem + OFF_V + s * TILE), pb = p0 + (j & 1) * TILE;
 #pragma unroll
         for (int k = 0; k < BKV / 16; k++) {
           const uint32_t poff = (k >> 2) * SUB + (k & 3) * 32;
-          mma_bf16(tO, desc_k_sw128(p0 + poff), desc_mn_sw128(v0 + k * 2048), id_o, (j | k) != 0);
+          mma_bf16(tO, desc_k_sw128(pb + poff), desc_mn_sw128(v0 + k * 2048), id_o, (j | k) != 0);
         }
-        mma_commit(o_done);
+        mma_commit(&o_done[j & 1]);
         mma_commit(&kv_empty[s]);
       }
     }
@@ -194,31 +199,36 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row = row0 + r;                  // row inside the sequence
     const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t *prow = smem + OFF_P + r * 128;    // row r of both 64-key boxes
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and running sum
     bool ok = true;
     for (int j = 0; j < n_kv && ok; j++) {
       if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sbase = tS + (j & 1) * 128 + lane_off;
       const int kbase = j * BKV;
-      // pass 1: row max of the masked, scaled scores
+      // the whole score row in one round trip
+      uint32_t v[BKV];
+      tmem_ld32(sbase + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+      tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_ld32(sbase + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+      tmem_ld32(sbase + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+      tmem_ld_wait();
       float tmax = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(sbase + c, v);
-        tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; i++)
-          if (kbase + c + i <= t_row) tmax = fmaxf(tmax, __uint_as_float(v[i]) * a.scale_log2);
+      for (int i = 0; i < BKV; i++) {
+        const float x = (kbase + i <= t_row) ? __uint_as_float(v[i]) * a.scale_log2 : -INFINITY;
+        v[i] = __float_as_uint(x);
+        tmax = fmaxf(tmax, x);
       }
-      const float m_new = fmaxf(m, tmax);
-      const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
-      // the previous P.V must be finished before O or the P buffer change
-      if (j > 0 && !mbar_wait(o_done, (j - 1) & 1, abort_flag, a.status)) { ok = false; break; }
-      tc_fence_after();
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
+      const float m_new = need ? tmax : m;
+      const float alpha = (need && m != -INFINITY) ? exp2f(m - m_new) : 1.f;
+      // P buffer j&1 is free once P_{j-2} V_{j-2} is done
+      if (j >= 2 && !mbar_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O must hold every earlier P V before it is rescaled
+        if (!mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           uint32_t o[32];
@@ -230,37 +240,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tmem_st_wait();
       }
-      // pass 2: p = exp2(s*scale_log2 - m_new), bf16 into the swizzled P tile
+      // p = exp2(s - m_new) in bf16 into the swizzled P tile j&1
+      uint8_t *prow = smem + OFF_P + (j & 1) * TILE + r * 128;
       float sum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(sbase + c, v);
-        tmem_ld_wait();
-        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = (kbase + c + i <= t_row) ? exp2f(__uint_as_float(v[i]) * a.scale_log2 - m_new) : 0.f;
-          float p1 = (kbase + c + i + 1 <= t_row) ? exp2f(__uint_as_float(v[i + 1]) * a.scale_log2 - m_new) : 0.f;
-          sum += p0 + p1;
-          pk[i / 2] = pack2(p0, p1);
-        }
-        // 32 keys = four 16-byte chunks; chunk index XOR (row & 7) (128-byte swizzle)
-        const int box = c >> 6;
+      for (int c = 0; c < BKV; c += 8) {
+        float pv[8];
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const int chunk = ((c & 63) >> 3) + q;
-          uint4 *dst = reinterpret_cast<uint4 *>(prow + box * SUB + ((chunk ^ (r & 7)) << 4));
-          *dst = make_uint4(pk[q * 4 + 0], pk[q * 4 + 1], pk[q * 4 + 2], pk[q * 4 + 3]);
+        for (int i = 0; i < 8; i++) {
+          const float x = __uint_as_float(v[c + i]);
+          pv[i] = x == -INFINITY ? 0.f : exp2f(x - m_new);
+          sum += pv[i];
         }
+        const int box = c >> 6, chunk = (c & 63) >> 3;
+        *reinterpret_cast<uint4 *>(prow + box * SUB + ((chunk ^ (r & 7)) << 4)) =
+            make_uint4(pack2(pv[0], pv[1]), pack2(pv[2], pv[3]), pack2(pv[4], pv[5]), pack2(pv[6], pv[7]));
       }
       l = l * alpha + sum;
       m = m_new;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
-    if (ok && mbar_wait(o_done, (n_kv - 1) & 1, abort_flag, a.status)) {
+    if (ok && mbar_wait(&o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, a.status)) {
       tc_fence_after();
       const float inv = 1.f / l;
       bf16 *dst = a.y + ((size_t)b * a.rows_per_seq + row) * HD;

@@ -72,7 +72,7 @@ struct nc_kv {
   int step_grid = 0;           // CTAs of the step kernel, 0 = not available
   CUtensorMap *step_maps = nullptr;  // device copy of the step kernel's tensor maps
   unsigned long long *step_bar = nullptr;  // its grid-barrier counter
-  float *step_ss = nullptr;    // [2*depth+1][32]
+  float *step_ss = nullptr;    // [2*depth+1][16][32] per-128-column sums of squares
   int attn_chunk = 0, attn_splits = 0;
   // CUDA graph of the last decode step's launches, replayed while the call's
   // pointers and batch stay the same

@@ -54,6 +54,7 @@ constexpr int XKB = 20;                // X staging capacity, 64-column blocks
 constexpr int THREADS = 192;
 constexpr int KT = 64;                 // keys per attention tile
 constexpr int NACC = 4;                // TMEM accumulators the K loop rotates over
+constexpr int SSN = 16;                // 128-column chunks of d_model (d <= 2048)
 
 constexpr int OFF_RING = 0;
 constexpr int OFF_X = OFF_RING + RING * SLOT;          // XKB * NB * 128 bytes
@@ -73,7 +74,7 @@ struct StepArgs {
   const int32_t *tokens, *positions;
   int32_t *len;
   float *x0, *x1;             // residual [32][d]: layer input, after attention
-  float *ss;                  // [2L + 1][32] sums of squares for each norm
+  float *ss;                  // [2L + 1][SSN][32]: per-128-column sums of squares for each norm
   bf16 *q, *y, *f;            // [32][H][128], [32][d], [32][F]
   bf16 *kc, *vc;              // [L][max_batch][max_seq][128]
   const float2 *rope;         // [max_seq][64]
@@ -398,7 +399,15 @@ __device__ void stage_x(const StepArgs &a, const Smem &s, uint8_t *xs, int type,
 
 // per-row scale 1/rms from a complete sum of squares
 __device__ void load_inv(const StepArgs &a, const Smem &s, const float *ss, int e) {
-  if (e < NB) s.inv[e] = e < a.B ? rsqrtf(ss[e] / a.d + a.eps) : 0.f;
+  if (e < NB) {
+    float v[SSN];
+#pragma unroll
+    for (int j = 0; j < SSN; j++) v[j] = (j < a.d / 128 && e < a.B) ? ss[j * 32 + e] : 0.f;
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < SSN; j++) sum += v[j];
+    s.inv[e] = e < a.B ? rsqrtf(sum / a.d + a.eps) : 0.f;
+  }
   epi_sync();
 }
 
@@ -444,7 +453,9 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
     }
   } else if (type == P_OPROJ || type == P_PROJ) {
     float *xout = type == P_OPROJ ? a.x1 : a.x0;
-    float *ss = a.ss + (size_t)(type == P_OPROJ ? 2 * layer + 1 : 2 * layer + 2) * 32;
+    // this tile's sum of squares: one slot per (tile, column), added up in a
+    // fixed order by the consumer, so results do not depend on timing
+    float *ss = a.ss + ((size_t)(type == P_OPROJ ? 2 * layer + 1 : 2 * layer + 2) * SSN + nt) * 32;
 #pragma unroll
     for (int j = 0; j < NB / CL; j++) {
       if (j < nb) {
@@ -458,7 +469,7 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
       float sum = tl[lane * (NB + 1) + j] + tl[(lane + 32) * (NB + 1) + j] + tl[(lane + 64) * (NB + 1) + j] +
                   tl[(lane + 96) * (NB + 1) + j];
       sum = warp_sum(sum);
-      if (lane == 0) atomicAdd(&ss[b0 + j], sum);
+      if (lane == 0) ss[b0 + j] = sum;
     }
   } else {  // P_QKV: one 128-wide head per tile: q heads, then k, then v
     const int head = nt;
@@ -807,11 +818,6 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
       int type, layer;
       phase_of(a, p, type, layer);
       if (type == P_EMBED) {
-        // sums of squares of norms 1..2L are accumulated later; norm 0 is
-        // written whole below
-        if (blockIdx.x == 0)
-          for (int i = 32 + e; i < (2 * a.L + 1) * 32; i += 128) a.ss[i] = 0.f;
-        epi_sync();
         for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
           int tok = a.tokens[b];
           if (tok < 0 || tok >= a.V) {
@@ -829,17 +835,16 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           epi_sync();
           const float tot = tl[0] + tl[1] + tl[2] + tl[3];
           const float inv = rsqrtf(tot / a.d + a.eps);
-          float sq2 = 0.f;
-          for (int i = e; i < a.d; i += 128) {
-            const float v = __bfloat162float(row[i]) * inv;
-            a.x0[(size_t)b * a.d + i] = v;
-            sq2 += v * v;
+          // x0 and its per-128-column sums of squares (norm 0 of layer 0)
+          epi_sync();
+          for (int j = 0; j < a.d / 128; j++) {
+            const float v = __bfloat162float(row[j * 128 + e]) * inv;
+            a.x0[(size_t)b * a.d + j * 128 + e] = v;
+            const float q = warp_sum(v * v);
+            if (lane == 0) tl[8 + 4 * j + (e >> 5)] = q;
           }
-          sq2 = warp_sum(sq2);
           epi_sync();
-          if (lane == 0) tl[e >> 5] = sq2;
-          epi_sync();
-          if (e == 0) a.ss[b] = tl[0] + tl[1] + tl[2] + tl[3];
+          if (e < a.d / 128) a.ss[(size_t)e * 32 + b] = tl[8 + 4 * e] + tl[9 + 4 * e] + tl[10 + 4 * e] + tl[11 + 4 * e];
           epi_sync();
         }
       } else if (type == P_ATTN) {
@@ -871,7 +876,8 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
         // linear layer: QKV, OPROJ, FC, PROJ (cluster split-K) or HEAD (full K)
         const Gemm g = gemm_of(a, type, layer, cid, ncl, rank);
         const bool norm = (type == P_QKV || type == P_FC || type == P_HEAD);
-        if (norm) load_inv(a, s, a.ss + (size_t)(type == P_QKV ? 2 * layer : type == P_FC ? 2 * layer + 1 : 2 * a.L) * 32, e);
+        if (norm)
+          load_inv(a, s, a.ss + (size_t)(type == P_QKV ? 2 * layer : type == P_FC ? 2 * layer + 1 : 2 * a.L) * SSN * 32, e);
         bool staged_once = false;
         for (int nt = g.nt0; nt < g.n_tiles && ok; nt += g.nt_step, units++) {
           for (int c0 = 0; c0 < g.nkb || (c0 == 0 && g.nkb == 0); c0 += XKB) {
@@ -974,7 +980,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
 bool make_map_bf16_k64(CUtensorMap *map, const void *ptr, int rows, int cols, int ld, int box_rows);
 
 bool decode_step_supported(const nc_config &c, int B) {
-  return decode_fast_supported(c, B) && c.n_head <= 16 && (c.n_head + 2) * 128 <= 64 * 128;
+  return decode_fast_supported(c, B) && c.n_head <= 16 && c.d_model / 128 <= SSN;
 }
 
 int decode_step_maps_count(const nc_config &c) { return 4 * c.depth + 1 + 2; }
