@@ -79,6 +79,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// 2^x (PTX ex2.approx.ftz: relative error ~2^-22, 2^-inf = 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -94,8 +101,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *q_full = bar;             // 1
   uint64_t *k_full = bar + 1;         // ST
   uint64_t *v_full = k_full + ST;     // ST
-  uint64_t *kv_empty = v_full + ST;   // ST
-  uint64_t *s_full = kv_empty + ST;   // 2
+  uint64_t *k_empty = v_full + ST;    // ST: K stage free once S = Q K^T is done
+  uint64_t *v_empty = k_empty + ST;   // ST: V stage free once P V is done
+  uint64_t *s_full = v_empty + ST;    // 2
   uint64_t *p_full = s_full + 2;      // 2 (128 arrivals), one per P buffer
   uint64_t *o_done = p_full + 2;      // 2, one per P buffer
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 2);
@@ -115,7 +123,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < ST; s++) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int i = 0; i < 2; i++) {
       mbar_init(&s_full[i], 1);
@@ -136,19 +145,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tO = tmem, tS = tmem + 128;
 
   if (warp == 0) {
+    // lane 0 streams K (and Q), lane 1 streams V: a V stage still in use by
+    // P V never holds back the next K tile
+    const int krow = b * a.max_seq;
     if (lane == 0) {
       const int qrow = b * a.rows_per_seq + row0;
-      const int krow = b * a.max_seq;
       mbar_arrive_expect_tx(q_full, TILE);
       tma_load_2d(smem + OFF_Q, &mapQ, 0, qrow, q_full);
       tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, qrow, q_full);
       for (int j = 0; j < n_kv; j++) {
         const int s = j % ST;
-        const uint32_t ph = (j / ST) & 1;
-        if (!mbar_wait(&kv_empty[s], ph ^ 1, abort_flag, a.status)) break;
+        if (!mbar_wait(&k_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(&k_full[s], TILE);
         tma_load_2d(smem + OFF_K + s * TILE, &mapK, 0, krow + j * BKV, &k_full[s]);
         tma_load_2d(smem + OFF_K + s * TILE + SUB, &mapK, 64, krow + j * BKV, &k_full[s]);
+      }
+    } else if (lane == 1) {
+      for (int j = 0; j < n_kv; j++) {
+        const int s = j % ST;
+        if (!mbar_wait(&v_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(&v_full[s], TILE);
         tma_load_2d(smem + OFF_V + s * TILE, &mapV, 0, krow + j * BKV, &v_full[s]);
         tma_load_2d(smem + OFF_V + s * TILE + SUB, &mapV, 64, krow + j * BKV, &v_full[s]);
@@ -173,6 +188,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mma_bf16(d, desc_k_sw128(q0 + off), desc_k_sw128(k0 + off), id_s, k != 0);
         }
         mma_commit(&s_full[j & 1]);
+        mma_commit(&k_empty[s]);
         return true;
       };
       if (ok) ok = issue_s(0);
@@ -189,7 +205,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mma_bf16(tO, desc_k_sw128(pb + poff), desc_mn_sw128(v0 + k * 2048), id_o, (j | k) != 0);
         }
         mma_commit(&o_done[j & 1]);
-        mma_commit(&kv_empty[s]);
+        mma_commit(&v_empty[s]);
       }
     }
   } else {
@@ -213,13 +229,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_ld32(sbase + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
       tmem_ld32(sbase + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
       tmem_ld_wait();
-      float tmax = -INFINITY;
+      // row max on the raw scores (the scale is positive); the causal mask only
+      // matters on tiles that reach past this row's position
+      const bool masked = kbase + BKV - 1 > t_row;
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+      if (masked) {
 #pragma unroll
-      for (int i = 0; i < BKV; i++) {
-        const float x = (kbase + i <= t_row) ? __uint_as_float(v[i]) * a.scale_log2 : -INFINITY;
-        v[i] = __float_as_uint(x);
-        tmax = fmaxf(tmax, x);
+        for (int i = 0; i < BKV; i++) {
+          if (kbase + i > t_row) v[i] = __float_as_uint(-INFINITY);
+          if (i & 1) mx1 = fmaxf(mx1, __uint_as_float(v[i]));
+          else mx0 = fmaxf(mx0, __uint_as_float(v[i]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < BKV; i += 2) {
+          mx0 = fmaxf(mx0, __uint_as_float(v[i]));
+          mx1 = fmaxf(mx1, __uint_as_float(v[i + 1]));
+        }
       }
+      const float tmax = fmaxf(mx0, mx1) * a.scale_log2;
       const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
       const float m_new = need ? tmax : m;
       const float alpha = (need && m != -INFINITY) ? exp2f(m - m_new) : 1.f;
@@ -242,20 +270,22 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // p = exp2(s - m_new) in bf16 into the swizzled P tile j&1
       uint8_t *prow = smem + OFF_P + (j & 1) * TILE + r * 128;
-      float sum = 0.f;
+      // p = 2^(s*scale - m): one FMA and one ex2 per score (masked scores are
+      // -inf and give 0)
+      const float nm = -m_new;
+      float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
       for (int c = 0; c < BKV; c += 8) {
         float pv[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
-          const float x = __uint_as_float(v[c + i]);
-          pv[i] = x == -INFINITY ? 0.f : exp2f(x - m_new);
-          sum += pv[i];
-        }
+        for (int i = 0; i < 8; i++) pv[i] = ex2(fmaf(__uint_as_float(v[c + i]), a.scale_log2, nm));
+        sum0 += (pv[0] + pv[2]) + (pv[4] + pv[6]);
+        sum1 += (pv[1] + pv[3]) + (pv[5] + pv[7]);
         const int box = c >> 6, chunk = (c & 63) >> 3;
         *reinterpret_cast<uint4 *>(prow + box * SUB + ((chunk ^ (r & 7)) << 4)) =
             make_uint4(pack2(pv[0], pv[1]), pack2(pv[2], pv[3]), pack2(pv[4], pv[5]), pack2(pv[6], pv[7]));
       }
+      const float sum = sum0 + sum1;
       l = l * alpha + sum;
       m = m_new;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
