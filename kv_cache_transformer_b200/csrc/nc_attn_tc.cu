@@ -39,9 +39,12 @@ constexpr int OFF_P = TILE;                  // 2 tiles (double-buffered P)
 constexpr int OFF_K = 3 * TILE;              // ST tiles
 constexpr int OFF_V = 3 * TILE + ST * TILE;  // ST tiles
 constexpr int OFF_BAR = 3 * TILE + 2 * ST * TILE;
+constexpr int OFF_XCH = OFF_BAR + 128;       // [2][2][128] fp32: row-max halves, then row-sum halves
 constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when the max grows by more than 2^8
-constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr int THREADS = 192;
+constexpr int SMEM_USED = OFF_XCH + 2 * 2 * 128 * 4;
+constexpr int SMEM_BYTES = 227 * 1024;       // the rest is slack for 1024-byte alignment
+constexpr int MAX_PAD = SMEM_BYTES - SMEM_USED;
+constexpr int THREADS = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (2 per row)
 constexpr uint32_t TMEM_COLS = 512;  // O: cols 0..127, S buffers: 128..255, 256..383
 
 struct AttnArgs {
@@ -96,7 +99,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                            const __grid_constant__ CUtensorMap mapV, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint32_t raw = smem_u32(smem_raw);
-  uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
+  const uint32_t pad = ((raw + 1023) & ~1023u) - raw;
+  if (pad > (uint32_t)MAX_PAD) {  // shared memory window not aligned as expected: report, do nothing
+    if (threadIdx.x == 0) atomicOr(a.status, (unsigned)NC_DEV_TIMEOUT);
+    return;
+  }
+  uint8_t *smem = smem_raw + pad;
+  float *xch = reinterpret_cast<float *>(smem + OFF_XCH);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint64_t *q_full = bar;             // 1
   uint64_t *k_full = bar + 1;         // ST
@@ -128,7 +137,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int i = 0; i < 2; i++) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
       mbar_init(&o_done[i], 1);
     }
     *abort_flag = 0;
@@ -209,56 +218,63 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    // softmax / correction / epilogue: thread <-> row
+    // softmax / correction / epilogue: two threads per row, each owning 64 of
+    // the tile's 128 keys (and 64 of the 128 output dims)
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
     const int row = row0 + r;                  // row inside the sequence
     const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and running sum
+    float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's running sum
     bool ok = true;
-    for (int j = 0; j < n_kv && ok; j++) {
-      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+    // every thread runs every iteration (a failed wait only clears `ok`), so
+    // the two named-barrier syncs per iteration always pair up
+    for (int j = 0; j < n_kv; j++) {
+      ok = ok && mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status);
       tc_fence_after();
-      const uint32_t sbase = tS + (j & 1) * 128 + lane_off;
-      const int kbase = j * BKV;
-      // the whole score row in one round trip
-      uint32_t v[BKV];
+      const uint32_t sbase = tS + (j & 1) * 128 + lane_off + half * 64;
+      const int kbase = j * BKV + half * 64;
+      uint32_t v[64];
       tmem_ld32(sbase + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
       tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_ld32(sbase + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
-      tmem_ld32(sbase + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
       tmem_ld_wait();
-      // row max on the raw scores (the scale is positive); the causal mask only
-      // matters on tiles that reach past this row's position
-      const bool masked = kbase + BKV - 1 > t_row;
+      // raw max of this half (the scale is positive); the causal mask only
+      // matters on tiles that reach past the row's position
+      const bool masked = kbase + 63 > t_row;
       float mx0 = -INFINITY, mx1 = -INFINITY;
       if (masked) {
 #pragma unroll
-        for (int i = 0; i < BKV; i++) {
+        for (int i = 0; i < 64; i++) {
           if (kbase + i > t_row) v[i] = __float_as_uint(-INFINITY);
           if (i & 1) mx1 = fmaxf(mx1, __uint_as_float(v[i]));
           else mx0 = fmaxf(mx0, __uint_as_float(v[i]));
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < BKV; i += 2) {
+        for (int i = 0; i < 64; i += 2) {
           mx0 = fmaxf(mx0, __uint_as_float(v[i]));
           mx1 = fmaxf(mx1, __uint_as_float(v[i + 1]));
         }
       }
-      const float tmax = fmaxf(mx0, mx1) * a.scale_log2;
+      // the two halves of the row agree on the row max (buffer j&1: the
+      // partner has read the previous use of it before arriving here again)
+      float *xm = xch + (j & 1) * 256;
+      xm[half * 128 + r] = fmaxf(mx0, mx1);
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float tmax = fmaxf(xm[r], xm[128 + r]) * a.scale_log2;
       const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
       const float m_new = need ? tmax : m;
       const float alpha = (need && m != -INFINITY) ? exp2f(m - m_new) : 1.f;
       // P buffer j&1 is free once P_{j-2} V_{j-2} is done
-      if (j >= 2 && !mbar_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+      if (j >= 2) ok = ok && mbar_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status);
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O must hold every earlier P V before it is rescaled
-        if (!mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        // O must hold every earlier P V before it is rescaled; this half
+        // rescales output dims half*64 .. +63
+        ok = ok && mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status);
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < HD; c += 32) {
+        for (int c = half * 64; c < half * 64 + 64; c += 32) {
           uint32_t o[32];
           tmem_ld32(tO + lane_off + c, o);
           tmem_ld_wait();
@@ -268,36 +284,40 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tmem_st_wait();
       }
-      // p = exp2(s - m_new) in bf16 into the swizzled P tile j&1
-      uint8_t *prow = smem + OFF_P + (j & 1) * TILE + r * 128;
       // p = 2^(s*scale - m): one FMA and one ex2 per score (masked scores are
-      // -inf and give 0)
+      // -inf and give 0), bf16 into box `half` of the swizzled P tile j&1
+      uint8_t *prow = smem + OFF_P + (j & 1) * TILE + half * SUB + r * 128;
       const float nm = -m_new;
       float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < BKV; c += 8) {
+      for (int c = 0; c < 64; c += 8) {
         float pv[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) pv[i] = ex2(fmaf(__uint_as_float(v[c + i]), a.scale_log2, nm));
         sum0 += (pv[0] + pv[2]) + (pv[4] + pv[6]);
         sum1 += (pv[1] + pv[3]) + (pv[5] + pv[7]);
-        const int box = c >> 6, chunk = (c & 63) >> 3;
-        *reinterpret_cast<uint4 *>(prow + box * SUB + ((chunk ^ (r & 7)) << 4)) =
+        const int chunk = c >> 3;
+        *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) =
             make_uint4(pack2(pv[0], pv[1]), pack2(pv[2], pv[3]), pack2(pv[4], pv[5]), pack2(pv[6], pv[7]));
       }
-      const float sum = sum0 + sum1;
-      l = l * alpha + sum;
+      l = l * alpha + (sum0 + sum1);
       m = m_new;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(&p_full[j & 1]);
     }
+    // row sum = both halves
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    float *xl = xch + 512 * 0;  // reuse buffer 0 (every exchange above has been read)
+    if (ok) xl[half * 128 + r] = l;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float lsum = xl[r] + xl[128 + r];
     if (ok && mbar_wait(&o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, a.status)) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      const float inv = 1.f / lsum;
       bf16 *dst = a.y + ((size_t)b * a.rows_per_seq + row) * HD;
 #pragma unroll 1
-      for (int c = 0; c < HD; c += 32) {
+      for (int c = half * 64; c < half * 64 + 64; c += 32) {
         uint32_t o[32];
         tmem_ld32(tO + lane_off + c, o);
         tmem_ld_wait();
