@@ -138,13 +138,21 @@ def dist_env():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank scalar (the timed region) over all ranks."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(units_per_rank: float, t_ms_max: float, world: int) -> float:
+    """Whole-job throughput of independent replicas: every rank processed
+    units_per_rank in at most t_ms_max milliseconds."""
+    return world * units_per_rank / (t_ms_max / 1e3)
 
 
 def barrier(world: int):
@@ -271,7 +279,7 @@ def run_ours(args):
     barrier(world)
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = t_ms / args.steps
-    value = world * args.steps * B * T / (t_ms / 1e3)
+    value = replica_throughput(args.steps * B * T, t_ms, world)
 
     fl = prefill_flops(cfg, B, T)
     gemm_ms = kms[nc.NC_K_GEMM] / args.steps  # GEMM time per step
@@ -433,6 +441,117 @@ def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local):
     }
 
 
+def run_decode_workload(args):
+    """d26 latency decode (B=1, 1024-token prompt, 512 greedy steps) or d30
+    rollout (256-token prompt, fork to 16 samples, 256 steps of argmax over
+    logits + Gumbel noise). One JSON line with decode tok/s and the HBM
+    roofline of a decode step."""
+    import numpy as np
+    import torch
+    import kv_cache_transformer_b200 as nc
+    import nc_synth as syn
+    from kv_cache_transformer_b200 import build as ncbuild
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    ncbuild.build()
+    peaks, peaks_src = load_peaks()
+    w = syn.WORKLOADS[args.workload]
+    cfg = w.model
+    model = nc.Model(cfg, syn.make_blob(cfg, w.weight_seed))
+    V, T, S = cfg.vocab, w.prompt_len, w.decode_steps
+    max_seq = T + S
+    prompts = torch.from_numpy(syn.prompt_tokens(w)).cuda()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    extra = {}
+    if w.fork:
+        n = w.fork
+        src = model.kv(1, max_seq)
+        dst = model.kv(n, max_seq)
+        tok1 = torch.empty((1,), dtype=torch.int32, device="cuda")
+        logits = torch.empty((n, V), dtype=torch.float32, device="cuda")
+        tok = torch.empty((n,), dtype=torch.int32, device="cuda")
+        # seeded Gumbel noise per step and sample, generated up front (an input)
+        noise = torch.from_numpy(np.stack([syn.gumbel(w.noise_seed, (n, V), stream=s_) for s_ in range(S)])).cuda()
+
+        def run_once():
+            model.prefill(src, prompts, 0, None, tok1)
+            src.fork_to(0, dst, 0, n)
+            tok.copy_(tok1.expand(n))
+            for s_ in range(S):
+                model.decode_step(dst, tok, None, noise[s_], logits, tok)
+
+        for _ in range(max(1, args.warmup // 3)):
+            run_once()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        model.prefill(src, prompts, 0, None, tok1)
+        e1.record(stream)
+        ef = torch.cuda.Event(enable_timing=True)
+        src.fork_to(0, dst, 0, n)
+        ef.record(stream)
+        tok.copy_(tok1.expand(n))
+        clocks = ClockSampler(local)
+        torch.cuda.synchronize()
+        clocks.start()
+        d0 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        n0 = nc.nc_launch_count()
+        for s_ in range(S):
+            model.decode_step(dst, tok, None, noise[s_], logits, tok)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        launches = nc.nc_launch_count() - n0
+        clk = clocks.stop()
+        assert model.status() == 0
+        B = n
+        extra = {"prefill_ms": e0.elapsed_time(e1), "fork_ms": e1.elapsed_time(ef),
+                 "fork_bytes": cfg.depth * 2 * T * cfg.head_dim * 2 * n}
+        ctx_avg = T + (S + 1) / 2.0
+    else:
+        kv = model.kv(w.batch, max_seq)
+        B = w.batch
+        logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
+        tok = torch.empty((B,), dtype=torch.int32, device="cuda")
+        for _ in range(max(1, args.warmup // 3)):
+            model.prefill(kv, prompts, 0, logits, tok)
+            for _s in range(min(S, 16)):
+                model.decode_step(kv, tok, None, None, logits, tok)
+        model.prefill(kv, prompts, 0, logits, tok)
+        clocks = ClockSampler(local)
+        torch.cuda.synchronize()
+        clocks.start()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        n0 = nc.nc_launch_count()
+        for _s in range(S):
+            model.decode_step(kv, tok, None, None, logits, tok)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        launches = nc.nc_launch_count() - n0
+        clk = clocks.stop()
+        assert model.status() == 0
+        ctx_avg = T + (S + 1) / 2.0
+    t_ms = d0.elapsed_time(d1)
+    by = decode_bytes(cfg, B, ctx_avg)
+    ms_step = t_ms / S
+    gbs = by["total"] / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": f"{args.workload} bf16 decode tok/s; % of HBM roofline", "value": B * S / (t_ms / 1e3),
+        "unit": "tok/s", "n_gpus": 1, "steps": S, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "batch": B, "prompt": T, "decode_steps": S,
+                   "fork": w.fork, "gumbel_noise": bool(w.fork)},
+        "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": by["total"],
+                     "peak_source": f"{peaks_src} hbm_gbs"},
+        "gpu_launches": int(launches), "clocks": clk, **extra,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -443,6 +562,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only", choices=("all", "decode"), default="all",
                     help="decode: skip the prefill timing (for profiling the decode kernels)")
+    ap.add_argument("--workload", choices=("d20", "d26_latency", "d30_rollout"), default="d20",
+                    help="d20: the headline prefill + decode line; d26_latency / d30_rollout: the other "
+                         "decode workloads, one JSON line each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=128,
                     help="tokens of one prompt the CPU oracle runs per sample")
@@ -451,6 +573,8 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload != "d20":
+        run_decode_workload(args)
     else:
         run_ours(args)
 
