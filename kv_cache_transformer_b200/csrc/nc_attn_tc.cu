@@ -39,16 +39,17 @@ constexpr int OFF_P = TILE;                  // 2 tiles (double-buffered P)
 constexpr int OFF_K = 3 * TILE;              // ST tiles
 constexpr int OFF_V = 3 * TILE + ST * TILE;  // ST tiles
 constexpr int OFF_BAR = 3 * TILE + 2 * ST * TILE;
-constexpr int OFF_XCH = OFF_BAR + 128;       // [2][2][128] fp32: row-max halves, then row-sum halves
+constexpr int OFF_XCH = OFF_BAR + 160;       // [2][2][128] fp32: row-max halves (x2); then the row-sum halves
 constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when the max grows by more than 2^8
 constexpr int SMEM_USED = OFF_XCH + 2 * 2 * 128 * 4;
+static_assert(SMEM_USED + 256 <= 227 * 1024, "shared memory budget");
 constexpr int SMEM_BYTES = 227 * 1024;       // the rest is slack for 1024-byte alignment
 constexpr int MAX_PAD = SMEM_BYTES - SMEM_USED;
 constexpr int THREADS = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (2 per row)
-constexpr uint32_t TMEM_COLS = 512;  // O: cols 0..127, S buffers: 128..255, 256..383
+constexpr uint32_t TMEM_COLS = 512;  // O accumulators: cols 0..255, S buffers: 256..511
 
 struct AttnArgs {
-  int T, H, max_seq;
+  int T, H, B, max_seq;
   int rows_per_seq;  // T*H
   float scale_log2;  // log2(e) / sqrt(hd)
   bf16 *y;           // [B*T*H, 128]
@@ -108,27 +109,36 @@ __global__ void __launch_bounds__(THREADS, 1)
   float *xch = reinterpret_cast<float *>(smem + OFF_XCH);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   uint64_t *q_full = bar;             // 1
-  uint64_t *k_full = bar + 1;         // ST
+  uint64_t *q_empty = bar + 1;        // 1: Q free once the item's last S is done
+  uint64_t *k_full = bar + 2;         // ST
   uint64_t *v_full = k_full + ST;     // ST
   uint64_t *k_empty = v_full + ST;    // ST: K stage free once S = Q K^T is done
   uint64_t *v_empty = k_empty + ST;   // ST: V stage free once P V is done
   uint64_t *s_full = v_empty + ST;    // 2
-  uint64_t *p_full = s_full + 2;      // 2 (128 arrivals), one per P buffer
+  uint64_t *p_full = s_full + 2;      // 2 (256 arrivals), one per P buffer
   uint64_t *o_done = p_full + 2;      // 2, one per P buffer
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_done + 2);
+  uint64_t *o_empty = o_done + 2;     // 2 (256 arrivals), one per O accumulator
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_empty + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_rt = (a.rows_per_seq + BR - 1) / BR;
-  const int rt = n_rt - 1 - blockIdx.x;  // heaviest tiles first
-  const int b = blockIdx.y;
-  const int row0 = rt * BR;              // first row inside the sequence
-  int t_max = (row0 + BR - 1) / a.H;
-  if (t_max > a.T - 1) t_max = a.T - 1;
-  const int n_kv = t_max / BKV + 1;
+  const int n_items = n_rt * a.B;
+
+  // work item i: row tile n_rt-1 - i/B of sequence i%B (heaviest first), the
+  // CTA takes items blockIdx.x, +gridDim.x, ...
+  auto item_of = [&](int i, int &b, int &row0, int &n_kv) {
+    const int rt = n_rt - 1 - i / a.B;
+    b = i % a.B;
+    row0 = rt * BR;
+    int t_max = (row0 + BR - 1) / a.H;
+    if (t_max > a.T - 1) t_max = a.T - 1;
+    n_kv = t_max / BKV + 1;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < ST; s++) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
@@ -139,6 +149,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 256);
       mbar_init(&o_done[i], 1);
+      mbar_init(&o_empty[i], 256);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -151,31 +162,43 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO = tmem, tS = tmem + 128;
+  const uint32_t tO0 = tmem, tS = tmem + 256;  // O accumulators at columns 0 and 128, S buffers at 256 and 384
 
   if (warp == 0) {
-    // lane 0 streams K (and Q), lane 1 streams V: a V stage still in use by
-    // P V never holds back the next K tile
-    const int krow = b * a.max_seq;
+    // lane 0 streams Q and K, lane 1 streams V, item after item
     if (lane == 0) {
-      const int qrow = b * a.rows_per_seq + row0;
-      mbar_arrive_expect_tx(q_full, TILE);
-      tma_load_2d(smem + OFF_Q, &mapQ, 0, qrow, q_full);
-      tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, qrow, q_full);
-      for (int j = 0; j < n_kv; j++) {
-        const int s = j % ST;
-        if (!mbar_wait(&k_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(&k_full[s], TILE);
-        tma_load_2d(smem + OFF_K + s * TILE, &mapK, 0, krow + j * BKV, &k_full[s]);
-        tma_load_2d(smem + OFF_K + s * TILE + SUB, &mapK, 64, krow + j * BKV, &k_full[s]);
+      int j = 0, it = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, it++) {
+        int b, row0, n_kv;
+        item_of(i, b, row0, n_kv);
+        const int krow = b * a.max_seq;
+        if (!mbar_wait(q_empty, (it & 1) ^ 1, abort_flag, a.status)) break;
+        mbar_arrive_expect_tx(q_full, TILE);
+        tma_load_2d(smem + OFF_Q, &mapQ, 0, b * a.rows_per_seq + row0, q_full);
+        tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, b * a.rows_per_seq + row0, q_full);
+        for (int jj = 0; jj < n_kv; jj++, j++) {
+          const int s = j % ST;
+          if (!mbar_wait(&k_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], TILE);
+          tma_load_2d(smem + OFF_K + s * TILE, &mapK, 0, krow + jj * BKV, &k_full[s]);
+          tma_load_2d(smem + OFF_K + s * TILE + SUB, &mapK, 64, krow + jj * BKV, &k_full[s]);
+        }
       }
     } else if (lane == 1) {
-      for (int j = 0; j < n_kv; j++) {
-        const int s = j % ST;
-        if (!mbar_wait(&v_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(&v_full[s], TILE);
-        tma_load_2d(smem + OFF_V + s * TILE, &mapV, 0, krow + j * BKV, &v_full[s]);
-        tma_load_2d(smem + OFF_V + s * TILE + SUB, &mapV, 64, krow + j * BKV, &v_full[s]);
+      int j = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
+        int b, row0, n_kv;
+        item_of(i, b, row0, n_kv);
+        const int krow = b * a.max_seq;
+        for (int jj = 0; jj < n_kv; jj++, j++) {
+          const int s = j % ST;
+          if (!mbar_wait(&v_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[s], TILE);
+          tma_load_2d(smem + OFF_V + s * TILE, &mapV, 0, krow + jj * BKV, &v_full[s]);
+          tma_load_2d(smem + OFF_V + s * TILE + SUB, &mapV, 64, krow + jj * BKV, &v_full[s]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -183,38 +206,55 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t id_s = idesc_bf16_f32(BR, BKV);
       const uint32_t id_o = idesc_bf16_f32(BR, HD) | (1u << 16);  // B (V) is MN-major
       const uint32_t q0 = smem_u32(smem + OFF_Q), p0 = smem_u32(smem + OFF_P);
-      bool ok = mbar_wait(q_full, 0, abort_flag, a.status);
-      // S_j = Q K_j^T into S buffer j % 2
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % ST;
-        if (!mbar_wait(&k_full[s], (j / ST) & 1, abort_flag, a.status)) return false;
+      // tile counters run across items; J indexes K/V stages, S and P buffers
+      int J = 0, it = 0;
+      bool ok = true;
+      auto issue_s = [&](int jg) -> bool {  // S_jg = Q K_jg^T into S buffer jg % 2
+        const int s = jg % ST;
+        if (!mbar_wait(&k_full[s], (jg / ST) & 1, abort_flag, a.status)) return false;
         tc_fence_after();
         const uint32_t k0 = smem_u32(smem + OFF_K + s * TILE);
-        const uint32_t d = tS + (j & 1) * 128;
+        const uint32_t d = tS + (jg & 1) * 128;
 #pragma unroll
         for (int k = 0; k < HD / 16; k++) {
           const uint32_t off = (k >> 2) * SUB + (k & 3) * 32;
           mma_bf16(d, desc_k_sw128(q0 + off), desc_k_sw128(k0 + off), id_s, k != 0);
         }
-        mma_commit(&s_full[j & 1]);
+        mma_commit(&s_full[jg & 1]);
         mma_commit(&k_empty[s]);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_kv && ok; j++) {
-        if (j + 1 < n_kv && !issue_s(j + 1)) break;
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, a.status)) break;
-        const int s = j % ST;
-        if (!mbar_wait(&v_full[s], (j / ST) & 1, abort_flag, a.status)) break;
+      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, it++) {
+        int b, row0, n_kv;
+        item_of(i, b, row0, n_kv);
+        const int ob = it & 1;
+        const uint32_t tO = tO0 + ob * 128;
+        if (!mbar_wait(q_full, it & 1, abort_flag, a.status)) break;
+        // the epilogue of item it-2 must have read this O accumulator
+        if (!mbar_wait(&o_empty[ob], ((it >> 1) & 1) ^ 1, abort_flag, a.status)) break;
         tc_fence_after();
-        const uint32_t v0 = smem_u32(smem + OFF_V + s * TILE), pb = p0 + (j & 1) * TILE;
+        if (!issue_s(J)) break;
+        for (int jj = 0; jj < n_kv && ok; jj++) {
+          const int jg = J + jj;
+          if (jj + 1 < n_kv) {
+            if (!issue_s(jg + 1)) { ok = false; break; }
+          } else {
+            mma_commit(q_empty);  // the last S of the item: Q may be reloaded
+          }
+          if (!mbar_wait(&p_full[jg & 1], (jg >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          const int s = jg % ST;
+          if (!mbar_wait(&v_full[s], (jg / ST) & 1, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t v0 = smem_u32(smem + OFF_V + s * TILE), pb = p0 + (jg & 1) * TILE;
 #pragma unroll
-        for (int k = 0; k < BKV / 16; k++) {
-          const uint32_t poff = (k >> 2) * SUB + (k & 3) * 32;
-          mma_bf16(tO, desc_k_sw128(pb + poff), desc_mn_sw128(v0 + k * 2048), id_o, (j | k) != 0);
+          for (int k = 0; k < BKV / 16; k++) {
+            const uint32_t poff = (k >> 2) * SUB + (k & 3) * 32;
+            mma_bf16(tO, desc_k_sw128(pb + poff), desc_mn_sw128(v0 + k * 2048), id_o, (jj | k) != 0);
+          }
+          mma_commit(&o_done[jg & 1]);
+          mma_commit(&v_empty[s]);
         }
-        mma_commit(&o_done[j & 1]);
-        mma_commit(&v_empty[s]);
+        J += n_kv;
       }
     }
   } else {
@@ -223,96 +263,105 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const int r = quarter * 32 + lane;
-    const int row = row0 + r;                  // row inside the sequence
-    const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's running sum
     bool ok = true;
+    int J = 0, it = 0;
     // every thread runs every iteration (a failed wait only clears `ok`), so
-    // the two named-barrier syncs per iteration always pair up
-    for (int j = 0; j < n_kv; j++) {
-      ok = ok && mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag, a.status);
-      tc_fence_after();
-      const uint32_t sbase = tS + (j & 1) * 128 + lane_off + half * 64;
-      const int kbase = j * BKV + half * 64;
-      uint32_t v[64];
-      tmem_ld32(sbase + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
-      tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_ld_wait();
-      // raw max of this half (the scale is positive); the causal mask only
-      // matters on tiles that reach past the row's position
-      const bool masked = kbase + 63 > t_row;
-      float mx0 = -INFINITY, mx1 = -INFINITY;
-      if (masked) {
-#pragma unroll
-        for (int i = 0; i < 64; i++) {
-          if (kbase + i > t_row) v[i] = __float_as_uint(-INFINITY);
-          if (i & 1) mx1 = fmaxf(mx1, __uint_as_float(v[i]));
-          else mx0 = fmaxf(mx0, __uint_as_float(v[i]));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; i += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(v[i]));
-          mx1 = fmaxf(mx1, __uint_as_float(v[i + 1]));
-        }
-      }
-      // the two halves of the row agree on the row max (buffer j&1: the
-      // partner has read the previous use of it before arriving here again)
-      float *xm = xch + (j & 1) * 256;
-      xm[half * 128 + r] = fmaxf(mx0, mx1);
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float tmax = fmaxf(xm[r], xm[128 + r]) * a.scale_log2;
-      const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
-      const float m_new = need ? tmax : m;
-      const float alpha = (need && m != -INFINITY) ? exp2f(m - m_new) : 1.f;
-      // P buffer j&1 is free once P_{j-2} V_{j-2} is done
-      if (j >= 2) ok = ok && mbar_wait(&o_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, a.status);
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O must hold every earlier P V before it is rescaled; this half
-        // rescales output dims half*64 .. +63
-        ok = ok && mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.status);
+    // the named-barrier syncs always pair up
+    for (int i = blockIdx.x; i < n_items; i += gridDim.x, it++) {
+      int b, row0, n_kv;
+      item_of(i, b, row0, n_kv);
+      const int ob = it & 1;
+      const uint32_t tO = tO0 + ob * 128;
+      const int row = row0 + r;  // row inside the sequence
+      const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
+      float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's running sum
+      for (int jj = 0; jj < n_kv; jj++) {
+        const int jg = J + jj;
+        ok = ok && mbar_wait(&s_full[jg & 1], (jg >> 1) & 1, abort_flag, a.status);
         tc_fence_after();
-#pragma unroll 1
-        for (int c = half * 64; c < half * 64 + 64; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + c, o);
-          tmem_ld_wait();
+        const uint32_t sbase = tS + (jg & 1) * 128 + lane_off + half * 64;
+        const int kbase = jj * BKV + half * 64;
+        uint32_t v[64];
+        tmem_ld32(sbase + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+        tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld_wait();
+        // raw max of this half (the scale is positive); the causal mask only
+        // matters on tiles that reach past the row's position
+        const bool masked = kbase + 63 > t_row;
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+        if (masked) {
 #pragma unroll
-          for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tO + lane_off + c, o);
+          for (int q = 0; q < 64; q++) {
+            if (kbase + q > t_row) v[q] = __float_as_uint(-INFINITY);
+            if (q & 1) mx1 = fmaxf(mx1, __uint_as_float(v[q]));
+            else mx0 = fmaxf(mx0, __uint_as_float(v[q]));
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 64; q += 2) {
+            mx0 = fmaxf(mx0, __uint_as_float(v[q]));
+            mx1 = fmaxf(mx1, __uint_as_float(v[q + 1]));
+          }
         }
-        tmem_st_wait();
-      }
-      // p = 2^(s*scale - m): one FMA and one ex2 per score (masked scores are
-      // -inf and give 0), bf16 into box `half` of the swizzled P tile j&1
-      uint8_t *prow = smem + OFF_P + (j & 1) * TILE + half * SUB + r * 128;
-      const float nm = -m_new;
-      float sum0 = 0.f, sum1 = 0.f;
+        // the two halves of the row agree on the row max (buffer jg&1: the
+        // partner has read the previous use of it before arriving here again)
+        float *xm = xch + (jg & 1) * 256;
+        xm[half * 128 + r] = fmaxf(mx0, mx1);
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        const float tmax = fmaxf(xm[r], xm[128 + r]) * a.scale_log2;
+        const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
+        const float m_new = need ? tmax : m;
+        const float alpha = (need && m != -INFINITY) ? exp2f(m - m_new) : 1.f;
+        // P buffer jg&1 is free once P_{jg-2} V_{jg-2} is done (any item)
+        if (jg >= 2) ok = ok && mbar_wait(&o_done[jg & 1], ((jg - 2) >> 1) & 1, abort_flag, a.status);
+        if (jj > 0 && __any_sync(0xffffffffu, need)) {
+          // O must hold every earlier P V of this item before it is rescaled;
+          // this half rescales output dims half*64 .. +63
+          ok = ok && mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1, abort_flag, a.status);
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = half * 64; c < half * 64 + 64; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + lane_off + c, o);
+            tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 64; c += 8) {
-        float pv[8];
+            for (int q = 0; q < 32; q++) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+            tmem_st32(tO + lane_off + c, o);
+          }
+          tmem_st_wait();
+        }
+        // p = 2^(s*scale - m): one FMA and one ex2 per score (masked scores
+        // are -inf and give 0), bf16 into box `half` of the swizzled P tile
+        uint8_t *prow = smem + OFF_P + (jg & 1) * TILE + half * SUB + r * 128;
+        const float nm = -m_new;
+        float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; i++) pv[i] = ex2(fmaf(__uint_as_float(v[c + i]), a.scale_log2, nm));
-        sum0 += (pv[0] + pv[2]) + (pv[4] + pv[6]);
-        sum1 += (pv[1] + pv[3]) + (pv[5] + pv[7]);
-        const int chunk = c >> 3;
-        *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) =
-            make_uint4(pack2(pv[0], pv[1]), pack2(pv[2], pv[3]), pack2(pv[4], pv[5]), pack2(pv[6], pv[7]));
+        for (int c = 0; c < 64; c += 8) {
+          float pv[8];
+#pragma unroll
+          for (int q = 0; q < 8; q++) pv[q] = ex2(fmaf(__uint_as_float(v[c + q]), a.scale_log2, nm));
+          sum0 += (pv[0] + pv[2]) + (pv[4] + pv[6]);
+          sum1 += (pv[1] + pv[3]) + (pv[5] + pv[7]);
+          const int chunk = c >> 3;
+          *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pack2(pv[0], pv[1]), pack2(pv[2], pv[3]), pack2(pv[4], pv[5]), pack2(pv[6], pv[7]));
+        }
+        l = l * alpha + (sum0 + sum1);
+        m = m_new;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(&p_full[jg & 1]);
       }
-      l = l * alpha + (sum0 + sum1);
-      m = m_new;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
-    }
-    // row sum = both halves
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    float *xl = xch + 512 * 0;  // reuse buffer 0 (every exchange above has been read)
-    if (ok) xl[half * 128 + r] = l;
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    const float lsum = xl[r] + xl[128 + r];
-    if (ok && mbar_wait(&o_done[(n_kv - 1) & 1], ((n_kv - 1) >> 1) & 1, abort_flag, a.status)) {
+      // row sum = both halves (the exchange slot is free: every max above has
+      // been read before this barrier)
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      float *xl = xch;  // both row-max slots have been read by now
+      xl[half * 128 + r] = l;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float lsum = xl[r] + xl[128 + r];
+      const int jl = J + n_kv - 1;
+      ok = ok && mbar_wait(&o_done[jl & 1], (jl >> 1) & 1, abort_flag, a.status);
       tc_fence_after();
       const float inv = 1.f / lsum;
       bf16 *dst = a.y + ((size_t)b * a.rows_per_seq + row) * HD;
@@ -321,19 +370,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t o[32];
         tmem_ld32(tO + lane_off + c, o);
         tmem_ld_wait();
-        if (row < a.rows_per_seq) {
+        if (ok && row < a.rows_per_seq) {
           uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
 #pragma unroll
           for (int q = 0; q < 4; q++) {
             float f[8];
 #pragma unroll
-            for (int i = 0; i < 8; i++) f[i] = __uint_as_float(o[q * 8 + i]) * inv;
+            for (int z = 0; z < 8; z++) f[z] = __uint_as_float(o[q * 8 + z]) * inv;
             d4[q] = make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&o_empty[ob]);
+      // keep the l exchange slot from being overwritten before the partner read it
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      J += n_kv;
     }
-    tc_fence_before();
   }
   __syncthreads();
   if (warp == 1) {
@@ -365,12 +418,20 @@ cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int
   AttnArgs a;
   a.T = T;
   a.H = H;
+  a.B = B;
   a.max_seq = max_seq;
   a.rows_per_seq = rows;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   a.y = (bf16 *)y;
   a.status = status;
-  dim3 grid((rows + BR - 1) / BR, B);
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const int items = ((rows + BR - 1) / BR) * B;
+  dim3 grid(items < sms ? items : sms);
   count_launch();
   attn_prefill_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, a);
   return cudaGetLastError();

@@ -312,14 +312,14 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
             t++;
             tc_fence_after();
             const uint32_t w0 = smem_u32(ring + slot * SLOT), x0 = smem_u32(xs + kb * NB * 128);
-            // consecutive k-blocks accumulate into different TMEM accumulators, so
-            // their MMAs do not wait on one another; the epilogue adds them up
-            const int kg = c0 + kb;
-            const uint32_t acc = tmem + (uint32_t)(kg % NACC) * NB;
-            const bool fresh = kg < NACC;
+            // the four 16-column steps of a block accumulate into four different
+            // TMEM accumulators, so consecutive MMAs do not wait on one another;
+            // the epilogue adds the accumulators up
+            const bool fresh = (c0 + kb) == 0;
 #pragma unroll
             for (int k = 0; k < 4; k++)
-              mma_bf16(acc, desc_k_sw128(w0 + 32 * k), desc_k_sw128(x0 + 32 * k), idesc, (fresh && k == 0) ? 0 : 1);
+              mma_bf16(tmem + (uint32_t)k * NB, desc_k_sw128(w0 + 32 * k), desc_k_sw128(x0 + 32 * k), idesc,
+                       fresh ? 0 : 1);
             first = false;
             mma_commit(&s.empty[slot]);
           }
@@ -901,7 +901,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           tc_fence_after();
           uint32_t r[NB];
           {
-            const int nacc = min(NACC, g.nkb);
+            const int nacc = g.nkb > 0 ? NACC : 1;
             tmem_ld32(tmem + lane_off, r);
             for (int q = 1; q < nacc; q++) {
               uint32_t r2[NB];

@@ -98,6 +98,7 @@ def _attn_ref(q, k, v, T):
     (2, 300, 13, 128, 20),   # d26 heads: rows per tile span partial positions
     (3, 77, 15, 128, 3),     # d30 heads, last row tile partial
     (2, 50, 2, 64, 0),       # head_dim 64: generic kernel
+    (8, 1024, 10, 128, 0),   # 640 row tiles: each CTA of the persistent kernel runs several
 ])
 def test_attention_prefill_matches_float64(B, T, H, hd, extra):
     import torch
