@@ -136,8 +136,74 @@ void attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm,
   nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->max_seq, kv->y, s);
 }
 
+// The fused prefill layer sequence of bf16 head_dim-128 models, when every
+// GEMM of the layer takes the tensor-core kernel:
+//   QKV  = GEMM(h) with RoPE + QK norm + cache append in its epilogue, h the
+//          normed x (layer 0) or bf16(x) scaled per row by its RMS factor
+//   attention
+//   x   += GEMM(y) (O projection), writing h = bf16(x) and row sums of squares
+//   f    = relu(GEMM(h) * rms factor)^2
+//   x   += GEMM(f) (MLP projection), again writing h and the sums of squares
+//          except in the last layer
+bool fused_layers_ok(const nc_model *m, const nc_kv *kv, int M, nc::RowMap rm) {
+  const nc_config &c = m->cfg;
+  const int d = c.d_model, q = c.n_head * 128, F = c.mlp_hidden;
+  return m->fast && !rm.pos && M >= 128 && kv->row_ss && nc::rowops_supported(c) &&
+         nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim) && nc::gemm_tc_supported(M, q + 256, d, d) &&
+         nc::gemm_tc_supported(M, d, q, q) && nc::gemm_tc_supported(M, F, d, d) && nc::gemm_tc_supported(M, d, F, F);
+}
+
+int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  const int d = c.d_model, H = c.n_head, F = c.mlp_hidden, q = H * 128;
+  nc::GemmFuse fz;
+  fz.eps = c.norm_eps;
+  fz.xb = kv->h;
+  fz.ss_out = kv->row_ss;
+  fz.rope = kv->rope;
+  fz.q = kv->q;
+  fz.T = rm.T;
+  fz.H = H;
+  fz.max_seq = kv->max_seq;
+  const int nss = (d + 255) / 256;
+  cudaError_t e = cudaSuccess;
+  auto gemm = [&](int epi, const void *A, int lda, const void *W, int N, int K, void *out) {
+    if (e == cudaSuccess)
+      e = nc::k_gemm_tc(epi, A, lda, W, M, N, K, out, N, 0.f, m->status, m->num_sms, s, &fz);
+  };
+  for (int l = 0; l < c.depth && e == cudaSuccess; l++) {
+    const nc_layer_w &w = m->layers[l];
+    fz.kc = layer_ptr(kv, kv->k, l);
+    fz.vc = layer_ptr(kv, kv->v, l);
+    if (l == 0) {
+      ProfScope p(m, NC_K_MISC, s);
+      norm_rows(m, kv, M, s);
+    }
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      fz.ss_in = kv->row_ss;
+      fz.nss = l == 0 ? 0 : nss;
+      gemm(nc::EPI_QKV, kv->h, d, w.wqkv, q + 256, d, nullptr);
+    }
+    if (e == cudaSuccess) {
+      ProfScope p(m, NC_K_ATTN, s);
+      attention(m, kv, fz.kc, fz.vc, M, rm, s);
+    }
+    {
+      ProfScope p(m, NC_K_GEMM, s);
+      gemm(nc::EPI_RESID_X, kv->y, q, w.wo, d, q, kv->x);
+      fz.nss = nss;
+      gemm(nc::EPI_RELU2, kv->h, d, w.wfc, F, d, kv->f);
+      gemm(l + 1 < c.depth ? nc::EPI_RESID_X : nc::EPI_RESID, kv->f, F, w.wproj, d, F, kv->x);
+    }
+  }
+  if (e != cudaSuccess) return nc::set_error(NC_ECUDA, "prefill GEMM launch failed");
+  return NC_OK;
+}
+
 // The transformer blocks for M rows already embedded into kv->x.
 int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
+  if (fused_layers_ok(m, kv, M, rm)) return run_blocks_fused(m, kv, M, rm, s);
   const nc_config &c = m->cfg;
   int d = c.d_model, H = c.n_head, Hkv = c.n_kv_head, hd = c.head_dim, F = c.mlp_hidden;
   int qkv_w = (H + 2 * Hkv) * hd;
@@ -423,6 +489,7 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   alloc(&kv->f, elem * rows * F);
   alloc((void **)&kv->logits, sizeof(float) * (size_t)max_batch * c.vocab);
   alloc((void **)&kv->pos_ws, sizeof(int32_t) * max_batch);
+  if (model->fast && nc::rowops_supported(c)) alloc((void **)&kv->row_ss, sizeof(float) * ((d + 255) / 256) * rows);
   kv->dec_fast = nc::decode_fast_supported(c, 1);
   if (kv->dec_fast) {
     int nb = max_batch < 32 ? max_batch : 32;
@@ -488,7 +555,7 @@ void nc_kv_destroy(nc_kv *kv) {
   void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
                 kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
                 kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl,     kv->step_maps, kv->step_bar,
-                kv->step_ss};
+                kv->step_ss, kv->row_ss};
   for (void *p : ps) cudaFree(p);
   delete kv;
 }
@@ -518,7 +585,8 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
     nc::k_embed_norm(c.dtype, d_tokens, M, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
   }
   nc::RowMap rm{T, nullptr};
-  run_blocks(m, kv, M, rm, s);
+  const int rc = run_blocks(m, kv, M, rm, s);
+  if (rc != NC_OK) return rc;
   float *logits;
   long long last_off, row_stride;
   if (logits_mode == 1) {

@@ -15,6 +15,10 @@
 //               its 32-lane TMEM quarter = 32 rows), epilogue math, stores,
 //               then release the accumulator so the next tile's MMAs run
 //               while this one drains.
+// Fused prefill epilogues (GemmFuse): the RMS factor of un-normed bf16(x)
+// rows applied to the accumulator; RoPE + QK norm + cache append of the qkv
+// projection; bf16(x) and per-tile sums of squares written beside the
+// residual update.
 // Every mbarrier wait is bounded (nc_sm100.cuh); a timeout sets
 // NC_DEV_TIMEOUT and all roles drain to the common exit, where TMEM is freed.
 #include "nc_internal.h"
@@ -30,7 +34,8 @@ constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr int EPI_BUF = 4 * 32 * 32 * 4;  // per epilogue warp: a 32 x 32 fp32 transpose buffer
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BUF;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
 struct GemmArgs {
@@ -39,6 +44,7 @@ struct GemmArgs {
   int ldo;
   float cap;
   uint32_t *status;
+  GemmFuse fz;
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -48,9 +54,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Apply the epilogue to 32 consecutive columns of one row.
+// Apply the STORE / RELU2 / SOFTCAP epilogue to 32 consecutive columns of one
+// row; `scale` is the row's RMS factor (1 when A is already normed).
 template <int EPI>
-__device__ __forceinline__ void epilogue32(const GemmArgs &g, int row, int col, const uint32_t (&r)[32]) {
+__device__ __forceinline__ void epilogue32(const GemmArgs &g, int row, int col, const uint32_t (&r)[32], float scale,
+                                           float &) {
   size_t o = (size_t)row * g.ldo + col;
   if (EPI == EPI_STORE || EPI == EPI_RELU2) {
     uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<bf16 *>(g.out) + o);
@@ -59,7 +67,7 @@ __device__ __forceinline__ void epilogue32(const GemmArgs &g, int row, int col, 
       float v[8];
 #pragma unroll
       for (int j = 0; j < 8; j++) {
-        float x = u2f(r[q * 8 + j]);
+        float x = u2f(r[q * 8 + j]) * scale;
         if (EPI == EPI_RELU2) {
           x = fmaxf(x, 0.f);
           x = x * x;
@@ -68,17 +76,6 @@ __device__ __forceinline__ void epilogue32(const GemmArgs &g, int row, int col, 
       }
       dst[q] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
                           pack_bf16(v[6], v[7]));
-    }
-  } else if (EPI == EPI_RESID) {
-    float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(g.out) + o);
-#pragma unroll
-    for (int q = 0; q < 8; q++) {
-      float4 x = dst[q];
-      x.x += u2f(r[q * 4 + 0]);
-      x.y += u2f(r[q * 4 + 1]);
-      x.z += u2f(r[q * 4 + 2]);
-      x.w += u2f(r[q * 4 + 3]);
-      dst[q] = x;
     }
   } else {  // EPI_SOFTCAP
     float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(g.out) + o);
@@ -91,6 +88,110 @@ __device__ __forceinline__ void epilogue32(const GemmArgs &g, int row, int col, 
       x.z = cap * tanhf(u2f(r[q * 4 + 2]) * inv);
       x.w = cap * tanhf(u2f(r[q * 4 + 3]) * inv);
       dst[q] = x;
+    }
+  }
+}
+
+// TMEM columns [col, col+32) of the warp's 32 rows -> registers (lane = row)
+// -> the warp's swizzled 32 x 32 shared buffer -> out[i] = float4 column
+// (lane & 7) of row 4i + (lane >> 3).
+__device__ __forceinline__ void transpose_chunk(uint32_t taddr, float *ebuf, int lane, float4 (&out)[8]) {
+  uint32_t r[32];
+  tmem_ld32(taddr, r);
+  tmem_ld_wait();
+#pragma unroll
+  for (int j = 0; j < 8; j++)
+    *reinterpret_cast<float4 *>(ebuf + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+        make_float4(u2f(r[4 * j]), u2f(r[4 * j + 1]), u2f(r[4 * j + 2]), u2f(r[4 * j + 3]));
+  __syncwarp();
+  const int q = lane & 7, rsub = lane >> 3;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const int rr = 4 * i + rsub;
+    out[i] = *reinterpret_cast<const float4 *>(ebuf + rr * 32 + ((q ^ (rr & 7)) << 2));
+  }
+  __syncwarp();
+}
+
+// EPI_QKV for one 128-column head of the warp's 32 rows (rbase + lane); the
+// head's accumulator columns start at TMEM address tcol, `scale` is the RMS
+// factor of this lane's row. Heads 0..H-1 are q, head H is k, head H+1 is v.
+// RoPE pairs element e with element e+64 and rotates by the angle of
+// (e, position); q and k are then RMS normed over their 128 elements. A
+// rotation keeps each pair's sum of squares, so the norm factor is taken from
+// the unrotated accumulator row (lane = row); the rotation, scaling and
+// stores then run on transposed chunks, lane = (row group, 4 columns).
+__device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane, int head, uint32_t tcol, float scale,
+                                         float *ebuf) {
+  const GemmFuse &f = g.fz;
+  const bool isv = head > f.H;
+  float fac = scale;
+  if (!isv) {
+    float ss = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < 4; j++) {
+      uint32_t r[32];
+      tmem_ld32(tcol + 32 * j, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int k = 0; k < 32; k++) ss += u2f(r[k]) * u2f(r[k]);
+    }
+    fac = scale * rsqrtf(scale * scale * ss * (1.0f / 128) + f.eps);
+  }
+  const int q = lane & 7, rsub = lane >> 3;
+  float facr[8];
+  bf16 *dst[8];
+  int pos[8];
+  bool ok[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const int row = rbase + 4 * i + rsub;
+    facr[i] = __shfl_sync(0xffffffffu, fac, 4 * i + rsub);
+    ok[i] = row < g.M;
+    const int b = row / f.T;
+    pos[i] = ok[i] ? row % f.T : 0;
+    const size_t crow = ((size_t)b * f.max_seq + pos[i]) * 128;
+    dst[i] = (head < f.H ? reinterpret_cast<bf16 *>(f.q) + ((size_t)row * f.H + head) * 128
+                         : reinterpret_cast<bf16 *>(head == f.H ? f.kc : f.vc) + crow) +
+             4 * q;
+  }
+  if (isv) {
+#pragma unroll 1
+    for (int c = 0; c < 4; c++) {
+      float4 v[8];
+      transpose_chunk(tcol + 32 * c, ebuf, lane, v);
+#pragma unroll
+      for (int i = 0; i < 8; i++)
+        if (ok[i])
+          *reinterpret_cast<uint2 *>(dst[i] + 32 * c) =
+              make_uint2(pack_bf16(v[i].x * facr[i], v[i].y * facr[i]), pack_bf16(v[i].z * facr[i], v[i].w * facr[i]));
+    }
+    return;
+  }
+#pragma unroll 1
+  for (int c = 0; c < 2; c++) {  // elements 32c + 4q .. +3 and their partners 64 + 32c + 4q .. +3
+    float4 t0[8], t1[8];         // (cos, sin) of the 4 pairs, per row
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float4 *cs = reinterpret_cast<const float4 *>(f.rope + (size_t)pos[i] * 64) + 16 * c + 2 * q;
+      t0[i] = cs[0];
+      t1[i] = cs[1];
+    }
+    float4 lo[8], hi[8];
+    transpose_chunk(tcol + 32 * c, ebuf, lane, lo);
+    transpose_chunk(tcol + 64 + 32 * c, ebuf, lane, hi);
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      if (!ok[i]) continue;
+      const float4 a = lo[i], h = hi[i], u = t0[i], w = t1[i];
+      const float F = facr[i];
+      const float l0 = a.x * u.x - h.x * u.y, h0 = a.x * u.y + h.x * u.x;
+      const float l1 = a.y * u.z - h.y * u.w, h1 = a.y * u.w + h.y * u.z;
+      const float l2 = a.z * w.x - h.z * w.y, h2 = a.z * w.y + h.z * w.x;
+      const float l3 = a.w * w.z - h.w * w.w, h3 = a.w * w.w + h.w * w.z;
+      *reinterpret_cast<uint2 *>(dst[i] + 32 * c) = make_uint2(pack_bf16(l0 * F, l1 * F), pack_bf16(l2 * F, l3 * F));
+      *reinterpret_cast<uint2 *>(dst[i] + 64 + 32 * c) =
+          make_uint2(pack_bf16(h0 * F, h1 * F), pack_bf16(h2 * F, h3 * F));
     }
   }
 }
@@ -194,17 +295,111 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, local++) {
       const int acc = local & 1;
       const uint32_t accphase = (local >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], accphase, abort_flag, g.status)) break;
-      tc_fence_after();
       const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
       const int row = m0 + quarter * 32 + lane;
+      const bool rok = row < g.M;
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      if constexpr (EPI == EPI_RESID || EPI == EPI_RESID_X) {
+        // x += acc over the tile's 8 chunks of 32 columns. Each chunk goes
+        // TMEM -> registers (lane = row) -> a swizzled shared buffer, and is
+        // read back with lane = (row group, float4 column), so that every
+        // global access of a warp covers 4 rows x 128 contiguous bytes. The
+        // residual is read 4 chunks ahead, the first 4 before the
+        // accumulator is ready.
+        float *ebuf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + quarter * 1024;
+        const int q = lane & 7, rsub = lane >> 3;
+        const int rbase = m0 + quarter * 32;
+        float *xt = reinterpret_cast<float *>(g.out) + (size_t)rbase * g.ldo + n0 + 4 * q;
+        bf16 *xbt = reinterpret_cast<bf16 *>(g.fz.xb) + (size_t)rbase * g.ldo + n0 + 4 * q;
+        float4 xp[4][8];
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+#pragma unroll
+          for (int i = 0; i < 8; i++)
+            if (rbase + 4 * i + rsub < g.M && n0 + 32 * c < g.N)
+              xp[c][i] = *reinterpret_cast<const float4 *>(xt + (size_t)(4 * i + rsub) * g.ldo + 32 * c);
+        if (!mbar_wait(&tfull[acc], accphase, abort_flag, g.status)) break;
+        tc_fence_after();
+        float ssl[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) ssl[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+          uint32_t r[32];
+          tmem_ld32(tbase + 32 * c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; j++)
+            *reinterpret_cast<float4 *>(ebuf + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+                make_float4(u2f(r[4 * j]), u2f(r[4 * j + 1]), u2f(r[4 * j + 2]), u2f(r[4 * j + 3]));
+          __syncwarp();
+          if (n0 + 32 * c < g.N) {
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+              const int rr = 4 * i + rsub;
+              const float4 a = *reinterpret_cast<const float4 *>(ebuf + rr * 32 + ((q ^ (rr & 7)) << 2));
+              if (rbase + rr < g.M) {
+                float4 x = xp[c & 3][i];
+                x.x += a.x;
+                x.y += a.y;
+                x.z += a.z;
+                x.w += a.w;
+                *reinterpret_cast<float4 *>(xt + (size_t)rr * g.ldo + 32 * c) = x;
+                if (EPI == EPI_RESID_X) {
+                  *reinterpret_cast<uint2 *>(xbt + (size_t)rr * g.ldo + 32 * c) =
+                      make_uint2(pack_bf16(x.x, x.y), pack_bf16(x.z, x.w));
+                  ssl[i] += x.x * x.x + x.y * x.y + x.z * x.z + x.w * x.w;
+                }
+              }
+            }
+          }
+          __syncwarp();
+          if (c + 4 < 8 && n0 + 32 * (c + 4) < g.N)
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+              if (rbase + 4 * i + rsub < g.M)
+                xp[c & 3][i] = *reinterpret_cast<const float4 *>(xt + (size_t)(4 * i + rsub) * g.ldo + 32 * (c + 4));
+        }
+        if (EPI == EPI_RESID_X) {
+          // row sums: the 8 lanes of a row group hold its 8 float4 columns
+#pragma unroll
+          for (int i = 0; i < 8; i++) {
+            float v = ssl[i];
+            v += __shfl_xor_sync(0xffffffffu, v, 1);
+            v += __shfl_xor_sync(0xffffffffu, v, 2);
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            if (q == 0 && rbase + 4 * i + rsub < g.M) g.fz.ss_out[(size_t)(n0 / BN) * g.M + rbase + 4 * i + rsub] = v;
+          }
+        }
+      } else {
+        float scale = 1.f;
+        if (EPI == EPI_STORE || EPI == EPI_RELU2 || EPI == EPI_QKV) {
+          if (g.fz.nss > 0 && rok) {
+            float t = 0.f;
+            for (int j = 0; j < g.fz.nss; j++) t += g.fz.ss_in[(size_t)j * g.M + row];  // fixed order
+            scale = rsqrtf(t / g.K + g.fz.eps);
+          }
+        }
+        if (!mbar_wait(&tfull[acc], accphase, abort_flag, g.status)) break;
+        tc_fence_after();
+        if constexpr (EPI == EPI_QKV) {
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tbase + c, r);
-        tmem_ld_wait();
-        if (row < g.M && n0 + c < g.N) epilogue32<EPI>(g, row, n0 + c, r);
+          for (int hh = 0; hh < BN / 128; hh++) {
+            const int head = n0 / 128 + hh;
+            if (head >= g.fz.H + 2) break;  // the same for the whole warp
+            qkv_head(g, m0 + quarter * 32, lane, head, tbase + hh * 128, scale,
+                     reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + quarter * 1024);
+          }
+        } else {
+          float ss = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(tbase + c, r);
+            tmem_ld_wait();
+            if (rok && n0 + c < g.N) epilogue32<EPI>(g, row, n0 + c, r, scale, ss);
+          }
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -271,18 +466,22 @@ static cudaError_t launch_tc(const CUtensorMap &ma, const CUtensorMap &mw, const
 }
 
 cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
-                      float cap, uint32_t *status, int num_sms, cudaStream_t s) {
+                      float cap, uint32_t *status, int num_sms, cudaStream_t s, const GemmFuse *fz) {
   if (!gemm_tc_supported(M, N, K, lda)) return cudaErrorInvalidValue;
+  if ((epi == EPI_QKV || epi == EPI_RESID_X) && !fz) return cudaErrorInvalidValue;
+  if (epi == EPI_QKV && N != (fz->H + 2) * 128) return cudaErrorInvalidValue;
   CUtensorMap ma, mw;
   if (!make_map_bf16_k64(&ma, A, M, K, lda, BM) || !make_map_bf16_k64(&mw, W, N, K, K, BN))
     return cudaErrorInvalidValue;
-  GemmArgs g{M, N, K, out, ldo, cap, status};
+  GemmArgs g{M, N, K, out, ldo, cap, status, fz ? *fz : GemmFuse{}};
   int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   int grid = tiles < num_sms ? tiles : num_sms;
   switch (epi) {
     case EPI_STORE: return launch_tc<EPI_STORE>(ma, mw, g, grid, s);
     case EPI_RELU2: return launch_tc<EPI_RELU2>(ma, mw, g, grid, s);
     case EPI_RESID: return launch_tc<EPI_RESID>(ma, mw, g, grid, s);
+    case EPI_QKV: return launch_tc<EPI_QKV>(ma, mw, g, grid, s);
+    case EPI_RESID_X: return launch_tc<EPI_RESID_X>(ma, mw, g, grid, s);
     default: return launch_tc<EPI_SOFTCAP>(ma, mw, g, grid, s);
   }
 }

@@ -68,6 +68,7 @@ struct nc_kv {
   float *cand_v = nullptr;     // [V/128][32] per-tile argmax winners
   int *cand_i = nullptr;
   float *xl = nullptr;         // [32][d] last-position rows of a prefill, for the fused lm_head
+  float *row_ss = nullptr;     // [ceil(d/256)][max_rows] per-256-column sums of squares of x rows (prefill)
   // whole-step decode kernel (nc_step.cu)
   int step_grid = 0;           // CTAs of the step kernel, 0 = not available
   CUtensorMap *step_maps = nullptr;  // device copy of the step kernel's tensor maps
@@ -95,7 +96,30 @@ int set_error(int code, const char *msg);
 extern std::atomic<unsigned long long> g_launches;
 inline void count_launch(unsigned long long n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
-enum Epi { EPI_STORE = 0, EPI_RELU2 = 1, EPI_RESID = 2, EPI_SOFTCAP = 3 };
+enum Epi { EPI_STORE = 0, EPI_RELU2 = 1, EPI_RESID = 2, EPI_SOFTCAP = 3, EPI_QKV = 4, EPI_RESID_X = 5 };
+
+// Extra operands of the fused prefill epilogues of the tensor-core GEMM.
+//  ss_in/nss   the A rows are bf16(x) of an un-normed residual row: every
+//              accumulator row is scaled by 1/sqrt(sum_j ss_in[j*M + row]/K + eps)
+//              (nss = 0: A is already normed, no scaling); EPI_STORE, EPI_RELU2
+//              and EPI_QKV
+//  EPI_QKV     columns are the q heads, the k head and the v head (128 each):
+//              RoPE + RMS norm of q and k, q to q[row][H][128], k and v to the
+//              caches at (row / T, row % T) with row pitch 128, max_seq rows
+//              per sequence
+//  EPI_RESID_X x += acc as EPI_RESID, plus xb = bf16(x) (row pitch N) and
+//              ss_out[tile_n*M + row] = sum of squares of the new x over the
+//              tile's 256 columns
+struct GemmFuse {
+  const float *ss_in = nullptr;
+  int nss = 0;
+  float eps = 0.f;
+  void *xb = nullptr;
+  float *ss_out = nullptr;
+  const float2 *rope = nullptr;
+  void *q = nullptr, *kc = nullptr, *vc = nullptr;
+  int T = 1, H = 0, max_seq = 0;
+};
 
 // ---- generic kernels (any even head_dim; fp32 or bf16 storage) ----
 void k_prefill_begin(int32_t *len, uint8_t *valid, int B, int T, cudaStream_t s);
@@ -123,7 +147,7 @@ void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_
 // ---- sm_100a tensor-core GEMM (nc_gemm_tc.cu) ----
 bool gemm_tc_supported(int M, int N, int K, int lda);
 cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
-                      float cap, uint32_t *status, int num_sms, cudaStream_t s);
+                      float cap, uint32_t *status, int num_sms, cudaStream_t s, const GemmFuse *fz = nullptr);
 
 
 // ---- sm_100a causal MQA prefill attention (nc_attn_tc.cu) ----

@@ -47,34 +47,40 @@ __global__ void __launch_bounds__(256) rows_norm_kernel(const float *x, int rows
     dst[c * 32 + lane] = make_uint2(pack_bf(v[c].x * inv, v[c].y * inv), pack_bf(v[c].z * inv, v[c].w * inv));
 }
 
-// One warp per (row, head) of qkv [M][(H+2)*128]: lane l owns the pairs
-// (2l, 64+2l) and (2l+1, 65+2l).
-__global__ void __launch_bounds__(256) rope_qk_kernel(const bf16 *qkv, int M, int T, int H, const float2 *rope,
-                                                      bf16 *q_out, bf16 *kc, bf16 *vc, int max_seq, float eps) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  const int nh = H + 2;
-  if (gw >= M * nh) return;
-  const int m = gw / nh, head = gw % nh;
+// One warp per row of qkv [M][(H+2)*128]: every head's loads are issued
+// before any is used, the RoPE (cos, sin) of the row's position is read once;
+// lane l owns the pairs (2l, 64+2l) and (2l+1, 65+2l) of each head.
+template <int NH>
+__global__ void __launch_bounds__(256) rope_qk_kernel(const bf16 *qkv, int M, int T, const float2 *rope, bf16 *q_out,
+                                                      bf16 *kc, bf16 *vc, int max_seq, float eps) {
+  constexpr int H = NH - 2;
+  const int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (m >= M) return;
   const int b = m / T, pos = m % T;
-  const bf16 *src = qkv + ((size_t)m * nh + head) * 128;
-  const uint32_t lo = reinterpret_cast<const uint32_t *>(src)[lane];       // elements 2l, 2l+1
-  const uint32_t hi = reinterpret_cast<const uint32_t *>(src + 64)[lane];  // elements 64+2l, 65+2l
-  if (head == H + 1) {  // v: copied to the cache unchanged
-    uint32_t *dst = reinterpret_cast<uint32_t *>(vc + ((size_t)b * max_seq + pos) * 128);
-    dst[lane] = lo;
-    dst[32 + lane] = hi;
-    return;
+  const uint32_t *src = reinterpret_cast<const uint32_t *>(qkv + (size_t)m * NH * 128);
+  uint32_t lo[NH], hi[NH];
+#pragma unroll
+  for (int h = 0; h < NH; h++) {
+    lo[h] = src[h * 64 + lane];       // elements 2l, 2l+1 of head h
+    hi[h] = src[h * 64 + 32 + lane];  // elements 64+2l, 65+2l
   }
-  const float2 a = unpack_bf(lo), c = unpack_bf(hi);
-  const float2 cs0 = rope[(size_t)pos * 64 + 2 * lane], cs1 = rope[(size_t)pos * 64 + 2 * lane + 1];
-  const float r0 = a.x * cs0.x - c.x * cs0.y, r64 = a.x * cs0.y + c.x * cs0.x;
-  const float r1 = a.y * cs1.x - c.y * cs1.y, r65 = a.y * cs1.y + c.y * cs1.x;
-  float ss = warp_sum(r0 * r0 + r1 * r1 + r64 * r64 + r65 * r65);
-  const float inv = rsqrtf(ss * (1.0f / 128) + eps);
-  uint32_t *dst = head < H ? reinterpret_cast<uint32_t *>(q_out + ((size_t)m * H + head) * 128)
-                           : reinterpret_cast<uint32_t *>(kc + ((size_t)b * max_seq + pos) * 128);
-  dst[lane] = pack_bf(r0 * inv, r1 * inv);
-  dst[32 + lane] = pack_bf(r64 * inv, r65 * inv);
+  const float4 cs = reinterpret_cast<const float4 *>(rope + (size_t)pos * 64)[lane];  // pairs 2l and 2l+1
+  const size_t crow = ((size_t)b * max_seq + pos) * 128;
+#pragma unroll
+  for (int h = 0; h < NH - 1; h++) {  // q heads and the k head: RoPE + RMS norm
+    const float2 a = unpack_bf(lo[h]), c = unpack_bf(hi[h]);
+    const float r0 = a.x * cs.x - c.x * cs.y, r64 = a.x * cs.y + c.x * cs.x;
+    const float r1 = a.y * cs.z - c.y * cs.w, r65 = a.y * cs.w + c.y * cs.z;
+    const float ss = warp_sum(r0 * r0 + r1 * r1 + r64 * r64 + r65 * r65);
+    const float inv = rsqrtf(ss * (1.0f / 128) + eps);
+    uint32_t *dst = h < H ? reinterpret_cast<uint32_t *>(q_out + ((size_t)m * H + h) * 128)
+                          : reinterpret_cast<uint32_t *>(kc + crow);
+    dst[lane] = pack_bf(r0 * inv, r1 * inv);
+    dst[32 + lane] = pack_bf(r64 * inv, r65 * inv);
+  }
+  uint32_t *dv = reinterpret_cast<uint32_t *>(vc + crow);  // v: copied unchanged
+  dv[lane] = lo[NH - 1];
+  dv[32 + lane] = hi[NH - 1];
 }
 
 // Row r of xl = row r*stride + offset of x; ss[j][r] = sum of squares of its
@@ -98,7 +104,7 @@ __global__ void gather_rows_ss_kernel(const float *x, int d, int stride, int off
 
 bool rowops_supported(const nc_config &c) {
   return c.dtype == NC_BF16 && c.head_dim == 128 && c.n_kv_head == 1 && c.d_model % 128 == 0 &&
-         c.d_model / 128 <= 16;
+         c.d_model / 128 <= 16 && c.n_head <= 16;
 }
 
 cudaError_t k_rows_norm_bf16(const float *x, int rows, int d, float eps, void *h, cudaStream_t s) {
@@ -120,10 +126,20 @@ cudaError_t k_rows_norm_bf16(const float *x, int rows, int d, float eps, void *h
 cudaError_t k_rope_qk_bf16(const void *qkv, int M, int T, int H, const float2 *rope, void *q_out, void *kc, void *vc,
                            int max_seq, float eps, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  const long long warps = (long long)M * (H + 2);
+  const unsigned grid = (unsigned)((M + 7) / 8);
   count_launch();
-  rope_qk_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>((const bf16 *)qkv, M, T, H, rope, (bf16 *)q_out,
-                                                             (bf16 *)kc, (bf16 *)vc, max_seq, eps);
+  switch (H + 2) {
+#define NC_ROPE_CASE(NH)                                                                                        \
+  case NH:                                                                                                       \
+    rope_qk_kernel<NH><<<grid, 256, 0, s>>>((const bf16 *)qkv, M, T, rope, (bf16 *)q_out, (bf16 *)kc, (bf16 *)vc, \
+                                            max_seq, eps);                                                      \
+    break;
+    NC_ROPE_CASE(3) NC_ROPE_CASE(4) NC_ROPE_CASE(5) NC_ROPE_CASE(6) NC_ROPE_CASE(7) NC_ROPE_CASE(8)
+    NC_ROPE_CASE(9) NC_ROPE_CASE(10) NC_ROPE_CASE(11) NC_ROPE_CASE(12) NC_ROPE_CASE(13) NC_ROPE_CASE(14)
+    NC_ROPE_CASE(15) NC_ROPE_CASE(16) NC_ROPE_CASE(17) NC_ROPE_CASE(18)
+#undef NC_ROPE_CASE
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -36,6 +36,11 @@ def test_tiny_batch_with_ragged_prompt_length():
     (syn.D20, 3, 160, 3, [0, 2]),
     (syn.D26, 1, 72, 3, [0]),
     (syn.D30, 2, 40, 2, [1]),
+    # >= 128 prompt rows: the fused prefill epilogues, with a partial last
+    # 256-column tile of the residual (d 1664, 1920) and of the qkv projection
+    # (15 and 17 heads of 128) and a partial last 128-row tile
+    (syn.D26, 2, 100, 2, [1]),
+    (syn.D30, 1, 130, 1, [0]),
 ])
 def test_bf16_models_short_context(cfg, B, T, steps, seqs):
     prompts = syn.tokens_zipf(21, (B, T), cfg.vocab)
