@@ -92,48 +92,46 @@ inline void *layer_ptr(const nc_kv *kv, void *base, int l) {
   return (char *)base + (size_t)l * kv->layer_elems * kv->model->elem;
 }
 
+// Each step below takes its sm_100a kernel when the shapes allow it and the
+// generic kernel otherwise; a failed launch of either is returned (never
+// retried on the other kernel, so a broken fast path cannot hide).
+
 // Linear layer out (epi) A[M,K] * W[N,K]^T: tcgen05 kernel for bf16 models
 // once there is at least one full 128-row tile, the generic kernel otherwise.
-void linear(nc_model *m, int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
-            float cap, const uint8_t *valid, cudaStream_t s) {
-  if (m->fast && M >= 128 && !valid && nc::gemm_tc_supported(M, N, K, lda)) {
-    if (nc::k_gemm_tc(epi, A, lda, W, M, N, K, out, ldo, cap, m->status, m->num_sms, s) == cudaSuccess) return;
-    cudaGetLastError();
-  }
+cudaError_t linear(nc_model *m, int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out,
+                   int ldo, float cap, const uint8_t *valid, cudaStream_t s) {
+  if (m->fast && M >= 128 && !valid && nc::gemm_tc_supported(M, N, K, lda))
+    return nc::k_gemm_tc(epi, A, lda, W, M, N, K, out, ldo, cap, m->status, m->num_sms, s);
   nc::k_gemm_generic(m->cfg.dtype, epi, A, lda, W, M, N, K, out, ldo, cap, valid, s);
+  return cudaGetLastError();
 }
 
 // h = bf16/fp32 rmsnorm of the M rows of x.
-void norm_rows(nc_model *m, nc_kv *kv, int M, cudaStream_t s) {
+cudaError_t norm_rows(nc_model *m, nc_kv *kv, int M, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (nc::rowops_supported(c) && nc::k_rows_norm_bf16(kv->x, M, c.d_model, c.norm_eps, kv->h, s) == cudaSuccess)
-    return;
-  cudaGetLastError();
+  if (nc::rowops_supported(c)) return nc::k_rows_norm_bf16(kv->x, M, c.d_model, c.norm_eps, kv->h, s);
   nc::k_rmsnorm_rows(c.dtype, kv->x, M, c.d_model, 1, 0, c.norm_eps, kv->h, s);
+  return cudaGetLastError();
 }
 
 // RoPE + QK norm of the M rows of kv->qkv, q out, K/V appended to the cache.
-void rope_append(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
+cudaError_t rope_append(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (!rm.pos && nc::rowops_supported(c) &&
-      nc::k_rope_qk_bf16(kv->qkv, M, rm.T, c.n_head, kv->rope, kv->q, kc, vc, kv->max_seq, c.norm_eps, s) ==
-          cudaSuccess)
-    return;
-  cudaGetLastError();
+  if (!rm.pos && nc::rowops_supported(c))
+    return nc::k_rope_qk_bf16(kv->qkv, M, rm.T, c.n_head, kv->rope, kv->q, kc, vc, kv->max_seq, c.norm_eps, s);
   nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->rope, kv->q, kc, vc,
                            kv->max_seq, kv->valid, c.norm_eps, s);
+  return cudaGetLastError();
 }
 
 // Causal MQA attention of the M rows in kv->q against layer cache kc/vc.
-void attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
+cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (m->fast && !rm.pos && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim)) {
-    if (nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, kv->max_batch, kv->max_seq, kv->y, m->status,
-                              s) == cudaSuccess)
-      return;
-    cudaGetLastError();
-  }
+  if (m->fast && !rm.pos && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
+    return nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, kv->max_batch, kv->max_seq, kv->y,
+                                 m->status, s);
   nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->max_seq, kv->y, s);
+  return cudaGetLastError();
 }
 
 // The fused prefill layer sequence of bf16 head_dim-128 models, when every
@@ -177,7 +175,7 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
     fz.vc = layer_ptr(kv, kv->v, l);
     if (l == 0) {
       ProfScope p(m, NC_K_MISC, s);
-      norm_rows(m, kv, M, s);
+      e = norm_rows(m, kv, M, s);
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
@@ -187,7 +185,7 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
     }
     if (e == cudaSuccess) {
       ProfScope p(m, NC_K_ATTN, s);
-      attention(m, kv, fz.kc, fz.vc, M, rm, s);
+      e = attention(m, kv, fz.kc, fz.vc, M, rm, s);
     }
     {
       ProfScope p(m, NC_K_GEMM, s);
@@ -197,7 +195,7 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
       gemm(l + 1 < c.depth ? nc::EPI_RESID_X : nc::EPI_RESID, kv->f, F, w.wproj, d, F, kv->x);
     }
   }
-  if (e != cudaSuccess) return nc::set_error(NC_ECUDA, "prefill GEMM launch failed");
+  if (e != cudaSuccess) return nc::set_error(NC_ECUDA, cudaGetErrorString(e));
   return NC_OK;
 }
 
@@ -207,50 +205,39 @@ int run_blocks(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
   int d = c.d_model, H = c.n_head, Hkv = c.n_kv_head, hd = c.head_dim, F = c.mlp_hidden;
   int qkv_w = (H + 2 * Hkv) * hd;
-  for (int l = 0; l < c.depth; l++) {
+  cudaError_t e = cudaSuccess;
+  auto step = [&](int cls, auto &&launch) {
+    if (e != cudaSuccess) return;
+    ProfScope p(m, cls, s);
+    e = launch();
+  };
+  for (int l = 0; l < c.depth && e == cudaSuccess; l++) {
     const nc_layer_w &w = m->layers[l];
     void *kc = layer_ptr(kv, kv->k, l), *vc = layer_ptr(kv, kv->v, l);
-    {
-      ProfScope p(m, NC_K_MISC, s);
-      norm_rows(m, kv, M, s);
-    }
-    {
-      ProfScope p(m, NC_K_GEMM, s);
-      linear(m, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s);
-    }
-    {
-      ProfScope p(m, NC_K_MISC, s);
-      rope_append(m, kv, kc, vc, M, rm, s);
-    }
-    {
-      ProfScope p(m, NC_K_ATTN, s);
-      attention(m, kv, kc, vc, M, rm, s);
-    }
-    {
-      ProfScope p(m, NC_K_GEMM, s);
-      linear(m, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s);
-    }
-    {
-      ProfScope p(m, NC_K_MISC, s);
-      norm_rows(m, kv, M, s);
-    }
-    {
-      ProfScope p(m, NC_K_GEMM, s);
-      linear(m, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s);
-      linear(m, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s);
-    }
+    step(NC_K_MISC, [&] { return norm_rows(m, kv, M, s); });
+    step(NC_K_GEMM, [&] { return linear(m, nc::EPI_STORE, kv->h, d, w.wqkv, M, qkv_w, d, kv->qkv, qkv_w, 0.f, nullptr, s); });
+    step(NC_K_MISC, [&] { return rope_append(m, kv, kc, vc, M, rm, s); });
+    step(NC_K_ATTN, [&] { return attention(m, kv, kc, vc, M, rm, s); });
+    step(NC_K_GEMM, [&] { return linear(m, nc::EPI_RESID, kv->y, H * hd, w.wo, M, d, H * hd, kv->x, d, 0.f, nullptr, s); });
+    step(NC_K_MISC, [&] { return norm_rows(m, kv, M, s); });
+    step(NC_K_GEMM, [&] { return linear(m, nc::EPI_RELU2, kv->h, d, w.wfc, M, F, d, kv->f, F, 0.f, nullptr, s); });
+    step(NC_K_GEMM, [&] { return linear(m, nc::EPI_RESID, kv->f, F, w.wproj, M, d, F, kv->x, d, 0.f, nullptr, s); });
   }
+  if (e != cudaSuccess) return nc::set_error(NC_ECUDA, cudaGetErrorString(e));
   return NC_OK;
 }
 
 // Final norm of `rows` rows of x (row r taken from x row r*stride + offset),
 // lm_head with softcap into logits (row-major, ldo = V), argmax into next.
-void run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, float *logits, const uint8_t *valid,
-              cudaStream_t s) {
+cudaError_t run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, float *logits, const uint8_t *valid,
+                     cudaStream_t s) {
   const nc_config &c = m->cfg;
   ProfScope p(m, NC_K_HEAD, s);
   nc::k_rmsnorm_rows(c.dtype, kv->x, rows, c.d_model, stride, offset, c.norm_eps, kv->h, s);
-  linear(m, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab, c.softcap, valid, s);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return linear(m, nc::EPI_SOFTCAP, kv->h, c.d_model, m->wlm, rows, c.vocab, c.d_model, logits, c.vocab, c.softcap,
+                valid, s);
 }
 
 // The decode step on the sm_100a decode kernels (bf16, head_dim 128, B <= 32).
@@ -589,14 +576,15 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
   if (rc != NC_OK) return rc;
   float *logits;
   long long last_off, row_stride;
+  cudaError_t eh = cudaSuccess;
   if (logits_mode == 1) {
     if (d_logits) {
-      run_head(m, kv, M, 1, 0, d_logits, nullptr, s);
+      eh = run_head(m, kv, M, 1, 0, d_logits, nullptr, s);
       logits = d_logits;
       last_off = (long long)(T - 1) * c.vocab;
       row_stride = (long long)T * c.vocab;
     } else {
-      run_head(m, kv, B, T, T - 1, kv->logits, nullptr, s);
+      eh = run_head(m, kv, B, T, T - 1, kv->logits, nullptr, s);
       logits = kv->logits;
       last_off = 0;
       row_stride = c.vocab;
@@ -615,10 +603,11 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
       if (e != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(e));
       return NC_OK;
     }
-    run_head(m, kv, B, T, T - 1, logits, nullptr, s);
+    eh = run_head(m, kv, B, T, T - 1, logits, nullptr, s);
     last_off = 0;
     row_stride = c.vocab;
   }
+  if (eh != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(eh));
   if (d_next) {
     ProfScope p(m, NC_K_HEAD, s);
     nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
@@ -649,8 +638,10 @@ int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_
     nc::k_embed_norm(c.dtype, d_tokens, B, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
   }
   nc::RowMap rm{1, d_positions};
-  run_blocks(m, kv, B, rm, s);
-  run_head(m, kv, B, 1, 0, logits, kv->valid, s);
+  const int rc = run_blocks(m, kv, B, rm, s);
+  if (rc != NC_OK) return rc;
+  const cudaError_t eh = run_head(m, kv, B, 1, 0, logits, kv->valid, s);
+  if (eh != cudaSuccess) return fail(NC_ECUDA, "decode head launch failed: %s", cudaGetErrorString(eh));
   if (d_next) {
     ProfScope p(m, NC_K_HEAD, s);
     nc::k_argmax_rows(logits, B, c.vocab, c.vocab, d_noise, d_next, kv->valid, s);
@@ -731,10 +722,11 @@ int nc_attention_prefill_bf16(const void *d_q, const void *d_k, const void *d_v,
   int rc = kernel_status_init(&status, &sms);
   if (rc) return rc;
   cudaStream_t s = as_stream(stream);
-  if (nc::attn_prefill_tc_supported(H, 1, hd) &&
-      nc::k_attn_prefill_tc(d_q, d_k, d_v, B, T, H, B, max_seq, d_y, status, s) == cudaSuccess)
+  if (nc::attn_prefill_tc_supported(H, 1, hd)) {
+    const cudaError_t e = nc::k_attn_prefill_tc(d_q, d_k, d_v, B, T, H, B, max_seq, d_y, status, s);
+    if (e != cudaSuccess) return fail(NC_ECUDA, "attention launch failed: %s", cudaGetErrorString(e));
     return NC_OK;
-  cudaGetLastError();
+  }
   nc::RowMap rm{T, nullptr};
   nc::k_attention_generic(NC_BF16, d_q, d_k, d_v, rm, B * T, H, 1, hd, max_seq, d_y, s);
   NC_CUDA_TRY(cudaGetLastError());
@@ -784,10 +776,11 @@ int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K,
   int rc = kernel_status_init(&status, &sms);
   if (rc) return rc;
   cudaStream_t s = as_stream(stream);
-  if (M >= 128 && nc::gemm_tc_supported(M, N, K, lda) &&
-      nc::k_gemm_tc(epi, d_A, lda, d_W, M, N, K, d_out, ldo, cap, status, sms, s) == cudaSuccess)
+  if (M >= 128 && nc::gemm_tc_supported(M, N, K, lda)) {
+    const cudaError_t e = nc::k_gemm_tc(epi, d_A, lda, d_W, M, N, K, d_out, ldo, cap, status, sms, s);
+    if (e != cudaSuccess) return fail(NC_ECUDA, "GEMM launch failed: %s", cudaGetErrorString(e));
     return NC_OK;
-  cudaGetLastError();
+  }
   nc::k_gemm_generic(NC_BF16, epi, d_A, lda, d_W, M, N, K, d_out, ldo, cap, nullptr, s);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;

@@ -3,21 +3,27 @@
 // With one KV head, the H query heads of a position all read the same keys
 // and values (the feature list's multi-query attention). The queries of a
 // sequence, stored [T, H, hd], are therefore one [T*H, hd] matrix whose row
-// r = t*H + h belongs to position t. A CTA takes 128 consecutive rows
-// (about 128/H positions, every head) and streams the sequence's K/V tiles
-// once for all of them:
-//   S  = Q K^T          (tcgen05, M=128 rows, N=128 keys, K=hd=128) -> TMEM
-//   P  = exp(S*scale - m) with the causal mask key <= t(row), online max/sum
-//   O += P V            (tcgen05, A = P from shared memory, B = V read
-//                        MN-major straight from the cache layout)  -> TMEM
-// and finally y = O / l in bf16.
-// Warp roles (192 threads): warp 0 TMA producer (Q once, K/V tiles through a
-// 2-stage ring), warp 1 TMEM allocator + MMA issuer (S_{j+1} is issued before
-// P_j is consumed), warps 2-5 softmax / O rescale / epilogue, one thread per
-// row. P is double-buffered, so the softmax of tile j+1 overlaps P_j V_j, and
-// O is rescaled only when a row's running max grows by more than 2^8 (the
-// probabilities of a tile are then at most 256, exact in fp32 and bf16).
-// Waits are bounded as in the GEMM.
+// r = t*H + h belongs to position t. A work item is 256 consecutive rows of
+// one sequence, two 128-row Q tiles (A and B) that share every K/V tile:
+//   S_t  = Q_t K_j^T       (tcgen05, M=128 rows, N=128 keys, K=hd) -> TMEM
+//   P_t  = 2^(S_t*scale*log2e - m) with the causal mask key <= t(row), online
+//          max/sum, bf16 pairs written back into the upper half of S_t's
+//          TMEM columns
+//   O_t += P_t V_j         (tcgen05 with A read from TMEM, B = V read
+//                           MN-major straight from the cache layout) -> TMEM
+// and finally y = O_t / l in bf16.
+// Warp roles (320 threads): warp 0 TMA (one thread: the Q tiles of each item,
+// then K_j and V_j alternately through a 4-slot ring), warp 1 TMEM
+// allocator + MMA issuer, warps 2-5 softmax of tile A and warps 6-9 of tile B,
+// one thread per row. Per key tile the MMA issuer runs PV_A(j), S_A(j+1),
+// PV_B(j), S_B(j+1): while one warpgroup exponentiates, the tensor core works
+// for the other. S_t(j+1) overwrites the TMEM columns PV_t(j) reads P from;
+// tcgen05.mma operations of one CTA run in issue order, so it is issued right
+// after PV_t(j) with no wait in between. O is rescaled only when a row's
+// running max grows by more than 2^8 (the probabilities of a tile are then at
+// most 256, exact in fp32 and bf16). Items are ordered heaviest first and dealt
+// to the CTAs in zig-zag rounds, which evens out the causal work per CTA.
+// Every wait is bounded as in the GEMM.
 #include "nc_internal.h"
 #include "nc_sm100.cuh"
 
@@ -28,25 +34,24 @@ bool make_map_bf16_k64(CUtensorMap *map, const void *ptr, int rows, int cols, in
 
 namespace {
 
-constexpr int HD = 128;           // head dim handled here
-constexpr int BR = 128;           // rows (position, head) per CTA
-constexpr int BKV = 128;          // keys per tile
-constexpr int ST = 2;             // K/V stages
-constexpr int SUB = 128 * 64 * 2; // one 128-row x 64-column swizzled box: 16 KB
-constexpr int TILE = 2 * SUB;     // 128 x 128 bf16: 32 KB
-constexpr int OFF_Q = 0;
-constexpr int OFF_P = TILE;                  // 2 tiles (double-buffered P)
-constexpr int OFF_K = 3 * TILE;              // ST tiles
-constexpr int OFF_V = 3 * TILE + ST * TILE;  // ST tiles
-constexpr int OFF_BAR = 3 * TILE + 2 * ST * TILE;
-constexpr int OFF_XCH = OFF_BAR + 160;       // [2][2][128] fp32: row-max halves (x2); then the row-sum halves
+constexpr int HD = 128;            // head dim handled here
+constexpr int BR = 128;            // rows (position, head) per Q tile
+constexpr int ITEM = 2 * BR;       // rows per work item: Q tiles A and B
+constexpr int BKV = 128;           // keys per K/V tile
+constexpr int NSLOT = 4;           // K/V ring slots (K_j and V_j alternate)
+constexpr int SUB = 128 * 64 * 2;  // one 128-row x 64-column swizzled box: 16 KB
+constexpr int TILE = 2 * SUB;      // 128 x 128 bf16: 32 KB
+constexpr int OFF_Q = 0;           // Q_A, Q_B
+constexpr int OFF_KV = 2 * TILE;   // NSLOT tiles
+constexpr int OFF_BAR = OFF_KV + NSLOT * TILE;
+constexpr int SMEM_USED = OFF_BAR + 256;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 constexpr float RESCALE_LOG2 = 8.0f;         // rescale O when the max grows by more than 2^8
-constexpr int SMEM_USED = OFF_XCH + 2 * 2 * 128 * 4;
-static_assert(SMEM_USED + 256 <= 227 * 1024, "shared memory budget");
-constexpr int SMEM_BYTES = 227 * 1024;       // the rest is slack for 1024-byte alignment
-constexpr int MAX_PAD = SMEM_BYTES - SMEM_USED;
-constexpr int THREADS = 320;                 // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (2 per row)
-constexpr uint32_t TMEM_COLS = 512;  // O accumulators: cols 0..255, S buffers: 256..511
+constexpr int THREADS = 320;
+// TMEM columns: S of tile t at 128t (P of tile t at 128t + 64, bf16 pairs),
+// O of tile t at 256 + 128t
+constexpr uint32_t TMEM_COLS = 512;
 
 struct AttnArgs {
   int T, H, B, max_seq;
@@ -68,6 +73,16 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// D (TMEM) (+)= A (TMEM, bf16 pairs per 32-bit column, K-major) * B (shared)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -95,61 +110,54 @@ __device__ __forceinline__ uint32_t pack2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// round r of the zig-zag deal of items to G CTAs: CTA c takes item
+// r*G + c in even rounds and r*G + G-1-c in odd ones
+__device__ __forceinline__ int item_at(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+
 __global__ void __launch_bounds__(THREADS, 1)
     attn_prefill_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                            const __grid_constant__ CUtensorMap mapV, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint32_t raw = smem_u32(smem_raw);
-  const uint32_t pad = ((raw + 1023) & ~1023u) - raw;
-  if (pad > (uint32_t)MAX_PAD) {  // shared memory window not aligned as expected: report, do nothing
-    if (threadIdx.x == 0) atomicOr(a.status, (unsigned)NC_DEV_TIMEOUT);
-    return;
-  }
-  uint8_t *smem = smem_raw + pad;
-  float *xch = reinterpret_cast<float *>(smem + OFF_XCH);
+  uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
   uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *q_full = bar;             // 1
-  uint64_t *q_empty = bar + 1;        // 1: Q free once the item's last S is done
-  uint64_t *k_full = bar + 2;         // ST
-  uint64_t *v_full = k_full + ST;     // ST
-  uint64_t *k_empty = v_full + ST;    // ST: K stage free once S = Q K^T is done
-  uint64_t *v_empty = k_empty + ST;   // ST: V stage free once P V is done
-  uint64_t *s_full = v_empty + ST;    // 2
-  uint64_t *p_full = s_full + 2;      // 2 (256 arrivals), one per P buffer
-  uint64_t *o_done = p_full + 2;      // 2, one per P buffer
-  uint64_t *o_empty = o_done + 2;     // 2 (256 arrivals), one per O accumulator
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_empty + 2);
+  uint64_t *q_full = bar;               // 1
+  uint64_t *q_empty = bar + 1;          // 1: Q tiles free once the item's last S is done
+  uint64_t *kv_full = bar + 2;          // NSLOT
+  uint64_t *kv_empty = kv_full + NSLOT; // NSLOT
+  uint64_t *s_full = kv_empty + NSLOT;  // 2, per Q tile
+  uint64_t *p_full = s_full + 2;        // 2 (128 arrivals)
+  uint64_t *o_done = p_full + 2;        // 2: every P V of the tile so far is done
+  uint64_t *o_free = o_done + 2;        // 2 (128 arrivals): the item's O has been read
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_free + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_rt = (a.rows_per_seq + BR - 1) / BR;
-  const int n_items = n_rt * a.B;
+  const int n_pairs = (a.rows_per_seq + ITEM - 1) / ITEM;
+  const int n_items = n_pairs * a.B;
+  const int G = gridDim.x, c = blockIdx.x;
 
-  // work item i: row tile n_rt-1 - i/B of sequence i%B (heaviest first), the
-  // CTA takes items blockIdx.x, +gridDim.x, ...
+  // item i: rows 256*pp .. of sequence b, pp heaviest first; n_kv key tiles
   auto item_of = [&](int i, int &b, int &row0, int &n_kv) {
-    const int rt = n_rt - 1 - i / a.B;
+    const int pp = n_pairs - 1 - i / a.B;
     b = i % a.B;
-    row0 = rt * BR;
-    int t_max = (row0 + BR - 1) / a.H;
-    if (t_max > a.T - 1) t_max = a.T - 1;
-    n_kv = t_max / BKV + 1;
+    row0 = pp * ITEM;
+    const int last = min(row0 + ITEM, a.rows_per_seq) - 1;
+    n_kv = (last / a.H) / BKV + 1;
   };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int s = 0; s < ST; s++) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_empty[s], 1);
+    for (int s = 0; s < NSLOT; s++) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; i++) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 256);
-      mbar_init(&o_done[i], 1);
-      mbar_init(&o_empty[i], 256);
+    for (int t = 0; t < 2; t++) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_done[t], 1);
+      mbar_init(&o_free[t], 128);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -162,216 +170,203 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tO0 = tmem, tS = tmem + 256;  // O accumulators at columns 0 and 128, S buffers at 256 and 384
 
   if (warp == 0) {
-    // lane 0 streams Q and K, lane 1 streams V, item after item
+    // one thread issues every load in consumption order: the item's Q tiles
+    // (once its predecessor's last S is done), then K_j, V_j, K_{j+1}, ...
+    // through the ring (a second lane with its own waits would share this
+    // warp's issue slot and stall behind the first)
     if (lane == 0) {
-      int j = 0, it = 0;
+      uint32_t n = 0;
       bool ok = true;
-      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, it++) {
+      for (int r = 0, it = 0; ok; r++, it++) {
+        const int i = item_at(r, c, G);
+        if (i >= n_items) break;
         int b, row0, n_kv;
         item_of(i, b, row0, n_kv);
-        const int krow = b * a.max_seq;
         if (!mbar_wait(q_empty, (it & 1) ^ 1, abort_flag, a.status)) break;
-        mbar_arrive_expect_tx(q_full, TILE);
-        tma_load_2d(smem + OFF_Q, &mapQ, 0, b * a.rows_per_seq + row0, q_full);
-        tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, b * a.rows_per_seq + row0, q_full);
-        for (int jj = 0; jj < n_kv; jj++, j++) {
-          const int s = j % ST;
-          if (!mbar_wait(&k_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&k_full[s], TILE);
-          tma_load_2d(smem + OFF_K + s * TILE, &mapK, 0, krow + jj * BKV, &k_full[s]);
-          tma_load_2d(smem + OFF_K + s * TILE + SUB, &mapK, 64, krow + jj * BKV, &k_full[s]);
-        }
-      }
-    } else if (lane == 1) {
-      int j = 0;
-      bool ok = true;
-      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x) {
-        int b, row0, n_kv;
-        item_of(i, b, row0, n_kv);
+        mbar_arrive_expect_tx(q_full, 2 * TILE);
+        const int qrow = b * a.rows_per_seq + row0;
+        tma_load_2d(smem + OFF_Q, &mapQ, 0, qrow, q_full);
+        tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, qrow, q_full);
+        tma_load_2d(smem + OFF_Q + TILE, &mapQ, 0, qrow + BR, q_full);
+        tma_load_2d(smem + OFF_Q + TILE + SUB, &mapQ, 64, qrow + BR, q_full);
         const int krow = b * a.max_seq;
-        for (int jj = 0; jj < n_kv; jj++, j++) {
-          const int s = j % ST;
-          if (!mbar_wait(&v_empty[s], ((j / ST) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&v_full[s], TILE);
-          tma_load_2d(smem + OFF_V + s * TILE, &mapV, 0, krow + jj * BKV, &v_full[s]);
-          tma_load_2d(smem + OFF_V + s * TILE + SUB, &mapV, 64, krow + jj * BKV, &v_full[s]);
-        }
+        for (int j = 0; j < n_kv && ok; j++)
+          for (int w = 0; w < 2; w++, n++) {
+            const int s = n % NSLOT;
+            if (!mbar_wait(&kv_empty[s], ((n / NSLOT) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+            mbar_arrive_expect_tx(&kv_full[s], TILE);
+            const CUtensorMap *map = w ? &mapV : &mapK;
+            tma_load_2d(smem + OFF_KV + s * TILE, map, 0, krow + j * BKV, &kv_full[s]);
+            tma_load_2d(smem + OFF_KV + s * TILE + SUB, map, 64, krow + j * BKV, &kv_full[s]);
+          }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(BR, BKV);
       const uint32_t id_o = idesc_bf16_f32(BR, HD) | (1u << 16);  // B (V) is MN-major
-      const uint32_t q0 = smem_u32(smem + OFF_Q), p0 = smem_u32(smem + OFF_P);
-      // tile counters run across items; J indexes K/V stages, S and P buffers
-      int J = 0, it = 0;
+      const uint32_t q0 = smem_u32(smem + OFF_Q);
+      uint32_t n = 0;  // K/V ring position
+      int g = 0;       // key tiles done so far, over all items
       bool ok = true;
-      auto issue_s = [&](int jg) -> bool {  // S_jg = Q K_jg^T into S buffer jg % 2
-        const int s = jg % ST;
-        if (!mbar_wait(&k_full[s], (jg / ST) & 1, abort_flag, a.status)) return false;
+      auto take = [&](uint32_t &addr, int &slot) -> bool {
+        slot = n % NSLOT;
+        if (!mbar_wait(&kv_full[slot], (n / NSLOT) & 1, abort_flag, a.status)) return false;
+        n++;
+        addr = smem_u32(smem + OFF_KV + slot * TILE);
         tc_fence_after();
-        const uint32_t k0 = smem_u32(smem + OFF_K + s * TILE);
-        const uint32_t d = tS + (jg & 1) * 128;
+        return true;
+      };
+      auto issue_s = [&](int t, uint32_t k0) {  // S_t = Q_t K^T
+        const uint32_t qa = q0 + t * TILE;
 #pragma unroll
         for (int k = 0; k < HD / 16; k++) {
           const uint32_t off = (k >> 2) * SUB + (k & 3) * 32;
-          mma_bf16(d, desc_k_sw128(q0 + off), desc_k_sw128(k0 + off), id_s, k != 0);
+          mma_bf16(tmem + t * 128, desc_k_sw128(qa + off), desc_k_sw128(k0 + off), id_s, k != 0);
         }
-        mma_commit(&s_full[jg & 1]);
-        mma_commit(&k_empty[s]);
-        return true;
+        mma_commit(&s_full[t]);
       };
-      for (int i = blockIdx.x; i < n_items && ok; i += gridDim.x, it++) {
+      for (int r = 0, it = 0; ok; r++, it++) {
+        const int i = item_at(r, c, G);
+        if (i >= n_items) break;
         int b, row0, n_kv;
         item_of(i, b, row0, n_kv);
-        const int ob = it & 1;
-        const uint32_t tO = tO0 + ob * 128;
         if (!mbar_wait(q_full, it & 1, abort_flag, a.status)) break;
-        // the epilogue of item it-2 must have read this O accumulator
-        if (!mbar_wait(&o_empty[ob], ((it >> 1) & 1) ^ 1, abort_flag, a.status)) break;
-        tc_fence_after();
-        if (!issue_s(J)) break;
-        for (int jj = 0; jj < n_kv && ok; jj++) {
-          const int jg = J + jj;
-          if (jj + 1 < n_kv) {
-            if (!issue_s(jg + 1)) { ok = false; break; }
-          } else {
-            mma_commit(q_empty);  // the last S of the item: Q may be reloaded
-          }
-          if (!mbar_wait(&p_full[jg & 1], (jg >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-          const int s = jg % ST;
-          if (!mbar_wait(&v_full[s], (jg / ST) & 1, abort_flag, a.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t v0 = smem_u32(smem + OFF_V + s * TILE), pb = p0 + (jg & 1) * TILE;
+        uint32_t kaddr, vaddr;
+        int kslot, vslot;
+        if (!take(kaddr, kslot)) break;
+        issue_s(0, kaddr);
+        issue_s(1, kaddr);
+        mma_commit(&kv_empty[kslot]);
+        if (n_kv == 1) mma_commit(q_empty);
+        for (int j = 0; j < n_kv && ok; j++, g++) {
+          if (!take(vaddr, vslot)) { ok = false; break; }
+          for (int t = 0; t < 2 && ok; t++) {
+            if (!mbar_wait(&p_full[t], g & 1, abort_flag, a.status)) { ok = false; break; }
+            // the epilogue of the previous item must have read O_t
+            if (j == 0 && !mbar_wait(&o_free[t], (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t pa = tmem + t * 128 + 64;
 #pragma unroll
-          for (int k = 0; k < BKV / 16; k++) {
-            const uint32_t poff = (k >> 2) * SUB + (k & 3) * 32;
-            mma_bf16(tO, desc_k_sw128(pb + poff), desc_mn_sw128(v0 + k * 2048), id_o, (jj | k) != 0);
+            for (int k = 0; k < BKV / 16; k++)
+              mma_bf16_ts(tmem + 256 + t * 128, pa + k * 8, desc_mn_sw128(vaddr + k * 2048), id_o, (j | k) != 0);
+            mma_commit(&o_done[t]);
+            if (t == 1) mma_commit(&kv_empty[vslot]);
+            if (j + 1 < n_kv) {
+              if (t == 0 && !take(kaddr, kslot)) { ok = false; break; }
+              issue_s(t, kaddr);
+              if (t == 1) {
+                mma_commit(&kv_empty[kslot]);
+                if (j + 2 == n_kv) mma_commit(q_empty);  // the item's last S
+              }
+            }
           }
-          mma_commit(&o_done[jg & 1]);
-          mma_commit(&v_empty[s]);
         }
-        J += n_kv;
       }
     }
   } else {
-    // softmax / correction / epilogue: two threads per row, each owning 64 of
-    // the tile's 128 keys (and 64 of the 128 output dims)
-    const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
+    // softmax of Q tile t, one thread per row; then the item's epilogue
+    const int t = (warp - 2) >> 2;
+    const int quarter = warp & 3;  // this warp's TMEM lane quarter
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + t * 128 + lane_off, tO = tmem + 256 + t * 128 + lane_off;
     bool ok = true;
-    int J = 0, it = 0;
-    // every thread runs every iteration (a failed wait only clears `ok`), so
-    // the named-barrier syncs always pair up
-    for (int i = blockIdx.x; i < n_items; i += gridDim.x, it++) {
+    int g = 0;
+    for (int rr = 0;; rr++) {
+      const int i = item_at(rr, c, G);
+      if (i >= n_items) break;
       int b, row0, n_kv;
       item_of(i, b, row0, n_kv);
-      const int ob = it & 1;
-      const uint32_t tO = tO0 + ob * 128;
-      const int row = row0 + r;  // row inside the sequence
+      const int row = row0 + t * BR + r;  // row inside the sequence
       const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
-      float m = -INFINITY, l = 0.f;  // reference max (scaled, log2 units) and this half's running sum
-      for (int jj = 0; jj < n_kv; jj++) {
-        const int jg = J + jj;
-        ok = ok && mbar_wait(&s_full[jg & 1], (jg >> 1) & 1, abort_flag, a.status);
+      float m = -INFINITY, l = 0.f;  // running max (scaled, log2 units) and sum
+      for (int j = 0; j < n_kv; j++, g++) {
+        ok = ok && mbar_wait(&s_full[t], g & 1, abort_flag, a.status);
         tc_fence_after();
-        const uint32_t sbase = tS + (jg & 1) * 128 + lane_off + half * 64;
-        const int kbase = jj * BKV + half * 64;
-        uint32_t v[64];
-        tmem_ld32(sbase + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
-        tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        tmem_ld_wait();
-        // raw max of this half (the scale is positive); the causal mask only
-        // matters on tiles that reach past the row's position
-        const bool masked = kbase + 63 > t_row;
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-        if (masked) {
+        // pass 1: raw row max (the scale is positive), 64 columns at a time;
+        // the causal mask only matters on a tile that reaches past the
+        // row's position
+        const int kbase = j * BKV;
+        const bool masked = kbase + BKV - 1 > t_row;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int h = 0; h < 2; h++) {
+          uint32_t v[64];
+          tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 64; q++) {
-            if (kbase + q > t_row) v[q] = __float_as_uint(-INFINITY);
-            if (q & 1) mx1 = fmaxf(mx1, __uint_as_float(v[q]));
-            else mx0 = fmaxf(mx0, __uint_as_float(v[q]));
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 64; q += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(v[q]));
-            mx1 = fmaxf(mx1, __uint_as_float(v[q + 1]));
+            const float x = (masked && kbase + h * 64 + q > t_row) ? -INFINITY : __uint_as_float(v[q]);
+            mx[q & 3] = fmaxf(mx[q & 3], x);
           }
         }
-        // the two halves of the row agree on the row max (buffer jg&1: the
-        // partner has read the previous use of it before arriving here again)
-        float *xm = xch + (jg & 1) * 256;
-        xm[half * 128 + r] = fmaxf(mx0, mx1);
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        const float tmax = fmaxf(xm[r], xm[128 + r]) * a.scale_log2;
+        const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
         const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
         const float m_new = need ? tmax : m;
         const float alpha = (need && m != -INFINITY) ? exp2f(m - m_new) : 1.f;
-        // P buffer jg&1 is free once P_{jg-2} V_{jg-2} is done (any item)
-        if (jg >= 2) ok = ok && mbar_wait(&o_done[jg & 1], ((jg - 2) >> 1) & 1, abort_flag, a.status);
-        if (jj > 0 && __any_sync(0xffffffffu, need)) {
-          // O must hold every earlier P V of this item before it is rescaled;
-          // this half rescales output dims half*64 .. +63
-          ok = ok && mbar_wait(&o_done[(jg - 1) & 1], ((jg - 1) >> 1) & 1, abort_flag, a.status);
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O must hold every earlier P V of this item before it is rescaled
+          ok = ok && mbar_wait(&o_done[t], (g - 1) & 1, abort_flag, a.status);
           tc_fence_after();
 #pragma unroll 1
-          for (int c = half * 64; c < half * 64 + 64; c += 32) {
+          for (int cc = 0; cc < HD; cc += 32) {
             uint32_t o[32];
-            tmem_ld32(tO + lane_off + c, o);
+            tmem_ld32(tO + cc, o);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; q++) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-            tmem_st32(tO + lane_off + c, o);
+            tmem_st32(tO + cc, o);
           }
-          tmem_st_wait();
         }
-        // p = 2^(s*scale - m): one FMA and one ex2 per score (masked scores
-        // are -inf and give 0), bf16 into box `half` of the swizzled P tile
-        uint8_t *prow = smem + OFF_P + (jg & 1) * TILE + half * SUB + r * 128;
+        // pass 2: p = 2^(s*scale - m), one FMA and one ex2 per score (masked
+        // scores give 0), bf16 pairs into the P columns 64..127 of this S
+        // buffer. Keys 64..127 go first: their P lands on S columns 96..127,
+        // already read; keys 0..63 then land on columns 64..95.
         const float nm = -m_new;
-        float sum0 = 0.f, sum1 = 0.f;
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+        for (int hh = 0; hh < 2; hh++) {
+          const int h = 1 - hh;
+          uint32_t v[64];
+          tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_ld_wait();
+          uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          float pv[8];
-#pragma unroll
-          for (int q = 0; q < 8; q++) pv[q] = ex2(fmaf(__uint_as_float(v[c + q]), a.scale_log2, nm));
-          sum0 += (pv[0] + pv[2]) + (pv[4] + pv[6]);
-          sum1 += (pv[1] + pv[3]) + (pv[5] + pv[7]);
-          const int chunk = c >> 3;
-          *reinterpret_cast<uint4 *>(prow + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pack2(pv[0], pv[1]), pack2(pv[2], pv[3]), pack2(pv[4], pv[5]), pack2(pv[6], pv[7]));
+          for (int q = 0; q < 32; q++) {
+            const int k0 = kbase + h * 64 + 2 * q;
+            const float s0 = (masked && k0 > t_row) ? -INFINITY : __uint_as_float(v[2 * q]);
+            const float s1 = (masked && k0 + 1 > t_row) ? -INFINITY : __uint_as_float(v[2 * q + 1]);
+            const float p0 = ex2(fmaf(s0, a.scale_log2, nm));
+            const float p1 = ex2(fmaf(s1, a.scale_log2, nm));
+            sum[(2 * q) & 3] += p0;
+            sum[(2 * q + 1) & 3] += p1;
+            pk[q] = pack2(p0, p1);
+          }
+          tmem_st32(tS + 64 + h * 32, pk);
         }
-        l = l * alpha + (sum0 + sum1);
+        l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
         m = m_new;
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[jg & 1]);
+        mbar_arrive(&p_full[t]);
       }
-      // row sum = both halves (the exchange slot is free: every max above has
-      // been read before this barrier)
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      float *xl = xch;  // both row-max slots have been read by now
-      xl[half * 128 + r] = l;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float lsum = xl[r] + xl[128 + r];
-      const int jl = J + n_kv - 1;
-      ok = ok && mbar_wait(&o_done[jl & 1], (jl >> 1) & 1, abort_flag, a.status);
+      // epilogue: y = O / l
+      ok = ok && mbar_wait(&o_done[t], (g - 1) & 1, abort_flag, a.status);
       tc_fence_after();
-      const float inv = 1.f / lsum;
+      const float inv = 1.f / l;
       bf16 *dst = a.y + ((size_t)b * a.rows_per_seq + row) * HD;
 #pragma unroll 1
-      for (int c = half * 64; c < half * 64 + 64; c += 32) {
+      for (int cc = 0; cc < HD; cc += 32) {
         uint32_t o[32];
-        tmem_ld32(tO + lane_off + c, o);
+        tmem_ld32(tO + cc, o);
         tmem_ld_wait();
         if (ok && row < a.rows_per_seq) {
-          uint4 *d4 = reinterpret_cast<uint4 *>(dst + c);
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + cc);
 #pragma unroll
           for (int q = 0; q < 4; q++) {
             float f[8];
@@ -382,10 +377,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&o_empty[ob]);
-      // keep the l exchange slot from being overwritten before the partner read it
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      J += n_kv;
+      mbar_arrive(&o_free[t]);
     }
   }
   __syncthreads();
@@ -430,7 +422,7 @@ cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  const int items = ((rows + BR - 1) / BR) * B;
+  const int items = ((rows + ITEM - 1) / ITEM) * B;
   dim3 grid(items < sms ? items : sms);
   count_launch();
   attn_prefill_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, a);

@@ -118,6 +118,28 @@ def test_attention_prefill_matches_float64(B, T, H, hd, extra):
     assert np.all(err <= 1e-2 + 2.0 ** -8 * np.abs(want)), f"max err {err.max():.3g}"
 
 
+@pytest.mark.parametrize("B,T,H", [(2, 600, 10), (1, 2048, 4)])
+def test_attention_prefill_growing_scores_rescale_the_output(B, T, H):
+    """Keys whose norm grows along the sequence push every row's running max
+    up tile after tile, so the online softmax rescales its output again and
+    again (the random-key cases above rarely need it)."""
+    import torch
+    import kv_cache_transformer_b200 as nc
+    g = torch.Generator().manual_seed(7 * T + H)
+    q = torch.randn(B, T, H, 128, generator=g).to(torch.bfloat16)
+    ramp = (1.0 + torch.arange(T, dtype=torch.float32) / 48.0).view(1, T, 1)
+    k = (torch.randn(B, T, 128, generator=g) * ramp).to(torch.bfloat16)
+    v = torch.randn(B, T, 128, generator=g).to(torch.bfloat16)
+    y = torch.full((B, T, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nc.nc_attention_prefill_bf16(q.cuda(), k.cuda(), v.cuda(), y)
+    torch.cuda.synchronize()
+    want = _attn_ref(q, k, v, T).numpy()
+    got = y.cpu().double().numpy()
+    err = np.abs(got - want)
+    assert np.all(np.isfinite(got))
+    assert np.all(err <= 1e-2 + 2.0 ** -8 * np.abs(want)), f"max err {err.max():.3g}"
+
+
 def _decode_ref(q, k, v, pos):
     import torch
     out = torch.zeros(q.shape, dtype=torch.float64)
