@@ -61,27 +61,34 @@ struct AttnArgs {
   uint32_t *status;
 };
 
-// Shared-memory descriptor for an MN-major operand (V: keys x dims, dims
-// contiguous) written by TMA with 128-byte swizzle as two boxes of 64 dims:
-// 8-key groups 1024 B apart (stride byte offset), the second 64-dim box 16 KB
-// further (leading byte offset).
-__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
-  d |= (uint64_t)(SUB >> 4) << 16;   // leading byte offset: next 64-element MN chunk
-  d |= (uint64_t)(1024 >> 4) << 32;  // stride byte offset: next 8-row K group
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
+// Shared-memory descriptors split into 32-bit words: the low word holds the
+// start address (>> 4) and the leading byte offset, the high word the stride
+// byte offset, version and swizzle mode, the same for every tile here, so an
+// MMA's operands cost one add each (the MMA warp shares its issue slots with
+// two softmax warps).
+constexpr uint32_t DESC_HI = (1024u >> 4) | (1u << 14) | (2u << 29);  // bits 32..63
+__device__ __forceinline__ uint32_t desc_lo_k(uint32_t smem_addr) { return ((smem_addr >> 4) & 0x3FFF) | (1u << 16); }
+__device__ __forceinline__ uint32_t desc_lo_mn(uint32_t smem_addr) {
+  return ((smem_addr >> 4) & 0x3FFF) | ((uint32_t)(SUB >> 4) << 16);
+}
+
+// D (TMEM) (+)= A (shared) * B (shared), descriptors given as low words
+__device__ __forceinline__ void mma_ss(uint32_t tmem_d, uint32_t alo, uint32_t blo, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n .reg .b64 da, db;\n setp.ne.b32 p, %4, 0;\n mov.b64 da, {%1, %5};\n"
+      " mov.b64 db, {%2, %5};\n tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n}" ::"r"(tmem_d),
+      "r"(alo), "r"(blo), "r"(idesc), "r"(accumulate), "n"(DESC_HI)
+      : "memory");
 }
 
 // D (TMEM) (+)= A (TMEM, bf16 pairs per 32-bit column, K-major) * B (shared)
-__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t accumulate) {
+__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint32_t blo, uint32_t idesc,
+                                       uint32_t accumulate) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      "{\n .reg .pred p;\n .reg .b64 db;\n setp.ne.b32 p, %4, 0;\n mov.b64 db, {%2, %5};\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n}" ::"r"(tmem_d),
+      "r"(tmem_a), "r"(blo), "r"(idesc), "r"(accumulate), "n"(DESC_HI)
       : "memory");
 }
 
@@ -103,6 +110,13 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack2(float a, float b) {
@@ -207,7 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(BR, BKV);
       const uint32_t id_o = idesc_bf16_f32(BR, HD) | (1u << 16);  // B (V) is MN-major
-      const uint32_t q0 = smem_u32(smem + OFF_Q);
+      const uint32_t qlo = desc_lo_k(smem_u32(smem + OFF_Q));
       uint32_t n = 0;  // K/V ring position
       int g = 0;       // key tiles done so far, over all items
       bool ok = true;
@@ -220,11 +234,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         return true;
       };
       auto issue_s = [&](int t, uint32_t k0) {  // S_t = Q_t K^T
-        const uint32_t qa = q0 + t * TILE;
+        const uint32_t qa = qlo + ((t * TILE) >> 4), kb = desc_lo_k(k0);
 #pragma unroll
         for (int k = 0; k < HD / 16; k++) {
-          const uint32_t off = (k >> 2) * SUB + (k & 3) * 32;
-          mma_bf16(tmem + t * 128, desc_k_sw128(qa + off), desc_k_sw128(k0 + off), id_s, k != 0);
+          const uint32_t off = ((k >> 2) * SUB + (k & 3) * 32) >> 4;
+          mma_ss(tmem + t * 128, qa + off, kb + off, id_s, k != 0);
         }
         mma_commit(&s_full[t]);
       };
@@ -248,10 +262,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             // the epilogue of the previous item must have read O_t
             if (j == 0 && !mbar_wait(&o_free[t], (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t pa = tmem + t * 128 + 64;
+            const uint32_t pa = tmem + t * 128 + 64, vb = desc_lo_mn(vaddr);
 #pragma unroll
             for (int k = 0; k < BKV / 16; k++)
-              mma_bf16_ts(tmem + 256 + t * 128, pa + k * 8, desc_mn_sw128(vaddr + k * 2048), id_o, (j | k) != 0);
+              mma_ts(tmem + 256 + t * 128, pa + k * 8, vb + ((k * 2048) >> 4), id_o, (j | k) != 0);
             mma_commit(&o_done[t]);
             if (t == 1) mma_commit(&kv_empty[vslot]);
             if (j + 1 < n_kv) {
@@ -298,10 +312,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
           tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
           tmem_ld_wait();
+          if (masked) {  // a tile on the diagonal
+            const int kh = kbase + h * 64;
 #pragma unroll
-          for (int q = 0; q < 64; q++) {
-            const float x = (masked && kbase + h * 64 + q > t_row) ? -INFINITY : __uint_as_float(v[q]);
-            mx[q & 3] = fmaxf(mx[q & 3], x);
+            for (int q = 0; q < 64; q++) {
+              const float x = kh + q > t_row ? -INFINITY : __uint_as_float(v[q]);
+              mx[q & 3] = fmaxf(mx[q & 3], x);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 64; q += 8) {
+              mx[0] = max3(mx[0], __uint_as_float(v[q]), __uint_as_float(v[q + 1]));
+              mx[1] = max3(mx[1], __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
+              mx[2] = max3(mx[2], __uint_as_float(v[q + 4]), __uint_as_float(v[q + 5]));
+              mx[3] = max3(mx[3], __uint_as_float(v[q + 6]), __uint_as_float(v[q + 7]));
+            }
           }
         }
         const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
@@ -336,16 +361,27 @@ __global__ void __launch_bounds__(THREADS, 1)
           tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
           tmem_ld_wait();
           uint32_t pk[32];
+          if (masked) {
+            const int kh = kbase + h * 64;
 #pragma unroll
-          for (int q = 0; q < 32; q++) {
-            const int k0 = kbase + h * 64 + 2 * q;
-            const float s0 = (masked && k0 > t_row) ? -INFINITY : __uint_as_float(v[2 * q]);
-            const float s1 = (masked && k0 + 1 > t_row) ? -INFINITY : __uint_as_float(v[2 * q + 1]);
-            const float p0 = ex2(fmaf(s0, a.scale_log2, nm));
-            const float p1 = ex2(fmaf(s1, a.scale_log2, nm));
-            sum[(2 * q) & 3] += p0;
-            sum[(2 * q + 1) & 3] += p1;
-            pk[q] = pack2(p0, p1);
+            for (int q = 0; q < 32; q++) {
+              const float s0 = kh + 2 * q > t_row ? -INFINITY : __uint_as_float(v[2 * q]);
+              const float s1 = kh + 2 * q + 1 > t_row ? -INFINITY : __uint_as_float(v[2 * q + 1]);
+              const float p0 = ex2(fmaf(s0, a.scale_log2, nm));
+              const float p1 = ex2(fmaf(s1, a.scale_log2, nm));
+              sum[(2 * q) & 3] += p0;
+              sum[(2 * q + 1) & 3] += p1;
+              pk[q] = pack2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; q++) {
+              const float p0 = ex2(fmaf(__uint_as_float(v[2 * q]), a.scale_log2, nm));
+              const float p1 = ex2(fmaf(__uint_as_float(v[2 * q + 1]), a.scale_log2, nm));
+              sum[(2 * q) & 3] += p0;
+              sum[(2 * q + 1) & 3] += p1;
+              pk[q] = pack2(p0, p1);
+            }
           }
           tmem_st32(tS + 64 + h * 32, pk);
         }
