@@ -270,21 +270,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(&tempty[acc], accphase ^ 1, abort_flag, g.status)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
+        // a wait's result takes ~160 cycles even when the stage is full, so
+        // the next stage is probed before this stage's MMAs are issued and
+        // its answer is read after them
+        bool ready = mbar_try_wait(smem_u32(&full[stage]), phase);
         for (int kb = 0; kb < kblocks; kb++) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, g.status)) {
+          if (!ready && !mbar_wait(&full[stage], phase, abort_flag, g.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
+          const int nstage = stage + 1 == STAGES ? 0 : stage + 1;
+          const uint32_t nphase = stage + 1 == STAGES ? phase ^ 1 : phase;
+          const bool next_ready = kb + 1 < kblocks && mbar_try_wait(smem_u32(&full[nstage]), nphase);
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES), w0 = smem_u32(sW + stage * B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; k++)
             mma_bf16(d, desc_k_sw128(a0 + 32 * k), desc_k_sw128(w0 + 32 * k), idesc, (kb | k) != 0);
           mma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
+          stage = nstage;
+          phase = nphase;
+          ready = next_ready;
         }
         mma_commit(&tfull[acc]);
       }

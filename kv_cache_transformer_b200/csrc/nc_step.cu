@@ -141,14 +141,17 @@ __device__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, volatile int *
   }
 }
 
-// Grid barrier among the compute threads of every CTA (bounded).
-__device__ bool grid_sync(const StepArgs &a, volatile int *abort_flag, int e) {
+// Grid barrier among the compute threads of every CTA (bounded), the one
+// after phase p. The counter is zeroed before every launch, so the barrier is
+// complete once it reaches (p + 1) * grid: each CTA adds 1 with a release
+// reduction (no returned value, no round trip; the CTA barrier before it
+// orders the other compute threads' writes ahead of it) and polls with
+// acquire loads.
+__device__ bool grid_sync(const StepArgs &a, volatile int *abort_flag, int e, int p) {
   epi_sync();
   if (e == 0) {
-    __threadfence();
-    const unsigned long long n = (unsigned long long)a.grid;
-    const unsigned long long old = atomicAdd(a.bar, 1ull);
-    const unsigned long long target = (old / n + 1) * n;
+    const unsigned long long target = (unsigned long long)(p + 1) * (unsigned long long)a.grid;
+    asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(a.bar) : "memory");
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0;; ++it) {
       unsigned long long v;
@@ -163,7 +166,6 @@ __device__ bool grid_sync(const StepArgs &a, volatile int *abort_flag, int e) {
         }
       }
     }
-    __threadfence();
   }
   epi_sync();
   return *abort_flag == 0;
@@ -306,11 +308,15 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
           xr++;
           tc_fence_after();
           const int cn = min(XKB, g.nkb - c0);
+          // a wait's result takes ~160 cycles even when the slot is full: the
+          // next slot is probed before this slot's MMAs, its answer read after
+          bool ready = cn > 0 && mbar_try_wait(smem_u32(&s.full[t % RING]), (t / RING) & 1);
           for (int kb = 0; kb < cn; kb++) {
             const uint32_t slot = t % RING;
-            if (!mbar_wait(&s.full[slot], (t / RING) & 1, s.abort_flag, a.status)) return;
+            if (!ready && !mbar_wait(&s.full[slot], (t / RING) & 1, s.abort_flag, a.status)) return;
             t++;
             tc_fence_after();
+            ready = kb + 1 < cn && mbar_try_wait(smem_u32(&s.full[t % RING]), (t / RING) & 1);
             const uint32_t w0 = smem_u32(ring + slot * SLOT), x0 = smem_u32(xs + kb * NB * 128);
             // the four 16-column steps of a block accumulate into four different
             // TMEM accumulators, so consecutive MMAs do not wait on one another;
@@ -341,7 +347,10 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
 }
 
 // ------------------------------------------------- compute-side helpers
-// X staging: X[b][kb*64 + c] for this pass, NB rows, 128-byte swizzled.
+// X staging: X[b][kb*64 + c] for this pass, NB rows, 128-byte swizzled. The
+// normed inputs (QKV, FC, HEAD) are staged as bf16(x); their RMS factor is
+// applied to the accumulator column in the epilogue, so staging does not
+// wait for the row sums.
 // Loads are issued in batches of U per thread before any is consumed, so a
 // pass costs a few L2 round trips instead of one per item.
 __device__ void stage_x(const StepArgs &a, const Smem &s, uint8_t *xs, int type, int kb_begin, int nkb, int e) {
@@ -370,9 +379,8 @@ __device__ void stage_x(const StepArgs &a, const Smem &s, uint8_t *xs, int type,
         const int idx = base + u * 128;
         if (idx >= total) break;
         const int c = idx & 7, b = (idx >> 3) % NB, kbl = idx / (8 * NB);
-        const float r = s.inv[b];
-        const uint4 v = make_uint4(pack_bf(p[u].x * r, p[u].y * r), pack_bf(p[u].z * r, p[u].w * r),
-                                   pack_bf(q[u].x * r, q[u].y * r), pack_bf(q[u].z * r, q[u].w * r));
+        const uint4 v = make_uint4(pack_bf(p[u].x, p[u].y), pack_bf(p[u].z, p[u].w), pack_bf(q[u].x, q[u].y),
+                                   pack_bf(q[u].z, q[u].w));
         *reinterpret_cast<uint4 *>(xs + kbl * NB * 128 + b * 128 + ((c ^ (b & 7)) << 4)) = v;
       }
     } else {
@@ -447,7 +455,7 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
 #pragma unroll
     for (int j = 0; j < NB / CL; j++) {
       if (j < nb) {
-        const float v = fmaxf(tl[e * (NB + 1) + j], 0.f);
+        const float v = fmaxf(tl[e * (NB + 1) + j] * s.inv[b0 + j], 0.f);
         a.f[(size_t)(b0 + j) * a.F + col] = __float2bfloat16_rn(v * v);
       }
     }
@@ -483,7 +491,8 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
         rot[j] = 0.f;
         if (j < nb) {
           const float2 cs = pre.cs[j];
-          const float v = tl[e * (NB + 1) + j], u = tl[(e ^ 64) * (NB + 1) + j];
+          const float r = s.inv[b0 + j];
+          const float v = tl[e * (NB + 1) + j] * r, u = tl[(e ^ 64) * (NB + 1) + j] * r;
           rot[j] = e < 64 ? v * cs.x - u * cs.y : u * cs.y + v * cs.x;
         }
       }
@@ -514,7 +523,8 @@ __device__ void gemm_epilogue(const StepArgs &a, const Smem &s, int type, int la
       for (int j = 0; j < nb; j++) {
         const int b = b0 + j;
         if (s.valid[b])
-          a.vc[lay + ((size_t)b * a.max_seq + s.pos[b]) * 128 + e] = __float2bfloat16_rn(tl[e * (NB + 1) + j]);
+          a.vc[lay + ((size_t)b * a.max_seq + s.pos[b]) * 128 + e] =
+              __float2bfloat16_rn(tl[e * (NB + 1) + j] * s.inv[b]);
       }
     }
   }
@@ -533,7 +543,7 @@ __device__ void head_epilogue(const StepArgs &a, const Smem &s, int nt, const ui
 #pragma unroll
   for (int b = 0; b < NB; b++) {
     if (b < a.B) {
-      const float z = a.cap * tanhf(__uint_as_float(r[b]) * inv);
+      const float z = a.cap * tanhf(__uint_as_float(r[b]) * s.inv[b] * inv);
       if (s.valid[b]) a.logits[(size_t)b * a.V + col] = z;
       tl[n * (NB + 1) + b] = z + nz[b];
     }
@@ -876,8 +886,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
         // linear layer: QKV, OPROJ, FC, PROJ (cluster split-K) or HEAD (full K)
         const Gemm g = gemm_of(a, type, layer, cid, ncl, rank);
         const bool norm = (type == P_QKV || type == P_FC || type == P_HEAD);
-        if (norm)
-          load_inv(a, s, a.ss + (size_t)(type == P_QKV ? 2 * layer : type == P_FC ? 2 * layer + 1 : 2 * a.L) * SSN * 32, e);
+        bool inv_ready = !norm;
         bool staged_once = false;
         for (int nt = g.nt0; nt < g.n_tiles && ok; nt += g.nt_step, units++) {
           for (int c0 = 0; c0 < g.nkb || (c0 == 0 && g.nkb == 0); c0 += XKB) {
@@ -896,6 +905,11 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
             if (g.nkb == 0) break;
           }
           if (!ok) break;
+          if (!inv_ready) {  // the row factors, computed while the MMAs run
+            load_inv(a, s, a.ss + (size_t)(type == P_QKV ? 2 * layer : type == P_FC ? 2 * layer + 1 : 2 * a.L) * SSN * 32,
+                     e);
+            inv_ready = true;
+          }
           t += g.nkb;  // the unit's weight tiles went through the ring (consumed by the MMA warp)
           if (!mbar_wait(s.acc_full, units & 1, s.abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
@@ -960,7 +974,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           epi_sync();
         }
       }
-      if (ok && p + 1 < P) ok = grid_sync(a, s.abort_flag, e);
+      if (ok && p + 1 < P) ok = grid_sync(a, s.abort_flag, e, p);
     }
     if (x_pending && ok) {
       mbar_wait(s.x_free, xf & 1, s.abort_flag, a.status);
