@@ -163,7 +163,7 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
   fz.T = rm.T;
   fz.H = H;
   fz.max_seq = kv->max_seq;
-  const int nss = (d + 255) / 256;
+  const int nss = (d + 127) / 128;
   cudaError_t e = cudaSuccess;
   auto gemm = [&](int epi, const void *A, int lda, const void *W, int N, int K, void *out) {
     if (e == cudaSuccess)
@@ -476,7 +476,7 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   alloc(&kv->f, elem * rows * F);
   alloc((void **)&kv->logits, sizeof(float) * (size_t)max_batch * c.vocab);
   alloc((void **)&kv->pos_ws, sizeof(int32_t) * max_batch);
-  if (model->fast && nc::rowops_supported(c)) alloc((void **)&kv->row_ss, sizeof(float) * ((d + 255) / 256) * rows);
+  if (model->fast && nc::rowops_supported(c)) alloc((void **)&kv->row_ss, sizeof(float) * ((d + 127) / 128) * rows);
   kv->dec_fast = nc::decode_fast_supported(c, 1);
   if (kv->dec_fast) {
     int nb = max_batch < 32 ? max_batch : 32;

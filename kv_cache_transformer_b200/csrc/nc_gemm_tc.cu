@@ -5,16 +5,16 @@
 // accumulation in tensor memory (TMEM).
 //
 // Persistent kernel, one CTA per SM, 128 x 256 output tiles walked with a
-// static stride of gridDim.x. Warp roles (192 threads):
+// static stride of gridDim.x. Warp roles (320 threads):
 //   warp 0      TMA producer: A and W tiles of 64 K-columns (128-byte
 //               swizzle) into a 4-stage shared-memory ring;
 //   warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma (M=128,
 //               N=256, K=16) per stage into one of two TMEM accumulators
 //               (2 x 256 fp32 columns), tcgen05.commit frees the stage;
-//   warps 2-5   epilogue: tcgen05.ld of the finished accumulator (each warp
-//               its 32-lane TMEM quarter = 32 rows), epilogue math, stores,
-//               then release the accumulator so the next tile's MMAs run
-//               while this one drains.
+//   warps 2-9   epilogue: tcgen05.ld of the finished accumulator (each warp
+//               its 32-lane TMEM quarter = 32 rows, and one 128-column half),
+//               epilogue math, stores, then release the accumulator so the
+//               next tile's MMAs run while this one drains.
 // Fused prefill epilogues (GemmFuse): the RMS factor of un-normed bf16(x)
 // rows applied to the accumulator; RoPE + QK norm + cache append of the qkv
 // projection; bf16(x) and per-tile sums of squares written beside the
@@ -33,8 +33,10 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;
-constexpr int EPI_BUF = 4 * 32 * 32 * 4;  // per epilogue warp: a 32 x 32 fp32 transpose buffer
+constexpr int EPI_WARPS = 8;   // two per TMEM lane quarter, one per 128-column half of the tile
+constexpr int HC = BN / 2;      // columns per epilogue warp
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr int EPI_BUF = EPI_WARPS * 32 * 32 * 4;  // per epilogue warp: a 32 x 32 fp32 transpose buffer
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BUF;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 
@@ -140,21 +142,21 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
   }
   const int q = lane & 7, rsub = lane >> 3;
   float facr[8];
-  bf16 *dst[8];
-  int pos[8];
-  bool ok[8];
+  int pos[8], crow[8];  // position, and cache row b*max_seq + position
 #pragma unroll
   for (int i = 0; i < 8; i++) {
     const int row = rbase + 4 * i + rsub;
     facr[i] = __shfl_sync(0xffffffffu, fac, 4 * i + rsub);
-    ok[i] = row < g.M;
     const int b = row / f.T;
-    pos[i] = ok[i] ? row % f.T : 0;
-    const size_t crow = ((size_t)b * f.max_seq + pos[i]) * 128;
-    dst[i] = (head < f.H ? reinterpret_cast<bf16 *>(f.q) + ((size_t)row * f.H + head) * 128
-                         : reinterpret_cast<bf16 *>(head == f.H ? f.kc : f.vc) + crow) +
-             4 * q;
+    pos[i] = row < g.M ? row - b * f.T : 0;
+    crow[i] = row < g.M ? b * f.max_seq + pos[i] : 0;
   }
+  auto dst_of = [&](int i) -> bf16 * {
+    const int row = rbase + 4 * i + rsub;
+    return (head < f.H ? reinterpret_cast<bf16 *>(f.q) + ((size_t)row * f.H + head) * 128
+                       : reinterpret_cast<bf16 *>(head == f.H ? f.kc : f.vc) + (size_t)crow[i] * 128) +
+           4 * q;
+  };
   if (isv) {
 #pragma unroll 1
     for (int c = 0; c < 4; c++) {
@@ -162,36 +164,30 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
       transpose_chunk(tcol + 32 * c, ebuf, lane, v);
 #pragma unroll
       for (int i = 0; i < 8; i++)
-        if (ok[i])
-          *reinterpret_cast<uint2 *>(dst[i] + 32 * c) =
+        if (rbase + 4 * i + rsub < g.M)
+          *reinterpret_cast<uint2 *>(dst_of(i) + 32 * c) =
               make_uint2(pack_bf16(v[i].x * facr[i], v[i].y * facr[i]), pack_bf16(v[i].z * facr[i], v[i].w * facr[i]));
     }
     return;
   }
 #pragma unroll 1
   for (int c = 0; c < 2; c++) {  // elements 32c + 4q .. +3 and their partners 64 + 32c + 4q .. +3
-    float4 t0[8], t1[8];         // (cos, sin) of the 4 pairs, per row
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      const float4 *cs = reinterpret_cast<const float4 *>(f.rope + (size_t)pos[i] * 64) + 16 * c + 2 * q;
-      t0[i] = cs[0];
-      t1[i] = cs[1];
-    }
     float4 lo[8], hi[8];
     transpose_chunk(tcol + 32 * c, ebuf, lane, lo);
     transpose_chunk(tcol + 64 + 32 * c, ebuf, lane, hi);
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-      if (!ok[i]) continue;
-      const float4 a = lo[i], h = hi[i], u = t0[i], w = t1[i];
+      if (rbase + 4 * i + rsub >= g.M) continue;
+      const float4 *cs = reinterpret_cast<const float4 *>(f.rope + (size_t)pos[i] * 64) + 16 * c + 2 * q;
+      const float4 a = lo[i], h = hi[i], u = cs[0], w = cs[1];  // (cos, sin) of the 4 pairs
       const float F = facr[i];
       const float l0 = a.x * u.x - h.x * u.y, h0 = a.x * u.y + h.x * u.x;
       const float l1 = a.y * u.z - h.y * u.w, h1 = a.y * u.w + h.y * u.z;
       const float l2 = a.z * w.x - h.z * w.y, h2 = a.z * w.y + h.z * w.x;
       const float l3 = a.w * w.z - h.w * w.w, h3 = a.w * w.w + h.w * w.z;
-      *reinterpret_cast<uint2 *>(dst[i] + 32 * c) = make_uint2(pack_bf16(l0 * F, l1 * F), pack_bf16(l2 * F, l3 * F));
-      *reinterpret_cast<uint2 *>(dst[i] + 64 + 32 * c) =
-          make_uint2(pack_bf16(h0 * F, h1 * F), pack_bf16(h2 * F, h3 * F));
+      bf16 *d = dst_of(i);
+      *reinterpret_cast<uint2 *>(d + 32 * c) = make_uint2(pack_bf16(l0 * F, l1 * F), pack_bf16(l2 * F, l3 * F));
+      *reinterpret_cast<uint2 *>(d + 64 + 32 * c) = make_uint2(pack_bf16(h0 * F, h1 * F), pack_bf16(h2 * F, h3 * F));
     }
   }
 }
@@ -223,7 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; a++) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * EPI_WARPS);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -296,41 +292,46 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else {
-    const int quarter = warp & 3;  // this warp's TMEM lane quarter
+    const int ew = warp - 2;       // epilogue warp 0..7
+    const int quarter = warp & 3;  // its TMEM lane quarter (a warp reaches lanes 32*(warp%4) .. +31)
+    const int half = ew >> 2;      // its 128-column half of the tile
+    float *ebuf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + ew * 1024;
     int local = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, local++) {
       const int acc = local & 1;
       const uint32_t accphase = (local >> 1) & 1;
       const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+      const int nh = n0 + half * HC;  // first column of this warp's half
       const int row = m0 + quarter * 32 + lane;
       const bool rok = row < g.M;
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN + half * HC;
       if constexpr (EPI == EPI_RESID || EPI == EPI_RESID_X) {
-        // x += acc over the tile's 8 chunks of 32 columns. Each chunk goes
+        // x += acc over the half's 4 chunks of 32 columns. Each chunk goes
         // TMEM -> registers (lane = row) -> a swizzled shared buffer, and is
         // read back with lane = (row group, float4 column), so that every
         // global access of a warp covers 4 rows x 128 contiguous bytes. The
-        // residual is read 4 chunks ahead, the first 4 before the
+        // residual is read 2 chunks ahead (cur / nxt), the first 2 before the
         // accumulator is ready.
-        float *ebuf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + quarter * 1024;
         const int q = lane & 7, rsub = lane >> 3;
         const int rbase = m0 + quarter * 32;
-        float *xt = reinterpret_cast<float *>(g.out) + (size_t)rbase * g.ldo + n0 + 4 * q;
-        bf16 *xbt = reinterpret_cast<bf16 *>(g.fz.xb) + (size_t)rbase * g.ldo + n0 + 4 * q;
-        float4 xp[4][8];
-#pragma unroll
-        for (int c = 0; c < 4; c++)
+        float *xt = reinterpret_cast<float *>(g.out) + (size_t)rbase * g.ldo + nh + 4 * q;
+        bf16 *xbt = reinterpret_cast<bf16 *>(g.fz.xb) + (size_t)rbase * g.ldo + nh + 4 * q;
+        float4 cur[8], nxt[8];
+        auto load_chunk = [&](int c, float4 (&dst)[8]) {
 #pragma unroll
           for (int i = 0; i < 8; i++)
-            if (rbase + 4 * i + rsub < g.M && n0 + 32 * c < g.N)
-              xp[c][i] = *reinterpret_cast<const float4 *>(xt + (size_t)(4 * i + rsub) * g.ldo + 32 * c);
+            if (rbase + 4 * i + rsub < g.M && nh + 32 * c < g.N)
+              dst[i] = *reinterpret_cast<const float4 *>(xt + (size_t)(4 * i + rsub) * g.ldo + 32 * c);
+        };
+        load_chunk(0, cur);
+        load_chunk(1, nxt);
         if (!mbar_wait(&tfull[acc], accphase, abort_flag, g.status)) break;
         tc_fence_after();
         float ssl[8];
 #pragma unroll
         for (int i = 0; i < 8; i++) ssl[i] = 0.f;
-#pragma unroll
-        for (int c = 0; c < 8; c++) {
+#pragma unroll 1
+        for (int c = 0; c < HC / 32; c++) {
           uint32_t r[32];
           tmem_ld32(tbase + 32 * c, r);
           tmem_ld_wait();
@@ -339,13 +340,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             *reinterpret_cast<float4 *>(ebuf + lane * 32 + ((j ^ (lane & 7)) << 2)) =
                 make_float4(u2f(r[4 * j]), u2f(r[4 * j + 1]), u2f(r[4 * j + 2]), u2f(r[4 * j + 3]));
           __syncwarp();
-          if (n0 + 32 * c < g.N) {
+          if (nh + 32 * c < g.N) {
 #pragma unroll
             for (int i = 0; i < 8; i++) {
               const int rr = 4 * i + rsub;
               const float4 a = *reinterpret_cast<const float4 *>(ebuf + rr * 32 + ((q ^ (rr & 7)) << 2));
               if (rbase + rr < g.M) {
-                float4 x = xp[c & 3][i];
+                float4 x = cur[i];
                 x.x += a.x;
                 x.y += a.y;
                 x.z += a.z;
@@ -360,21 +361,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
           __syncwarp();
-          if (c + 4 < 8 && n0 + 32 * (c + 4) < g.N)
 #pragma unroll
-            for (int i = 0; i < 8; i++)
-              if (rbase + 4 * i + rsub < g.M)
-                xp[c & 3][i] = *reinterpret_cast<const float4 *>(xt + (size_t)(4 * i + rsub) * g.ldo + 32 * (c + 4));
+          for (int i = 0; i < 8; i++) cur[i] = nxt[i];
+          if (c + 2 < HC / 32) load_chunk(c + 2, nxt);
         }
-        if (EPI == EPI_RESID_X) {
-          // row sums: the 8 lanes of a row group hold its 8 float4 columns
+        if (EPI == EPI_RESID_X && nh < g.N) {
+          // row sums over the half: the 8 lanes of a row group hold its 8 float4 columns
 #pragma unroll
           for (int i = 0; i < 8; i++) {
             float v = ssl[i];
             v += __shfl_xor_sync(0xffffffffu, v, 1);
             v += __shfl_xor_sync(0xffffffffu, v, 2);
             v += __shfl_xor_sync(0xffffffffu, v, 4);
-            if (q == 0 && rbase + 4 * i + rsub < g.M) g.fz.ss_out[(size_t)(n0 / BN) * g.M + rbase + 4 * i + rsub] = v;
+            if (q == 0 && rbase + 4 * i + rsub < g.M)
+              g.fz.ss_out[(size_t)(nh / HC) * g.M + rbase + 4 * i + rsub] = v;
           }
         }
       } else {
@@ -389,21 +389,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(&tfull[acc], accphase, abort_flag, g.status)) break;
         tc_fence_after();
         if constexpr (EPI == EPI_QKV) {
-#pragma unroll 1
-          for (int hh = 0; hh < BN / 128; hh++) {
-            const int head = n0 / 128 + hh;
-            if (head >= g.fz.H + 2) break;  // the same for the whole warp
-            qkv_head(g, m0 + quarter * 32, lane, head, tbase + hh * 128, scale,
-                     reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + quarter * 1024);
-          }
+          const int head = nh / 128;  // one head per half
+          if (head < g.fz.H + 2) qkv_head(g, m0 + quarter * 32, lane, head, tbase, scale, ebuf);
         } else {
           float ss = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = 0; c < HC; c += 32) {
             uint32_t r[32];
             tmem_ld32(tbase + c, r);
             tmem_ld_wait();
-            if (rok && n0 + c < g.N) epilogue32<EPI>(g, row, n0 + c, r, scale, ss);
+            if (rok && nh + c < g.N) epilogue32<EPI>(g, row, nh + c, r, scale, ss);
           }
         }
       }

@@ -68,7 +68,7 @@ struct nc_kv {
   float *cand_v = nullptr;     // [V/128][32] per-tile argmax winners
   int *cand_i = nullptr;
   float *xl = nullptr;         // [32][d] last-position rows of a prefill, for the fused lm_head
-  float *row_ss = nullptr;     // [ceil(d/256)][max_rows] per-256-column sums of squares of x rows (prefill)
+  float *row_ss = nullptr;     // [ceil(d/128)][max_rows] per-128-column sums of squares of x rows (prefill)
   // whole-step decode kernel (nc_step.cu)
   int step_grid = 0;           // CTAs of the step kernel, 0 = not available
   CUtensorMap *step_maps = nullptr;  // device copy of the step kernel's tensor maps
@@ -108,8 +108,8 @@ enum Epi { EPI_STORE = 0, EPI_RELU2 = 1, EPI_RESID = 2, EPI_SOFTCAP = 3, EPI_QKV
 //              caches at (row / T, row % T) with row pitch 128, max_seq rows
 //              per sequence
 //  EPI_RESID_X x += acc as EPI_RESID, plus xb = bf16(x) (row pitch N) and
-//              ss_out[tile_n*M + row] = sum of squares of the new x over the
-//              tile's 256 columns
+//              ss_out[j*M + row] = sum of squares of the new x over columns
+//              128j .. 128j+127
 struct GemmFuse {
   const float *ss_in = nullptr;
   int nss = 0;
