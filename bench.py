@@ -78,6 +78,15 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------- clocks
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of the
+# prefill GEMMs, the mean over the QKV, O-proj, MLP fc and MLP proj launches of
+# one layer (one of each per layer, so also the mean over a step's 80 launches),
+# from an ncu capture (cold L2; writes still in L2 at kernel end not counted)
+# of `python bench.py --no-decode --no-cpu-baseline --steps 1 --warmup 3` with
+# -k regex:gemm_tc -s 240 -c 4. To be re-taken whenever nc_gemm_tc.cu changes.
+GEMM_DRAM_BYTES_PER_LAUNCH = (54_963_200 + 196_754_176 + 166_150_400 + 388_773_632) / 4
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -95,7 +104,12 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            # nvidia-smi takes a moment to start: wait (up to 5 s) for its
+            # first sample, so the samples cover the timed region
+            t_end = time.time() + 5.0
+            while time.time() < t_end and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
 
@@ -289,7 +303,7 @@ def run_ours(args):
     roofline = {
         "bound": "tensor", "kernel": "prefill linear-layer GEMMs (QKV, O, fc relu^2, proj)",
         "achieved": gemm_tflops, "peak": peak_tc, "unit": "TFLOP/s", "frac": gemm_tflops / peak_tc,
-        "traffic": None, "peak_source": f"{peaks_src} bf16_tflops_sustained",
+        "traffic": GEMM_DRAM_BYTES_PER_LAUNCH, "peak_source": f"{peaks_src} bf16_tflops_sustained",
         "flops_per_launch": fl["gemm"] / max(gemm_launch_per_step, 1),
         "ms_per_launch": gemm_ms / max(gemm_launch_per_step, 1),
         "launches_per_step": gemm_launch_per_step,
