@@ -61,7 +61,7 @@ constexpr int OFF_X = OFF_RING + RING * SLOT;          // XKB * NB * 128 bytes
 constexpr int OFF_RED = OFF_X + XKB * NB * 128;         // 16 KB, read by cluster peers
 constexpr int OFF_TL = OFF_RED + 16384;                 // [128][NB+1] fp32
 constexpr int OFF_BAR = OFF_TL + 128 * (NB + 1) * 4;
-constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+constexpr int SMEM_BYTES = OFF_BAR + 1024 + 1024;  // barriers and per-row tables, then alignment slack
 
 enum Phase { P_EMBED = 0, P_QKV, P_ATTN, P_OPROJ, P_FC, P_PROJ, P_HEAD, P_MERGE };
 
@@ -88,7 +88,8 @@ struct StepArgs {
 };
 
 struct Smem {
-  uint64_t *full, *empty, *x_ready, *x_free, *acc_full, *acc_empty, *red_full, *red_free;
+  uint64_t *full, *empty, *x_ready, *x_free, *red_full, *red_free;
+  uint64_t *acc_full, *acc_empty;  // [2] each: one per TMEM accumulator set
   uint32_t *tmem_slot;
   int *abort_flag;
   int *pos, *valid;  // [32]
@@ -299,41 +300,60 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
     phase_of(a, p, type, layer);
     if (type == P_QKV || type == P_OPROJ || type == P_FC || type == P_PROJ || type == P_HEAD) {
       const Gemm g = gemm_of(a, type, layer, cid, ncl, rank);
-      for (int nt = g.nt0; nt < g.n_tiles; nt += g.nt_step, units++) {
-        if (!mbar_wait(s.acc_empty, (units & 1) ^ 1, s.abort_flag, a.status)) return;
+      // When this CTA's K range fits the staging buffer, X is staged once for
+      // every n-tile of the phase (they all multiply the same X slice)
+      const bool single = g.nkb <= XKB && g.nt0 < g.n_tiles;
+      if (single) {
+        if (!mbar_wait(s.x_ready, xr & 1, s.abort_flag, a.status)) return;
+        xr++;
         tc_fence_after();
-        bool first = true;
-        for (int c0 = 0; c0 < g.nkb || (c0 == 0 && g.nkb == 0); c0 += XKB) {
-          if (!mbar_wait(s.x_ready, xr & 1, s.abort_flag, a.status)) return;
-          xr++;
-          tc_fence_after();
-          const int cn = min(XKB, g.nkb - c0);
-          // a wait's result takes ~160 cycles even when the slot is full: the
-          // next slot is probed before this slot's MMAs, its answer read after
-          bool ready = cn > 0 && mbar_try_wait(smem_u32(&s.full[t % RING]), (t / RING) & 1);
-          for (int kb = 0; kb < cn; kb++) {
-            const uint32_t slot = t % RING;
-            if (!ready && !mbar_wait(&s.full[slot], (t / RING) & 1, s.abort_flag, a.status)) return;
-            t++;
-            tc_fence_after();
-            ready = kb + 1 < cn && mbar_try_wait(smem_u32(&s.full[t % RING]), (t / RING) & 1);
-            const uint32_t w0 = smem_u32(ring + slot * SLOT), x0 = smem_u32(xs + kb * NB * 128);
-            // the four 16-column steps of a block accumulate into four different
-            // TMEM accumulators, so consecutive MMAs do not wait on one another;
-            // the epilogue adds the accumulators up
-            const bool fresh = (c0 + kb) == 0;
-#pragma unroll
-            for (int k = 0; k < 4; k++)
-              mma_bf16(tmem + (uint32_t)k * NB, desc_k_sw128(w0 + 32 * k), desc_k_sw128(x0 + 32 * k), idesc,
-                       fresh ? 0 : 1);
-            first = false;
-            mma_commit(&s.empty[slot]);
-          }
-          mma_commit(s.x_free);
-          if (g.nkb == 0) break;
-        }
-        mma_commit(s.acc_full);
       }
+      // k-blocks kb_lo .. kb_lo + cn - 1 of this unit, X staged from kb_lo
+      auto issue = [&](uint32_t acc0, int kb_lo, int cn, bool fresh0) -> bool {
+        // a wait's result takes ~160 cycles even when the slot is full: the
+        // next slot is probed before this slot's MMAs, its answer read after
+        bool ready = cn > 0 && mbar_try_wait(smem_u32(&s.full[t % RING]), (t / RING) & 1);
+        for (int kb = 0; kb < cn; kb++) {
+          const uint32_t slot = t % RING;
+          if (!ready && !mbar_wait(&s.full[slot], (t / RING) & 1, s.abort_flag, a.status)) return false;
+          t++;
+          tc_fence_after();
+          ready = kb + 1 < cn && mbar_try_wait(smem_u32(&s.full[t % RING]), (t / RING) & 1);
+          const uint32_t w0 = smem_u32(ring + slot * SLOT), x0 = smem_u32(xs + (kb_lo + kb) * NB * 128);
+          // the four 16-column steps of a block accumulate into four different
+          // TMEM accumulators, so consecutive MMAs do not wait on one another;
+          // the epilogue adds the accumulators up
+          const bool fresh = fresh0 && kb == 0;
+#pragma unroll
+          for (int k = 0; k < 4; k++)
+            mma_bf16(acc0 + (uint32_t)k * NB, desc_k_sw128(w0 + 32 * k), desc_k_sw128(x0 + 32 * k), idesc,
+                     fresh ? 0 : 1);
+          mma_commit(&s.empty[slot]);
+        }
+        return true;
+      };
+      for (int nt = g.nt0; nt < g.n_tiles; nt += g.nt_step, units++) {
+        // two accumulator sets: this unit's MMAs may run while the compute
+        // warps still reduce and store the previous unit
+        const uint32_t set = units & 1;
+        if (!mbar_wait(&s.acc_empty[set], ((units >> 1) & 1) ^ 1, s.abort_flag, a.status)) return;
+        tc_fence_after();
+        const uint32_t acc0 = tmem + set * (uint32_t)(NACC * NB);
+        if (single) {
+          if (!issue(acc0, 0, g.nkb, true)) return;
+        } else {
+          for (int c0 = 0; c0 < g.nkb || (c0 == 0 && g.nkb == 0); c0 += XKB) {
+            if (!mbar_wait(s.x_ready, xr & 1, s.abort_flag, a.status)) return;
+            xr++;
+            tc_fence_after();
+            if (!issue(acc0, 0, min(XKB, g.nkb - c0), c0 == 0)) return;
+            mma_commit(s.x_free);
+            if (g.nkb == 0) break;
+          }
+        }
+        mma_commit(&s.acc_full[set]);
+      }
+      if (single) mma_commit(s.x_free);  // X is free once every unit's MMAs are done
     } else if (type == P_ATTN) {
       // the compute warps consume this phase's ring slots; keep the count
       for (int b = cid; b < a.B; b += ncl) {
@@ -760,11 +780,11 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     s.empty = b + RING;
     s.x_ready = b + 2 * RING;
     s.x_free = s.x_ready + 1;
-    s.acc_full = s.x_ready + 2;
-    s.acc_empty = s.x_ready + 3;
-    s.red_full = s.x_ready + 4;
-    s.red_free = s.x_ready + 5;
-    s.tmem_slot = reinterpret_cast<uint32_t *>(s.x_ready + 6);
+    s.acc_full = s.x_ready + 2;   // [2]
+    s.acc_empty = s.x_ready + 4;  // [2]
+    s.red_full = s.x_ready + 6;
+    s.red_free = s.x_ready + 7;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(s.x_ready + 8);
     s.abort_flag = reinterpret_cast<int *>(s.tmem_slot + 1);
     s.pos = s.abort_flag + 1;
     s.valid = s.pos + 32;
@@ -784,8 +804,10 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     }
     mbar_init(s.x_ready, 1);
     mbar_init(s.x_free, 1);
-    mbar_init(s.acc_full, 1);
-    mbar_init(s.acc_empty, 128);
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 128);
+    }
     mbar_init(s.red_full, CL);
     mbar_init(s.red_free, CL);
     *s.abort_flag = 0;
@@ -803,7 +825,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     s.pos[b] = ok ? p : 0;
     s.valid[b] = ok;
   }
-  if (warp == 1) tmem_alloc(s.tmem_slot, NB * NACC);
+  if (warp == 1) tmem_alloc(s.tmem_slot, 2 * NB * NACC);
   tc_fence_before();
   __syncthreads();
   cluster.sync();  // peers' barriers are initialised before any remote arrive
@@ -887,39 +909,52 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
         const Gemm g = gemm_of(a, type, layer, cid, ncl, rank);
         const bool norm = (type == P_QKV || type == P_FC || type == P_HEAD);
         bool inv_ready = !norm;
-        bool staged_once = false;
-        for (int nt = g.nt0; nt < g.n_tiles && ok; nt += g.nt_step, units++) {
-          for (int c0 = 0; c0 < g.nkb || (c0 == 0 && g.nkb == 0); c0 += XKB) {
-            if (x_pending) {
-              if (!mbar_wait(s.x_free, xf & 1, s.abort_flag, a.status)) { ok = false; break; }
-              xf++;
-              x_pending = false;
-            }
-            const int cn = min(XKB, g.nkb - c0);
-            const bool reuse = (type == P_HEAD && staged_once && g.nkb <= XKB);
-            if (!reuse && cn > 0) stage_x(a, s, xs, type, g.kb0 + c0, cn, e);
-            staged_once = true;
-            epi_sync();
-            if (e == 0) mbar_arrive(s.x_ready);
-            x_pending = true;
-            if (g.nkb == 0) break;
+        const bool single = g.nkb <= XKB && g.nt0 < g.n_tiles;  // X staged once for the phase
+        if (single) {
+          if (x_pending) {
+            if (!mbar_wait(s.x_free, xf & 1, s.abort_flag, a.status)) { ok = false; }
+            xf++;
+            x_pending = false;
           }
-          if (!ok) break;
+          if (ok && g.nkb > 0) stage_x(a, s, xs, type, g.kb0, g.nkb, e);
+          epi_sync();
+          if (e == 0) mbar_arrive(s.x_ready);
+          x_pending = true;
+        }
+        for (int nt = g.nt0; nt < g.n_tiles && ok; nt += g.nt_step, units++) {
+          if (!single) {
+            for (int c0 = 0; c0 < g.nkb || (c0 == 0 && g.nkb == 0); c0 += XKB) {
+              if (x_pending) {
+                if (!mbar_wait(s.x_free, xf & 1, s.abort_flag, a.status)) { ok = false; break; }
+                xf++;
+                x_pending = false;
+              }
+              const int cn = min(XKB, g.nkb - c0);
+              if (cn > 0) stage_x(a, s, xs, type, g.kb0 + c0, cn, e);
+              epi_sync();
+              if (e == 0) mbar_arrive(s.x_ready);
+              x_pending = true;
+              if (g.nkb == 0) break;
+            }
+            if (!ok) break;
+          }
           if (!inv_ready) {  // the row factors, computed while the MMAs run
             load_inv(a, s, a.ss + (size_t)(type == P_QKV ? 2 * layer : type == P_FC ? 2 * layer + 1 : 2 * a.L) * SSN * 32,
                      e);
             inv_ready = true;
           }
           t += g.nkb;  // the unit's weight tiles went through the ring (consumed by the MMA warp)
-          if (!mbar_wait(s.acc_full, units & 1, s.abort_flag, a.status)) { ok = false; break; }
+          const uint32_t set = units & 1;
+          if (!mbar_wait(&s.acc_full[set], (units >> 1) & 1, s.abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t tacc = tmem + set * (uint32_t)(NACC * NB) + lane_off;
           uint32_t r[NB];
           {
             const int nacc = g.nkb > 0 ? NACC : 1;
-            tmem_ld32(tmem + lane_off, r);
+            tmem_ld32(tacc, r);
             for (int q = 1; q < nacc; q++) {
               uint32_t r2[NB];
-              tmem_ld32(tmem + lane_off + (uint32_t)q * NB, r2);
+              tmem_ld32(tacc + (uint32_t)q * NB, r2);
               tmem_ld_wait();
 #pragma unroll
               for (int j = 0; j < NB; j++) r[j] = __float_as_uint(__uint_as_float(r[j]) + __uint_as_float(r2[j]));
@@ -927,7 +962,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
             tmem_ld_wait();
           }
           tc_fence_before();
-          mbar_arrive(s.acc_empty);
+          mbar_arrive(&s.acc_empty[set]);
           if (g.nkb == 0)
             for (int j = 0; j < NB; j++) r[j] = 0u;  // this rank holds no k-blocks
           if (type == P_HEAD) {
@@ -985,7 +1020,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
   cluster.sync();  // no CTA leaves while a peer may still read its shared memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, NB * NACC);
+    tmem_dealloc(tmem, 2 * NB * NACC);
   }
 }
 
