@@ -251,7 +251,7 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
     ProfScope p(m, NC_K_STEP, s);
     return nc::k_decode_step(m, B, kv->max_batch, kv->max_seq, kv->step_maps, tokens, positions, kv->len, kv->x,
                              kv->xl, kv->step_ss, kv->q, kv->y, kv->f, kv->k, kv->v, kv->rope, logits, noise, next,
-                             kv->cand_v, kv->cand_i, kv->step_bar, kv->step_grid, s);
+                             kv->cand_v, kv->cand_i, kv->step_bar, kv->step_part, kv->step_grid, s);
   }
   {
     ProfScope p(m, NC_K_MISC, s);
@@ -494,9 +494,10 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
       const int nmaps = nc::decode_step_maps_count(c);
       std::vector<CUtensorMap> maps(nmaps);
       alloc((void **)&kv->step_maps, sizeof(CUtensorMap) * nmaps);
-      alloc((void **)&kv->step_bar, sizeof(unsigned long long));
+      alloc((void **)&kv->step_bar, nc::decode_step_bar_bytes());
+      alloc((void **)&kv->step_part, sizeof(float) * nc::decode_step_part_floats(model->num_sms));
       alloc((void **)&kv->step_ss, sizeof(float) * (size_t)(2 * c.depth + 1) * 16 * 32);
-      if (e == cudaSuccess) e = cudaMemset(kv->step_bar, 0, sizeof(unsigned long long));
+      if (e == cudaSuccess) e = cudaMemset(kv->step_bar, 0, nc::decode_step_bar_bytes());
       if (e == cudaSuccess && nc::decode_step_build_maps(model, kv->k, kv->v, max_batch, max_seq, maps.data())) {
         e = cudaMemcpy(kv->step_maps, maps.data(), sizeof(CUtensorMap) * nmaps, cudaMemcpyHostToDevice);
         if (e == cudaSuccess) kv->step_grid = nc::decode_step_grid(model->num_sms);
@@ -542,7 +543,7 @@ void nc_kv_destroy(nc_kv *kv) {
   void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
                 kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
                 kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl,     kv->step_maps, kv->step_bar,
-                kv->step_ss, kv->row_ss};
+                kv->step_ss, kv->row_ss, kv->step_part};
   for (void *p : ps) cudaFree(p);
   delete kv;
 }

@@ -72,7 +72,8 @@ struct nc_kv {
   // whole-step decode kernel (nc_step.cu)
   int step_grid = 0;           // CTAs of the step kernel, 0 = not available
   CUtensorMap *step_maps = nullptr;  // device copy of the step kernel's tensor maps
-  unsigned long long *step_bar = nullptr;  // its grid-barrier counter
+  unsigned long long *step_bar = nullptr;  // its grid-barrier counter and split counters
+  float *step_part = nullptr;  // split-K partials of its MLP proj phase
   float *step_ss = nullptr;    // [2*depth+1][16][32] per-128-column sums of squares
   int attn_chunk = 0, attn_splits = 0;
   // CUDA graph of the last decode step's launches, replayed while the call's
@@ -193,6 +194,8 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
                           const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
                           float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
                           const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          int grid, cudaStream_t s);
+                          float *split_part, int grid, cudaStream_t s);
+size_t decode_step_bar_bytes();              // grid-barrier word + split counters, zeroed per launch
+size_t decode_step_part_floats(int num_sms);  // split-K partials of the MLP proj phase
 
 }  // namespace nc

@@ -55,6 +55,8 @@ constexpr int THREADS = 192;
 constexpr int KT = 64;                 // keys per attention tile
 constexpr int NACC = 4;                // TMEM accumulators the K loop rotates over
 constexpr int SSN = 16;                // 128-column chunks of d_model (d <= 2048)
+constexpr int SPLIT_TILES = 16;        // MLP proj n-tiles (d / 128) the cross-cluster K split supports
+constexpr int SPLIT_MAX = 4;           // clusters per MLP proj n-tile at most
 
 constexpr int OFF_RING = 0;
 constexpr int OFF_X = OFF_RING + RING * SLOT;          // XKB * NB * 128 bytes
@@ -83,7 +85,9 @@ struct StepArgs {
   int32_t *next;              // [B] or null
   float *cand_v;              // [V/128][32]
   int *cand_i;
-  unsigned long long *bar;    // grid barrier counter
+  unsigned long long *bar;    // grid barrier counter, followed by split_cnt
+  unsigned *split_cnt;        // [SPLIT_TILES][CL]: arrivals of the K-split MLP proj partials
+  float *split_part;          // [n_tiles * S][CL][128][NB/CL]: their partial sums
   uint32_t *status;
 };
 
@@ -187,6 +191,7 @@ struct Gemm {
   int N, K, kb_total, n_tiles;
   int kb0, nkb;           // this CTA's k-blocks (split over the cluster; full K for HEAD)
   int nt0, nt_step;       // this CTA's n-tiles: nt0, nt0 + nt_step, ...
+  int S, split;           // K also split over S clusters per n-tile; this cluster's part
   const CUtensorMap *map;
 };
 
@@ -199,11 +204,29 @@ __device__ __forceinline__ Gemm gemm_of(const StepArgs &a, int type, int layer, 
   else { g.N = a.V; g.K = a.d; g.map = a.wmaps + 4 * a.L; }
   g.kb_total = g.K / 64;
   g.n_tiles = g.N / 128;
+  g.S = 1;
+  g.split = 0;
   if (type == P_HEAD) {
     g.kb0 = 0;
     g.nkb = g.kb_total;
     g.nt0 = cid * CL + rank;
     g.nt_step = ncl * CL;
+  } else if (type == P_PROJ && ncl >= 2 * g.n_tiles && g.n_tiles <= SPLIT_TILES) {
+    // few n-tiles, long K: S clusters per n-tile, each a contiguous K range
+    // split again over its CTAs; the partials are summed after the phase's
+    // cluster reduction by the last of the S clusters to arrive
+    g.S = min(ncl / g.n_tiles, SPLIT_MAX);
+    if (cid < g.n_tiles * g.S) {
+      g.split = cid / g.n_tiles;
+      g.nt0 = cid % g.n_tiles;
+    } else {
+      g.nt0 = g.n_tiles;  // no work in this phase
+    }
+    g.nt_step = g.n_tiles;
+    const int s0 = g.split * g.kb_total / g.S, s1 = (g.split + 1) * g.kb_total / g.S;
+    const int kbs = (s1 - s0 + CL - 1) / CL;
+    g.kb0 = s0 + rank * kbs;
+    g.nkb = max(0, min(kbs, s1 - g.kb0));
   } else {
     const int kbs = (g.kb_total + CL - 1) / CL;
     g.kb0 = rank * kbs;
@@ -1005,6 +1028,46 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           epi_sync();
           if (e < CL) mbar_arrive_remote(s.red_free, e);
           rounds++;
+          if (g.S > 1) {
+            // K split over S clusters: publish this cluster's partial of
+            // (n-tile, rank); the last of the S to arrive adds them up in
+            // split order (independent of the arrival order) and runs the
+            // epilogue, the others are done
+            constexpr int NC = NB / CL;
+            float *part = a.split_part + ((size_t)(nt * g.S + g.split) * CL + rank) * 128 * NC;
+#pragma unroll
+            for (int j = 0; j < NC; j++) part[e * NC + j] = tl[e * (NB + 1) + j];
+            epi_sync();
+            if (e == 0) {
+              unsigned old;
+              asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                           : "=r"(old)
+                           : "l"(a.split_cnt + nt * CL + rank)
+                           : "memory");
+              *s.flag = old == (unsigned)((layer + 1) * g.S - 1) ? 1 : 0;
+            }
+            epi_sync();
+            if (!*s.flag) {
+              epi_sync();  // s.flag is rewritten by the next unit
+              continue;
+            }
+            float sum[NC];
+#pragma unroll
+            for (int j = 0; j < NC; j++) sum[j] = 0.f;
+            for (int q = 0; q < g.S; q++) {
+              if (q == g.split) {
+#pragma unroll
+                for (int j = 0; j < NC; j++) sum[j] += tl[e * (NB + 1) + j];
+              } else {
+                const float *src = a.split_part + ((size_t)(nt * g.S + q) * CL + rank) * 128 * NC + e * NC;
+#pragma unroll
+                for (int j = 0; j < NC; j++) sum[j] += __ldcg(src + j);
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < NC; j++) tl[e * (NB + 1) + j] = sum[j];
+            epi_sync();
+          }
           if (b1 > b0) gemm_epilogue(a, s, type, layer, nt, tl, b0, b1, e, pre);
           epi_sync();
         }
@@ -1027,6 +1090,13 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
 }  // namespace
 
 bool make_map_bf16_k64(CUtensorMap *map, const void *ptr, int rows, int cols, int ld, int box_rows);
+
+size_t decode_step_bar_bytes() { return sizeof(unsigned long long) + sizeof(unsigned) * SPLIT_TILES * CL; }
+
+size_t decode_step_part_floats(int num_sms) {
+  // n_tiles * S <= clusters; each (tile, split, rank) holds 128 rows x NB/CL columns
+  return (size_t)(num_sms / CL + 1) * CL * 128 * (NB / CL);
+}
 
 bool decode_step_supported(const nc_config &c, int B) {
   return decode_fast_supported(c, B) && c.n_head <= 16 && c.d_model / 128 <= SSN;
@@ -1089,7 +1159,7 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
                           const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
                           float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
                           const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          int grid, cudaStream_t s) {
+                          float *split_part, int grid, cudaStream_t s) {
   const nc_config &c = m->cfg;
   StepArgs a;
   a.L = c.depth;
@@ -1125,9 +1195,11 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
   a.cand_v = cand_v;
   a.cand_i = cand_i;
   a.bar = bar;
+  a.split_cnt = reinterpret_cast<unsigned *>(bar + 1);
+  a.split_part = split_part;
   a.status = m->status;
-  // grid-barrier counter from zero for every step
-  cudaError_t e = cudaMemsetAsync(bar, 0, sizeof(unsigned long long), s);
+  // grid-barrier counter and split counters from zero for every step
+  cudaError_t e = cudaMemsetAsync(bar, 0, decode_step_bar_bytes(), s);
   if (e != cudaSuccess) return e;
   count_launch();
   decode_step_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(a);
