@@ -992,38 +992,45 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
             head_epilogue(a, s, nt, r, tl, n, e);
             continue;
           }
-          // cluster reduction over the K split: each CTA finishes NB/CL columns
+          // cluster reduction over the K split: each CTA finishes NB/CL batch
+          // columns. Every CTA pushes the columns rank q finishes straight into
+          // q's inbox (red, laid out [source rank][row][NB/CL]) and arrives on
+          // q's red_full; q then adds its inbox up from local shared memory.
+          // (red_free: every destination has read its inbox of the last round.)
+          constexpr int NC = NB / CL;
           if (!mbar_wait_cluster(s.red_free, (rounds & 1) ^ 1, s.abort_flag, a.status)) { ok = false; break; }
 #pragma unroll
-          for (int j = 0; j < NB; j++) red[n * NB + j] = __uint_as_float(r[j]);
+          for (int q = 0; q < CL; q++) {
+            float4 *dst = reinterpret_cast<float4 *>(cluster.map_shared_rank(red, q) + (rank * 128 + n) * NC);
+#pragma unroll
+            for (int j4 = 0; j4 < NC / 4; j4++)
+              dst[j4] = make_float4(__uint_as_float(r[q * NC + 4 * j4]), __uint_as_float(r[q * NC + 4 * j4 + 1]),
+                                    __uint_as_float(r[q * NC + 4 * j4 + 2]), __uint_as_float(r[q * NC + 4 * j4 + 3]));
+          }
           epi_sync();
           if (e < CL) mbar_arrive_remote(s.red_full, e);
-          const int b0 = rank * (NB / CL), b1 = min(a.B, b0 + NB / CL);
+          const int b0 = rank * NC, b1 = min(a.B, b0 + NC);
           EpiPre pre;
           epi_preload(a, s, type, nt, b0, b1, e, pre);
           if (!mbar_wait_cluster(s.red_full, rounds & 1, s.abort_flag, a.status)) { ok = false; break; }
           {
-            float pv[CL][NB / CL];
+            float sum[NC];
+#pragma unroll
+            for (int j = 0; j < NC; j++) sum[j] = 0.f;
 #pragma unroll
             for (int q = 0; q < CL; q++) {
-              const float4 *src =
-                  reinterpret_cast<const float4 *>(cluster.map_shared_rank(red, q) + e * NB + rank * (NB / CL));
+              const float4 *src = reinterpret_cast<const float4 *>(red + (q * 128 + e) * NC);
 #pragma unroll
-              for (int j4 = 0; j4 < NB / CL / 4; j4++) {
+              for (int j4 = 0; j4 < NC / 4; j4++) {
                 const float4 v4 = src[j4];
-                pv[q][4 * j4 + 0] = v4.x;
-                pv[q][4 * j4 + 1] = v4.y;
-                pv[q][4 * j4 + 2] = v4.z;
-                pv[q][4 * j4 + 3] = v4.w;
+                sum[4 * j4 + 0] += v4.x;
+                sum[4 * j4 + 1] += v4.y;
+                sum[4 * j4 + 2] += v4.z;
+                sum[4 * j4 + 3] += v4.w;
               }
             }
 #pragma unroll
-            for (int j = 0; j < NB / CL; j++) {
-              float sum = 0.f;
-#pragma unroll
-              for (int q = 0; q < CL; q++) sum += pv[q][j];
-              tl[e * (NB + 1) + j] = sum;
-            }
+            for (int j = 0; j < NC; j++) tl[e * (NB + 1) + j] = sum[j];
           }
           epi_sync();
           if (e < CL) mbar_arrive_remote(s.red_free, e);
@@ -1033,7 +1040,6 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
             // (n-tile, rank); the last of the S to arrive adds them up in
             // split order (independent of the arrival order) and runs the
             // epilogue, the others are done
-            constexpr int NC = NB / CL;
             float *part = a.split_part + ((size_t)(nt * g.S + g.split) * CL + rank) * 128 * NC;
 #pragma unroll
             for (int j = 0; j < NC; j++) part[e * NC + j] = tl[e * (NB + 1) + j];
