@@ -742,9 +742,11 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
       }
     }
     epi_sync();
-    // this CTA's state -> its red buffer, then the cluster merge
+    // this CTA's state (m, l, O per head row) is pushed into the inbox of the
+    // rank that finishes that head (head h -> rank h % CL, inbox laid out
+    // [source rank][h / CL][130]); the owner merges its inbox locally
     if (!mbar_wait_cluster(s.red_free, (rounds & 1) ^ 1, s.abort_flag, a.status)) return false;
-    for (int idx = e; idx < 16 * 128; idx += 128) {
+    for (int idx = e; idx < a.H * 128; idx += 128) {
       const int row = idx >> 7, col = idx & 127;
       float M = -INFINITY;
 #pragma unroll
@@ -757,23 +759,25 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
         Ls += f * cw[w * 16 * 130 + row * 130 + 1];
         O += f * cw[w * 16 * 130 + row * 130 + 2 + col];
       }
-      red[row * 130 + 2 + col] = O;
+      float *dst = cluster.map_shared_rank(red, row % CL) + (rank * (16 / CL) + row / CL) * 130;
+      dst[2 + col] = O;
       if (col == 0) {
-        red[row * 130 + 0] = M;
-        red[row * 130 + 1] = Ls;
+        dst[0] = M;
+        dst[1] = Ls;
       }
     }
     epi_sync();
     if (e < CL) mbar_arrive_remote(s.red_full, e);
     if (!mbar_wait_cluster(s.red_full, rounds & 1, s.abort_flag, a.status)) return false;
     for (int h = rank; h < a.H; h += CL) {
+      const int slot = h / CL;
       float M = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < CL; q++) M = fmaxf(M, cluster.map_shared_rank(red, q)[h * 130]);
+      for (int q = 0; q < CL; q++) M = fmaxf(M, red[(q * (16 / CL) + slot) * 130]);
       float Ls = 0.f, O = 0.f;
 #pragma unroll
       for (int q = 0; q < CL; q++) {
-        const float *pr = cluster.map_shared_rank(red, q) + h * 130;
+        const float *pr = red + (q * (16 / CL) + slot) * 130;
         const float f = pr[0] == -INFINITY ? 0.f : exp2f(pr[0] - M);
         Ls += f * pr[1];
         O += f * pr[2 + e];
