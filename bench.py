@@ -87,6 +87,13 @@ def load_peaks():
 GEMM_DRAM_BYTES_PER_LAUNCH = (54_963_200 + 196_754_176 + 166_150_400 + 388_773_632) / 4
 
 
+# DRAM bytes of one whole-step decode launch (d20, 32 sequences at context
+# 2051): dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of
+# `python bench.py --only decode --decode-steps 4 --warmup 3` with
+# -k regex:decode_step -s 3 -c 1. To be re-taken whenever nc_step.cu changes.
+DECODE_STEP_DRAM_BYTES = 1_528_550_000 + 10_848_768
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -439,7 +446,7 @@ def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local):
         "config": {"workload": "d20_decode: 32 sequences prefilled to 2048 Zipf tokens, 128 greedy steps "
                                "(positions 2048..2175), CUDA-graph replay", "batch": B, "ctx": [T, T + S]},
         "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": DECODE_STEP_DRAM_BYTES,
                      "bytes_per_step": by["total"], "peak_source": f"{peaks_src} hbm_gbs"},
         "kernel_rooflines_profiled": {
             "note": "event-timed pass without the graph; ms per step per class",
@@ -558,8 +565,8 @@ def run_decode_workload(args):
         "config": {"workload": args.workload, "batch": B, "prompt": T, "decode_steps": S,
                    "fork": w.fork, "gumbel_noise": bool(w.fork)},
         "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": by["total"],
-                     "peak_source": f"{peaks_src} hbm_gbs"},
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "bytes_per_step": by["total"], "peak_source": f"{peaks_src} hbm_gbs"},
         "gpu_launches": int(launches), "clocks": clk, **extra,
     }
     if rank == 0:
