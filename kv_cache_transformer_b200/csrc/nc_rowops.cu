@@ -3,9 +3,11 @@
 //
 //   rows_norm_bf16     h = bf16(x / sqrt(mean(x^2) + eps)), one warp per row,
 //                      16-byte loads / 8-byte stores
-//   rope_qk_bf16       one warp per (row, head): RoPE on split-half pairs,
-//                      RMS norm of every q head and the k head, q out, k and
-//                      v appended to the row's sequence in the cache
+//   rope_qk_bf16       one warp per row: RoPE on split-half pairs, RMS norm
+//                      of every q head and the k head, q out, k and v
+//                      appended to the row's sequence in the cache (the
+//                      unfused prefill path; the fused one does this in the
+//                      QKV GEMM epilogue)
 //   gather_rows_ss     copy selected rows of x (the last position of each
 //                      prompt) and their per-128-column sums of squares, the
 //                      input the fused lm_head + softcap + argmax kernel of

@@ -6,20 +6,28 @@
 // cache once) take ~0.24 ms on a B200. Launching each link as its own kernel
 // costs more than the bytes. Here one kernel runs the whole step:
 //
-//  * 148 CTAs (one per SM) in clusters of CL = 4, one phase per link,
-//    separated by a grid barrier (global counter, bounded spin);
+//  * as many 4-CTA clusters as the occupancy query places (33 on a B200:
+//    132 CTAs, one per SM), one phase per link, separated by a grid barrier
+//    (a counter zeroed before each launch, release increments, acquire
+//    polling, bounded);
 //  * warp 0 is a TMA producer that walks the same phase program as everyone
 //    and streams every weight tile and KV-cache tile this CTA will need into
 //    a 6-slot shared-memory ring, running ahead across phase barriers —
 //    neither weights nor the cached keys depend on the step's activations
 //    (the one new key per sequence is patched in from global memory);
 //  * warp 1 issues the tensor-core work of linear layers: swap-AB tcgen05
-//    MMA, M = 128 weight rows, N = 32 batch columns, fp32 in TMEM;
-//  * warps 2-5 stage the normalised activations, read the accumulators and
-//    run the epilogues and the attention; the four CTAs of a cluster split
-//    K (linears) or the keys (attention) and reduce their partial results
-//    through distributed shared memory, each CTA finishing a quarter of the
-//    batch columns (linears) or of the heads (attention).
+//    MMA, M = 128 weight rows, N = 32 batch columns, fp32 in TMEM, two
+//    accumulator sets so a CTA's next weight tile overlaps the current one's
+//    reduction and epilogue;
+//  * warps 2-5 stage the activations (once per phase: every weight tile of a
+//    phase multiplies the same slice), read the accumulators and run the
+//    epilogues and the attention. The four CTAs of a cluster split K
+//    (linears) or the keys (attention); each CTA pushes the batch columns
+//    (linears) or heads (attention) another CTA finishes straight into that
+//    CTA's shared-memory inbox, so the finishing CTA reduces locally. The MLP
+//    projection, with few weight tiles and a long K, also splits K over
+//    several clusters per tile; the last cluster to arrive adds the partials
+//    in split order.
 //
 // Phases: EMBED | depth x [QKV | ATTN | OPROJ | FC | PROJ] | HEAD | MERGE.
 //   EMBED  validate positions, x0 = rmsnorm(wte[token]), sum of squares
