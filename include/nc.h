@@ -27,6 +27,18 @@
  *  - The library owns the weights, KV caches and workspaces it allocates;
  *    calls on one model/cache must not overlap on different streams.
  *  - Only one GPU is used: the device current when the model is created.
+ *  - A call whose shapes take one of the sm_100a kernels returns NC_ECUDA if
+ *    that kernel fails to launch; the work is never retried on another
+ *    kernel.
+ *
+ * Numerics. fp32 models compute in fp32 throughout. bf16 models keep the
+ * weights, the activations fed to each matrix product and the KV cache in
+ * bf16, and accumulate, keep the residual stream and produce logits in fp32.
+ * On the sm_100a prefill path, an RMS norm followed by a linear layer is
+ * evaluated as (bf16(x) . W) * (1 / rms(x)) rather than bf16(x / rms(x)) . W.
+ * Both round each input once, so the error is of the same size; the
+ * results differ in the last bf16 bits. The QK-norm factor is taken before
+ * RoPE, which keeps each pair's sum of squares.
  */
 #ifndef NC_H
 #define NC_H
