@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "d20 bf16 prefill tok/s & decode tok/s (B=32); % of HBM / tensor-core roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16, the vendor's figure
+NOMINAL_HBM_GBS = 8000.0
 
 
 # ------------------------------------------------------------ accounting
@@ -183,14 +185,22 @@ def barrier(world: int):
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_prefill_sample(cfg, blob, prompts, n_tokens: int):
-    """Time the oracle's prefill of the first n_tokens of prompt 0; -> (tok/s, seconds, threads)."""
+def oracle_prefill_sample(cfg, blob, prompts, n_tokens: int, threads: int | None = None):
+    """Time the oracle's prefill of the first n_tokens of prompt 0 on `threads`
+    host threads (all by default); -> (tok/s, seconds, threads used)."""
     import oracle as orc
-    om = orc.OracleModel(cfg, blob)
-    t0 = time.perf_counter()
-    om.forward_full(prompts[0, :n_tokens], all_positions=False)
-    dt = time.perf_counter() - t0
-    return n_tokens / dt, dt, orc.num_threads()
+    full = orc.num_threads()
+    if threads:
+        orc.set_threads(threads)
+    try:
+        om = orc.OracleModel(cfg, blob)
+        used = orc.num_threads()
+        t0 = time.perf_counter()
+        om.forward_full(prompts[0, :n_tokens], all_positions=False)
+        dt = time.perf_counter() - t0
+    finally:
+        orc.set_threads(full)
+    return n_tokens / dt, dt, used
 
 
 def run_reference(args):
@@ -306,11 +316,15 @@ def run_ours(args):
     gemm_ms = kms[nc.NC_K_GEMM] / args.steps  # GEMM time per step
     gemm_launch_per_step = kn[nc.NC_K_GEMM] / args.steps
     gemm_tflops = fl["gemm"] / (gemm_ms / 1e3) / 1e12
-    peak_tc = peaks["bf16_tflops_sustained"]
+    # the burst peak (cuBLAS bf16 at full clock) is the denominator; the
+    # sustained figure was measured over seconds at a lower, power-capped
+    # clock than a prefill step runs at, so it is only reported beside it
+    peak_tc = peaks["bf16_tflops"]
     roofline = {
         "bound": "tensor", "kernel": "prefill linear-layer GEMMs (QKV, O, fc relu^2, proj)",
         "achieved": gemm_tflops, "peak": peak_tc, "unit": "TFLOP/s", "frac": gemm_tflops / peak_tc,
-        "traffic": GEMM_DRAM_BYTES_PER_LAUNCH, "peak_source": f"{peaks_src} bf16_tflops_sustained",
+        "traffic": GEMM_DRAM_BYTES_PER_LAUNCH, "peak_source": f"{peaks_src} bf16_tflops (burst)",
+        "frac_of_sustained": gemm_tflops / peaks["bf16_tflops_sustained"],
         "flops_per_launch": fl["gemm"] / max(gemm_launch_per_step, 1),
         "ms_per_launch": gemm_ms / max(gemm_launch_per_step, 1),
         "launches_per_step": gemm_launch_per_step,
@@ -349,13 +363,23 @@ def run_ours(args):
     if not args.no_decode:
         decode = run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local)
 
+    # ---------------- the other decode workloads (d26 latency, d30 rollout)
+    workloads = None
+    if not args.no_workloads:
+        workloads = {name: decode_workload(name, args, world, local, peaks, peaks_src)
+                     for name in ("d26_latency", "d30_rollout")}
+
     # ---------------- CPU oracle on a bounded sample (rank 0, N = 1)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tps, secs, thr = oracle_prefill_sample(cfg, blob, prompts_np, args.ref_tokens)
+        n1 = max(8, args.ref_tokens // 8)
+        tps1, secs1, _ = oracle_prefill_sample(cfg, blob, prompts_np, n1, threads=1)
         cpu = {"value": tps, "unit": "tok/s", "cores": thr, "kind": "oracle",
                "sample": f"oracle prefill of the first {args.ref_tokens} tokens of prompt 0 "
-                         f"({secs:.1f} s on {thr} threads)"}
+                         f"({secs:.1f} s on {thr} threads)",
+               "single_core": {"value": tps1, "unit": "tok/s", "cores": 1,
+                               "sample": f"first {n1} tokens of prompt 0 ({secs1:.1f} s on 1 thread)"}}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
@@ -367,9 +391,10 @@ def run_ours(args):
                    "l2": "inputs larger than L2 (1.0 GB of weights streamed per step)"},
         "roofline": roofline,
         "step_tflops": step_tflops, "step_frac_of_peak": step_tflops / peak_tc,
+        "step_frac_of_nominal": step_tflops / NOMINAL_BF16_TFLOPS,
         "kernel_time_share": kernel_share,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches), "clocks": clk,
-        "decode": decode,
+        "decode": decode, "workloads": workloads,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -422,61 +447,88 @@ def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local):
     t_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = t_ms / S
 
-    # per-class breakdown from a separate profiled pass (events between launches,
-    # no graph), over the same positions
-    prefill()
-    model.profile(True)
-    model.profile_read()
-    for _ in range(S):
-        step()
-    kms, kn = model.profile_read()
-    model.profile(False)
-    prof_ms_step = float(kms.sum()) / S
-
     by = decode_bytes(cfg, B, T + (S + 1) / 2.0)
     gbs = by["total"] / (ms_step / 1e3) / 1e9
-    gemm_ms = kms[nc.NC_K_GEMM] / S
-    gemm_gbs = by["weights_linear"] / (gemm_ms / 1e3) / 1e9
-    attn_ms = kms[nc.NC_K_ATTN] / S
-    attn_gbs = (by["kv_read"] + by["kv_write"]) / (attn_ms / 1e3) / 1e9
-    head_ms = kms[nc.NC_K_HEAD] / S
-    head_gbs = (by["weights_head"] + by["logits"]) / (head_ms / 1e3) / 1e9
+
+    # per-phase breakdown of one step of the whole-step kernel from its
+    # timestamp trace (nc_decode_trace), at context ~2050, outside the timed loop
+    prefill()
+    for _ in range(2):
+        step()
+    trace = decode_phase_trace(kv, step, cfg.depth)
+
     return {
         "value": world * B * S / (t_ms / 1e3), "unit": "tok/s", "ms_per_step": ms_step, "steps": S,
         "config": {"workload": "d20_decode: 32 sequences prefilled to 2048 Zipf tokens, 128 greedy steps "
                                "(positions 2048..2175), CUDA-graph replay", "batch": B, "ctx": [T, T + S]},
-        "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": gbs, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": DECODE_STEP_DRAM_BYTES,
-                     "bytes_per_step": by["total"], "peak_source": f"{peaks_src} hbm_gbs"},
-        "kernel_rooflines_profiled": {
-            "note": "event-timed pass without the graph; ms per step per class",
-            "ms_per_step": prof_ms_step,
-            "gemm": {"ms": gemm_ms, "GB/s": gemm_gbs, "bytes": by["weights_linear"],
-                     "launches_per_step": float(kn[nc.NC_K_GEMM]) / S},
-            "attn": {"ms": attn_ms, "GB/s": attn_gbs, "bytes": by["kv_read"] + by["kv_write"],
-                     "launches_per_step": float(kn[nc.NC_K_ATTN]) / S},
-            "head": {"ms": head_ms, "GB/s": head_gbs, "bytes": by["weights_head"] + by["logits"],
-                     "launches_per_step": float(kn[nc.NC_K_HEAD]) / S},
-            "misc_ms": kms[nc.NC_K_MISC] / S},
+        "roofline": {"bound": "hbm", "kernel": "whole decode step (one persistent kernel per step)",
+                     "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "traffic": DECODE_STEP_DRAM_BYTES,
+                     "bytes_per_step": by["total"], "bytes": by, "peak_source": f"{peaks_src} hbm_gbs"},
+        "phase_trace": trace,
         "gpu_launches": int(launches), "clocks": clk,
     }
 
 
-def run_decode_workload(args):
+def decode_phase_trace(kv, step, depth: int):
+    """Run step() once with the step kernel's phase timestamps on and reduce
+    them to microseconds per phase type (summed over the layers): the median
+    over CTAs of each phase's span and of its parts. None when the cache has
+    no whole-step kernel."""
+    import numpy as np
+    import torch
+    grid, P = kv.trace(None)
+    if grid == 0:
+        return None
+    buf = torch.zeros(grid * P * 8, dtype=torch.int64, device="cuda")
+    kv.trace(buf)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    step()
+    e1.record()
+    torch.cuda.synchronize()
+    kv.trace(None)
+    event_us = 1e3 * e0.elapsed_time(e1)
+    tr = buf.cpu().numpy().reshape(grid, P, 8).astype(np.float64)
+    tr[tr == 0] = np.nan
+    t0 = np.nanmin(tr[:, 0, 0])
+    tr = (tr - t0) / 1e3  # us from the first phase start
+    kinds = ["embed"] + [k for _ in range(depth) for k in ("qkv", "attn", "oproj", "fc", "proj")] + ["head", "merge"]
+    start = tr[:, :, 0]
+    parts = ("stage", "first_acc", "reduce", "epilogue")
+    out = {}
+    for p, kind in enumerate(kinds):
+        rec = out.setdefault(kind, {"phases": 0, "span": 0.0, "barrier": 0.0, **{k: 0.0 for k in parts}})
+        rec["phases"] += 1
+        end = start[:, p + 1] if p + 1 < P else tr[:, p, 4]
+        rec["span"] += float(np.nanmedian(end - start[:, p]))
+        if p + 1 < P:
+            rec["barrier"] += float(np.nanmedian(start[:, p + 1] - tr[:, p, 4]))
+        for j, k in enumerate(parts):
+            d = tr[:, p, j + 1] - tr[:, p, j]
+            if np.any(np.isfinite(d)):
+                rec[k] += float(np.nanmedian(d))
+    for rec in out.values():
+        for k in list(rec):
+            if isinstance(rec[k], float):
+                rec[k] = round(rec[k], 2)
+    span = float(np.nanmax(tr[:, P - 1, 4]))
+    return {"note": "us per step by phase type, summed over layers; span = median over CTAs of a phase's "
+                    "start-to-next-start, barrier = work done to next start; parts are medians over the CTAs "
+                    "that reached them", "grid": grid, "kernel_span_us": round(span, 1),
+            "event_us": round(event_us, 1), "by_phase": out}
+
+
+def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src) -> dict:
     """d26 latency decode (B=1, 1024-token prompt, 512 greedy steps) or d30
-    rollout (256-token prompt, fork to 16 samples, 256 steps of argmax over
-    logits + Gumbel noise). One JSON line with decode tok/s and the HBM
-    roofline of a decode step."""
+    rollout (256-token prompt prefilled once, forked to 16 samples, 256 steps
+    of argmax over logits + Gumbel noise): decode tok/s over all ranks and the
+    HBM roofline of a decode step."""
     import numpy as np
     import torch
     import kv_cache_transformer_b200 as nc
     import nc_synth as syn
-    from kv_cache_transformer_b200 import build as ncbuild
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    ncbuild.build()
-    peaks, peaks_src = load_peaks()
-    w = syn.WORKLOADS[args.workload]
+    w = syn.WORKLOADS[name]
     cfg = w.model
     model = nc.Model(cfg, syn.make_blob(cfg, w.weight_seed))
     V, T, S = cfg.vocab, w.prompt_len, w.decode_steps
@@ -484,26 +536,33 @@ def run_decode_workload(args):
     prompts = torch.from_numpy(syn.prompt_tokens(w)).cuda()
     stream = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     extra = {}
+    caches = []
     if w.fork:
         n = w.fork
         src = model.kv(1, max_seq)
         dst = model.kv(n, max_seq)
+        caches = [src, dst]
         tok1 = torch.empty((1,), dtype=torch.int32, device="cuda")
         logits = torch.empty((n, V), dtype=torch.float32, device="cuda")
         tok = torch.empty((n,), dtype=torch.int32, device="cuda")
         # seeded Gumbel noise per step and sample, generated up front (an input)
         noise = torch.from_numpy(np.stack([syn.gumbel(w.noise_seed, (n, V), stream=s_) for s_ in range(S)])).cuda()
 
-        def run_once():
+        def start():
             model.prefill(src, prompts, 0, None, tok1)
             src.fork_to(0, dst, 0, n)
             tok.copy_(tok1.expand(n))
-            for s_ in range(S):
-                model.decode_step(dst, tok, None, noise[s_], logits, tok)
 
+        def step(s_):
+            model.decode_step(dst, tok, None, noise[s_], logits, tok)
+
+        B = n
         for _ in range(max(1, args.warmup // 3)):
-            run_once()
+            start()
+            for s_ in range(S):
+                step(s_)
         torch.cuda.synchronize()
         e0.record(stream)
         model.prefill(src, prompts, 0, None, tok1)
@@ -512,63 +571,72 @@ def run_decode_workload(args):
         src.fork_to(0, dst, 0, n)
         ef.record(stream)
         tok.copy_(tok1.expand(n))
-        clocks = ClockSampler(local)
         torch.cuda.synchronize()
-        clocks.start()
-        d0 = torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        n0 = nc.nc_launch_count()
-        for s_ in range(S):
-            model.decode_step(dst, tok, None, noise[s_], logits, tok)
-        d1 = torch.cuda.Event(enable_timing=True)
-        d1.record(stream)
-        torch.cuda.synchronize()
-        launches = nc.nc_launch_count() - n0
-        clk = clocks.stop()
-        assert model.status() == 0
-        B = n
         extra = {"prefill_ms": e0.elapsed_time(e1), "fork_ms": e1.elapsed_time(ef),
                  "fork_bytes": cfg.depth * 2 * T * cfg.head_dim * 2 * n}
-        ctx_avg = T + (S + 1) / 2.0
     else:
         kv = model.kv(w.batch, max_seq)
+        caches = [kv]
         B = w.batch
         logits = torch.empty((B, V), dtype=torch.float32, device="cuda")
         tok = torch.empty((B,), dtype=torch.int32, device="cuda")
-        for _ in range(max(1, args.warmup // 3)):
+
+        def start():
             model.prefill(kv, prompts, 0, logits, tok)
-            for _s in range(min(S, 16)):
-                model.decode_step(kv, tok, None, None, logits, tok)
-        model.prefill(kv, prompts, 0, logits, tok)
-        clocks = ClockSampler(local)
-        torch.cuda.synchronize()
-        clocks.start()
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        n0 = nc.nc_launch_count()
-        for _s in range(S):
+
+        def step(s_):
             model.decode_step(kv, tok, None, None, logits, tok)
-        d1.record(stream)
-        torch.cuda.synchronize()
-        launches = nc.nc_launch_count() - n0
-        clk = clocks.stop()
-        assert model.status() == 0
-        ctx_avg = T + (S + 1) / 2.0
-    t_ms = d0.elapsed_time(d1)
+
+        for _ in range(max(1, args.warmup // 3)):
+            start()
+            for s_ in range(min(S, 16)):
+                step(s_)
+        start()
+    clocks = ClockSampler(local)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.start()
+    n0 = nc.nc_launch_count()
+    d0.record(stream)
+    for s_ in range(S):
+        step(s_)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    launches = nc.nc_launch_count() - n0
+    clk = clocks.stop()
+    assert model.status() == 0
+    barrier(world)
+    t_ms = max_over_ranks(d0.elapsed_time(d1), world)
+    ctx_avg = T + (S + 1) / 2.0
     by = decode_bytes(cfg, B, ctx_avg)
     ms_step = t_ms / S
     gbs = by["total"] / (ms_step / 1e3) / 1e9
-    line = {
-        "metric": f"{args.workload} bf16 decode tok/s; % of HBM roofline", "value": B * S / (t_ms / 1e3),
-        "unit": "tok/s", "n_gpus": 1, "steps": S, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "batch": B, "prompt": T, "decode_steps": S,
-                   "fork": w.fork, "gumbel_noise": bool(w.fork)},
+    for c in caches:
+        c.close()
+    model.close()
+    return {
+        "metric": f"{name} bf16 decode tok/s; % of HBM roofline", "value": world * B * S / (t_ms / 1e3),
+        "unit": "tok/s", "n_gpus": world, "steps": S, "ms_per_step": ms_step, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": name, "batch": B, "prompt": T, "decode_steps": S, "fork": w.fork,
+                   "gumbel_noise": bool(w.fork)},
         "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                      "bytes_per_step": by["total"], "peak_source": f"{peaks_src} hbm_gbs"},
         "gpu_launches": int(launches), "clocks": clk, **extra,
     }
+
+
+def run_decode_workload(args):
+    """One JSON line for --workload d26_latency | d30_rollout."""
+    import torch
+    from kv_cache_transformer_b200 import build as ncbuild
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    ncbuild.build()
+    peaks, peaks_src = load_peaks()
+    line = decode_workload(args.workload, args, 1, local, peaks, peaks_src)
+    line["warmup"] = args.warmup
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -587,6 +655,7 @@ def main():
                     help="d20: the headline prefill + decode line; d26_latency / d30_rollout: the other "
                          "decode workloads, one JSON line each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the d26 latency and d30 rollout lines")
     ap.add_argument("--ref-tokens", type=int, default=128,
                     help="tokens of one prompt the CPU oracle runs per sample")
     args = ap.parse_args()

@@ -109,7 +109,11 @@ int nc_device_status(nc_model *model, uint32_t *out_bits);
  * plus the workspace prefill/decode need (sized for max_batch*max_seq
  * prefill rows). Layout per layer: K and V [max_batch][max_seq][Hkv*hd] of
  * the model's dtype, K stored after RoPE and QK norm. All lengths start at
- * 0. Errors: NC_EINVAL, NC_ENOMEM, NC_ECUDA. */
+ * 0. A bf16 decode step of up to 32 sequences runs as one persistent kernel
+ * (NC_K_STEP); with the environment variable NC_DECODE_STEP_KERNEL=0 set
+ * when the cache is created, it runs as one launch per layer step instead
+ * (a diagnostic switch: same results within the stated tolerances).
+ * Errors: NC_EINVAL, NC_ENOMEM, NC_ECUDA. */
 int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out);
 
 /* Free a cache (waits for the device). NULL is ignored. */
@@ -171,6 +175,23 @@ int nc_profile_enable(nc_model *model, int on);
  * last read; then resets them. Synchronises the device. Either output may be
  * NULL. */
 int nc_profile_read(nc_model *model, double *ms, long long *launches);
+
+/* Phase timestamps of the whole-step decode kernel (NC_K_STEP). With d_buf
+ * non-NULL, every later nc_decode_step on `kv` that runs that kernel writes,
+ * for each CTA c and phase p, eight %globaltimer readings (ns) to
+ * d_buf[(c * phases + p) * 8 + slot]: slot 0 phase start (after the previous
+ * grid barrier), 1 inputs staged (linear phases) or first cache tile in
+ * (attention), 2 first accumulator complete (linear) or keys done
+ * (attention), 3 cluster reduction / merge done, 4 phase work done (barrier
+ * entry), 5 and 6 the TMA producer's first and last load of the phase, 7 the
+ * MMA issuer's last commit of the phase. Slots a CTA does not reach in a
+ * phase keep their old contents (clear the buffer first). Phases are EMBED,
+ * then per layer QKV, ATTN, O-proj, MLP fc, MLP proj, then HEAD and MERGE.
+ * d_buf = NULL turns tracing off. *grid and *phases (host, may be NULL)
+ * receive the kernel's CTA count and phase count; d_buf needs grid * phases
+ * * 8 words. Errors: NC_EINVAL, NC_EUNSUP (no step kernel on this cache),
+ * NC_ERANGE (buffer too small). */
+int nc_decode_trace(nc_kv *kv, unsigned long long *d_buf, size_t n_words, int *grid, int *phases);
 
 /* Number of kernels this library has launched in this process so far
  * (a CUDA graph replay counts each of its kernel nodes). */

@@ -68,8 +68,10 @@ int nc_attention_decode_bf16(const void *d_q, const void *d_k, const void *d_v, 
  * every GPU that loads the library until the process exits); no call
  * allocates or frees device memory. Limits: B <= 32, H <= 16, and max_seq
  * small enough for 16 key splits (the split rule grows the chunk to fit).
- * The first call on each device looks up the array's device address, so
- * make that first call before any stream capture. All calls share the one
+ * Every call looks up the array's device address on the current device
+ * (a host-side query), so a device reset in between is harmless; the first
+ * call on a device also loads the library's code there, so make that first
+ * call before any stream capture. All calls share the one
  * array: calls that overlap on the GPU (other streams, other threads) race
  * and must be serialised by the caller. Errors: NC_EINVAL (null pointer, bad
  * shape, B or max_seq beyond the limits), NC_ECUDA. */

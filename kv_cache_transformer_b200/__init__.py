@@ -35,7 +35,7 @@ EXPORTS = (
     "nc_kv_lengths", "nc_prefill", "nc_decode_step", "nc_kv_fork", "nc_last_error",
     "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
     "nc_attention_prefill_bf16", "nc_attention_decode_workspace_bytes", "nc_attention_decode_bf16",
-    "nc_attention_decode_bf16_static",
+    "nc_attention_decode_bf16_static", "nc_decode_trace",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_STEP, NC_K_COUNT = 0, 1, 2, 3, 4, 5
@@ -90,6 +90,7 @@ def lib() -> ctypes.CDLL:
             L.nc_attention_decode_workspace_bytes.restype = ctypes.c_size_t
             L.nc_attention_decode_bf16.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp, sz, vp]
             L.nc_attention_decode_bf16_static.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp]
+            L.nc_decode_trace.argtypes = [vp, vp, sz, ctypes.POINTER(i), ctypes.POINTER(i)]
             for name in EXPORTS:
                 if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error", "nc_launch_count",
                                 "nc_attention_decode_workspace_bytes"):
@@ -201,6 +202,18 @@ def nc_decode_step(model_h, kv_h, tokens, positions, noise=None, logits=None, ne
 
 def nc_kv_fork(src_h, src_seq: int, dst_h, dst_first: int, n: int, stream=None):
     _check(lib().nc_kv_fork(src_h, int(src_seq), dst_h, int(dst_first), int(n), _stream(stream)))
+
+
+def nc_decode_trace(kv_h, buf=None):
+    """Point the whole-step decode kernel's phase timestamps at `buf` (a CUDA
+    int64 tensor of at least grid * phases * 8 elements), or turn them off
+    (buf=None). -> (grid, phases)."""
+    import torch
+    g, p = ctypes.c_int(), ctypes.c_int()
+    ptr = None if buf is None else _dptr(buf, torch.int64, name="trace buffer")
+    n = 0 if buf is None else buf.numel()
+    _check(lib().nc_decode_trace(kv_h, ptr, n, ctypes.byref(g), ctypes.byref(p)))
+    return g.value, p.value
 
 
 def nc_profile_enable(model_h, on: bool = True):
@@ -343,3 +356,7 @@ class KVCache:
 
     def fork_to(self, src_seq: int, dst: "KVCache", dst_first: int, n: int, stream=None):
         nc_kv_fork(self._h, src_seq, dst.handle, dst_first, n, stream)
+
+    def trace(self, buf=None):
+        """Phase timestamps of later decode steps into `buf` (see nc_decode_trace)."""
+        return nc_decode_trace(self._h, buf)

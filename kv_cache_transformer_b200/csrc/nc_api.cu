@@ -1,11 +1,15 @@
 // nc_api.cu — the C ABI (include/nc.h): objects, argument checks, and the
 // prefill / decode / fork call sequences over the engine's kernels.
 #include <math.h>
+#include <stdlib.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
 
+#include <map>
+#include <mutex>
 #include <string>
+#include <utility>
 
 #include "nc_internal.h"
 #include "nc_kernels.h"
@@ -251,7 +255,8 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
     ProfScope p(m, NC_K_STEP, s);
     return nc::k_decode_step(m, B, kv->max_batch, kv->max_seq, kv->step_maps, tokens, positions, kv->len, kv->x,
                              kv->xl, kv->step_ss, kv->q, kv->y, kv->f, kv->k, kv->v, kv->rope, logits, noise, next,
-                             kv->cand_v, kv->cand_i, kv->step_bar, kv->step_part, kv->step_grid, s);
+                             kv->cand_v, kv->cand_i, kv->step_bar, kv->step_part, kv->step_grid, kv->step_trace,
+                             s);
   }
   {
     ProfScope p(m, NC_K_MISC, s);
@@ -366,6 +371,20 @@ int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *po
 namespace nc {
 // Record a message for nc_last_error() from other translation units.
 int set_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
+cudaError_t ensure_smem_attr(const void *func, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, size_t> done;
+  std::lock_guard<std::mutex> lock(mu);
+  size_t &have = done[std::make_pair(func, dev)];
+  if (bytes <= have) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
 }  // namespace nc
 
 extern "C" {
@@ -501,6 +520,8 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
       if (e == cudaSuccess && nc::decode_step_build_maps(model, kv->k, kv->v, max_batch, max_seq, maps.data())) {
         e = cudaMemcpy(kv->step_maps, maps.data(), sizeof(CUtensorMap) * nmaps, cudaMemcpyHostToDevice);
         if (e == cudaSuccess) kv->step_grid = nc::decode_step_grid(model->num_sms);
+        const char *sw = getenv("NC_DECODE_STEP_KERNEL");
+        if (sw && sw[0] == '0') kv->step_grid = 0;  // per-kernel decode launches instead
       }
     }
   }
@@ -667,6 +688,24 @@ int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *
                 dst->v, dst->layer_elems, dst->max_seq, dst_first, n, dst->len, c.depth, c.n_kv_head * c.head_dim,
                 src->model->status, as_stream(stream));
   NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+int nc_decode_trace(nc_kv *kv, unsigned long long *d_buf, size_t n_words, int *grid, int *phases) {
+  if (!kv) return fail(NC_EINVAL, "kv is NULL");
+  const nc_config &c = kv->model->cfg;
+  const int g = kv->step_grid, P = 3 + 5 * c.depth;
+  if (grid) *grid = g;
+  if (phases) *phases = P;
+  if (d_buf && g == 0) return fail(NC_EUNSUP, "this cache has no whole-step decode kernel to trace");
+  if (d_buf && n_words < (size_t)g * P * 8)
+    return fail(NC_ERANGE, "trace buffer holds %zu words, the step kernel writes %zu", n_words, (size_t)g * P * 8);
+  kv->step_trace = d_buf;
+  if (kv->graph) {  // the captured launch carries the old trace pointer
+    cudaGraphExecDestroy(kv->graph);
+    kv->graph = nullptr;
+  }
+  kv->graph_ready = false;
   return NC_OK;
 }
 

@@ -437,11 +437,9 @@ cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int
       !make_map_bf16_k64(&mk, kc, max_batch * max_seq, HD, HD, BKV) ||
       !make_map_bf16_k64(&mv, vc, max_batch * max_seq, HD, HD, BKV))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  {
+    const cudaError_t e = ensure_smem_attr((const void *)attn_prefill_tc_kernel, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   AttnArgs a;
   a.T = T;

@@ -713,12 +713,9 @@ void plan_split(int n_tiles, int kblocks, int num_sms, int &splits, int &kbs) {
 template <int NB, int SRC, int EPI>
 cudaError_t launch_dec_linear_t(const CUtensorMap &map, DecLinArgs &a, int num_sms, cudaStream_t s) {
   size_t smem = dec_linear_smem<NB>(a.kbs);
-  static size_t attr_set = 0;
-  if (smem > attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(dec_linear_kernel<NB, SRC, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  {
+    const cudaError_t e = ensure_smem_attr((const void *)dec_linear_kernel<NB, SRC, EPI>, smem);
     if (e != cudaSuccess) return e;
-    attr_set = smem;
   }
   int per_sm = smem * 2 + 2048 <= 227 * 1024 ? 2 : 1;
   int grid = a.units < per_sm * num_sms ? a.units : per_sm * num_sms;
@@ -849,11 +846,9 @@ cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int3
   a.counters = counters;
   a.y = (bf16 *)y;
   const size_t smem = 4 * ATILE;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(dec_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    const cudaError_t e = ensure_smem_attr((const void *)dec_attn_kernel, smem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   return launch_pdl(dec_attn_kernel, dim3(splits, B), dim3(ATHREADS), smem, s, a);
 }

@@ -455,11 +455,9 @@ bool gemm_tc_supported(int M, int N, int K, int lda) {
 template <int EPI>
 static cudaError_t launch_tc(const CUtensorMap &ma, const CUtensorMap &mw, const GemmArgs &g, int grid,
                              cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  {
+    const cudaError_t e = ensure_smem_attr((const void *)gemm_tc_kernel<EPI>, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   count_launch();
   gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ma, mw, g);

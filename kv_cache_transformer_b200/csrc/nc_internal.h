@@ -75,6 +75,7 @@ struct nc_kv {
   unsigned long long *step_bar = nullptr;  // its grid-barrier counter and split counters
   float *step_part = nullptr;  // split-K partials of its MLP proj phase
   float *step_ss = nullptr;    // [2*depth+1][16][32] per-128-column sums of squares
+  unsigned long long *step_trace = nullptr;  // caller's phase-timestamp buffer (nc_decode_trace), or null
   int attn_chunk = 0, attn_splits = 0;
   // CUDA graph of the last decode step's launches, replayed while the call's
   // pointers and batch stay the same
@@ -92,6 +93,11 @@ namespace nc {
 
 // Set the message returned by nc_last_error(); returns code.
 int set_error(int code, const char *msg);
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the
+// current device. The attribute is per device, so it is tracked per (kernel,
+// device); thread-safe.
+cudaError_t ensure_smem_attr(const void *func, size_t bytes);
 
 // Kernels launched by this library (nc_launch_count).
 extern std::atomic<unsigned long long> g_launches;
@@ -194,7 +200,7 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
                           const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
                           float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
                           const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          float *split_part, int grid, cudaStream_t s);
+                          float *split_part, int grid, unsigned long long *trace, cudaStream_t s);
 size_t decode_step_bar_bytes();              // grid-barrier word + split counters, zeroed per launch
 size_t decode_step_part_floats(int num_sms);  // split-K partials of the MLP proj phase
 

@@ -11,8 +11,6 @@
 // and no call here allocates or frees device memory.
 #include <stdio.h>
 
-#include <mutex>
-
 #include "nc_internal.h"
 #include "nc_kernels.h"
 
@@ -25,30 +23,21 @@ constexpr size_t kPartFloats = (size_t)kStaticMaxBatch * kStaticMaxSplits * 16 *
 // Split-KV partials (m, l, O per head row), then one counter per sequence.
 static __device__ __align__(256) float g_decode_scratch[kPartFloats + kStaticMaxBatch];
 
-constexpr int kMaxDevices = 64;
-void *g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Device address of g_decode_scratch on the current device, looked up once
-// per device. In host code the array's name is only a host-side handle, so
-// the kernel must be given this address instead.
+// Device address of g_decode_scratch on the current device. In host code the
+// array's name is only a host-side handle, so the kernel must be given this
+// address instead. It is looked up on every call (a host-side query, cheap):
+// a cached address would dangle after cudaDeviceReset unloads the module.
+// The first lookup on a device loads the library's module there, which is
+// why the first call on each device belongs before any stream capture.
 int scratch_address(void **out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return nc::set_error(NC_ECUDA, cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return nc::set_error(NC_EINVAL, "device ordinal beyond the static scratch table");
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || !p) {
-      char msg[160];
-      snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
-      return nc::set_error(NC_ECUDA, msg);
-    }
-    g_scratch_addr[dev] = p;
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || !p) {
+    char msg[160];
+    snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    return nc::set_error(NC_ECUDA, msg);
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return NC_OK;
 }
 

@@ -97,7 +97,17 @@ struct StepArgs {
   unsigned *split_cnt;        // [SPLIT_TILES][CL]: arrivals of the K-split MLP proj partials
   float *split_part;          // [n_tiles * S][CL][128][NB/CL]: their partial sums
   uint32_t *status;
+  unsigned long long *trace;  // [grid][phases][8] phase timestamps (ns), or null
 };
+
+// Phase timestamps for nc_decode_trace: slot 0 phase start (after the last
+// barrier), 1 activations staged / first cache tile in, 2 first accumulator
+// complete, 3 last cluster reduction done, 4 epilogue done (barrier entry),
+// 5 producer's first load of the phase, 6 its last load, 7 the MMA issuer's
+// last commit of the phase. Only written when a trace buffer is set.
+__device__ __forceinline__ void trace_mark(const StepArgs &a, int p, int slot) {
+  if (a.trace) a.trace[((size_t)blockIdx.x * (3 + 5 * a.L) + p) * 8 + slot] = global_ns();
+}
 
 struct Smem {
   uint64_t *full, *empty, *x_ready, *x_free, *red_full, *red_free;
@@ -293,13 +303,17 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int ci
     phase_of(a, p, type, layer);
     if (type == P_QKV || type == P_OPROJ || type == P_FC || type == P_PROJ || type == P_HEAD) {
       const Gemm g = gemm_of(a, type, layer, cid, ncl, rank);
+      bool first = true;
       for (int nt = g.nt0; nt < g.n_tiles; nt += g.nt_step)
         for (int kb = g.kb0; kb < g.kb0 + g.nkb; kb++) {
           uint32_t slot;
           if (!take(slot)) return;
+          if (first) trace_mark(a, p, 5);
+          first = false;
           mbar_arrive_expect_tx(&s.full[slot], SLOT);
           tma_load_2d(ring + slot * SLOT, g.map, kb * 64, nt * 128, &s.full[slot]);
         }
+      trace_mark(a, p, 6);
     } else if (type == P_ATTN) {
       for (int b = cid; b < a.B; b += ncl) {
         if (!s.valid[b]) continue;
@@ -310,12 +324,14 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int ci
           for (int which = 0; which < 2; which++) {
             uint32_t slot;
             if (!take(slot)) return;
+            if (key == k0 && which == 0 && b == cid) trace_mark(a, p, 5);
             mbar_arrive_expect_tx(&s.full[slot], SLOT);
             uint8_t *dst = ring + slot * SLOT;
             tma_load_2d(dst, a.kvmaps + which, 0, row0 + key, &s.full[slot]);
             tma_load_2d(dst + 8192, a.kvmaps + which, 64, row0 + key, &s.full[slot]);
           }
       }
+      trace_mark(a, p, 6);
     }
   }
 }
@@ -385,6 +401,7 @@ __device__ void mma_issuer(const StepArgs &a, const Smem &s, uint8_t *ring, uint
         mma_commit(&s.acc_full[set]);
       }
       if (single) mma_commit(s.x_free);  // X is free once every unit's MMAs are done
+      trace_mark(a, p, 7);
     } else if (type == P_ATTN) {
       // the compute warps consume this phase's ring slots; keep the count
       for (int b = cid; b < a.B; b += ncl) {
@@ -651,6 +668,7 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
       t++;
       if (!mbar_wait(&s.full[ks_], kph, s.abort_flag, a.status)) return false;
       if (!mbar_wait(&s.full[vs_], vph, s.abort_flag, a.status)) return false;
+      if (e == 0 && b == cid && key0 == k0) trace_mark(a, 2 + 5 * layer, 1);
       uint8_t *K = ring + ks_ * SLOT, *V = ring + vs_ * SLOT;
       // the key/value written by this step's QKV phase may postdate the
       // prefetch: copy that row from the cache
@@ -728,6 +746,7 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
         mbar_arrive(&s.empty[vs_]);
       }
     }
+    if (e == 0 && b == cid) trace_mark(a, 2 + 5 * layer, 2);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -777,6 +796,7 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
     epi_sync();
     if (e < CL) mbar_arrive_remote(s.red_full, e);
     if (!mbar_wait_cluster(s.red_full, rounds & 1, s.abort_flag, a.status)) return false;
+    if (e == 0) trace_mark(a, 2 + 5 * layer, 3);
     for (int h = rank; h < a.H; h += CL) {
       const int slot = h / CL;
       float M = -INFINITY;
@@ -884,6 +904,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     for (int p = 0; p < P && ok; p++) {
       int type, layer;
       phase_of(a, p, type, layer);
+      if (e == 0) trace_mark(a, p, 0);
       if (type == P_EMBED) {
         for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
           int tok = a.tokens[b];
@@ -953,7 +974,10 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           }
           if (ok && g.nkb > 0) stage_x(a, s, xs, type, g.kb0, g.nkb, e);
           epi_sync();
-          if (e == 0) mbar_arrive(s.x_ready);
+          if (e == 0) {
+            mbar_arrive(s.x_ready);
+            trace_mark(a, p, 1);
+          }
           x_pending = true;
         }
         for (int nt = g.nt0; nt < g.n_tiles && ok; nt += g.nt_step, units++) {
@@ -982,6 +1006,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           const uint32_t set = units & 1;
           if (!mbar_wait(&s.acc_full[set], (units >> 1) & 1, s.abort_flag, a.status)) { ok = false; break; }
           tc_fence_after();
+          if (e == 0 && nt == g.nt0) trace_mark(a, p, 2);
           const uint32_t tacc = tmem + set * (uint32_t)(NACC * NB) + lane_off;
           uint32_t r[NB];
           {
@@ -1025,6 +1050,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           EpiPre pre;
           epi_preload(a, s, type, nt, b0, b1, e, pre);
           if (!mbar_wait_cluster(s.red_full, rounds & 1, s.abort_flag, a.status)) { ok = false; break; }
+          if (e == 0) trace_mark(a, p, 3);
           {
             float sum[NC];
 #pragma unroll
@@ -1090,6 +1116,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
           epi_sync();
         }
       }
+      if (e == 0) trace_mark(a, p, 4);
       if (ok && p + 1 < P) ok = grid_sync(a, s.abort_flag, e, p);
     }
     if (x_pending && ok) {
@@ -1145,12 +1172,10 @@ bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *v
 
 // Number of CTAs: whole clusters, at most one CTA per SM, all co-resident.
 int decode_step_grid(int num_sms) {
-  static int cached = -1;
-  if (cached >= 0) return cached;
-  cudaError_t e = cudaFuncSetAttribute(decode_step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  cudaError_t e = ensure_smem_attr((const void *)decode_step_kernel, SMEM_BYTES);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return cached = 0;
+    return 0;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((num_sms / CL) * CL);
@@ -1167,17 +1192,17 @@ int decode_step_grid(int num_sms) {
   e = cudaOccupancyMaxActiveClusters(&clusters, decode_step_kernel, &cfg);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return cached = 0;
+    return 0;
   }
   if (clusters > num_sms / CL) clusters = num_sms / CL;
-  return cached = clusters * CL;
+  return clusters * CL;
 }
 
 cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, const CUtensorMap *maps_dev,
                           const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
                           float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
                           const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          float *split_part, int grid, cudaStream_t s) {
+                          float *split_part, int grid, unsigned long long *trace, cudaStream_t s) {
   const nc_config &c = m->cfg;
   StepArgs a;
   a.L = c.depth;
@@ -1216,6 +1241,7 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
   a.split_cnt = reinterpret_cast<unsigned *>(bar + 1);
   a.split_part = split_part;
   a.status = m->status;
+  a.trace = trace;
   // grid-barrier counter and split counters from zero for every step
   cudaError_t e = cudaMemsetAsync(bar, 0, decode_step_bar_bytes(), s);
   if (e != cudaSuccess) return e;

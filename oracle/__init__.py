@@ -76,6 +76,8 @@ def lib():
             L.orc_argmax.restype = i32
             L.orc_argmax.argtypes = [vp, vp, ip]
             L.orc_num_threads.restype = ip
+            L.orc_set_threads.argtypes = [ip]
+            L.orc_set_threads.restype = None
             _lib = L
     return _lib
 
@@ -87,6 +89,11 @@ def _p(a: np.ndarray):
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops (results do not depend on it)."""
+    lib().orc_set_threads(int(n))
 
 
 # ---------------------------------------------------------------- primitives

@@ -376,3 +376,14 @@ int orc_num_threads(void) {
   return 1;
 #endif
 }
+
+/* Threads of the parallel loops from now on (n >= 1). Every output element
+ * is computed by one thread in a fixed order, so results do not depend on it. */
+void orc_set_threads(int n) {
+#ifdef _OPENMP
+  extern void omp_set_num_threads(int);
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}

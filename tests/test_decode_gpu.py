@@ -152,3 +152,71 @@ def test_d20_decode_workload_full_context_sampled():
     prompts = syn.prompt_tokens(w)
     worst = greedy_session(cfg, blob_for(cfg), prompts, 2, [31], max_seq=w.prompt_len + w.decode_steps)
     assert worst <= TOL_BF16
+
+
+@pytest.mark.parametrize("cfg,B,T,steps", [(SMALL, 5, 40, 4), (syn.D20, 3, 70, 3)])
+def test_per_kernel_decode_path_matches_oracle(monkeypatch, cfg, B, T, steps):
+    """The decode step as one launch per layer step (the path a cache takes
+    when the whole-step kernel cannot be placed), forced with the
+    NC_DECODE_STEP_KERNEL=0 switch, against the oracle."""
+    import kv_cache_transformer_b200 as nc
+    monkeypatch.setenv("NC_DECODE_STEP_KERNEL", "0")
+    blob = blob_for(cfg)
+    prompts = syn.tokens_zipf(60 + B, (B, T), cfg.vocab)
+    run = Run(cfg, blob, B, T + steps + 1)
+    _, nxt = run.prefill(prompts)
+    om = orc.OracleModel(cfg, blob)
+    seqs = [om.new_seq(T + steps + 1) for _ in range(B)]
+    for b in range(B):
+        seqs[b].prefill(prompts[b])
+    cur = nxt.copy()
+    run.model.profile(True)
+    run.model.profile_read()
+    for s in range(steps):
+        lg, nn = run.decode(cur, np.full(B, T + s, np.int32))
+        for b in (0, B - 1):
+            ref = seqs[b].step(int(cur[b]))
+            check_logits(lg[b], ref, TOL_BF16, f"per-kernel step {s} seq {b}")
+            check_token(int(nn[b]), ref, None, f"per-kernel step {s} seq {b}")
+        for b in range(1, B - 1):
+            seqs[b].step(int(cur[b]))
+        cur = nn
+    _, launches = run.model.profile_read()
+    run.model.profile(False)
+    assert launches[nc.NC_K_STEP] == 0 and launches[nc.NC_K_GEMM] == 4 * cfg.depth * steps
+    assert run.status() == 0
+
+
+def test_decode_step_trace_fills_and_fits_the_event_time():
+    """nc_decode_trace: every CTA stamps every phase, phases follow one
+    another, the kernel's span lies inside the event-timed step, and tracing
+    does not change the results."""
+    import torch
+    cfg = syn.D20
+    blob = blob_for(cfg)
+    B, T = 4, 16
+    prompts = syn.tokens_zipf(66, (B, T), cfg.vocab)
+    a, b_ = Run(cfg, blob, B, T + 2), Run(cfg, blob, B, T + 2)
+    _, na = a.prefill(prompts)
+    _, nb = b_.prefill(prompts)
+    assert np.array_equal(na, nb)
+    grid, P = a.kv.trace(None)
+    assert grid > 0 and P == 3 + 5 * cfg.depth
+    buf = torch.zeros(grid * P * 8, dtype=torch.int64, device="cuda")
+    a.kv.trace(buf)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    la, ta = a.decode(na, np.full(B, T, np.int32))
+    e1.record()
+    torch.cuda.synchronize()
+    a.kv.trace(None)
+    lb, tb = b_.decode(nb, np.full(B, T, np.int32))
+    assert np.array_equal(la, lb) and np.array_equal(ta, tb), "tracing changed the results"
+    tr = buf.cpu().numpy().reshape(grid, P, 8)
+    assert np.all(tr[:, :, 0] > 0) and np.all(tr[:, :, 4] > 0), "a CTA skipped a phase stamp"
+    assert np.all(tr[:, :, 4] >= tr[:, :, 0])
+    assert np.all(np.diff(tr[:, :, 0], axis=1) >= 0), "phase starts out of order"
+    span_us = (tr[:, -1, 4].max() - tr[:, 0, 0].min()) / 1e3
+    event_us = 1e3 * e0.elapsed_time(e1)
+    assert 0.5 * event_us <= span_us <= event_us, (span_us, event_us)
+    assert a.status() == 0

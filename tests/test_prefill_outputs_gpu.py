@@ -1,0 +1,114 @@
+"""GPU parity of the outputs around the token pick: every-position logits of
+bf16 models (the tcgen05 GEMM with the softcap epilogue), the next token with
+additive noise on each of the library's argmax paths, and the tie rule
+(lowest index wins) on logits that tie exactly.
+
+Paths covered (nc.h, nc_prefill):
+  logits_mode 0, bf16, B <= 32  -> fused final norm + lm_head + softcap + argmax
+  logits_mode 1, bf16           -> norm + softcap GEMM over all rows, then the
+                                   row argmax kernel
+  fp32 model                    -> generic head, then the row argmax kernel
+  decode step, bf16             -> the whole-step kernel's head and merge
+"""
+import numpy as np
+import pytest
+
+import nc_synth as syn
+import oracle as orc
+from nc_harness import Run, check_logits, check_token, tol_for
+
+pytestmark = pytest.mark.gpu
+
+SMALL = syn.ModelConfig(depth=2, d_model=256, n_head=2, n_kv_head=1, head_dim=128, mlp_hidden=512, vocab=1024,
+                        dtype="bf16")
+_blobs = {}
+
+
+def blob_for(cfg):
+    if cfg not in _blobs:
+        _blobs[cfg] = syn.make_blob(cfg, 0)
+    return _blobs[cfg]
+
+
+def first_argmax(z: np.ndarray) -> int:
+    """Index of the largest value, the lowest one among equals (the rule nc.h states)."""
+    return int(np.flatnonzero(z == z.max())[0])
+
+
+@pytest.mark.parametrize("cfg,B,T,seqs", [
+    (syn.D20, 2, 136, [0, 1]),  # 272 rows: two full 128-row tiles and a partial one
+    (syn.D30, 1, 130, [0]),     # 15 heads, d 1920: partial last 256-column tile
+])
+def test_bf16_all_position_logits_match_oracle(cfg, B, T, seqs):
+    prompts = syn.tokens_zipf(41, (B, T), cfg.vocab)
+    run = Run(cfg, blob_for(cfg), B, T + 1)
+    lg, nxt = run.prefill(prompts, all_logits=True)
+    assert run.status() == 0
+    om = orc.OracleModel(cfg, blob_for(cfg))
+    for b in seqs:
+        ref = om.new_seq(T + 1).prefill(prompts[b], all_positions=True)
+        check_logits(lg[b], ref, tol_for(cfg), f"seq {b} all positions")
+        assert int(nxt[b]) == first_argmax(lg[b, -1]), f"seq {b}: next token is not the argmax of its logits"
+        check_token(int(nxt[b]), ref[-1], None, f"seq {b}")
+
+
+@pytest.mark.parametrize("cfg,B,T,mode", [
+    (SMALL, 3, 40, 0),      # fused lm_head + argmax with noise
+    (SMALL, 3, 40, 1),      # all-position logits, then the row argmax with noise
+    (syn.D20, 2, 24, 0),    # fused path over 512 vocabulary tiles
+    (syn.TINY, 2, 17, 0),   # fp32 model: generic head, row argmax
+])
+def test_prefill_next_token_with_noise(cfg, B, T, mode):
+    prompts = syn.tokens_zipf(43, (B, T), cfg.vocab)
+    noise = syn.gumbel(5, (B, cfg.vocab), stream=3)
+    run = Run(cfg, blob_for(cfg), B, T + 1)
+    lg, nxt = run.prefill(prompts, all_logits=bool(mode), noise=noise)
+    assert run.status() == 0
+    last = lg[:, -1] if mode else lg
+    om = orc.OracleModel(cfg, blob_for(cfg))
+    for b in range(B):
+        # the pick is the argmax of the kernel's own logits + noise, in fp32
+        z = (last[b].astype(np.float32) + noise[b].astype(np.float32)).astype(np.float32)
+        assert int(nxt[b]) == first_argmax(z), f"seq {b}: token {nxt[b]} != argmax(logits + noise)"
+        ref = om.new_seq(T + 1).prefill(prompts[b])
+        check_logits(last[b], ref, tol_for(cfg), f"seq {b}")
+        check_token(int(nxt[b]), ref, noise[b], f"seq {b} with noise")
+
+
+def _paired_head_blob(cfg):
+    """The model's blob with lm_head rows duplicated in pairs (row 2k+1 = row
+    2k), so every logit has an exact twin at the next index."""
+    blob = blob_for(cfg).copy()
+    off, rows, cols = syn.tensor_offsets(cfg)["wlm"]
+    w = blob[off:off + rows * cols].reshape(rows, cols)
+    w[1::2] = w[0::2]
+    return blob
+
+
+@pytest.mark.parametrize("cfg", [SMALL, syn.TINY])
+def test_exact_ties_pick_the_lowest_index(cfg):
+    B, T, steps = 3, 20, 3
+    blob = _paired_head_blob(cfg)
+    prompts = syn.tokens_zipf(47, (B, T), cfg.vocab)
+    # noise tied in the same pairs keeps every tie through the noisy pick
+    noise = np.repeat(syn.gumbel(5, (B, cfg.vocab // 2), stream=9), 2, axis=1)
+
+    def check(lg, nxt, nz, what):
+        for b in range(B):
+            assert np.array_equal(lg[b, 0::2], lg[b, 1::2]), f"{what} seq {b}: twin rows gave different logits"
+            z = lg[b] if nz is None else (lg[b].astype(np.float32) + nz[b].astype(np.float32)).astype(np.float32)
+            want = first_argmax(z)
+            assert want % 2 == 0
+            assert int(nxt[b]) == want, f"{what} seq {b}: token {nxt[b]}, the lowest tied index is {want}"
+
+    for mode in (0, 1):
+        for nz in (None, noise):
+            run = Run(cfg, blob, B, T + steps + 1)
+            lg, nxt = run.prefill(prompts, all_logits=bool(mode), noise=nz)
+            check(lg[:, -1] if mode else lg, nxt, nz, f"prefill mode {mode} noise {nz is not None}")
+            cur = nxt.copy()
+            for s in range(steps):
+                lg2, n2 = run.decode(cur, np.full(B, T + s, np.int32), nz)
+                check(lg2, n2, nz, f"decode step {s} noise {nz is not None}")
+                cur = n2
+            assert run.status() == 0
