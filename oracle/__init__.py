@@ -76,6 +76,8 @@ def lib():
             L.orc_argmax.restype = i32
             L.orc_argmax.argtypes = [vp, vp, ip]
             L.orc_num_threads.restype = ip
+            L.orc_sample_topk.restype = i32
+            L.orc_sample_topk.argtypes = [vp, vp, ip, ctypes.c_float, ip]
             L.orc_set_threads.argtypes = [ip]
             L.orc_set_threads.restype = None
             _lib = L
@@ -89,6 +91,15 @@ def _p(a: np.ndarray):
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def sample_topk(z, g=None, temperature: float = 1.0, top_k: int = 0) -> int:
+    """Sampled pick over fp32 logits z [n]: argmax over the top_k largest z of
+    fl(fl(z / temperature) + g) (g fp32 Gumbel noise or None), lowest index on
+    ties; temperature 0 is argmax z. See orc_sample_topk in nc_oracle.c."""
+    z = np.ascontiguousarray(z, dtype=np.float32)
+    gg = None if g is None else np.ascontiguousarray(g, dtype=np.float32)
+    return int(lib().orc_sample_topk(_p(z), None if gg is None else _p(gg), z.size, float(temperature), int(top_k)))
 
 
 def set_threads(n: int) -> None:

@@ -133,6 +133,54 @@ int orc_argmax(const double *v, const float *g, int n) {
   return best;
 }
 
+/* Sampled token pick with temperature and top-k. The launch article lists
+ * sampling in the Engine ("高效推理") and gives no details; the reading is the
+ * usual one: keep the top_k largest logits (top_k <= 0 or >= n keeps all;
+ * at a tie on the cut the lower index is kept) and draw from the softmax of
+ * z / temperature over them. With g_v i.i.d. standard Gumbel noise the draw
+ * is argmax_v (z_v / temperature + g_v) (Gumbel-max), so the noise is an
+ * input, as for orc_argmax. temperature == 0 is the greedy pick argmax_v z_v.
+ * The decision is taken in fp32, the precision of the logits it is made on:
+ * score_v = fl(fl(z_v / temperature) + g_v), lowest index on ties. */
+static const float *g_sample_z;  /* key of the ordering below (qsort has no context argument) */
+
+static int by_logit_desc(const void *a, const void *b) {
+  const int i = *(const int *)a, j = *(const int *)b;
+  const float zi = g_sample_z[i], zj = g_sample_z[j];
+  if (zi > zj) return -1;
+  if (zi < zj) return 1;
+  return (i > j) - (i < j);
+}
+
+int orc_sample_topk(const float *z, const float *g, int n, float temperature, int top_k) {
+  if (n <= 0) return -1;
+  if (temperature == 0.0f) {
+    int best = 0;
+    for (int i = 1; i < n; i++)
+      if (z[i] > z[best]) best = i;
+    return best;
+  }
+  const int k = (top_k <= 0 || top_k >= n) ? n : top_k;
+  int *order = (int *)malloc(sizeof(int) * (size_t)n);
+  if (!order) return -1;
+  for (int i = 0; i < n; i++) order[i] = i;
+  g_sample_z = z;
+  qsort(order, (size_t)n, sizeof(int), by_logit_desc);
+  int best = -1;
+  float best_s = 0.0f;
+  for (int r = 0; r < k; r++) {
+    const int v = order[r];
+    const float scaled = z[v] / temperature;
+    const float s = scaled + (g ? g[v] : 0.0f);
+    if (best < 0 || s > best_s || (s == best_s && v < best)) {
+      best = v;
+      best_s = s;
+    }
+  }
+  free(order);
+  return best;
+}
+
 /* ----------------------------------------------------------------- model */
 orc_model *orc_model_create(const orc_config *c, const void *blob) {
   if (!c || !blob || c->depth < 0 || c->d_model <= 0 || c->n_head <= 0 || c->n_kv_head <= 0 ||

@@ -335,3 +335,52 @@ def test_pages_figures_pin_the_width_reading():
     # the oracle's own parameter count agrees with the blob layout
     m = orc.OracleModel(syn.TINY, BLOB)
     assert BLOB.size == syn.param_count(syn.TINY) == 491_520
+
+
+# ------------------------------------------------------ sampled token pick
+def _first_max(a):
+    return int(np.flatnonzero(a == a.max())[0])
+
+
+def test_sample_topk_special_cases_reduce_to_argmax():
+    # temperature 0: the greedy pick, whatever the noise and k
+    z = RNG.standard_normal(300).astype(np.float32)
+    g = syn.gumbel(11, (300,), stream=1)
+    assert orc.sample_topk(z, g, 0.0, 7) == _first_max(z)
+    # k = 1: only the largest logit is a candidate
+    assert orc.sample_topk(z, g, 0.6, 1) == _first_max(z)
+    # k = n (and k = 0), temperature 1: argmax of z + g, the pick the engine
+    # makes without sampling parameters
+    want = _first_max((z + g).astype(np.float32))
+    assert orc.sample_topk(z, g, 1.0, 0) == want == orc.sample_topk(z, g, 1.0, 300)
+    # no noise: any temperature > 0 and any k keep the greedy pick
+    assert orc.sample_topk(z, None, 2.5, 40) == _first_max(z)
+
+
+def test_sample_topk_membership_and_ties():
+    z = np.array([3.0, 5.0, 5.0, 5.0, 1.0], np.float32)
+    # k = 2 keeps the two lowest indices of the three tied 5s: index 3 is out
+    # however large its noise, and equal scores go to the lower index
+    assert orc.sample_topk(z, np.array([0, 0, 0, 9, 0], np.float32), 1.0, 2) == 1
+    assert orc.sample_topk(z, np.array([0, 0, 0.5, 9, 0], np.float32), 1.0, 2) == 2
+    # k = 3 lets index 3 in
+    assert orc.sample_topk(z, np.array([0, 0, 0, 9, 0], np.float32), 1.0, 3) == 3
+    # the lowest logit can win only once it is a candidate
+    g = np.array([0, 0, 0, 0, 50], np.float32)
+    assert orc.sample_topk(z, g, 1.0, 4) != 4 and orc.sample_topk(z, g, 1.0, 5) == 4
+
+
+def test_sample_topk_draws_follow_the_tempered_topk_softmax():
+    # Gumbel-max: with i.i.d. standard Gumbel noise the pick is distributed as
+    # softmax(z / T) over the top-k logits and never picks outside them
+    z = np.array([0.5, 2.0, 1.0, -1.0, 1.5, 0.2], np.float32)
+    T, k, n = 0.8, 4, 40000
+    g = syn.gumbel(21, (n, z.size), stream=0)
+    counts = np.bincount([orc.sample_topk(z, g[i], T, k) for i in range(n)], minlength=z.size)
+    keep = np.argsort(-z, kind="stable")[:k]
+    p = np.zeros(z.size)
+    e = np.exp((z[keep].astype(np.float64) - z.max()) / T)
+    p[keep] = e / e.sum()
+    freq = counts / n
+    assert np.all(counts[p == 0] == 0)
+    assert np.all(np.abs(freq - p) <= 4.5 * np.sqrt(p * (1 - p) / n) + 1e-3), (freq, p)
