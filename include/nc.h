@@ -156,6 +156,20 @@ int nc_decode_step(nc_model *model, nc_kv *kv, const int32_t *d_tokens, const in
  * NC_ECUDA. */
 int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream);
 
+/* Sampled token pick for nc_prefill and nc_decode_step on this cache. The
+ * launch article's Engine samples its tokens ("高效推理"; the pages give no
+ * details); the usual temperature / top-k reading is taken. From now on
+ * d_next[b] is the argmax, over the top_k largest logits of row b (all of
+ * them when top_k == 0 or >= V; at a tie on the cut the lower index is
+ * kept), of fl(fl(logit / temperature) + d_noise[b, v]) in fp32, lowest
+ * index on ties. With d_noise i.i.d. standard Gumbel this draws from
+ * softmax(logits / temperature) restricted to the top_k (Gumbel-max); with
+ * d_noise NULL the noise is 0. temperature 0 is the greedy pick argmax of
+ * the logits. temperature 1 with top_k 0 (the default) is the plain
+ * argmax(logits + noise) pick. The logits returned are unchanged (softcapped,
+ * untempered). Errors: NC_EINVAL (temperature < 0 or not finite, top_k < 0). */
+int nc_kv_set_sampling(nc_kv *kv, float temperature, int top_k);
+
 /* ---- tracing ----
  * Kernel classes for nc_profile_read. */
 #define NC_K_GEMM 0   /* linear layers: QKV, O-proj, MLP fc, MLP proj */

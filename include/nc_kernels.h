@@ -59,6 +59,19 @@ size_t nc_attention_decode_workspace_bytes(int B, int max_seq);
 int nc_attention_decode_bf16(const void *d_q, const void *d_k, const void *d_v, const int32_t *d_pos, int B, int H,
                              int max_seq, void *d_y, void *d_workspace, size_t workspace_bytes, void *stream);
 
+/* Sampled token pick over fp32 logits (the pick nc_kv_set_sampling turns on
+ * inside the engine): d_next[b] = argmax, over the top_k largest logits of
+ * row b (all when top_k == 0 or >= V; at a tie on the cut the lower index is
+ * kept), of fl(fl(d_logits[b, v] / temperature) + d_noise[b, v]), lowest
+ * index on ties; temperature 0 gives argmax of the logits. d_logits rows are
+ * row_stride floats apart (row_stride >= V); d_noise fp32 [B, V] contiguous
+ * or NULL (no noise); d_next int32 [B]. One CTA per row re-reads the row from
+ * memory four times (radix select of the cut, then the pick). Errors:
+ * NC_EINVAL (null logits or next, B or V < 1, row_stride < V, temperature < 0
+ * or not finite, top_k < 0), NC_ECUDA. */
+int nc_sample_topk(const float *d_logits, int B, int V, long long row_stride, const float *d_noise, float temperature,
+                   int top_k, int32_t *d_next, void *stream);
+
 /* nc_attention_decode_bf16 without a workspace argument, for callers that
  * cannot allocate device memory (a serving runtime whose allocator owns all
  * of it, a plugin host without a workspace hook, a fixed-footprint

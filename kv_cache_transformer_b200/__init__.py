@@ -35,7 +35,7 @@ EXPORTS = (
     "nc_kv_lengths", "nc_prefill", "nc_decode_step", "nc_kv_fork", "nc_last_error",
     "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
     "nc_attention_prefill_bf16", "nc_attention_decode_workspace_bytes", "nc_attention_decode_bf16",
-    "nc_attention_decode_bf16_static", "nc_decode_trace",
+    "nc_attention_decode_bf16_static", "nc_decode_trace", "nc_kv_set_sampling", "nc_sample_topk",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_STEP, NC_K_COUNT = 0, 1, 2, 3, 4, 5
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
             L.nc_attention_decode_bf16.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp, sz, vp]
             L.nc_attention_decode_bf16_static.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp]
             L.nc_decode_trace.argtypes = [vp, vp, sz, ctypes.POINTER(i), ctypes.POINTER(i)]
+            L.nc_kv_set_sampling.argtypes = [vp, ctypes.c_float, i]
+            L.nc_sample_topk.argtypes = [vp, i, i, ctypes.c_longlong, vp, ctypes.c_float, i, vp, vp]
             for name in EXPORTS:
                 if name not in ("nc_model_destroy", "nc_kv_destroy", "nc_last_error", "nc_launch_count",
                                 "nc_attention_decode_workspace_bytes"):
@@ -202,6 +204,21 @@ def nc_decode_step(model_h, kv_h, tokens, positions, noise=None, logits=None, ne
 
 def nc_kv_fork(src_h, src_seq: int, dst_h, dst_first: int, n: int, stream=None):
     _check(lib().nc_kv_fork(src_h, int(src_seq), dst_h, int(dst_first), int(n), _stream(stream)))
+
+
+def nc_kv_set_sampling(kv_h, temperature: float = 1.0, top_k: int = 0):
+    _check(lib().nc_kv_set_sampling(kv_h, float(temperature), int(top_k)))
+
+
+def nc_sample_topk(logits, next, noise=None, temperature: float = 1.0, top_k: int = 0, stream=None):
+    """next[b] = sampled pick over fp32 CUDA logits [B, V] (rows may be strided: logits.stride(0))."""
+    import torch
+    B, V = logits.shape
+    if logits.dtype != torch.float32 or logits.stride(1) != 1 or not logits.is_cuda:
+        raise TypeError("logits must be a CUDA float32 tensor with unit inner stride")
+    _check(lib().nc_sample_topk(ctypes.c_void_p(logits.data_ptr()), int(B), int(V), int(logits.stride(0)),
+                                _dptr(noise, torch.float32, B * V, "noise"), float(temperature), int(top_k),
+                                _dptr(next, torch.int32, B, "next"), _stream(stream)))
 
 
 def nc_decode_trace(kv_h, buf=None):
@@ -356,6 +373,10 @@ class KVCache:
 
     def fork_to(self, src_seq: int, dst: "KVCache", dst_first: int, n: int, stream=None):
         nc_kv_fork(self._h, src_seq, dst.handle, dst_first, n, stream)
+
+    def set_sampling(self, temperature: float = 1.0, top_k: int = 0):
+        """Sampled token pick for later prefill/decode calls on this cache (see nc_kv_set_sampling)."""
+        nc_kv_set_sampling(self._h, temperature, top_k)
 
     def trace(self, buf=None):
         """Phase timestamps of later decode steps into `buf` (see nc_decode_trace)."""

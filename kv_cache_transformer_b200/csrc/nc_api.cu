@@ -244,6 +244,15 @@ cudaError_t run_head(nc_model *m, nc_kv *kv, int rows, int stride, int offset, f
                 valid, s);
 }
 
+// With sampling parameters set on the cache (nc_kv_set_sampling), replace the
+// argmax pick in next[] by the sampled pick over the same logits and noise.
+cudaError_t sampled_pick(nc_model *m, nc_kv *kv, const float *logits, int B, int V, long long stride,
+                         const float *noise, const uint8_t *valid, int32_t *next, cudaStream_t s) {
+  if (!next || !kv->sampling()) return cudaSuccess;
+  ProfScope p(m, NC_K_HEAD, s);
+  return nc::k_sample_topk(logits, B, V, stride, noise, kv->temperature, kv->top_k, valid, next, s);
+}
+
 // The decode step on the sm_100a decode kernels (bf16, head_dim 128, B <= 32).
 cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *positions, int B,
                                  const float *noise, float *logits, int32_t *next, cudaStream_t s) {
@@ -252,11 +261,14 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
   const float eps = c.norm_eps;
   cudaError_t e;
   if (kv->step_grid > 0 && nc::decode_step_supported(c, B)) {
-    ProfScope p(m, NC_K_STEP, s);
-    return nc::k_decode_step(m, B, kv->max_batch, kv->max_seq, kv->step_maps, tokens, positions, kv->len, kv->x,
-                             kv->xl, kv->step_ss, kv->q, kv->y, kv->f, kv->k, kv->v, kv->rope, logits, noise, next,
-                             kv->cand_v, kv->cand_i, kv->step_bar, kv->step_part, kv->step_grid, kv->step_trace,
-                             s);
+    {
+      ProfScope p(m, NC_K_STEP, s);
+      e = nc::k_decode_step(m, B, kv->max_batch, kv->max_seq, kv->step_maps, tokens, positions, kv->len, kv->x,
+                            kv->xl, kv->step_ss, kv->q, kv->y, kv->f, kv->k, kv->v, kv->rope, logits, noise, next,
+                            kv->cand_v, kv->cand_i, kv->step_bar, kv->step_part, kv->step_grid, kv->step_trace,
+                            kv->valid, s);
+    }
+    return e == cudaSuccess ? sampled_pick(m, kv, logits, B, V, V, noise, kv->valid, next, s) : e;
   }
   {
     ProfScope p(m, NC_K_MISC, s);
@@ -296,11 +308,14 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
       if (e != cudaSuccess) return e;
     }
   }
-  ProfScope p(m, NC_K_HEAD, s);
-  return nc::k_dec_linear(0 /*norm*/, 3 /*lmhead*/, m->wlm, V, d, B, kv->x, kv->ss, 32, eps, nullptr, kv->part,
-                          kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq, H, kv->pos_ws,
-                          kv->valid, kv->rope, logits, noise, c.softcap, kv->cand_v, kv->cand_i, next, m->status, sms,
-                          s);
+  {
+    ProfScope p(m, NC_K_HEAD, s);
+    e = nc::k_dec_linear(0 /*norm*/, 3 /*lmhead*/, m->wlm, V, d, B, kv->x, kv->ss, 32, eps, nullptr, kv->part,
+                         kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq, H, kv->pos_ws,
+                         kv->valid, kv->rope, logits, noise, c.softcap, kv->cand_v, kv->cand_i, next, m->status, sms,
+                         s);
+  }
+  return e == cudaSuccess ? sampled_pick(m, kv, logits, B, V, V, noise, kv->valid, next, s) : e;
 }
 
 // Replay the cached graph of the decode step when the call matches the last
@@ -322,6 +337,8 @@ int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *po
   key.logits = logits;
   key.next = next;
   key.B = B;
+  key.temperature = kv->temperature;
+  key.top_k = kv->top_k;
   const bool same = memcmp(&key, &kv->graph_key, sizeof key) == 0;
   if (!same || !kv->graph_ready) {
     // a new call shape runs directly; the graph is captured once it repeats
@@ -622,6 +639,7 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
                              nullptr, kv->part, kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq,
                              c.n_head, kv->pos_ws, kv->valid, kv->rope, logits, d_noise, c.softcap, kv->cand_v,
                              kv->cand_i, d_next, m->status, m->num_sms, s);
+      if (e == cudaSuccess) e = sampled_pick(m, kv, logits, B, c.vocab, c.vocab, d_noise, nullptr, d_next, s);
       if (e != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(e));
       return NC_OK;
     }
@@ -631,8 +649,12 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
   }
   if (eh != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(eh));
   if (d_next) {
-    ProfScope p(m, NC_K_HEAD, s);
-    nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
+    if (kv->sampling()) {
+      NC_CUDA_TRY(sampled_pick(m, kv, logits + last_off, B, c.vocab, row_stride, d_noise, nullptr, d_next, s));
+    } else {
+      ProfScope p(m, NC_K_HEAD, s);
+      nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
+    }
   }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
@@ -665,8 +687,12 @@ int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_
   const cudaError_t eh = run_head(m, kv, B, 1, 0, logits, kv->valid, s);
   if (eh != cudaSuccess) return fail(NC_ECUDA, "decode head launch failed: %s", cudaGetErrorString(eh));
   if (d_next) {
-    ProfScope p(m, NC_K_HEAD, s);
-    nc::k_argmax_rows(logits, B, c.vocab, c.vocab, d_noise, d_next, kv->valid, s);
+    if (kv->sampling()) {
+      NC_CUDA_TRY(sampled_pick(m, kv, logits, B, c.vocab, c.vocab, d_noise, kv->valid, d_next, s));
+    } else {
+      ProfScope p(m, NC_K_HEAD, s);
+      nc::k_argmax_rows(logits, B, c.vocab, c.vocab, d_noise, d_next, kv->valid, s);
+    }
   }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
@@ -688,6 +714,15 @@ int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *
                 dst->v, dst->layer_elems, dst->max_seq, dst_first, n, dst->len, c.depth, c.n_kv_head * c.head_dim,
                 src->model->status, as_stream(stream));
   NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+int nc_kv_set_sampling(nc_kv *kv, float temperature, int top_k) {
+  if (!kv) return fail(NC_EINVAL, "kv is NULL");
+  if (!(temperature >= 0.f) || !isfinite(temperature)) return fail(NC_EINVAL, "temperature must be finite and >= 0");
+  if (top_k < 0) return fail(NC_EINVAL, "top_k must be >= 0");
+  kv->temperature = temperature;
+  kv->top_k = top_k;
   return NC_OK;
 }
 
@@ -803,6 +838,18 @@ int nc_attention_decode_bf16(const void *d_q, const void *d_k, const void *d_v, 
   cudaError_t e = nc::k_dec_attn(d_q, d_k, d_v, d_pos, nullptr, B, H, max_seq, chunk, splits, pf, counters, d_y,
                                  as_stream(stream));
   if (e != cudaSuccess) return fail(NC_ECUDA, "decode attention launch: %s", cudaGetErrorString(e));
+  return NC_OK;
+}
+
+int nc_sample_topk(const float *d_logits, int B, int V, long long row_stride, const float *d_noise, float temperature,
+                   int top_k, int32_t *d_next, void *stream) {
+  if (!d_logits || !d_next) return fail(NC_EINVAL, "null pointer");
+  if (B < 1 || V < 1 || row_stride < V) return fail(NC_EINVAL, "bad shape (B, V >= 1, row_stride >= V)");
+  if (!(temperature >= 0.f) || !isfinite(temperature)) return fail(NC_EINVAL, "temperature must be finite and >= 0");
+  if (top_k < 0) return fail(NC_EINVAL, "top_k must be >= 0");
+  const cudaError_t e =
+      nc::k_sample_topk(d_logits, B, V, row_stride, d_noise, temperature, top_k, nullptr, d_next, as_stream(stream));
+  if (e != cudaSuccess) return fail(NC_ECUDA, "sampling launch failed: %s", cudaGetErrorString(e));
   return NC_OK;
 }
 

@@ -76,6 +76,11 @@ struct nc_kv {
   float *step_part = nullptr;  // split-K partials of its MLP proj phase
   float *step_ss = nullptr;    // [2*depth+1][16][32] per-128-column sums of squares
   unsigned long long *step_trace = nullptr;  // caller's phase-timestamp buffer (nc_decode_trace), or null
+  // sampled token pick (nc_kv_set_sampling): temperature 1 and top_k 0 are
+  // the plain argmax(logits + noise)
+  float temperature = 1.f;
+  int top_k = 0;
+  bool sampling() const { return temperature != 1.f || top_k > 0; }
   int attn_chunk = 0, attn_splits = 0;
   // CUDA graph of the last decode step's launches, replayed while the call's
   // pointers and batch stay the same
@@ -84,6 +89,8 @@ struct nc_kv {
   struct GraphKey {
     const void *tokens, *positions, *noise, *logits, *next;
     int B;
+    float temperature;
+    int top_k;
   } graph_key = {};
   bool graph_ready = false;    // graph_key has run once directly
   unsigned long long graph_kernels = 0;
@@ -190,6 +197,14 @@ cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int3
                        cudaStream_t s);
 
 
+// ---- sampled token pick (nc_sample.cu) ----
+// next[b] = argmax over the top_k largest logits of row b (all when top_k <= 0
+// or >= V; the lower index on a tie at the cut) of fl(fl(z / temperature) +
+// noise), lowest index on ties; temperature 0 is argmax z. Logit rows are
+// `stride` floats apart, noise rows V; rows with valid[b] == 0 are skipped.
+cudaError_t k_sample_topk(const float *logits, int B, int V, long long stride, const float *noise, float temperature,
+                          int top_k, const uint8_t *valid, int32_t *next, cudaStream_t s);
+
 // ---- whole decode step in one persistent kernel (nc_step.cu) ----
 bool decode_step_supported(const nc_config &c, int B);
 int decode_step_maps_count(const nc_config &c);
@@ -200,7 +215,8 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
                           const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
                           float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
                           const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          float *split_part, int grid, unsigned long long *trace, cudaStream_t s);
+                          float *split_part, int grid, unsigned long long *trace, uint8_t *valid_out,
+                          cudaStream_t s);
 size_t decode_step_bar_bytes();              // grid-barrier word + split counters, zeroed per launch
 size_t decode_step_part_floats(int num_sms);  // split-K partials of the MLP proj phase
 

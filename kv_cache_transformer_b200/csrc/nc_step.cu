@@ -98,6 +98,7 @@ struct StepArgs {
   float *split_part;          // [n_tiles * S][CL][128][NB/CL]: their partial sums
   uint32_t *status;
   unsigned long long *trace;  // [grid][phases][8] phase timestamps (ns), or null
+  uint8_t *valid_out;         // [B]: 1 where the sequence's position was valid (written by CTA 0)
 };
 
 // Phase timestamps for nc_decode_trace: slot 0 phase start (after the last
@@ -879,6 +880,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(THREADS, 1) decode_
     }
     s.pos[b] = ok ? p : 0;
     s.valid[b] = ok;
+    if (blockIdx.x == 0 && b < a.B) a.valid_out[b] = (uint8_t)ok;
   }
   if (warp == 1) tmem_alloc(s.tmem_slot, 2 * NB * NACC);
   tc_fence_before();
@@ -1202,7 +1204,8 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
                           const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
                           float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
                           const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          float *split_part, int grid, unsigned long long *trace, cudaStream_t s) {
+                          float *split_part, int grid, unsigned long long *trace, uint8_t *valid_out,
+                          cudaStream_t s) {
   const nc_config &c = m->cfg;
   StepArgs a;
   a.L = c.depth;
@@ -1242,6 +1245,7 @@ cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, 
   a.split_part = split_part;
   a.status = m->status;
   a.trace = trace;
+  a.valid_out = valid_out;
   // grid-barrier counter and split counters from zero for every step
   cudaError_t e = cudaMemsetAsync(bar, 0, decode_step_bar_bytes(), s);
   if (e != cudaSuccess) return e;
