@@ -56,12 +56,14 @@ def prefill_flops(cfg, B: int, T: int) -> dict:
     return {"gemm": lin, "attn": attn, "head": head, "total": lin + attn + head}
 
 
-def decode_bytes(cfg, B: int, ctx_avg: float) -> dict:
-    """Algorithmic HBM bytes of one decode step (bf16 weights and cache, fp32 logits)."""
+def decode_bytes(cfg, B: int, ctx_avg: float, shared_rows: int = 0) -> dict:
+    """Algorithmic HBM bytes of one decode step (bf16 weights and cache, fp32
+    logits). shared_rows: key/value rows every sequence reads from one shared
+    prefix (nc_kv_fork_shared), counted once."""
     kd = cfg.n_kv_head * cfg.head_dim
     w_lin = 2 * linear_params(cfg)
     w_head = 2 * cfg.vocab * cfg.d_model
-    kv_read = cfg.depth * B * ctx_avg * kd * 2 * 2
+    kv_read = cfg.depth * (shared_rows + B * (ctx_avg - shared_rows)) * kd * 2 * 2
     kv_write = cfg.depth * B * kd * 2 * 2
     logits = 4 * B * cfg.vocab
     total = w_lin + w_head + kv_read + kv_write + logits
@@ -93,7 +95,7 @@ GEMM_DRAM_BYTES_PER_LAUNCH = (54_963_200 + 196_754_176 + 166_150_400 + 388_773_6
 # 2051): dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of
 # `python bench.py --only decode --decode-steps 4 --warmup 3` with
 # -k regex:decode_step -s 3 -c 1. To be re-taken whenever nc_step.cu changes.
-DECODE_STEP_DRAM_BYTES = 1_528_550_000 + 10_848_768
+DECODE_STEP_DRAM_BYTES = None  # re-taken from an ncu capture of the current kernel
 
 
 class ClockSampler:
@@ -368,6 +370,8 @@ def run_ours(args):
     if not args.no_workloads:
         workloads = {name: decode_workload(name, args, world, local, peaks, peaks_src)
                      for name in ("d26_latency", "d30_rollout")}
+        workloads["d30_rollout_shared_prefix"] = decode_workload("d30_rollout", args, world, local, peaks, peaks_src,
+                                                                 shared=True)
 
     # ---------------- CPU oracle on a bounded sample (rank 0, N = 1)
     cpu = None
@@ -519,7 +523,7 @@ def decode_phase_trace(kv, step, depth: int):
             "event_us": round(event_us, 1), "by_phase": out}
 
 
-def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src) -> dict:
+def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src, shared: bool = False) -> dict:
     """d26 latency decode (B=1, 1024-token prompt, 512 greedy steps) or d30
     rollout (256-token prompt prefilled once, forked to 16 samples, 256 steps
     of argmax over logits + Gumbel noise): decode tok/s over all ranks and the
@@ -550,9 +554,11 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src) -
         # seeded Gumbel noise per step and sample, generated up front (an input)
         noise = torch.from_numpy(np.stack([syn.gumbel(w.noise_seed, (n, V), stream=s_) for s_ in range(S)])).cuda()
 
+        fork = src.fork_shared_to if shared else src.fork_to
+
         def start():
             model.prefill(src, prompts, 0, None, tok1)
-            src.fork_to(0, dst, 0, n)
+            fork(0, dst, 0, n)
             tok.copy_(tok1.expand(n))
 
         def step(s_):
@@ -568,13 +574,17 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src) -
         model.prefill(src, prompts, 0, None, tok1)
         e1.record(stream)
         ef = torch.cuda.Event(enable_timing=True)
-        src.fork_to(0, dst, 0, n)
+        fork(0, dst, 0, n)
         ef.record(stream)
         tok.copy_(tok1.expand(n))
         torch.cuda.synchronize()
+        shared_rows = T // 64 * 64 if shared else 0
         extra = {"prefill_ms": e0.elapsed_time(e1), "fork_ms": e1.elapsed_time(ef),
-                 "fork_bytes": cfg.depth * 2 * T * cfg.head_dim * 2 * n}
+                 "fork_bytes": cfg.depth * 2 * (T - shared_rows) * cfg.head_dim * 2 * n,
+                 "fork_kind": "nc_kv_fork_shared (prefix rows read from the source)" if shared
+                 else "nc_kv_fork (copy)"}
     else:
+        shared_rows = 0
         kv = model.kv(w.batch, max_seq)
         caches = [kv]
         B = w.batch
@@ -608,7 +618,7 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src) -
     barrier(world)
     t_ms = max_over_ranks(d0.elapsed_time(d1), world)
     ctx_avg = T + (S + 1) / 2.0
-    by = decode_bytes(cfg, B, ctx_avg)
+    by = decode_bytes(cfg, B, ctx_avg, shared_rows)
     ms_step = t_ms / S
     gbs = by["total"] / (ms_step / 1e3) / 1e9
     for c in caches:

@@ -131,7 +131,8 @@ int nc_kv_lengths(const nc_kv *kv, int n, int32_t *out);
  *   d_next    int32 [B]: argmax over the vocabulary of the last position's
  *             logits (+ d_noise[b,:] if given), lowest index on ties;
  *   d_noise   fp32 [B,V] additive noise for d_next (e.g. Gumbel), or NULL.
- * Errors: NC_EINVAL (null kv/model/tokens, B or T < 1, bad logits_mode),
+ * Errors: NC_EINVAL (null kv/model/tokens, B or T < 1, bad logits_mode, a
+ * sequence among 0..B-1 is the shared prefix of another, nc_kv_fork_shared),
  * NC_ERANGE (B > max_batch, T > max_seq), NC_ECUDA. */
 int nc_prefill(nc_model *model, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode,
                float *d_logits, int32_t *d_next, const float *d_noise, void *stream);
@@ -155,6 +156,27 @@ int nc_decode_step(nc_model *model, nc_kv *kv, const int32_t *d_tokens, const in
  * Errors: NC_EINVAL, NC_ERANGE (indices out of range, len > dst max_seq),
  * NC_ECUDA. */
 int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream);
+
+/* Fork by sharing the prefix (the RL rollouts of the launch article's
+ * pipeline list sample many continuations of one prompt, and the lineage
+ * page's GRPO stage does the same): like nc_kv_fork, with the same results
+ * in every later call, but the destinations get no copy of the source's
+ * first P key/value rows of every layer, P = its length rounded down to a
+ * multiple of 64. Their attention reads those rows from the source sequence
+ * in `src` (one read of the shared rows serves every sample through the L2
+ * cache), and only the remaining len - P < 64 rows are copied. If the source
+ * sequence itself reads a shared prefix, the destinations read the same one
+ * (P is the source's). src and dst may be the same cache.
+ * The link lasts until the destination is replaced (nc_prefill over it, a
+ * fork into it) or its cache is destroyed. While any sequence reads shared
+ * rows from a sequence, that sequence may take decode steps (they append
+ * past the shared rows) but may not be replaced: nc_prefill and the forks
+ * return NC_EINVAL. A cache reads shared rows from one cache at a time. A
+ * source cache destroyed while others still read from it keeps its memory
+ * until the last such link ends.
+ * Errors: as nc_kv_fork, plus NC_EINVAL (the prefix's sequence among the
+ * destinations, dst already shares prefixes with another cache). */
+int nc_kv_fork_shared(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream);
 
 /* Sampled token pick for nc_prefill and nc_decode_step on this cache. The
  * launch article's Engine samples its tokens ("高效推理"; the pages give no

@@ -36,6 +36,7 @@ EXPORTS = (
     "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
     "nc_attention_prefill_bf16", "nc_attention_decode_workspace_bytes", "nc_attention_decode_bf16",
     "nc_attention_decode_bf16_static", "nc_decode_trace", "nc_kv_set_sampling", "nc_sample_topk",
+    "nc_kv_fork_shared",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_STEP, NC_K_COUNT = 0, 1, 2, 3, 4, 5
@@ -78,6 +79,7 @@ def lib() -> ctypes.CDLL:
             L.nc_prefill.argtypes = [vp, vp, vp, i, i, i, vp, vp, vp, vp]
             L.nc_decode_step.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp]
             L.nc_kv_fork.argtypes = [vp, i, vp, i, i, vp]
+            L.nc_kv_fork_shared.argtypes = [vp, i, vp, i, i, vp]
             L.nc_last_error.restype = ctypes.c_char_p
             L.nc_last_error.argtypes = []
             L.nc_profile_enable.argtypes = [vp, i]
@@ -233,6 +235,10 @@ def nc_decode_trace(kv_h, buf=None):
     return g.value, p.value
 
 
+def nc_kv_fork_shared(src_h, src_seq: int, dst_h, dst_first: int, n: int, stream=None):
+    _check(lib().nc_kv_fork_shared(src_h, int(src_seq), dst_h, int(dst_first), int(n), _stream(stream)))
+
+
 def nc_profile_enable(model_h, on: bool = True):
     _check(lib().nc_profile_enable(model_h, 1 if on else 0))
 
@@ -373,6 +379,10 @@ class KVCache:
 
     def fork_to(self, src_seq: int, dst: "KVCache", dst_first: int, n: int, stream=None):
         nc_kv_fork(self._h, src_seq, dst.handle, dst_first, n, stream)
+
+    def fork_shared_to(self, src_seq: int, dst: "KVCache", dst_first: int, n: int, stream=None):
+        """Fork sequence src_seq into dst[dst_first:dst_first+n] sharing its prefix rows (nc_kv_fork_shared)."""
+        nc_kv_fork_shared(self._h, src_seq, dst.handle, dst_first, n, stream)
 
     def set_sampling(self, temperature: float = 1.0, top_k: int = 0):
         """Sampled token pick for later prefill/decode calls on this cache (see nc_kv_set_sampling)."""

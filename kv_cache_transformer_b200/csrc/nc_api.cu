@@ -96,6 +96,63 @@ inline void *layer_ptr(const nc_kv *kv, void *base, int l) {
   return (char *)base + (size_t)l * kv->layer_elems * kv->model->elem;
 }
 
+// Where layer l's shared-prefix rows of kv's sequences live (len == nullptr
+// when kv has no links).
+nc::KvPrefix prefix_view(const nc_kv *kv, int l) {
+  nc::KvPrefix p;
+  const nc_kv *r = kv->prefix_src;
+  if (!r) return p;
+  p.k = layer_ptr(r, r->k, l);
+  p.v = layer_ptr(r, r->v, l);
+  p.seq = kv->pre_seq;
+  p.len = kv->pre_len;
+  p.max_seq = r->max_seq;
+  return p;
+}
+
+void free_kv(nc_kv *kv);
+
+void free_kv(nc_kv *kv) {
+  cudaDeviceSynchronize();
+  if (kv->graph) cudaGraphExecDestroy(kv->graph);
+  if (kv->cap_stream) cudaStreamDestroy(kv->cap_stream);
+  void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
+                kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
+                kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl,     kv->step_maps, kv->step_ws,
+                kv->row_ss,   kv->pre_seq, kv->pre_len};
+  for (void *p : ps) cudaFree(p);
+  delete kv;
+}
+
+// Sequence b of kv stops reading rows of its prefix cache (host bookkeeping;
+// the device table is reset by the kernel that replaces the sequence). A
+// source cache destroyed while linked is freed with its last link.
+void unlink_seq(nc_kv *kv, int b) {
+  if (kv->link_seq.empty() || kv->link_seq[b] < 0) return;
+  nc_kv *src = kv->prefix_src;
+  src->dep_count[kv->link_seq[b]]--;
+  src->n_dependents--;
+  kv->link_seq[b] = -1;
+  if (--kv->n_links == 0) kv->prefix_src = nullptr;
+  if (src->destroy_pending && src->n_dependents == 0) free_kv(src);
+}
+
+// Sequences [first, first + n) of kv are about to be replaced: refuse if
+// another sequence still reads shared rows from one of them (links from
+// sequences inside the range itself end with the replacement).
+bool replace_blocked(const nc_kv *kv, int first, int n, int *who) {
+  for (int b = first; b < first + n; b++) {
+    int inside = 0;
+    if (kv->prefix_src == kv)
+      for (int b2 = first; b2 < first + n; b2++) inside += kv->link_seq[b2] == b;
+    if (kv->dep_count[b] - inside > 0) {
+      *who = b;
+      return true;
+    }
+  }
+  return false;
+}
+
 // Each step below takes its sm_100a kernel when the shapes allow it and the
 // generic kernel otherwise; a failed launch of either is returned (never
 // retried on the other kernel, so a broken fast path cannot hide).
@@ -128,13 +185,21 @@ cudaError_t rope_append(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::R
   return cudaGetLastError();
 }
 
+// The layer whose K cache starts at kc.
+int layer_of(const nc_kv *kv, const void *kc) {
+  return (int)(((const char *)kc - (const char *)kv->k) / (ptrdiff_t)(kv->layer_elems * kv->model->elem));
+}
+
 // Causal MQA attention of the M rows in kv->q against layer cache kc/vc.
 cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
   if (m->fast && !rm.pos && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
     return nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, kv->max_batch, kv->max_seq, kv->y,
                                  m->status, s);
-  nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->max_seq, kv->y, s);
+  // decode rows may read shared-prefix rows; prefill rows replace their sequences
+  const nc::KvPrefix pre = rm.pos ? prefix_view(kv, layer_of(kv, kc)) : nc::KvPrefix{};
+  nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->max_seq, kv->y, s,
+                          &pre);
   return cudaGetLastError();
 }
 
@@ -263,10 +328,10 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
   if (kv->step_grid > 0 && nc::decode_step_supported(c, B)) {
     {
       ProfScope p(m, NC_K_STEP, s);
-      e = nc::k_decode_step(m, B, kv->max_batch, kv->max_seq, kv->step_maps, tokens, positions, kv->len, kv->x,
-                            kv->xl, kv->step_ss, kv->q, kv->y, kv->f, kv->k, kv->v, kv->rope, logits, noise, next,
-                            kv->cand_v, kv->cand_i, kv->step_bar, kv->step_part, kv->step_grid, kv->step_trace,
-                            kv->valid, s);
+      const nc_kv *pre = kv->prefix_src ? kv->prefix_src : kv;
+      e = nc::k_decode_step(m, kv->step_plan, B, kv->max_batch, kv->max_seq, kv->step_maps, kv->step_ws, tokens,
+                            positions, kv->len, kv->k, kv->v, kv->rope, logits, noise, next, kv->step_trace,
+                            kv->valid, kv->pre_seq, kv->pre_len, pre->max_batch, pre->max_seq, s);
     }
     return e == cudaSuccess ? sampled_pick(m, kv, logits, B, V, V, noise, kv->valid, next, s) : e;
   }
@@ -288,8 +353,9 @@ cudaError_t decode_fast_launches(nc_model *m, nc_kv *kv, const int32_t *tokens, 
     }
     {
       ProfScope p(m, NC_K_ATTN, s);
+      const nc::KvPrefix pre = prefix_view(kv, l);
       e = nc::k_dec_attn(kv->q, kc, vc, kv->pos_ws, kv->valid, B, H, kv->max_seq, kv->attn_chunk, kv->attn_splits,
-                         kv->part, kv->counters, kv->y, s);
+                         kv->part, kv->counters, kv->y, s, &pre);
       if (e != cudaSuccess) return e;
     }
     {
@@ -512,6 +578,10 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   alloc(&kv->f, elem * rows * F);
   alloc((void **)&kv->logits, sizeof(float) * (size_t)max_batch * c.vocab);
   alloc((void **)&kv->pos_ws, sizeof(int32_t) * max_batch);
+  alloc((void **)&kv->pre_seq, sizeof(int32_t) * max_batch);
+  alloc((void **)&kv->pre_len, sizeof(int32_t) * max_batch);
+  kv->link_seq.assign(max_batch, -1);
+  kv->dep_count.assign(max_batch, 0);
   if (model->fast && nc::rowops_supported(c)) alloc((void **)&kv->row_ss, sizeof(float) * ((d + 127) / 128) * rows);
   kv->dec_fast = nc::decode_fast_supported(c, 1);
   if (kv->dec_fast) {
@@ -526,17 +596,16 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
     if (e == cudaSuccess) e = cudaMemset(kv->counters, 0, sizeof(unsigned) * 1024);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&kv->cap_stream, cudaStreamNonBlocking);
     // whole-step kernel: tensor maps of the weights and of this cache
-    if (e == cudaSuccess && nc::decode_step_supported(c, 1)) {
+    if (e == cudaSuccess && nc::decode_step_plan(c, model->num_sms, &kv->step_plan)) {
       const int nmaps = nc::decode_step_maps_count(c);
       std::vector<CUtensorMap> maps(nmaps);
       alloc((void **)&kv->step_maps, sizeof(CUtensorMap) * nmaps);
-      alloc((void **)&kv->step_bar, nc::decode_step_bar_bytes());
-      alloc((void **)&kv->step_part, sizeof(float) * nc::decode_step_part_floats(model->num_sms));
-      alloc((void **)&kv->step_ss, sizeof(float) * (size_t)(2 * c.depth + 1) * 16 * 32);
-      if (e == cudaSuccess) e = cudaMemset(kv->step_bar, 0, nc::decode_step_bar_bytes());
-      if (e == cudaSuccess && nc::decode_step_build_maps(model, kv->k, kv->v, max_batch, max_seq, maps.data())) {
+      alloc(&kv->step_ws, kv->step_plan.ws_bytes);
+      if (e == cudaSuccess) e = cudaMemset(kv->step_ws, 0, kv->step_plan.ws_bytes);
+      if (e == cudaSuccess && nc::decode_step_build_maps(model, kv->k, kv->v, max_batch, max_seq, kv->step_plan,
+                                                          kv->step_ws, maps.data())) {
         e = cudaMemcpy(kv->step_maps, maps.data(), sizeof(CUtensorMap) * nmaps, cudaMemcpyHostToDevice);
-        if (e == cudaSuccess) kv->step_grid = nc::decode_step_grid(model->num_sms);
+        if (e == cudaSuccess) kv->step_grid = nc::decode_step_grid(kv->step_plan, model->num_sms);
         const char *sw = getenv("NC_DECODE_STEP_KERNEL");
         if (sw && sw[0] == '0') kv->step_grid = 0;  // per-kernel decode launches instead
       }
@@ -546,6 +615,8 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   if (e == cudaSuccess) e = cudaMemset(kv->k, 0, cache_bytes);
   if (e == cudaSuccess) e = cudaMemset(kv->v, 0, cache_bytes);
   if (e == cudaSuccess) e = cudaMemset(kv->len, 0, sizeof(int32_t) * max_batch);
+  if (e == cudaSuccess) e = cudaMemset(kv->pre_seq, 0, sizeof(int32_t) * max_batch);
+  if (e == cudaSuccess) e = cudaMemset(kv->pre_len, 0, sizeof(int32_t) * max_batch);
   if (e == cudaSuccess) e = cudaMemset(kv->valid, 0, max_batch);
   if (e == cudaSuccess) {
     // RoPE table: angle pos * base^(-2i/hd) in double, stored as (cos, sin).
@@ -573,17 +644,18 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   return NC_OK;
 }
 
+
 void nc_kv_destroy(nc_kv *kv) {
   if (!kv) return;
   cudaDeviceSynchronize();
-  if (kv->graph) cudaGraphExecDestroy(kv->graph);
-  if (kv->cap_stream) cudaStreamDestroy(kv->cap_stream);
-  void *ps[] = {kv->k,      kv->v,      kv->len,  kv->valid,    kv->rope,   kv->x,     kv->h,
-                kv->qkv,    kv->q,      kv->y,    kv->f,        kv->logits, kv->pos_ws, kv->ss,
-                kv->part,   kv->counters, kv->cand_v, kv->cand_i, kv->xl,     kv->step_maps, kv->step_bar,
-                kv->step_ss, kv->row_ss, kv->step_part};
-  for (void *p : ps) cudaFree(p);
-  delete kv;
+  // this cache's own links end; a cache others still read from is freed
+  // with their last link
+  for (int b = 0; b < (int)kv->link_seq.size(); b++) unlink_seq(kv, b);
+  if (kv->n_dependents > 0) {
+    kv->destroy_pending = true;
+    return;
+  }
+  free_kv(kv);
 }
 
 int nc_kv_lengths(const nc_kv *kv, int n, int32_t *out) {
@@ -602,12 +674,16 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
   if (logits_mode != 0 && logits_mode != 1) return fail(NC_EINVAL, "logits_mode must be 0 (last) or 1 (all)");
   if (B > kv->max_batch) return fail(NC_ERANGE, "B=%d > max_batch=%d", B, kv->max_batch);
   if (T > kv->max_seq) return fail(NC_ERANGE, "T=%d > max_seq=%d", T, kv->max_seq);
+  int who = -1;
+  if (replace_blocked(kv, 0, B, &who))
+    return fail(NC_EINVAL, "sequence %d is the shared prefix of another sequence (nc_kv_fork_shared)", who);
+  for (int b = 0; b < B; b++) unlink_seq(kv, b);
   const nc_config &c = m->cfg;
   cudaStream_t s = as_stream(stream);
   int M = B * T;
   {
     ProfScope p(m, NC_K_MISC, s);
-    nc::k_prefill_begin(kv->len, kv->valid, B, T, s);
+    nc::k_prefill_begin(kv->len, kv->valid, kv->pre_len, B, T, s);
     nc::k_embed_norm(c.dtype, d_tokens, M, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
   }
   nc::RowMap rm{T, nullptr};
@@ -698,7 +774,8 @@ int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_
   return NC_OK;
 }
 
-int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream) {
+namespace {
+int kv_fork_impl(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, bool shared, void *stream) {
   if (!src || !dst) return fail(NC_EINVAL, "null cache");
   if (src->model != dst->model) return fail(NC_EINVAL, "caches belong to different models");
   if (n < 1) return fail(NC_EINVAL, "n must be >= 1");
@@ -708,13 +785,65 @@ int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *
     return fail(NC_ERANGE, "destination max_seq %d < source max_seq %d", dst->max_seq, src->max_seq);
   if (src == dst && src_seq >= dst_first && src_seq < dst_first + n)
     return fail(NC_EINVAL, "source sequence is among the destinations");
+  int who = -1;
+  if (replace_blocked(dst, dst_first, n, &who))
+    return fail(NC_EINVAL, "sequence %d is the shared prefix of another sequence (nc_kv_fork_shared)", who);
+  // shared rows are read from the source's own prefix sequence if it has one
+  nc_kv *root = shared && src->link_seq[src_seq] >= 0 ? src->prefix_src : src;
+  const int root_seq = shared && src->link_seq[src_seq] >= 0 ? src->link_seq[src_seq] : src_seq;
+  if (shared) {
+    if (root == dst && root_seq >= dst_first && root_seq < dst_first + n)
+      return fail(NC_EINVAL, "the shared prefix's sequence is among the destinations");
+    int inside = 0;
+    for (int b = dst_first; b < dst_first + n; b++) inside += dst->link_seq[b] >= 0;
+    if (dst->prefix_src && dst->prefix_src != root && dst->n_links - inside > 0)
+      return fail(NC_EINVAL, "the destination cache already shares prefixes with another cache");
+  }
   const nc_config &c = src->model->cfg;
-  ProfScope p(src->model, NC_K_MISC, as_stream(stream));
-  nc::k_kv_fork((int)src->model->elem, src->k, src->v, src->layer_elems, src->max_seq, src_seq, src->len, dst->k,
-                dst->v, dst->layer_elems, dst->max_seq, dst_first, n, dst->len, c.depth, c.n_kv_head * c.head_dim,
-                src->model->status, as_stream(stream));
+  cudaStream_t s = as_stream(stream);
+  // the source's shared rows, as they are before any link changes below
+  const nc::KvPrefix src_pre = prefix_view(src, 0);
+  const size_t pre_layer = src->prefix_src ? src->prefix_src->layer_elems : 0;
+  for (int b = dst_first; b < dst_first + n; b++) unlink_seq(dst, b);
+  if (shared) {
+    if (dst->prefix_src != root) {
+      // the step kernel reads shared rows through the prefix cache's maps
+      if (dst->step_maps && dst->step_grid > 0) {
+        std::vector<CUtensorMap> pm(2);
+        if (!nc::decode_step_prefix_maps(root->k, root->v, c, root->max_batch, root->max_seq, pm.data()))
+          return fail(NC_ECUDA, "tensor maps of the shared prefix");
+        NC_CUDA_TRY(cudaMemcpy(dst->step_maps + nc::decode_step_prefix_map_index(c), pm.data(),
+                               sizeof(CUtensorMap) * 2, cudaMemcpyHostToDevice));
+      }
+      if (dst->graph) {  // the captured step carries the old prefix shape
+        cudaGraphExecDestroy(dst->graph);
+        dst->graph = nullptr;
+      }
+      dst->graph_ready = false;
+    }
+    dst->prefix_src = root;
+    for (int b = dst_first; b < dst_first + n; b++) {
+      dst->link_seq[b] = root_seq;
+      dst->n_links++;
+      root->dep_count[root_seq]++;
+      root->n_dependents++;
+    }
+  }
+  ProfScope p(src->model, NC_K_MISC, s);
+  nc::k_kv_fork((int)src->model->elem, src->k, src->v, src->layer_elems, src->max_seq, src_seq, src->len, src_pre,
+                pre_layer, dst->k, dst->v, dst->layer_elems, dst->max_seq, dst_first, n, dst->len, dst->pre_seq,
+                dst->pre_len, shared, c.depth, c.n_kv_head * c.head_dim, src->model->status, s);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
+}
+}  // namespace
+
+int nc_kv_fork(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream) {
+  return kv_fork_impl(src, src_seq, dst, dst_first, n, false, stream);
+}
+
+int nc_kv_fork_shared(nc_kv *src, int src_seq, nc_kv *dst, int dst_first, int n, void *stream) {
+  return kv_fork_impl(src, src_seq, dst, dst_first, n, true, stream);
 }
 
 int nc_kv_set_sampling(nc_kv *kv, float temperature, int top_k) {

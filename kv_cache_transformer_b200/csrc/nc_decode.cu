@@ -440,6 +440,7 @@ struct DecAttnArgs {
   float *part;          // [B][splits][16][130]: m, l, O[128] per head row
   unsigned *counters;   // [B]
   bf16 *y;              // [B][H][128]
+  KvPrefix pre;         // shared prefixes (pre.len null: none)
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -491,6 +492,10 @@ __global__ void __launch_bounds__(ATHREADS) dec_attn_kernel(DecAttnArgs a) {
   const int n_tiles = k_end > k_begin ? (k_end - k_begin + AKT - 1) / AKT : 0;
   const bf16 *Kb = a.kc + (size_t)b * a.max_seq * 128;
   const bf16 *Vb = a.vc + (size_t)b * a.max_seq * 128;
+  // keys below the shared length live in the prefix cache's sequence
+  const int plen = a.pre.len ? a.pre.len[b] : 0;
+  const bf16 *PK = plen ? (const bf16 *)a.pre.k + (size_t)a.pre.seq[b] * a.pre.max_seq * 128 : Kb;
+  const bf16 *PV = plen ? (const bf16 *)a.pre.v + (size_t)a.pre.seq[b] * a.pre.max_seq * 128 : Vb;
 
   auto load_tile = [&](int it, int stage) {
     const int key0 = k_begin + it * AKT;
@@ -500,8 +505,9 @@ __global__ void __launch_bounds__(ATHREADS) dec_attn_kernel(DecAttnArgs a) {
       const int key = key0 + r;
       const bool in = key < k_end;
       const size_t off = (size_t)(in ? key : 0) * 128 + c * 8;
-      cp_async16(kd + atile_off(r, c), Kb + off, in);
-      cp_async16(vd + atile_off(r, c), Vb + off, in);
+      const bool sh = in && key < plen;
+      cp_async16(kd + atile_off(r, c), (sh ? PK : Kb) + off, in);
+      cp_async16(vd + atile_off(r, c), (sh ? PV : Vb) + off, in);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
@@ -830,8 +836,9 @@ cudaError_t k_dec_linear(int src, int epi, const void *W, int N, int K, int B, c
 
 cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int32_t *pos, const uint8_t *valid, int B,
                        int H, int max_seq, int chunk, int splits, float *part, unsigned *counters, void *y,
-                       cudaStream_t s) {
+                       cudaStream_t s, const KvPrefix *pre) {
   DecAttnArgs a;
+  a.pre = pre ? *pre : KvPrefix{};
   a.q = (const bf16 *)q;
   a.kc = (const bf16 *)kc;
   a.vc = (const bf16 *)vc;

@@ -18,17 +18,18 @@ namespace nc {
 std::atomic<unsigned long long> g_launches{0};
 
 // --------------------------------------------------------------- sequences
-__global__ void prefill_begin_kernel(int32_t *len, uint8_t *valid, int B, int T) {
+__global__ void prefill_begin_kernel(int32_t *len, uint8_t *valid, int32_t *pre_len, int B, int T) {
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) {
     len[b] = T;
     valid[b] = 1;
+    pre_len[b] = 0;  // a replaced sequence owns all its rows
   }
 }
 
-void k_prefill_begin(int32_t *len, uint8_t *valid, int B, int T, cudaStream_t s) {
+void k_prefill_begin(int32_t *len, uint8_t *valid, int32_t *pre_len, int B, int T, cudaStream_t s) {
   count_launch();
-  prefill_begin_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, valid, B, T);
+  prefill_begin_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, valid, pre_len, B, T);
 }
 
 // A decode row is valid iff its position is the sequence's current length and
@@ -250,7 +251,7 @@ void k_rope_qknorm_append(int dtype, const void *qkv, RowMap rm, int M, int H, i
 // 0..pos of its sequence (exact scores kept in shared memory).
 template <typename T>
 __global__ void attn_generic_kernel(const T *q, const T *kc, const T *vc, RowMap rm, int H, int Hkv, int hd,
-                                    int max_seq, T *y) {
+                                    int max_seq, T *y, KvPrefix pre) {
   extern __shared__ float sm[];
   __shared__ float red[32];
   int m = blockIdx.x, h = blockIdx.y;
@@ -262,10 +263,15 @@ __global__ void attn_generic_kernel(const T *q, const T *kc, const T *vc, RowMap
   __syncthreads();
   const T *K = kc + (size_t)b * max_seq * kd + g * hd;
   const T *V = vc + (size_t)b * max_seq * kd + g * hd;
+  // rows below the shared length live in the prefix cache's sequence
+  const int plen = pre.len ? pre.len[b] : 0;
+  const T *PK = plen ? (const T *)pre.k + (size_t)pre.seq[b] * pre.max_seq * kd + g * hd : K;
+  const T *PV = plen ? (const T *)pre.v + (size_t)pre.seq[b] * pre.max_seq * kd + g * hd : V;
   float scale = 1.0f / sqrtf((float)hd), mx = -INFINITY;
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
     float dot = 0.f;
-    for (int e = 0; e < hd; e++) dot = fmaf(qs[e], to_f32(K[(size_t)j * kd + e]), dot);
+    const T *Kj = (j < plen ? PK : K) + (size_t)j * kd;
+    for (int e = 0; e < hd; e++) dot = fmaf(qs[e], to_f32(Kj[e]), dot);
     s[j] = dot * scale;
     mx = fmaxf(mx, s[j]);
   }
@@ -280,14 +286,15 @@ __global__ void attn_generic_kernel(const T *q, const T *kc, const T *vc, RowMap
   __syncthreads();
   for (int e = threadIdx.x; e < hd; e += blockDim.x) {
     float acc = 0.f;
-    for (int j = 0; j < n; j++) acc = fmaf(s[j], to_f32(V[(size_t)j * kd + e]), acc);
+    for (int j = 0; j < n; j++) acc = fmaf(s[j], to_f32((j < plen ? PV : V)[(size_t)j * kd + e]), acc);
     y[((size_t)m * H + h) * hd + e] = from_f32<T>(acc / z);
   }
 }
 
 void k_attention_generic(int dtype, const void *q, const void *kc, const void *vc, RowMap rm, int M, int H,
-                         int Hkv, int hd, int max_seq, void *y, cudaStream_t s) {
+                         int Hkv, int hd, int max_seq, void *y, cudaStream_t s, const KvPrefix *pre) {
   if (M <= 0) return;
+  const KvPrefix pv = pre ? *pre : KvPrefix{};
   size_t smem = sizeof(float) * ((size_t)hd + max_seq);
   dim3 grid(M, H);
   if (dtype == NC_F32) {
@@ -295,13 +302,13 @@ void k_attention_generic(int dtype, const void *q, const void *kc, const void *v
       cudaFuncSetAttribute(attn_generic_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     count_launch();
     attn_generic_kernel<float><<<grid, 128, smem, s>>>((const float *)q, (const float *)kc, (const float *)vc, rm,
-                                                       H, Hkv, hd, max_seq, (float *)y);
+                                                       H, Hkv, hd, max_seq, (float *)y, pv);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(attn_generic_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     count_launch();
     attn_generic_kernel<bf16><<<grid, 128, smem, s>>>((const bf16 *)q, (const bf16 *)kc, (const bf16 *)vc, rm, H,
-                                                      Hkv, hd, max_seq, (bf16 *)y);
+                                                      Hkv, hd, max_seq, (bf16 *)y, pv);
   }
 }
 
@@ -340,47 +347,86 @@ void k_argmax_rows(const float *logits, int rows, int V, long long row_stride, c
 }
 
 // ------------------------------------------------------------------ fork
-// Copy rows [0, len) of sequence src_seq (every layer, K and V) into n
-// destination sequences; len is read on the device from src_len.
-__global__ void kv_fork_kernel(const uint32_t *src_k, const uint32_t *src_v, size_t src_layer_words,
-                               size_t src_seq_words, size_t src_off_words, const int32_t *src_len,
-                               uint32_t *dst_k, uint32_t *dst_v, size_t dst_layer_words, size_t dst_seq_words,
-                               int dst_first, int dst_max_seq, int32_t *dst_len, int row_words, uint32_t *status) {
-  int layer = blockIdx.y >> 1, which = blockIdx.y & 1, i = blockIdx.z;
-  int len = *src_len;
-  if (len > dst_max_seq) {
-    if (blockIdx.x == 0 && threadIdx.x == 0 && layer == 0 && which == 0) atomicOr(status, (unsigned)NC_DEV_BAD_POSITION);
-    len = dst_max_seq;
+struct ForkArgs {
+  const uint32_t *src_k, *src_v;          // source cache at layer 0, sequence src_seq
+  size_t src_layer_words;
+  const int32_t *src_len;                  // &len[src_seq]
+  const int32_t *src_pre_len, *src_pre_seq;  // &pre_len[src_seq], &pre_seq[src_seq] (null: none)
+  const uint32_t *pre_k, *pre_v;           // the source's prefix cache at layer 0
+  size_t pre_layer_words, pre_seq_words;
+  uint32_t *dst_k, *dst_v;                 // destination cache at layer 0
+  size_t dst_layer_words, dst_seq_words;
+  int dst_first, dst_max_seq, row_words, src_seq;
+  int32_t *dst_len, *dst_pre_seq, *dst_pre_len;
+  int shared;                              // 1: share the rows below the shared length
+  uint32_t *status;
+};
+
+// One (layer, K or V, destination) per blockIdx.(y, z): copy the rows the
+// destination owns; the source's rows below its own shared length come from
+// its prefix cache. Lengths and prefix tables are read on the device.
+__global__ void kv_fork_kernel(ForkArgs f) {
+  const int layer = blockIdx.y >> 1, which = blockIdx.y & 1, i = blockIdx.z;
+  int len = *f.src_len;
+  if (len > f.dst_max_seq) {
+    if (blockIdx.x == 0 && threadIdx.x == 0 && layer == 0 && which == 0) atomicOr(f.status, (unsigned)NC_DEV_BAD_POSITION);
+    len = f.dst_max_seq;
   }
   if (len < 0) len = 0;
-  const uint32_t *src = (which ? src_v : src_k) + layer * src_layer_words + src_off_words;
-  uint32_t *dst = (which ? dst_v : dst_k) + layer * dst_layer_words + (size_t)(dst_first + i) * dst_seq_words;
-  size_t total = (size_t)len * row_words;
-  for (size_t w = (size_t)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (size_t)gridDim.x * blockDim.x)
-    dst[w] = src[w];
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) dst_len[dst_first + i] = len;
+  const int spl = f.src_pre_len ? *f.src_pre_len : 0;  // rows of the source living in its prefix cache
+  const int first = f.shared ? (spl > 0 ? spl : len / 64 * 64) : 0;
+  const uint32_t *own = (which ? f.src_v : f.src_k) + layer * f.src_layer_words;
+  const uint32_t *pre = spl > 0 ? (which ? f.pre_v : f.pre_k) + layer * f.pre_layer_words +
+                                      (size_t)*f.src_pre_seq * f.pre_seq_words
+                                : own;
+  uint32_t *dst = (which ? f.dst_v : f.dst_k) + layer * f.dst_layer_words + (size_t)(f.dst_first + i) * f.dst_seq_words;
+  const size_t w0 = (size_t)first * f.row_words, total = (size_t)len * f.row_words, wsh = (size_t)spl * f.row_words;
+  for (size_t w = w0 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (size_t)gridDim.x * blockDim.x)
+    dst[w] = w < wsh ? pre[w] : own[w];
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    f.dst_len[f.dst_first + i] = len;
+    f.dst_pre_len[f.dst_first + i] = first;
+    f.dst_pre_seq[f.dst_first + i] = spl > 0 ? *f.src_pre_seq : f.src_seq;
+  }
 }
 
 void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_layer_elems, int src_max_seq,
-               int src_seq, const int32_t *src_len, void *dst_k, void *dst_v, size_t dst_layer_elems,
-               int dst_max_seq, int dst_first, int n, int32_t *dst_len, int depth, int kd, uint32_t *status,
+               int src_seq, const int32_t *src_len, const KvPrefix &src_pre, size_t pre_layer_elems, void *dst_k,
+               void *dst_v, size_t dst_layer_elems, int dst_max_seq, int dst_first, int n, int32_t *dst_len,
+               int32_t *dst_pre_seq, int32_t *dst_pre_len, bool shared, int depth, int kd, uint32_t *status,
                cudaStream_t s) {
   if (n <= 0) return;
-  size_t per = (size_t)elem_bytes / 2;  // 16-bit units per element
+  const size_t per = (size_t)elem_bytes / 2;  // 16-bit units per element
   // all row sizes are whole 32-bit words: kd is even
-  int row_words = (int)((size_t)kd * elem_bytes / 4);
-  size_t src_layer_words = src_layer_elems * per / 2, dst_layer_words = dst_layer_elems * per / 2;
-  size_t src_seq_words = (size_t)src_max_seq * row_words, dst_seq_words = (size_t)dst_max_seq * row_words;
+  const int row_words = (int)((size_t)kd * elem_bytes / 4);
+  ForkArgs f;
+  f.src_layer_words = src_layer_elems * per / 2;
+  const size_t src_seq_words = (size_t)src_max_seq * row_words;
+  f.src_k = (const uint32_t *)src_k + (size_t)src_seq * src_seq_words;
+  f.src_v = (const uint32_t *)src_v + (size_t)src_seq * src_seq_words;
+  f.src_len = src_len + src_seq;
+  f.src_pre_len = src_pre.len ? src_pre.len + src_seq : nullptr;
+  f.src_pre_seq = src_pre.seq ? src_pre.seq + src_seq : nullptr;
+  f.pre_k = (const uint32_t *)src_pre.k;
+  f.pre_v = (const uint32_t *)src_pre.v;
+  f.pre_layer_words = pre_layer_elems * per / 2;
+  f.pre_seq_words = (size_t)src_pre.max_seq * row_words;
+  f.dst_k = (uint32_t *)dst_k;
+  f.dst_v = (uint32_t *)dst_v;
+  f.dst_layer_words = dst_layer_elems * per / 2;
+  f.dst_seq_words = (size_t)dst_max_seq * row_words;
+  f.dst_first = dst_first;
+  f.dst_max_seq = dst_max_seq;
+  f.row_words = depth > 0 ? row_words : 0;
+  f.src_seq = src_seq;
+  f.dst_len = dst_len;
+  f.dst_pre_seq = dst_pre_seq;
+  f.dst_pre_len = dst_pre_len;
+  f.shared = shared ? 1 : 0;
+  f.status = status;
   dim3 grid(32, (unsigned)(depth > 0 ? depth * 2 : 1), (unsigned)n);
-  if (depth <= 0) {
-    // no layers: only the lengths change
-    grid.y = 1;
-  }
   count_launch();
-  kv_fork_kernel<<<grid, 256, 0, s>>>((const uint32_t *)src_k, (const uint32_t *)src_v, src_layer_words,
-                                      src_seq_words, (size_t)src_seq * src_seq_words, src_len + src_seq,
-                                      (uint32_t *)dst_k, (uint32_t *)dst_v, dst_layer_words, dst_seq_words,
-                                      dst_first, dst_max_seq, dst_len, depth > 0 ? row_words : 0, status);
+  kv_fork_kernel<<<grid, 256, 0, s>>>(f);
 }
 
 }  // namespace nc

@@ -41,6 +41,35 @@ struct nc_model {
   std::vector<cudaEvent_t> event_pool;
 };
 
+namespace nc {
+// Shared-prefix view for attention (nc_kv_fork_shared): key/value row j < len[b]
+// of sequence b is row j of sequence seq[b] of the prefix cache (k, v: that
+// cache's K and V at the layer being read, max_seq rows per sequence). len ==
+// nullptr: every row is the sequence's own.
+struct KvPrefix {
+  const void *k = nullptr, *v = nullptr;
+  const int32_t *seq = nullptr, *len = nullptr;
+  int max_seq = 0;
+};
+
+// Launch plan of the whole-step decode kernel (nc_step.cu): CTAs, the rows
+// each CTA owns in every linear phase, its shared-memory ring and the layout
+// of its device workspace.
+struct StepPlan {
+  int grid = 0;                      // CTAs, one per SM (0 = no plan)
+  int n_qkv = 0;                     // QKV units of 16 rows (8 RoPE pairs)
+  int r_o = 0, r_f = 0, r_p = 0;     // rows per CTA: O projection, MLP fc, MLP projection
+  int s_p = 0;                       // K splits of the MLP projection
+  int r_h = 0;                       // lm_head rows per CTA
+  int n_o = 0, n_f = 0, n_p = 0, n_h = 0;  // units of each phase
+  int slots = 0;                     // 16 KB ring slots
+  size_t smem = 0;                   // dynamic shared memory per CTA
+  size_t ws_bytes = 0;               // device workspace
+  size_t off_ctr = 0, off_x0 = 0, off_x1 = 0, off_xb0 = 0, off_xb1 = 0, off_y = 0, off_f = 0, off_qk = 0,
+         off_ss = 0, off_cv = 0, off_ci = 0, off_ap = 0, off_pp = 0;
+};
+}  // namespace nc
+
 struct nc_kv {
   nc_model *model = nullptr;
   int max_batch = 0, max_seq = 0;
@@ -71,11 +100,20 @@ struct nc_kv {
   float *row_ss = nullptr;     // [ceil(d/128)][max_rows] per-128-column sums of squares of x rows (prefill)
   // whole-step decode kernel (nc_step.cu)
   int step_grid = 0;           // CTAs of the step kernel, 0 = not available
+  nc::StepPlan step_plan;
   CUtensorMap *step_maps = nullptr;  // device copy of the step kernel's tensor maps
-  unsigned long long *step_bar = nullptr;  // its grid-barrier counter and split counters
-  float *step_part = nullptr;  // split-K partials of its MLP proj phase
-  float *step_ss = nullptr;    // [2*depth+1][16][32] per-128-column sums of squares
+  void *step_ws = nullptr;     // its workspace (activations, partials, counters)
   unsigned long long *step_trace = nullptr;  // caller's phase-timestamp buffer (nc_decode_trace), or null
+  // shared prefixes (nc_kv_fork_shared): sequence b reads its first
+  // pre_len[b] key/value rows of every layer from sequence pre_seq[b] of
+  // prefix_src (a multiple of 64; 0 = none)
+  int32_t *pre_seq = nullptr, *pre_len = nullptr;  // device [max_batch]
+  nc_kv *prefix_src = nullptr;   // the cache those rows live in (host bookkeeping below mirrors the device)
+  std::vector<int> link_seq;     // per sequence: the prefix_src sequence it reads from, -1 none
+  int n_links = 0;               // live links of this cache into prefix_src
+  std::vector<int> dep_count;    // per sequence: live links of any cache into it
+  int n_dependents = 0;          // live links of any cache into this one
+  bool destroy_pending = false;  // destroyed while links into it were live: freed with the last link
   // sampled token pick (nc_kv_set_sampling): temperature 1 and top_k 0 are
   // the plain argmax(logits + noise)
   float temperature = 1.f;
@@ -136,7 +174,7 @@ struct GemmFuse {
 };
 
 // ---- generic kernels (any even head_dim; fp32 or bf16 storage) ----
-void k_prefill_begin(int32_t *len, uint8_t *valid, int B, int T, cudaStream_t s);
+void k_prefill_begin(int32_t *len, uint8_t *valid, int32_t *pre_len, int B, int T, cudaStream_t s);
 void k_decode_begin(const int32_t *positions, int32_t *len, uint8_t *valid, int B, int max_seq,
                     uint32_t *status, cudaStream_t s);
 void k_embed_norm(int dtype, const int32_t *tokens, int M, const void *wte, int d, int vocab, float eps,
@@ -149,12 +187,21 @@ void k_rope_qknorm_append(int dtype, const void *qkv, RowMap rm, int M, int H, i
                           const float2 *rope, void *q_out, void *kc, void *vc, int max_seq,
                           const uint8_t *valid, float eps, cudaStream_t s);
 void k_attention_generic(int dtype, const void *q, const void *kc, const void *vc, RowMap rm, int M, int H,
-                         int Hkv, int hd, int max_seq, void *y, cudaStream_t s);
+                         int Hkv, int hd, int max_seq, void *y, cudaStream_t s, const KvPrefix *pre = nullptr);
 void k_argmax_rows(const float *logits, int rows, int V, long long row_stride, const float *noise,
                    int32_t *next, const uint8_t *valid, cudaStream_t s);
+// Copy (shared == false) or share (true) the rows of sequence src_seq into
+// sequences dst_first .. dst_first + n - 1. Copy: every row, the source's
+// shared rows read from its prefix cache (src_pre, layer 0 pointers, with
+// its per-layer stride pre_layer_elems); the destinations own all their rows.
+// Share: the destinations read rows below the shared length (the source's
+// own shared length if it has one, else its length rounded down to 64) from
+// the source's prefix sequence or the source itself (dst_pre_seq/len set on
+// the device) and get a copy of the rest.
 void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_layer_elems, int src_max_seq,
-               int src_seq, const int32_t *src_len, void *dst_k, void *dst_v, size_t dst_layer_elems,
-               int dst_max_seq, int dst_first, int n, int32_t *dst_len, int depth, int kd, uint32_t *status,
+               int src_seq, const int32_t *src_len, const KvPrefix &src_pre, size_t pre_layer_elems, void *dst_k,
+               void *dst_v, size_t dst_layer_elems, int dst_max_seq, int dst_first, int n, int32_t *dst_len,
+               int32_t *dst_pre_seq, int32_t *dst_pre_len, bool shared, int depth, int kd, uint32_t *status,
                cudaStream_t s);
 
 
@@ -194,7 +241,7 @@ void attn_decode_plan(int B, int max_seq, int num_sms, int *chunk, int *splits);
 size_t attn_decode_partial_floats(int B, int splits);
 cudaError_t k_dec_attn(const void *q, const void *kc, const void *vc, const int32_t *pos, const uint8_t *valid, int B,
                        int H, int max_seq, int chunk, int splits, float *part, unsigned *counters, void *y,
-                       cudaStream_t s);
+                       cudaStream_t s, const KvPrefix *pre = nullptr);
 
 
 // ---- sampled token pick (nc_sample.cu) ----
@@ -207,17 +254,18 @@ cudaError_t k_sample_topk(const float *logits, int B, int V, long long stride, c
 
 // ---- whole decode step in one persistent kernel (nc_step.cu) ----
 bool decode_step_supported(const nc_config &c, int B);
+bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *plan);
 int decode_step_maps_count(const nc_config &c);
+int decode_step_prefix_map_index(const nc_config &c);
+bool decode_step_prefix_maps(const void *kcache, const void *vcache, const nc_config &c, int max_batch, int max_seq,
+                             CUtensorMap *out);
 bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *vcache, int max_batch, int max_seq,
-                            CUtensorMap *out);
-int decode_step_grid(int num_sms);
-cudaError_t k_decode_step(const nc_model *m, int B, int max_batch, int max_seq, const CUtensorMap *maps_dev,
-                          const int32_t *tokens, const int32_t *positions, int32_t *len, float *x0, float *x1,
-                          float *ss, void *q, void *y, void *f, void *kc, void *vc, const float2 *rope, float *logits,
-                          const float *noise, int32_t *next, float *cand_v, int *cand_i, unsigned long long *bar,
-                          float *split_part, int grid, unsigned long long *trace, uint8_t *valid_out,
-                          cudaStream_t s);
-size_t decode_step_bar_bytes();              // grid-barrier word + split counters, zeroed per launch
-size_t decode_step_part_floats(int num_sms);  // split-K partials of the MLP proj phase
+                            const StepPlan &p, void *ws, CUtensorMap *out);
+int decode_step_grid(const StepPlan &p, int num_sms);
+cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_batch, int max_seq,
+                          const CUtensorMap *maps_dev, void *ws, const int32_t *tokens, const int32_t *positions,
+                          int32_t *len, void *kc, void *vc, const float2 *rope, float *logits, const float *noise,
+                          int32_t *next, unsigned long long *trace, uint8_t *valid_out, const int32_t *pre_seq,
+                          const int32_t *pre_len, int pmax_batch, int pmax_seq, cudaStream_t s);
 
 }  // namespace nc

@@ -112,3 +112,60 @@ def test_exact_ties_pick_the_lowest_index(cfg):
                 check(lg2, n2, nz, f"decode step {s} noise {nz is not None}")
                 cur = n2
             assert run.status() == 0
+
+
+@pytest.mark.parametrize("temp,k", [(0.0, 0), (1.0, 0), (1.0, 50), (0.7, 1000), (1.3, 1), (0.9, 65535)])
+def test_sample_topk_kernel_matches_oracle(temp, k):
+    """nc_sample_topk against the oracle's pick on the same fp32 logits and
+    noise: the decision is taken in fp32 on both sides, so it must agree
+    exactly; rows carry exact ties, some of them on the top-k cut."""
+    import torch
+    import kv_cache_transformer_b200 as nc
+    B, V = 5, 65536
+    rng = np.random.default_rng(int(1000 * temp) + k)
+    z = (rng.standard_normal((B, V)) * 3).astype(np.float32)
+    z[1, :] = np.float32(1.25)                     # every logit tied
+    z[2, 1000:3000] = z[2].max()                   # a block of tied maxima wider than k
+    z[3, ::7] = np.float32(0.5)                    # many ties in the middle of the order
+    z[4, 5] = np.float32(-0.0)
+    z[4, 6] = np.float32(0.0)
+    noise = syn.gumbel(17, (B, V), stream=int(10 * temp) + k)
+    stride = V + 96                                # rows of a wider logits buffer
+    buf = torch.zeros((B, stride), dtype=torch.float32)
+    buf[:, :V] = torch.from_numpy(z)
+    lg = buf.cuda()[:, :V]
+    nxt = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+    nc.nc_sample_topk(lg, nxt, torch.from_numpy(noise).cuda(), temp, k)
+    torch.cuda.synchronize()
+    got = nxt.cpu().numpy()
+    for b in range(B):
+        want = orc.sample_topk(z[b], noise[b], temp, k)
+        assert int(got[b]) == want, f"row {b}: kernel {got[b]}, oracle {want}"
+
+
+@pytest.mark.parametrize("temp,k", [(0.8, 20), (0.0, 0)])
+def test_engine_sampling_in_prefill_and_decode(temp, k):
+    """nc_kv_set_sampling: the engine's next tokens are the sampled pick over
+    the logits it returns (prefill and the whole-step decode), and those
+    logits still match the oracle."""
+    cfg = SMALL
+    B, T, steps = 4, 30, 3
+    prompts = syn.tokens_zipf(49, (B, T), cfg.vocab)
+    run = Run(cfg, blob_for(cfg), B, T + steps + 1)
+    run.kv.set_sampling(temp, k)
+    noise = syn.gumbel(5, (B, cfg.vocab), stream=20)
+    lg, nxt = run.prefill(prompts, noise=noise)
+    om = orc.OracleModel(cfg, blob_for(cfg))
+    seqs = [om.new_seq(T + steps + 1) for _ in range(B)]
+    for b in range(B):
+        check_logits(lg[b], seqs[b].prefill(prompts[b]), tol_for(cfg), f"prefill seq {b}")
+        assert int(nxt[b]) == orc.sample_topk(lg[b], noise[b], temp, k)
+    cur = nxt.copy()
+    for s in range(steps):
+        nz = syn.gumbel(5, (B, cfg.vocab), stream=21 + s)
+        lg2, n2 = run.decode(cur, np.full(B, T + s, np.int32), nz)
+        for b in range(B):
+            check_logits(lg2[b], seqs[b].step(int(cur[b])), tol_for(cfg), f"step {s} seq {b}")
+            assert int(n2[b]) == orc.sample_topk(lg2[b], nz[b], temp, k), f"step {s} seq {b}"
+        cur = n2
+    assert run.status() == 0
