@@ -137,6 +137,24 @@ int nc_kv_lengths(const nc_kv *kv, int n, int32_t *out);
 int nc_prefill(nc_model *model, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode,
                float *d_logits, int32_t *d_next, const float *d_noise, void *stream);
 
+/* Append a chunk: run d_tokens[B,T] at positions len[b] .. len[b] + T - 1
+ * of sequences 0..B-1, after whatever each already holds (its prompt,
+ * earlier chunks, decode steps). This is how the Engine feeds tokens into a
+ * running sequence (the launch article's "高效推理" item: tool use, whose
+ * outputs go back into the conversation). Each sequence's K/V rows for the
+ * chunk are appended and its length grows by T. Outputs as in nc_prefill:
+ * d_logits [B,V] for the chunk's last position (logits_mode 0) or [B,T,V]
+ * for all of its positions (1), d_next from the last position (+ d_noise,
+ * or the sampled pick of nc_kv_set_sampling). A sequence whose chunk does
+ * not fit (len + T > max_seq) is skipped: its cache and length stay
+ * unchanged, NC_DEV_BAD_POSITION is raised, and its outputs are not
+ * meaningful. A sequence reading a shared prefix (nc_kv_fork_shared) may be
+ * extended. The linear layers run on the tensor-core GEMM; RoPE/QK norm and
+ * attention over the cached prefix run on the shape-generic kernels.
+ * Errors: as nc_prefill. */
+int nc_prefill_extend(nc_model *model, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode,
+                      float *d_logits, int32_t *d_next, const float *d_noise, void *stream);
+
 /* Decode one token for each of sequences 0..B-1: d_tokens[B] are fed at
  * d_positions[B] (int32, device). positions[b] must equal sequence b's
  * current length (< max_seq); the token's K/V are appended there and the

@@ -36,7 +36,7 @@ EXPORTS = (
     "nc_profile_enable", "nc_profile_read", "nc_launch_count", "nc_gemm_bf16",
     "nc_attention_prefill_bf16", "nc_attention_decode_workspace_bytes", "nc_attention_decode_bf16",
     "nc_attention_decode_bf16_static", "nc_decode_trace", "nc_kv_set_sampling", "nc_sample_topk",
-    "nc_kv_fork_shared",
+    "nc_kv_fork_shared", "nc_prefill_extend",
 )
 NC_EPI_STORE, NC_EPI_RELU2, NC_EPI_RESID, NC_EPI_SOFTCAP = 0, 1, 2, 3
 NC_K_GEMM, NC_K_ATTN, NC_K_HEAD, NC_K_MISC, NC_K_STEP, NC_K_COUNT = 0, 1, 2, 3, 4, 5
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
             L.nc_kv_destroy.restype = None
             L.nc_kv_lengths.argtypes = [vp, i, vp]
             L.nc_prefill.argtypes = [vp, vp, vp, i, i, i, vp, vp, vp, vp]
+            L.nc_prefill_extend.argtypes = [vp, vp, vp, i, i, i, vp, vp, vp, vp]
             L.nc_decode_step.argtypes = [vp, vp, vp, vp, i, vp, vp, vp, vp]
             L.nc_kv_fork.argtypes = [vp, i, vp, i, i, vp]
             L.nc_kv_fork_shared.argtypes = [vp, i, vp, i, i, vp]
@@ -186,6 +187,18 @@ def nc_prefill(model_h, kv_h, tokens, logits_mode: int = 0, logits=None, next=No
     B, T = tokens.shape
     V = vocab
     _check(lib().nc_prefill(
+        model_h, kv_h, _dptr(tokens, torch.int32, name="tokens"), int(B), int(T), int(logits_mode),
+        _dptr(logits, torch.float32, None if V is None else (B * T * V if logits_mode else B * V), "logits"),
+        _dptr(next, torch.int32, B, "next"),
+        _dptr(noise, torch.float32, None if V is None else B * V, "noise"), _stream(stream)))
+
+
+def nc_prefill_extend(model_h, kv_h, tokens, logits_mode: int = 0, logits=None, next=None, noise=None, stream=None,
+                      vocab: int | None = None):
+    import torch
+    B, T = tokens.shape
+    V = vocab
+    _check(lib().nc_prefill_extend(
         model_h, kv_h, _dptr(tokens, torch.int32, name="tokens"), int(B), int(T), int(logits_mode),
         _dptr(logits, torch.float32, None if V is None else (B * T * V if logits_mode else B * V), "logits"),
         _dptr(next, torch.int32, B, "next"),
@@ -348,6 +361,10 @@ class Model:
 
     def prefill(self, kv: "KVCache", tokens, logits_mode: int = 0, logits=None, next=None, noise=None, stream=None):
         nc_prefill(self._h, kv.handle, tokens, logits_mode, logits, next, noise, stream, vocab=self.vocab)
+
+    def extend(self, kv: "KVCache", tokens, logits_mode: int = 0, logits=None, next=None, noise=None, stream=None):
+        """Append tokens [B, T] to sequences 0..B-1 at their current lengths (nc_prefill_extend)."""
+        nc_prefill_extend(self._h, kv.handle, tokens, logits_mode, logits, next, noise, stream, vocab=self.vocab)
 
     def decode_step(self, kv: "KVCache", tokens, positions, noise=None, logits=None, next=None, stream=None):
         nc_decode_step(self._h, kv.handle, tokens, positions, noise, logits, next, stream, vocab=self.vocab)

@@ -178,7 +178,7 @@ cudaError_t norm_rows(nc_model *m, nc_kv *kv, int M, cudaStream_t s) {
 // RoPE + QK norm of the M rows of kv->qkv, q out, K/V appended to the cache.
 cudaError_t rope_append(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (!rm.pos && nc::rowops_supported(c))
+  if (!rm.pos && !rm.off && nc::rowops_supported(c))
     return nc::k_rope_qk_bf16(kv->qkv, M, rm.T, c.n_head, kv->rope, kv->q, kc, vc, kv->max_seq, c.norm_eps, s);
   nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->rope, kv->q, kc, vc,
                            kv->max_seq, kv->valid, c.norm_eps, s);
@@ -193,11 +193,12 @@ int layer_of(const nc_kv *kv, const void *kc) {
 // Causal MQA attention of the M rows in kv->q against layer cache kc/vc.
 cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (m->fast && !rm.pos && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
+  if (m->fast && !rm.pos && !rm.off && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
     return nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, kv->max_batch, kv->max_seq, kv->y,
                                  m->status, s);
-  // decode rows may read shared-prefix rows; prefill rows replace their sequences
-  const nc::KvPrefix pre = rm.pos ? prefix_view(kv, layer_of(kv, kc)) : nc::KvPrefix{};
+  // decode rows and appended chunks may read shared-prefix rows; prefill rows
+  // replace their sequences
+  const nc::KvPrefix pre = (rm.pos || rm.off) ? prefix_view(kv, layer_of(kv, kc)) : nc::KvPrefix{};
   nc::k_attention_generic(c.dtype, kv->q, kc, vc, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->max_seq, kv->y, s,
                           &pre);
   return cudaGetLastError();
@@ -215,7 +216,7 @@ cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::Row
 bool fused_layers_ok(const nc_model *m, const nc_kv *kv, int M, nc::RowMap rm) {
   const nc_config &c = m->cfg;
   const int d = c.d_model, q = c.n_head * 128, F = c.mlp_hidden;
-  return m->fast && !rm.pos && M >= 128 && kv->row_ss && nc::rowops_supported(c) &&
+  return m->fast && !rm.pos && !rm.off && M >= 128 && kv->row_ss && nc::rowops_supported(c) &&
          nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim) && nc::gemm_tc_supported(M, q + 256, d, d) &&
          nc::gemm_tc_supported(M, d, q, q) && nc::gemm_tc_supported(M, F, d, d) && nc::gemm_tc_supported(M, d, F, F);
 }
@@ -446,6 +447,59 @@ int decode_fast(nc_model *m, nc_kv *kv, const int32_t *tokens, const int32_t *po
   }
   NC_CUDA_TRY(cudaGraphLaunch(kv->graph, s));
   nc::count_launch(kv->graph_kernels);
+  return NC_OK;
+}
+
+// The outputs of a prefill (or an appended chunk) whose B * T rows are in
+// kv->x: logits of the last or of every position, and the next token.
+int prefill_tail(nc_model *m, nc_kv *kv, int B, int T, int logits_mode, float *d_logits, int32_t *d_next,
+                 const float *d_noise, cudaStream_t s) {
+  const nc_config &c = m->cfg;
+  const int M = B * T;
+  float *logits;
+  long long last_off, row_stride;
+  cudaError_t eh = cudaSuccess;
+  if (logits_mode == 1) {
+    if (d_logits) {
+      eh = run_head(m, kv, M, 1, 0, d_logits, nullptr, s);
+      logits = d_logits;
+      last_off = (long long)(T - 1) * c.vocab;
+      row_stride = (long long)T * c.vocab;
+    } else {
+      eh = run_head(m, kv, B, T, T - 1, kv->logits, nullptr, s);
+      logits = kv->logits;
+      last_off = 0;
+      row_stride = c.vocab;
+    }
+  } else {
+    logits = d_logits ? d_logits : kv->logits;
+    if (kv->dec_fast && nc::decode_fast_supported(c, B)) {
+      // last rows -> fused norm + lm_head + softcap + argmax (the decode head kernel)
+      ProfScope p(m, NC_K_HEAD, s);
+      cudaError_t e = nc::k_gather_rows_ss(kv->x, B, c.d_model, T, T - 1, kv->xl, kv->ss, 32, s);
+      if (e == cudaSuccess)
+        e = nc::k_dec_linear(0 /*norm*/, 3 /*lmhead*/, m->wlm, c.vocab, c.d_model, B, kv->xl, kv->ss, 32, c.norm_eps,
+                             nullptr, kv->part, kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq,
+                             c.n_head, kv->pos_ws, kv->valid, kv->rope, logits, d_noise, c.softcap, kv->cand_v,
+                             kv->cand_i, d_next, m->status, m->num_sms, s);
+      if (e == cudaSuccess) e = sampled_pick(m, kv, logits, B, c.vocab, c.vocab, d_noise, nullptr, d_next, s);
+      if (e != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(e));
+      return NC_OK;
+    }
+    eh = run_head(m, kv, B, T, T - 1, logits, nullptr, s);
+    last_off = 0;
+    row_stride = c.vocab;
+  }
+  if (eh != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(eh));
+  if (d_next) {
+    if (kv->sampling()) {
+      NC_CUDA_TRY(sampled_pick(m, kv, logits + last_off, B, c.vocab, row_stride, d_noise, nullptr, d_next, s));
+    } else {
+      ProfScope p(m, NC_K_HEAD, s);
+      nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
+    }
+  }
+  NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
 
@@ -689,51 +743,29 @@ int nc_prefill(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, in
   nc::RowMap rm{T, nullptr};
   const int rc = run_blocks(m, kv, M, rm, s);
   if (rc != NC_OK) return rc;
-  float *logits;
-  long long last_off, row_stride;
-  cudaError_t eh = cudaSuccess;
-  if (logits_mode == 1) {
-    if (d_logits) {
-      eh = run_head(m, kv, M, 1, 0, d_logits, nullptr, s);
-      logits = d_logits;
-      last_off = (long long)(T - 1) * c.vocab;
-      row_stride = (long long)T * c.vocab;
-    } else {
-      eh = run_head(m, kv, B, T, T - 1, kv->logits, nullptr, s);
-      logits = kv->logits;
-      last_off = 0;
-      row_stride = c.vocab;
-    }
-  } else {
-    logits = d_logits ? d_logits : kv->logits;
-    if (kv->dec_fast && nc::decode_fast_supported(c, B)) {
-      // last rows -> fused norm + lm_head + softcap + argmax (the decode head kernel)
-      ProfScope p(m, NC_K_HEAD, s);
-      cudaError_t e = nc::k_gather_rows_ss(kv->x, B, c.d_model, T, T - 1, kv->xl, kv->ss, 32, s);
-      if (e == cudaSuccess)
-        e = nc::k_dec_linear(0 /*norm*/, 3 /*lmhead*/, m->wlm, c.vocab, c.d_model, B, kv->xl, kv->ss, 32, c.norm_eps,
-                             nullptr, kv->part, kv->counters, nullptr, nullptr, nullptr, nullptr, nullptr, kv->max_seq,
-                             c.n_head, kv->pos_ws, kv->valid, kv->rope, logits, d_noise, c.softcap, kv->cand_v,
-                             kv->cand_i, d_next, m->status, m->num_sms, s);
-      if (e == cudaSuccess) e = sampled_pick(m, kv, logits, B, c.vocab, c.vocab, d_noise, nullptr, d_next, s);
-      if (e != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(e));
-      return NC_OK;
-    }
-    eh = run_head(m, kv, B, T, T - 1, logits, nullptr, s);
-    last_off = 0;
-    row_stride = c.vocab;
+  return prefill_tail(m, kv, B, T, logits_mode, d_logits, d_next, d_noise, s);
+}
+
+int nc_prefill_extend(nc_model *m, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode,
+                      float *d_logits, int32_t *d_next, const float *d_noise, void *stream) {
+  if (!m || !kv || !d_tokens) return fail(NC_EINVAL, "null model, kv or tokens");
+  if (kv->model != m) return fail(NC_EINVAL, "kv belongs to another model");
+  if (B < 1 || T < 1) return fail(NC_EINVAL, "B and T must be >= 1");
+  if (logits_mode != 0 && logits_mode != 1) return fail(NC_EINVAL, "logits_mode must be 0 (last) or 1 (all)");
+  if (B > kv->max_batch) return fail(NC_ERANGE, "B=%d > max_batch=%d", B, kv->max_batch);
+  if (T > kv->max_seq) return fail(NC_ERANGE, "T=%d > max_seq=%d", T, kv->max_seq);
+  const nc_config &c = m->cfg;
+  cudaStream_t s = as_stream(stream);
+  const int M = B * T;
+  {
+    ProfScope p(m, NC_K_MISC, s);
+    nc::k_extend_begin(kv->len, kv->valid, kv->pos_ws, B, T, kv->max_seq, m->status, s);
+    nc::k_embed_norm(c.dtype, d_tokens, M, m->wte, c.d_model, c.vocab, c.norm_eps, kv->x, m->status, s);
   }
-  if (eh != cudaSuccess) return fail(NC_ECUDA, "prefill head launch failed: %s", cudaGetErrorString(eh));
-  if (d_next) {
-    if (kv->sampling()) {
-      NC_CUDA_TRY(sampled_pick(m, kv, logits + last_off, B, c.vocab, row_stride, d_noise, nullptr, d_next, s));
-    } else {
-      ProfScope p(m, NC_K_HEAD, s);
-      nc::k_argmax_rows(logits + last_off, B, c.vocab, row_stride, d_noise, d_next, nullptr, s);
-    }
-  }
-  NC_CUDA_TRY(cudaGetLastError());
-  return NC_OK;
+  nc::RowMap rm{T, nullptr, kv->pos_ws};  // rows at positions len[b] + t
+  const int rc = run_blocks(m, kv, M, rm, s);
+  if (rc != NC_OK) return rc;
+  return prefill_tail(m, kv, B, T, logits_mode, d_logits, d_next, d_noise, s);
 }
 
 int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_t *d_positions, int B,

@@ -71,12 +71,17 @@ __device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
 }
 
 // Which sequence / position a row of activations belongs to. Prefill rows
-// are m = b*T + t (position t); decode rows are m = b with position pos[b].
+// are m = b*T + t (position t, or off[b] + t when a chunk is appended to
+// sequences already holding off[b] tokens); decode rows are m = b with
+// position pos[b].
 struct RowMap {
-  int T;               // prefill prompt length (ignored for decode)
-  const int32_t *pos;  // decode positions [B], or nullptr for prefill
+  int T;                         // prefill prompt / chunk length (ignored for decode)
+  const int32_t *pos;            // decode positions [B], or nullptr for prefill
+  const int32_t *off = nullptr;  // chunk start of each sequence [B], or nullptr (from position 0)
   __device__ __forceinline__ int seq(int m) const { return pos ? m : m / T; }
-  __device__ __forceinline__ int position(int m) const { return pos ? pos[m] : m % T; }
+  __device__ __forceinline__ int position(int m) const {
+    return pos ? pos[m] : (off ? off[m / T] : 0) + m % T;
+  }
 };
 
 }  // namespace nc

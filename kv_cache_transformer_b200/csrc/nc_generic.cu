@@ -32,6 +32,27 @@ void k_prefill_begin(int32_t *len, uint8_t *valid, int32_t *pre_len, int B, int 
   prefill_begin_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, valid, pre_len, B, T);
 }
 
+// A chunk of T tokens is appended to sequence b at its current length:
+// off[b] = len[b]; the sequence takes part iff the chunk fits (len + T <=
+// max_seq), and then its length advances by T.
+__global__ void extend_begin_kernel(int32_t *len, uint8_t *valid, int32_t *off, int B, int T, int max_seq,
+                                    uint32_t *status) {
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const int l = len[b];
+  const bool ok = l >= 0 && l + T <= max_seq;
+  off[b] = ok ? l : 0;
+  valid[b] = ok ? 1 : 0;
+  if (ok) len[b] = l + T;
+  else atomicOr(status, (unsigned)NC_DEV_BAD_POSITION);
+}
+
+void k_extend_begin(int32_t *len, uint8_t *valid, int32_t *off, int B, int T, int max_seq, uint32_t *status,
+                    cudaStream_t s) {
+  count_launch();
+  extend_begin_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, valid, off, B, T, max_seq, status);
+}
+
 // A decode row is valid iff its position is the sequence's current length and
 // inside the cache; valid rows advance their length by one.
 __global__ void decode_begin_kernel(const int32_t *positions, int32_t *len, uint8_t *valid, int B, int max_seq,

@@ -175,6 +175,8 @@ struct GemmFuse {
 
 // ---- generic kernels (any even head_dim; fp32 or bf16 storage) ----
 void k_prefill_begin(int32_t *len, uint8_t *valid, int32_t *pre_len, int B, int T, cudaStream_t s);
+void k_extend_begin(int32_t *len, uint8_t *valid, int32_t *off, int B, int T, int max_seq, uint32_t *status,
+                    cudaStream_t s);
 void k_decode_begin(const int32_t *positions, int32_t *len, uint8_t *valid, int B, int max_seq,
                     uint32_t *status, cudaStream_t s);
 void k_embed_norm(int dtype, const int32_t *tokens, int M, const void *wte, int d, int vocab, float eps,

@@ -59,19 +59,21 @@ using namespace sm100;
 
 namespace {
 
-constexpr int NCW = 4;                  // compute warps
+constexpr int NCW = 8;                  // compute warps (two per SM sub-partition)
 constexpr int THREADS = 32 * (1 + NCW);  // warp 0: TMA producer
 constexpr int SLOT = 16384;             // ring slot bytes
 constexpr int KT = 64;                  // keys per attention tile
 constexpr int MAXB = 32;                // sequences per step: rows of every staged activation
 constexpr int MAX_SPLIT = 8;            // attention key splits per sequence
 constexpr int MAX_R = 64;               // weight rows per CTA in the K-split linears
-constexpr int HG = 64;                  // lm_head rows per pass (16 per compute warp)
+constexpr int HG = 64;                  // lm_head rows per pass (16 per warp of each warp group)
 constexpr int SMEM_CAP = 227 * 1024;
 constexpr int MISC = 2048;              // barriers and per-sequence tables
-constexpr int ATT_SCRATCH = NCW * 16 * 130 * 4 + 17 * 128 * 2 + 256;  // softmax states, q and k in bf16
 constexpr int CTR_BYTES = 2048;         // counters zeroed before each launch
 constexpr int AROW = 132;               // floats per attention state row: m, l, O[128], padding
+// attention scratch: the warps' softmax states, q and the new key in bf16,
+// per-row merge factors
+constexpr int ATT_SCRATCH = NCW * 16 * AROW * 4 + 17 * 128 * 2 + (NCW + 2) * 16 * 4;
 
 enum Phase { P_EMBED = 0, P_QKV, P_ATTN, P_OPROJ, P_FC, P_PROJ, P_HEAD, P_MERGE };
 
@@ -128,7 +130,7 @@ struct Smem {
   int *flag;
 };
 
-__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -304,18 +306,27 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint3
 // ------------------------------------------------------------- producer
 // Slot sizes: a linear unit of R rows puts kps = SLOT / (R * 128) k-blocks in
 // a slot (the lm_head: 2 k-blocks of 64 rows); attention puts one K or V tile
-// of 64 keys in a slot.
+// of 64 keys in a slot. The whole warp walks the program: lane 0 waits for a
+// free slot and arms its barrier, then each lane issues one of the slot's
+// tensor copies, so a slot's copies leave together.
 __device__ __forceinline__ int kps_of(int R) { return SLOT / (R * 128); }
 
-__device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
+__device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int lane) {
   uint64_t evict_first;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(evict_first));
   uint32_t t = 0;
-  auto take = [&](uint32_t &slot) -> bool {
+  // the next slot, armed for `bytes`; false once the pipeline has aborted
+  auto take = [&](uint32_t &slot, uint32_t bytes) -> bool {
     slot = t % a.slots;
     const uint32_t ph = (t / a.slots) & 1;
     t++;
-    return mbar_wait(&s.empty[slot], ph ^ 1, s.abort_flag, a.status);
+    int ok = 1;
+    if (lane == 0) {
+      ok = mbar_wait(&s.empty[slot], ph ^ 1, s.abort_flag, a.status) ? 1 : 0;
+      if (ok) mbar_arrive_expect_tx(&s.full[slot], bytes);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    return ok != 0;
   };
   const int c = blockIdx.x, P = n_phases(a);
   for (int p = 0; p < P; p++) {
@@ -335,18 +346,15 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
       for (int key = k0; key < k1; key += KT)
         for (int which = 0; which < 2; which++) {
           uint32_t slot;
-          if (!take(slot)) return;
-          if (first) trace_mark(a, p, 5);
+          if (!take(slot, SLOT)) return;
+          if (first && lane == 0) trace_mark(a, p, 5);
           first = false;
-          mbar_arrive_expect_tx(&s.full[slot], SLOT);
-          uint8_t *dst = ring + slot * SLOT;
           const bool sh = key < plen;
           const CUtensorMap *map = a.kvmaps + (sh ? 2 : 0) + which;
           const int row = (sh ? prow0 : row0) + key;
-          tma_load_2d(dst, map, 0, row, &s.full[slot]);
-          tma_load_2d(dst + 8192, map, 64, row, &s.full[slot]);
+          if (lane < 2) tma_load_2d(ring + slot * SLOT + lane * 8192, map, lane * 64, row, &s.full[slot]);
         }
-      trace_mark(a, p, 6);
+      if (lane == 0) trace_mark(a, p, 6);
     } else if (type == P_QKV || type == P_OPROJ || type == P_FC || type == P_PROJ || type == P_HEAD) {
       const Unit u = unit_of(a, type, layer, c);
       if (!u.active) continue;
@@ -354,38 +362,36 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
         const int rows = min(u.R, a.V - u.r0);
         for (int g0 = 0; g0 < rows; g0 += HG)
           for (int kb = 0; kb < u.nkb; kb += 2) {
-            uint32_t slot;
-            if (!take(slot)) return;
-            if (first) trace_mark(a, p, 5);
-            first = false;
             const int n = min(2, u.nkb - kb);
-            mbar_arrive_expect_tx(&s.full[slot], n * HG * 128);
-            for (int j = 0; j < n; j++)
-              tma_load_2d_hint(ring + slot * SLOT + j * HG * 128, u.map, (kb + j) * 64, u.r0 + g0, &s.full[slot],
+            uint32_t slot;
+            if (!take(slot, n * HG * 128)) return;
+            if (first && lane == 0) trace_mark(a, p, 5);
+            first = false;
+            if (lane < n)
+              tma_load_2d_hint(ring + slot * SLOT + lane * HG * 128, u.map, (kb + lane) * 64, u.r0 + g0, &s.full[slot],
                                evict_first);
           }
       } else {
         const int kps = kps_of(u.R);
         for (int ch = 0; ch < u.nkb; ch += kps) {
-          uint32_t slot;
-          if (!take(slot)) return;
-          if (first) trace_mark(a, p, 5);
-          first = false;
           const int n = min(kps, u.nkb - ch);
-          mbar_arrive_expect_tx(&s.full[slot], n * u.R * 128);
-          for (int j = 0; j < n; j++) {
-            uint8_t *dst = ring + slot * SLOT + j * u.R * 128;
-            const int x = (u.kb0 + ch + j) * 64;
-            if (type == P_QKV) {  // rows r0..r0+7 and their RoPE partners r0+64..r0+71
-              tma_load_2d_hint(dst, u.map, x, u.r0, &s.full[slot], evict_first);
-              tma_load_2d_hint(dst + 8 * 128, u.map, x, u.r0 + 64, &s.full[slot], evict_first);
-            } else {
-              tma_load_2d_hint(dst, u.map, x, u.r0, &s.full[slot], evict_first);
+          uint32_t slot;
+          if (!take(slot, n * u.R * 128)) return;
+          if (first && lane == 0) trace_mark(a, p, 5);
+          first = false;
+          if (type == P_QKV) {  // rows r0..r0+7 and their RoPE partners r0+64..r0+71: two boxes per k-block
+            if (lane < 2 * n) {
+              const int j = lane >> 1, hi = lane & 1;
+              tma_load_2d_hint(ring + slot * SLOT + j * u.R * 128 + hi * 8 * 128, u.map, (u.kb0 + ch + j) * 64,
+                               u.r0 + 64 * hi, &s.full[slot], evict_first);
             }
+          } else if (lane < n) {
+            tma_load_2d_hint(ring + slot * SLOT + lane * u.R * 128, u.map, (u.kb0 + ch + lane) * 64, u.r0,
+                             &s.full[slot], evict_first);
           }
         }
       }
-      trace_mark(a, p, 6);
+      if (lane == 0) trace_mark(a, p, 6);
     }
   }
 }
@@ -393,27 +399,29 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
 // ------------------------------------------------- compute-side helpers
 // Stage the phase's activation rows: nkb boxes of 64 columns x 32 rows from
 // k-block kb0 of the activation map into xs ([kb][32 rows][128 B], swizzled).
-// Issued by one thread after the barrier; the writers' data was released
-// through the grid barrier, the proxy fence orders it ahead of the copies.
-__device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CUtensorMap *amap, int kb0, int nkb) {
+// Issued by one warp right after the barrier (lane j issues boxes j, j + 32,
+// ...); the writers' data was released through the grid barrier, the proxy
+// fences order it ahead of the copies.
+__device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CUtensorMap *amap, int kb0, int nkb,
+                                            int lane) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  mbar_arrive_expect_tx(s.x_bar, nkb * MAXB * 128);
-  for (int j = 0; j < nkb; j++) tma_load_2d(xs + j * MAXB * 128, amap, (kb0 + j) * 64, 0, s.x_bar);
+  if (lane == 0) mbar_arrive_expect_tx(s.x_bar, nkb * MAXB * 128);
+  __syncwarp();
+  for (int j = lane; j < nkb; j += 32) tma_load_2d(xs + j * MAXB * 128, amap, (kb0 + j) * 64, 0, s.x_bar);
 }
 
 // 1/rms of each sequence's row from the per-CTA partial sums of squares of a
-// norm: units [0, nu) of ss[norm]. Four threads per sequence add a quarter of
-// the partials each, combined in a fixed order.
+// norm: units [0, nu) of ss[norm]. Eight threads per sequence load every
+// eighth partial (all loads first), combined in a fixed order.
 __device__ void load_inv(const StepArgs &a, const Smem &s, int norm, int nu, int e) {
-  const int b = e >> 2, q = e & 3;
+  const int b = e >> 3, q = e & 7;
   const float *src = a.ss + (size_t)norm * a.grid * 32;
-  // all loads first (nu <= grid <= 4 * 40), then the sum in unit order
-  constexpr int NL = 40;
+  constexpr int NL = 20;  // nu <= grid <= 8 * NL
   float v[NL];
 #pragma unroll
   for (int i = 0; i < NL; i++) {
-    const int u = q + 4 * i;
+    const int u = q + 8 * i;
     v[i] = u < nu ? __ldcg(src + (size_t)u * 32 + b) : 0.f;
   }
   float sum = 0.f;
@@ -421,6 +429,7 @@ __device__ void load_inv(const StepArgs &a, const Smem &s, int norm, int nu, int
   for (int i = 0; i < NL; i++) sum += v[i];
   sum += __shfl_xor_sync(0xffffffffu, sum, 1);
   sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+  sum += __shfl_xor_sync(0xffffffffu, sum, 4);
   if (q == 0) s.inv[b] = b < a.B ? rsqrtf(sum / a.d + a.eps) : 0.f;
 }
 
@@ -447,7 +456,7 @@ __device__ bool gemv_t(const StepArgs &a, const Smem &s, uint8_t *ring, const ui
     const uint8_t *wslot = ring + slot * SLOT;
     for (int j = 0; j < n; j++) {
       const int kb = ch + j;
-      if ((kb & (NCW - 1)) != warp) continue;
+      if (kb % NCW != warp) continue;
       const uint32_t wb = smem_u32(wslot + j * R * 128), xb = smem_u32(xs + kb * MAXB * 128);
       uint32_t af[4][MT][4], bf[4][NT][2];
 #pragma unroll
@@ -506,7 +515,7 @@ __device__ bool gemv_mt(const StepArgs &a, const Smem &s, uint8_t *ring, const u
 __device__ float *reduce_warps(float *red, int R, int MT, int e) {
   csync();
   float *out = red + (size_t)NCW * MAXB * R;
-  for (int i = e; i < MT * 16 * R; i += 128) {
+  for (int i = e; i < MT * 16 * R; i += 32 * NCW) {
     float v = red[i];
 #pragma unroll
     for (int w = 1; w < NCW; w++) v += red[(size_t)w * MAXB * R + i];
@@ -530,9 +539,11 @@ __device__ void write_ss(const StepArgs &a, const float *sq, int R, int norm, in
 // ------------------------------------------------------------ attention
 // Split `sp` of sequence b's keys: q and the new key get their QK norm here,
 // the new key is appended to the cache by the split that holds it, then
-// flash decoding over the split's tiles (mma.sync m16n8k16, rows = query
-// heads padded to 16), and the split's softmax state goes to apart; the last
-// split to arrive merges them in split order into y.
+// flash decoding over the split's 64-key tiles (mma.sync m16n8k16, rows =
+// query heads padded to 16): warp group g (warps 4g .. 4g+3) takes the tiles
+// of parity g, each warp 16 keys of a tile. The eight warps' softmax states
+// are merged (per-row factors first), the split's state goes to apart, and
+// the last split to arrive merges all splits in split order into y.
 __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
                                 uint32_t &t, uint32_t &xph, int p) {
   const int c = blockIdx.x;
@@ -540,24 +551,26 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
   const int b = c / a.splits, sp = c % a.splits;
   if (!s.valid[b]) return true;
   const int warp = e >> 5, lane = e & 31, g = lane >> 2, t4 = lane & 3;
+  const int grp = warp >> 2, wq = warp & 3;
   const size_t lay = (size_t)layer * a.max_batch * a.max_seq * 128;
   const int pos = s.pos[b], n_keys = pos + 1;
   int k0, k1;
   key_range(n_keys, sp, a.splits, k0, k1);
-  float *cw = reinterpret_cast<float *>(xs);                        // [4 warps][16 rows][130]
-  bf16 *qs = reinterpret_cast<bf16 *>(xs + NCW * 16 * 130 * 4);     // [17][128]: q heads, then the new key
+  float *cw = reinterpret_cast<float *>(xs);                                 // [8 warps][16 rows][AROW]
+  bf16 *qs = reinterpret_cast<bf16 *>(xs + NCW * 16 * AROW * 4);             // [17][128]: q heads, the new key
+  float *fac = reinterpret_cast<float *>(xs + NCW * 16 * AROW * 4 + 17 * 128 * 2);  // [NCW + 2][16]
   // QK norm of the H query heads and of the new key, in fp32, to bf16 (the
-  // warp's heads w, w+4, ... are loaded before any is used)
+  // warp's heads w, w+8, w+16 are loaded before any is used)
   {
-    float4 qv[5];
+    float4 qv[3];
 #pragma unroll
-    for (int i = 0; i < 5; i++) {
+    for (int i = 0; i < 3; i++) {
       const int h = warp + NCW * i;
       qv[i] = h <= a.H ? __ldcg(reinterpret_cast<const float4 *>(a.qk + ((size_t)b * (a.H + 1) + h) * 128) + lane)
                        : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int i = 0; i < 5; i++) {
+    for (int i = 0; i < 3; i++) {
       const int h = warp + NCW * i;
       if (h > a.H) break;
       const float4 v = qv[i];
@@ -584,11 +597,13 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
 #pragma unroll
   for (int i = 0; i < 16; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  for (int key0 = k0; key0 < k1; key0 += KT) {
+  int tile = 0;
+  for (int key0 = k0; key0 < k1; key0 += KT, tile++) {
     const uint32_t ks_ = t % a.slots, kph = (t / a.slots) & 1;
     t++;
     const uint32_t vs_ = t % a.slots, vph = (t / a.slots) & 1;
     t++;
+    // every warp waits for every tile (its arrival on the slot must follow the fill)
     mbar_wait(&s.full[ks_], kph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
     mbar_wait(&s.full[vs_], vph, s.abort_flag, a.status);
     if (e == 0 && key0 == k0) trace_mark(a, p, 1);
@@ -605,63 +620,65 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
       }
       csync();
     }
-    const uint32_t kb = smem_u32(K), vb = smem_u32(V);
-    const int kw = warp * 16;
-    const int kg = key0 + kw;
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    if ((tile & 1) == grp) {
+      const uint32_t kb = smem_u32(K), vb = smem_u32(V);
+      const int kw = wq * 16;
+      const int kg = key0 + kw;
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int ks = 0; ks < 8; ks++) {
-      const int key = kw + (lane & 7) + ((lane >> 4) << 3);
-      const int cc = 2 * ks + ((lane >> 3) & 1);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(kb + kv_tile_off(key, cc), b0, b1, b2, b3);
-      mma16816(s0, qa[ks], b0, b1);
-      mma16816(s1, qa[ks], b2, b3);
-    }
-    float v[8] = {s0[0], s0[1], s1[0], s1[1], s0[2], s0[3], s1[2], s1[3]};
-    const int kidx[4] = {kg + 2 * t4, kg + 2 * t4 + 1, kg + 8 + 2 * t4, kg + 9 + 2 * t4};
-    float mx0 = -INFINITY, mx1 = -INFINITY;
+      for (int ks = 0; ks < 8; ks++) {
+        const int key = kw + (lane & 7) + ((lane >> 4) << 3);
+        const int cc = 2 * ks + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + kv_tile_off(key, cc), b0, b1, b2, b3);
+        mma16816(s0, qa[ks], b0, b1);
+        mma16816(s1, qa[ks], b2, b3);
+      }
+      float v[8] = {s0[0], s0[1], s1[0], s1[1], s0[2], s0[3], s1[2], s1[3]};
+      const int kidx[4] = {kg + 2 * t4, kg + 2 * t4 + 1, kg + 8 + 2 * t4, kg + 9 + 2 * t4};
+      float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-      const bool in = kidx[i] < k1;
-      v[i] = in ? v[i] * a.scale_log2 : -INFINITY;
-      v[i + 4] = in ? v[i + 4] * a.scale_log2 : -INFINITY;
-      mx0 = fmaxf(mx0, v[i]);
-      mx1 = fmaxf(mx1, v[i + 4]);
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
-    float pp[8];
+      for (int i = 0; i < 4; i++) {
+        const bool in = kidx[i] < k1;
+        v[i] = in ? v[i] * a.scale_log2 : -INFINITY;
+        v[i + 4] = in ? v[i + 4] * a.scale_log2 : -INFINITY;
+        mx0 = fmaxf(mx0, v[i]);
+        mx1 = fmaxf(mx1, v[i + 4]);
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
+      const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
+      float pp[8];
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-      pp[i] = v[i] == -INFINITY ? 0.f : exp2f(v[i] - mn0);
-      pp[i + 4] = v[i + 4] == -INFINITY ? 0.f : exp2f(v[i + 4] - mn1);
-    }
-    l0 = l0 * al0 + pp[0] + pp[1] + pp[2] + pp[3];
-    l1 = l1 * al1 + pp[4] + pp[5] + pp[6] + pp[7];
-    m0 = mn0;
-    m1 = mn1;
+      for (int i = 0; i < 4; i++) {
+        pp[i] = v[i] == -INFINITY ? 0.f : exp2f(v[i] - mn0);
+        pp[i + 4] = v[i + 4] == -INFINITY ? 0.f : exp2f(v[i + 4] - mn1);
+      }
+      l0 = l0 * al0 + pp[0] + pp[1] + pp[2] + pp[3];
+      l1 = l1 * al1 + pp[4] + pp[5] + pp[6] + pp[7];
+      m0 = mn0;
+      m1 = mn1;
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-      o[i][0] *= al0;
-      o[i][1] *= al0;
-      o[i][2] *= al1;
-      o[i][3] *= al1;
-    }
-    uint32_t pa[4] = {pack_bf(pp[0], pp[1]), pack_bf(pp[4], pp[5]), pack_bf(pp[2], pp[3]), pack_bf(pp[6], pp[7])};
+      for (int i = 0; i < 16; i++) {
+        o[i][0] *= al0;
+        o[i][1] *= al0;
+        o[i][2] *= al1;
+        o[i][3] *= al1;
+      }
+      uint32_t pa[4] = {pack_bf(pp[0], pp[1]), pack_bf(pp[4], pp[5]), pack_bf(pp[2], pp[3]), pack_bf(pp[6], pp[7])};
 #pragma unroll
-    for (int dt = 0; dt < 16; dt += 2) {
-      const int key = kw + (lane & 7) + (((lane >> 3) & 1) << 3);
-      const int cc = dt + (lane >> 4);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(vb + kv_tile_off(key, cc), b0, b1, b2, b3);
-      mma16816(o[dt], pa, b0, b1);
-      mma16816(o[dt + 1], pa, b2, b3);
+      for (int dt = 0; dt < 16; dt += 2) {
+        const int key = kw + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int cc = dt + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + kv_tile_off(key, cc), b0, b1, b2, b3);
+        mma16816(o[dt], pa, b0, b1);
+        mma16816(o[dt + 1], pa, b2, b3);
+      }
     }
     __syncwarp();
     if (lane == 0) {
@@ -675,43 +692,45 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
   {
-    float *mine = cw + warp * 16 * 130;
+    float *mine = cw + warp * 16 * AROW;
     if (t4 == 0) {
-      mine[g * 130 + 0] = m0;
-      mine[g * 130 + 1] = l0;
-      mine[(g + 8) * 130 + 0] = m1;
-      mine[(g + 8) * 130 + 1] = l1;
+      mine[g * AROW + 0] = m0;
+      mine[g * AROW + 1] = l0;
+      mine[(g + 8) * AROW + 0] = m1;
+      mine[(g + 8) * AROW + 1] = l1;
     }
 #pragma unroll
     for (int dt = 0; dt < 16; dt++) {
       const int col = dt * 8 + 2 * t4;
-      mine[g * 130 + 2 + col] = o[dt][0];
-      mine[g * 130 + 2 + col + 1] = o[dt][1];
-      mine[(g + 8) * 130 + 2 + col] = o[dt][2];
-      mine[(g + 8) * 130 + 2 + col + 1] = o[dt][3];
+      *reinterpret_cast<float2 *>(mine + g * AROW + 2 + col) = make_float2(o[dt][0], o[dt][1]);
+      *reinterpret_cast<float2 *>(mine + (g + 8) * AROW + 2 + col) = make_float2(o[dt][2], o[dt][3]);
     }
   }
   csync();
-  // this split's state: the four warps' key quarters merged, to apart[b][sp]
+  // the eight warps' states merged: per-row factors, then the rows, to apart[b][sp]
   float *dst = a.apart + ((size_t)b * MAX_SPLIT + sp) * 16 * AROW;
-  for (int idx = e; idx < a.H * 128; idx += 128) {
-    const int row = idx >> 7, col = idx & 127;
+  if (e < a.H) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NCW; w++) M = fmaxf(M, cw[w * 16 * 130 + row * 130]);
-    float Ls = 0.f, O = 0.f;
+    for (int w = 0; w < NCW; w++) M = fmaxf(M, cw[(w * 16 + e) * AROW]);
+    float Ls = 0.f;
 #pragma unroll
     for (int w = 0; w < NCW; w++) {
-      const float mw = cw[w * 16 * 130 + row * 130];
+      const float mw = cw[(w * 16 + e) * AROW];
       const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
-      Ls += f * cw[w * 16 * 130 + row * 130 + 1];
-      O += f * cw[w * 16 * 130 + row * 130 + 2 + col];
+      fac[w * 16 + e] = f;
+      Ls += f * cw[(w * 16 + e) * AROW + 1];
     }
+    dst[e * AROW] = M;
+    dst[e * AROW + 1] = Ls;
+  }
+  csync();
+  for (int idx = e; idx < a.H * 128; idx += 32 * NCW) {
+    const int row = idx >> 7, col = idx & 127;
+    float O = 0.f;
+#pragma unroll
+    for (int w = 0; w < NCW; w++) O += fac[w * 16 + row] * cw[(w * 16 + row) * AROW + 2 + col];
     dst[row * AROW + 2 + col] = O;
-    if (col == 0) {
-      dst[row * AROW] = M;
-      dst[row * AROW + 1] = Ls;
-    }
   }
   csync();
   if (e == 0) {
@@ -721,9 +740,9 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
   }
   csync();
   if (*s.flag) {  // the last split: merge all splits in split order
-    // every split's H state rows in one bulk copy each, into the scratch
+    // every split's H state rows in one bulk copy each, over the warp states
     // (free now: this split's state is in apart)
-    float *st = reinterpret_cast<float *>(xs);  // [splits][H][AROW]
+    float *st = cw;  // [splits][H][AROW]
     const uint32_t rows_bytes = (uint32_t)(a.H * AROW * 4);
     if (e == 0) {
       asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -734,21 +753,27 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
     }
     mbar_wait(s.x_bar, xph & 1, s.abort_flag, a.status);
     xph++;
-    for (int idx = e; idx < a.H * 128; idx += 128) {
-      const int row = idx >> 7, col = idx & 127;
+    if (e < a.H) {
       float M = -INFINITY;
-      for (int q = 0; q < a.splits; q++) M = fmaxf(M, st[(q * a.H + row) * AROW]);
-      float Ls = 0.f, O = 0.f;
+      for (int q = 0; q < a.splits; q++) M = fmaxf(M, st[(q * a.H + e) * AROW]);
+      float Ls = 0.f;
       for (int q = 0; q < a.splits; q++) {
-        const float *pr = st + (q * a.H + row) * AROW;
-        const float f = pr[0] == -INFINITY ? 0.f : exp2f(pr[0] - M);
-        Ls += f * pr[1];
-        O += f * pr[2 + col];
+        const float mq = st[(q * a.H + e) * AROW];
+        const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
+        fac[q * 16 + e] = f;
+        Ls += f * st[(q * a.H + e) * AROW + 1];
       }
-      a.y[(size_t)b * a.d + row * 128 + col] = __float2bfloat16_rn(Ls > 0.f ? O / Ls : 0.f);
+      fac[NCW * 16 + e] = Ls > 0.f ? 1.f / Ls : 0.f;
+    }
+    csync();
+    for (int idx = e; idx < a.H * 128; idx += 32 * NCW) {
+      const int row = idx >> 7, col = idx & 127;
+      float O = 0.f;
+      for (int q = 0; q < a.splits; q++) O += fac[q * 16 + row] * st[(q * a.H + row) * AROW + 2 + col];
+      a.y[(size_t)b * a.d + row * 128 + col] = __float2bfloat16_rn(O * fac[NCW * 16 + row]);
     }
   }
-  csync();  // s.flag is rewritten by the next use
+  csync();  // s.flag and the scratch are rewritten by the next use
   if (e == 0) trace_mark(a, p, 3);
   return true;
 }
@@ -760,7 +785,7 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
 __device__ void qkv_epilogue(const StepArgs &a, const Smem &s, const float *sum, const Unit &u, int layer, int e) {
   const int head = u.r0 >> 7, j0 = u.r0 & 127;
   const size_t lay = (size_t)layer * a.max_batch * a.max_seq * 128;
-  for (int idx = e; idx < a.B * 8; idx += 128) {
+  for (int idx = e; idx < a.B * 8; idx += 32 * NCW) {
     const int b = idx >> 3, i = idx & 7;
     const float lo = sum[b * 16 + i] * s.inv[b], hi = sum[b * 16 + 8 + i] * s.inv[b];
     if (head <= a.H) {
@@ -779,12 +804,12 @@ __device__ void qkv_epilogue(const StepArgs &a, const Smem &s, const float *sum,
 // Residual: xout = xin + sum over the unit's rows (row r of the layer is
 // column r of the residual), bf16(xout), and this CTA's sums of squares.
 // The residual inputs of the rows this thread finishes, loaded at the start
-// of the phase (element i: index e + 128 i of the unit's [32][R] block).
-constexpr int XR = MAXB * MAX_R / 128;
+// of the phase (element i: index e + 256 i of the unit's [32][R] block).
+constexpr int XR = MAXB * MAX_R / (32 * NCW);
 __device__ __forceinline__ void load_resid(const StepArgs &a, const Unit &u, const float *xin, int e, float (&xr)[XR]) {
 #pragma unroll
   for (int i = 0; i < XR; i++) {
-    const int idx = e + 128 * i, b = idx / u.R, col = u.r0 + idx % u.R;
+    const int idx = e + 32 * NCW * i, b = idx / u.R, col = u.r0 + idx % u.R;
     xr[i] = (idx < MAXB * u.R && b < a.B && col < u.N) ? __ldcg(xin + (size_t)b * a.d + col) : 0.f;
   }
 }
@@ -793,7 +818,7 @@ __device__ void resid_epilogue(const StepArgs &a, float *sum, const Unit &u, con
                                bf16 *xbout, int norm, int e) {
 #pragma unroll
   for (int i = 0; i < XR; i++) {
-    const int idx = e + 128 * i;
+    const int idx = e + 32 * NCW * i;
     if (idx >= MAXB * u.R) break;
     const int b = idx / u.R, r = idx % u.R, col = u.r0 + r;
     float v = 0.f;
@@ -841,11 +866,15 @@ __device__ void head_group(const StepArgs &a, const Smem &s, const float (&acc)[
   }
 }
 
-// The lm_head rows of this CTA, 64 at a time (16 per warp: two n8 tiles),
-// full K from the ring; each group's logits and winners from registers.
+// The lm_head rows of this CTA, 64 at a time: warp w of group g takes rows
+// 16 (w % 4) .. +15 of the 64 and k-block g of every slot (a slot holds two),
+// full K from the ring. The halves are added in the group's last slot, which
+// is released only afterwards; group 0 then writes the group's logits and
+// keeps its winners.
 template <int MT>
-__device__ bool head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const uint8_t *xs, const Unit &u,
+__device__ void head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const uint8_t *xs, const Unit &u,
                           uint32_t &t, int warp, int lane, ArgMax (&best)[4]) {
+  const int grp = warp >> 2, wq = warp & 3;
   const int rows = min(u.R, a.V - u.r0);
   for (int g0 = 0; g0 < rows; g0 += HG) {
     float acc[MT][2][4];
@@ -853,14 +882,15 @@ __device__ bool head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
     for (int m = 0; m < MT; m++)
 #pragma unroll
       for (int n = 0; n < 2; n++) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.f;
+    uint32_t last_slot = 0;
     for (int kb2 = 0; kb2 < u.nkb; kb2 += 2) {
       const uint32_t slot = t % a.slots, ph = (t / a.slots) & 1;
       t++;
       mbar_wait(&s.full[slot], ph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
       const int n = min(2, u.nkb - kb2);
-      for (int j = 0; j < n; j++) {
-        const uint32_t wb = smem_u32(ring + slot * SLOT + j * HG * 128);
-        const uint32_t xb = smem_u32(xs + (kb2 + j) * MAXB * 128);
+      if (grp < n) {
+        const uint32_t wb = smem_u32(ring + slot * SLOT + grp * HG * 128);
+        const uint32_t xb = smem_u32(xs + (kb2 + grp) * MAXB * 128);
         uint32_t af[4][MT][4], bf[4][4];
 #pragma unroll
         for (int ks = 0; ks < 4; ks++) {
@@ -868,7 +898,7 @@ __device__ bool head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
           for (int m = 0; m < MT; m++)
             ldsm_x4(xb + swz(m * 16 + (lane & 15), 2 * ks + (lane >> 4)), af[ks][m][0], af[ks][m][1], af[ks][m][2],
                     af[ks][m][3]);
-          ldsm_x4(wb + swz(warp * 16 + (lane & 7) + ((lane >> 4) << 3), 2 * ks + ((lane >> 3) & 1)), bf[ks][0],
+          ldsm_x4(wb + swz(wq * 16 + (lane & 7) + ((lane >> 4) << 3), 2 * ks + ((lane >> 3) & 1)), bf[ks][0],
                   bf[ks][1], bf[ks][2], bf[ks][3]);
         }
 #pragma unroll
@@ -879,12 +909,42 @@ __device__ bool head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
             mma16816(acc[m][1], af[ks][m], bf[ks][2], bf[ks][3]);
           }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.empty[slot]);
+      if (kb2 + 2 < u.nkb) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[slot]);
+      } else {
+        last_slot = slot;
+      }
     }
-    head_group<MT>(a, s, acc, u.r0 + g0, warp, lane, best);
+    // group 1's half into group 0 through the last slot (every warp is done
+    // with its weights first)
+    float *scr = reinterpret_cast<float *>(ring + last_slot * SLOT) + (wq * 32 + lane) * (MT * 8);
+    csync();
+    if (grp == 1) {
+#pragma unroll
+      for (int m = 0; m < MT; m++)
+#pragma unroll
+        for (int n = 0; n < 2; n++)
+          *reinterpret_cast<float4 *>(scr + (m * 2 + n) * 4) = make_float4(acc[m][n][0], acc[m][n][1], acc[m][n][2], acc[m][n][3]);
+    }
+    csync();
+    if (grp == 0) {
+#pragma unroll
+      for (int m = 0; m < MT; m++)
+#pragma unroll
+        for (int n = 0; n < 2; n++) {
+          const float4 h = *reinterpret_cast<const float4 *>(scr + (m * 2 + n) * 4);
+          acc[m][n][0] += h.x;
+          acc[m][n][1] += h.y;
+          acc[m][n][2] += h.z;
+          acc[m][n][3] += h.w;
+        }
+      head_group<MT>(a, s, acc, u.r0 + g0, wq, lane, best);
+    }
+    csync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s.empty[last_slot]);
   }
-  return true;
 }
 
 // ------------------------------------------------------------ the kernel
@@ -896,7 +956,8 @@ __host__ __device__ constexpr int xreg_bytes(int d) {
               : (NCW + 1) * MAXB * MAX_R * 4);
 }
 
-__global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
+// 9 warps of at most 200 registers: one CTA per SM with every warp resident
+__global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
@@ -941,10 +1002,10 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
   __syncthreads();
 
   if (warp == 0) {
-    if (lane == 0) producer(a, s, ring);
+    producer(a, s, ring, lane);
   } else {
     const int e = threadIdx.x - 32;
-    const int cw = warp - 1;  // compute warp 0..3
+    const int cw = warp - 1;  // compute warp 0..7
     const int MT = a.B > 16 ? 2 : 1;
     uint32_t t = 0;           // ring slots consumed, in the producer's order
     uint32_t xph = 0;         // staging barrier phase
@@ -964,26 +1025,32 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
           }
           const bf16 *row = a.wte + (size_t)tok * a.d;
           float sq = 0.f;
-          for (int i = e; i < a.d; i += 128) {
+          for (int i = e; i < a.d; i += 32 * NCW) {
             const float v = __bfloat162float(row[i]);
             sq += v * v;
           }
           sq = warp_sum(sq);
           if (lane == 0) red[cw] = sq;
           csync();
-          const float inv = rsqrtf((red[0] + red[1] + red[2] + red[3]) / a.d + a.eps);
+          float tot = 0.f;
+          for (int w = 0; w < NCW; w++) tot += red[w];
+          const float inv = rsqrtf(tot / a.d + a.eps);
           float sq2 = 0.f;
-          for (int i = e; i < a.d; i += 128) {
+          for (int i = e; i < a.d; i += 32 * NCW) {
             const float v = __bfloat162float(row[i]) * inv;
             a.x0[(size_t)b * a.d + i] = v;
             a.xb0[(size_t)b * a.d + i] = __float2bfloat16_rn(v);
             sq2 += v * v;
           }
           sq2 = warp_sum(sq2);
-          if (lane == 0) red[4 + cw] = sq2;
+          if (lane == 0) red[NCW + cw] = sq2;
           csync();
           // norm 0 (the first layer's pre-attention norm) has one partial
-          if (e == 0) a.ss[b] = red[4] + red[5] + red[6] + red[7];
+          if (e == 0) {
+            float t2 = 0.f;
+            for (int w = 0; w < NCW; w++) t2 += red[NCW + w];
+            a.ss[b] = t2;
+          }
           csync();
         }
       } else if (type == P_ATTN) {
@@ -992,7 +1059,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
         for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
           if (!s.valid[b]) continue;
           ArgMax best{-INFINITY, 0x7fffffff};
-          for (int i = e; i < a.n_h; i += 128)
+          for (int i = e; i < a.n_h; i += 32 * NCW)
             best = argmax_merge(best, ArgMax{__ldcg(&a.cand_v[(size_t)i * 32 + b]), __ldcg(&a.cand_i[(size_t)i * 32 + b])});
           best = warp_argmax(best);
           if (lane == 0) {
@@ -1014,7 +1081,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
         // linear layer
         const Unit u = unit_of(a, type, layer, blockIdx.x);
         if (u.active) {
-          if (e == 0) stage_issue(s, xs, u.amap, u.kb0, u.nkb);
+          if (cw == 0) stage_issue(s, xs, u.amap, u.kb0, u.nkb, lane);
           float xr[XR];  // residual inputs of the rows this thread finishes
           if (type == P_OPROJ) load_resid(a, u, a.x0, e, xr);
           else if (type == P_PROJ) load_resid(a, u, a.x1, e, xr);
@@ -1030,7 +1097,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
             ArgMax best[4];
 #pragma unroll
             for (int i = 0; i < 4; i++) best[i] = ArgMax{-INFINITY, 0x7fffffff};
-            ok = MT == 2 ? head_rows<2>(a, s, ring, xs, u, t, cw, lane, best) : head_rows<1>(a, s, ring, xs, u, t, cw, lane, best);
+            if (MT == 2) head_rows<2>(a, s, ring, xs, u, t, cw, lane, best);
+            else head_rows<1>(a, s, ring, xs, u, t, cw, lane, best);
             if (e == 0) trace_mark(a, p, 2);
             // this CTA's winner per sequence: over the 4 lanes of a row group,
             // then over the warps
@@ -1070,7 +1138,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
               } else if (type == P_OPROJ) {
                 resid_epilogue(a, sum, u, xr, a.x1, a.xb1, 2 * layer + 1, e);
               } else if (type == P_FC) {
-                for (int idx = e; idx < a.B * u.R; idx += 128) {
+                for (int idx = e; idx < a.B * u.R; idx += 32 * NCW) {
                   const int b = idx / u.R, r = idx % u.R, col = u.r0 + r;
                   if (col < u.N) {
                     const float v = fmaxf(sum[idx] * s.inv[b], 0.f);
@@ -1079,7 +1147,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
                 }
               } else {  // P_PROJ: publish this split, the last of the splits finishes the rows
                 float *part = a.ppart + ((size_t)u.u * a.s_p + u.split) * MAXB * u.R;
-                for (int idx = e; idx < a.B * u.R; idx += 128) part[idx] = sum[idx];
+                for (int idx = e; idx < a.B * u.R; idx += 32 * NCW) part[idx] = sum[idx];
                 csync();
                 if (e == 0) {
                   unsigned old;
@@ -1103,7 +1171,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
                   }
                   mbar_wait(s.x_bar, xph & 1, s.abort_flag, a.status);
                   xph++;
-                  for (int idx = e; idx < a.B * u.R; idx += 128) {
+                  for (int idx = e; idx < a.B * u.R; idx += 32 * NCW) {
                     float v = 0.f;
                     for (int q = 0; q < a.s_p; q++) v += all[(size_t)q * MAXB * u.R + idx];
                     sum[idx] = v;

@@ -109,11 +109,15 @@ def test_shared_fork_within_one_cache_and_chained():
         r.copy_from(refs[2])
     c2 = np.full(2, int(cur[2]), np.int32)
     for s in range(2):
-        noise = syn.gumbel(5, (2, cfg.vocab), stream=300 + s)
+        # one noise row for both: the two forks must pick the same tokens
+        noise = np.repeat(syn.gumbel(5, (1, cfg.vocab), stream=300 + s), 2, axis=0)
         lg, nn = _decode(run.model, gen2, c2, noise)
-        assert np.array_equal(lg[0], lg[1]), "shared and copied second-generation forks differ"
+        errs = []
         for i in range(2):
-            check_logits(lg[i], r2[i].step(int(c2[i])), tol_for(cfg), f"gen2 seq {i} step {s}")
+            ref = r2[i].step(int(c2[i]))
+            errs.append(float(np.max(np.abs(lg[i] - ref))))
+        assert max(errs) <= tol_for(cfg), f"gen2 step {s}: max |logit error| shared {errs[0]:.3g}, copied {errs[1]:.3g}"
+        assert np.array_equal(lg[0], lg[1]), "shared and copied second-generation forks differ"
         c2 = nn.copy()
     assert run.status() == 0
     gen2.close()
