@@ -372,6 +372,8 @@ def run_ours(args):
                      for name in ("d26_latency", "d30_rollout")}
         workloads["d30_rollout_shared_prefix"] = decode_workload("d30_rollout", args, world, local, peaks, peaks_src,
                                                                  shared=True)
+        workloads["d20_extend"] = extend_workload(args, world, local, peaks, peaks_src)
+        workloads["sample_topk"] = sample_kernel_us(args)
 
     # ---------------- CPU oracle on a bounded sample (rank 0, N = 1)
     cpu = None
@@ -635,6 +637,77 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src, s
                      "bytes_per_step": by["total"], "peak_source": f"{peaks_src} hbm_gbs"},
         "gpu_launches": int(launches), "clocks": clk, **extra,
     }
+
+
+def extend_workload(args, world: int, local: int, peaks, peaks_src) -> dict:
+    """d20 chunked prefill: 8 sequences holding 2048-token prompts each take a
+    256-token chunk at their current length (nc_prefill_extend). tok/s of the
+    chunk tokens over all ranks; the chunk's FLOPs against the tensor peak."""
+    import torch
+    import kv_cache_transformer_b200 as nc
+    import nc_synth as syn
+    w = syn.WORKLOADS["d20_prefill"]
+    cfg = w.model
+    model = nc.Model(cfg, syn.make_blob(cfg, w.weight_seed))
+    B, T0, T1 = w.batch, w.prompt_len, 256
+    kv = model.kv(B, T0 + T1)
+    prompts = torch.from_numpy(syn.prompt_tokens(w)).cuda()
+    chunk = torch.from_numpy(syn.tokens_zipf(9, (B, T1), cfg.vocab)).cuda()
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    nxt = torch.empty((B,), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for it in range(args.warmup + max(2, args.steps // 5)):
+        model.prefill(kv, prompts, 0, logits, nxt)
+        e0.record(stream)
+        model.extend(kv, chunk, 0, logits, nxt)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            times.append(e0.elapsed_time(e1))
+    assert model.status() == 0
+    barrier(world)
+    t_ms = max_over_ranks(sum(times) / len(times), world)
+    lin = 2 * B * T1 * linear_params(cfg)
+    ctx_avg = T0 + (T1 + 1) / 2.0
+    attn = cfg.depth * B * T1 * 4 * cfg.n_head * cfg.head_dim * ctx_avg
+    flops = lin + attn + 2 * B * cfg.d_model * cfg.vocab
+    tf = flops / (t_ms / 1e3) / 1e12
+    kv.close()
+    model.close()
+    return {"metric": "d20 chunked prefill tok/s (256-token chunk after 2048)", "value": world * B * T1 / (t_ms / 1e3),
+            "unit": "tok/s", "n_gpus": world, "ms_per_chunk": t_ms, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "d20_extend", "batch": B, "prompt": T0, "chunk": T1},
+            "roofline": {"bound": "tensor", "kernel": "whole chunk", "achieved": tf, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"], "flops": flops,
+                         "peak_source": f"{peaks_src} bf16_tflops (burst)"}}
+
+
+def sample_kernel_us(args) -> dict:
+    """Device time of one nc_sample_topk over 32 rows of 65536 fp32 logits
+    (temperature 0.8, top_k 50) with Gumbel noise."""
+    import numpy as np
+    import torch
+    import kv_cache_transformer_b200 as nc
+    import nc_synth as syn
+    B, V = 32, 65536
+    lg = torch.from_numpy((np.random.default_rng(0).standard_normal((B, V)) * 3).astype(np.float32)).cuda()
+    nz = torch.from_numpy(syn.gumbel(5, (B, V), stream=0)).cuda()
+    nx = torch.empty((B,), dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        nc.nc_sample_topk(lg, nx, nz, 0.8, 50)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = 20
+    e0.record()
+    for _ in range(n):
+        nc.nc_sample_topk(lg, nx, nz, 0.8, 50)
+    e1.record()
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / n
+    return {"us_per_call": us, "rows": B, "vocab": V, "temperature": 0.8, "top_k": 50,
+            "bytes_per_call": 4 * B * V * 5, "GB/s": 4 * B * V * 5 / (us / 1e6) / 1e9,
+            "note": "the row is read four times (three radix passes, one pick) plus the noise once"}
 
 
 def run_decode_workload(args):

@@ -448,6 +448,28 @@ bool make_map_bf16_k64(CUtensorMap *map, const void *ptr, int rows, int cols, in
   return r == CUDA_SUCCESS;
 }
 
+// bf16 tensor map of rank 2..5 over `ptr`: dims[0] is the contiguous
+// dimension (64 elements = the 128-byte swizzle span), strides[i] the byte
+// stride of dims[i + 1] (any order, multiples of 16), box[i] the box extent
+// in each dimension; 128-byte swizzle, zero fill outside the tensor.
+bool make_map_bf16(CUtensorMap *map, const void *ptr, int rank, const uint64_t *dims, const uint64_t *strides,
+                   const uint32_t *box) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || rank < 2 || rank > 5) return false;
+  cuuint64_t d[5], st[4];
+  cuuint32_t bx[5], estr[5];
+  for (int i = 0; i < rank; i++) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    estr[i] = 1;
+    if (i + 1 < rank) st[i] = strides[i];
+  }
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), d, st, bx, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool gemm_tc_supported(int M, int N, int K, int lda) {
   return M > 0 && N > 0 && K > 0 && K % BK == 0 && N % 32 == 0 && lda % 8 == 0;
 }

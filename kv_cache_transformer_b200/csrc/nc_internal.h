@@ -66,7 +66,7 @@ struct StepPlan {
   size_t smem = 0;                   // dynamic shared memory per CTA
   size_t ws_bytes = 0;               // device workspace
   size_t off_ctr = 0, off_x0 = 0, off_x1 = 0, off_xb0 = 0, off_xb1 = 0, off_y = 0, off_f = 0, off_qk = 0,
-         off_ss = 0, off_cv = 0, off_ci = 0, off_ap = 0, off_pp = 0;
+         off_cv = 0, off_ci = 0, off_ap = 0, off_pp = 0;
 };
 }  // namespace nc
 

@@ -94,7 +94,6 @@ struct StepArgs {
   float *x0, *x1;             // [32][d] fp32 residual: layer input, after attention
   bf16 *xb0, *xb1, *y, *f;    // [32][d], [32][d], [32][d], [32][F]
   float *qk;                  // [32][H + 1][128]: q heads and k after RoPE, before QK norm
-  float *ss;                  // [2L + 1][grid][32]: per-CTA sums of squares for each norm
   bf16 *kc, *vc;              // [L][max_batch][max_seq][128]
   const float2 *rope;         // [max_seq][64]
   float *logits;              // [B][V]
@@ -127,6 +126,7 @@ struct Smem {
   int *abort_flag;
   int *pos, *valid;        // [32]
   float *inv;              // [32] per-sequence 1/rms of the phase's normed input
+  float *red_ss;           // [NCW][32] per-warp sums of squares of the staged rows
   int *flag;
 };
 
@@ -185,6 +185,7 @@ struct Unit {
   int u, split;   // unit index, K split (MLP projection)
   int r0, R, N;   // first row, rows per unit, rows of the layer
   int kb0, nkb;
+  int sbox;       // k-blocks of the activation map's box (what one staging copy brings)
   const CUtensorMap *map, *amap;
 };
 
@@ -193,6 +194,7 @@ __device__ __forceinline__ Unit unit_of(const StepArgs &a, int type, int layer, 
   u.active = false;
   u.split = 0;
   u.kb0 = 0;
+  u.sbox = a.d / 64;
   if (type == P_QKV) {
     u.N = (a.H + 2) * 128;
     u.R = 16;
@@ -230,6 +232,7 @@ __device__ __forceinline__ Unit unit_of(const StepArgs &a, int type, int layer, 
     const int kbt = a.F / 64, kbs = (kbt + a.s_p - 1) / a.s_p;
     u.kb0 = u.split * kbs;
     u.nkb = max(0, min(kbs, kbt - u.kb0));
+    u.sbox = kbs;
     u.map = a.wmaps + 4 * layer + 3;
     u.amap = a.amaps + 3;
   } else {  // P_HEAD
@@ -294,6 +297,34 @@ __device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorM
       : "memory");
 }
 
+// Tensor copies of rank 3 and 4 (one copy per ring slot, per cache tile, per
+// staging), with an L2 cache hint for the streamed weights.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_hint(void *dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d_hint(void *dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                                 uint64_t *bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // 1D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
 // completing on `bar`'s transaction count.
 __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
@@ -304,14 +335,17 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint3
 }
 
 // ------------------------------------------------------------- producer
-// Slot sizes: a linear unit of R rows puts kps = SLOT / (R * 128) k-blocks in
-// a slot (the lm_head: 2 k-blocks of 64 rows); attention puts one K or V tile
-// of 64 keys in a slot. The whole warp walks the program: lane 0 waits for a
-// free slot and arms its barrier, then each lane issues one of the slot's
-// tensor copies, so a slot's copies leave together.
-__device__ __forceinline__ int kps_of(int R) { return SLOT / (R * 128); }
+// Slot contents: a linear unit of R rows puts kps = SLOT / (R * 128) k-blocks
+// in a slot, [kb][R rows][128 B], as one tensor copy whose box spans the
+// k-blocks (the last slot of a unit may run past the unit's k-blocks: zero
+// fill past K, or a few bytes of the next split that nobody reads); the
+// lm_head puts 2 k-blocks of 64 rows; attention puts one K or V tile of 64
+// keys, [half][key][128 B]. Few, large copies keep the SM's queue of pending
+// tensor copies short, so the activations a phase stages are not queued
+// behind prefetched weights.
+__host__ __device__ __forceinline__ int kps_of(int R) { return SLOT / (R * 128); }
 
-__device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int lane) {
+__device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
   uint64_t evict_first;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(evict_first));
   uint32_t t = 0;
@@ -320,13 +354,9 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int la
     slot = t % a.slots;
     const uint32_t ph = (t / a.slots) & 1;
     t++;
-    int ok = 1;
-    if (lane == 0) {
-      ok = mbar_wait(&s.empty[slot], ph ^ 1, s.abort_flag, a.status) ? 1 : 0;
-      if (ok) mbar_arrive_expect_tx(&s.full[slot], bytes);
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    return ok != 0;
+    if (!mbar_wait(&s.empty[slot], ph ^ 1, s.abort_flag, a.status)) return false;
+    mbar_arrive_expect_tx(&s.full[slot], bytes);
+    return true;
   };
   const int c = blockIdx.x, P = n_phases(a);
   for (int p = 0; p < P; p++) {
@@ -347,14 +377,13 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int la
         for (int which = 0; which < 2; which++) {
           uint32_t slot;
           if (!take(slot, SLOT)) return;
-          if (first && lane == 0) trace_mark(a, p, 5);
+          if (first) trace_mark(a, p, 5);
           first = false;
           const bool sh = key < plen;
-          const CUtensorMap *map = a.kvmaps + (sh ? 2 : 0) + which;
-          const int row = (sh ? prow0 : row0) + key;
-          if (lane < 2) tma_load_2d(ring + slot * SLOT + lane * 8192, map, lane * 64, row, &s.full[slot]);
+          tma_load_3d(ring + slot * SLOT, a.kvmaps + (sh ? 2 : 0) + which, 0, (sh ? prow0 : row0) + key, 0,
+                      &s.full[slot]);
         }
-      if (lane == 0) trace_mark(a, p, 6);
+      trace_mark(a, p, 6);
     } else if (type == P_QKV || type == P_OPROJ || type == P_FC || type == P_PROJ || type == P_HEAD) {
       const Unit u = unit_of(a, type, layer, c);
       if (!u.active) continue;
@@ -362,75 +391,73 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring, int la
         const int rows = min(u.R, a.V - u.r0);
         for (int g0 = 0; g0 < rows; g0 += HG)
           for (int kb = 0; kb < u.nkb; kb += 2) {
-            const int n = min(2, u.nkb - kb);
             uint32_t slot;
-            if (!take(slot, n * HG * 128)) return;
-            if (first && lane == 0) trace_mark(a, p, 5);
+            if (!take(slot, 2 * HG * 128)) return;
+            if (first) trace_mark(a, p, 5);
             first = false;
-            if (lane < n)
-              tma_load_2d_hint(ring + slot * SLOT + lane * HG * 128, u.map, (kb + lane) * 64, u.r0 + g0, &s.full[slot],
-                               evict_first);
+            tma_load_3d_hint(ring + slot * SLOT, u.map, 0, u.r0 + g0, kb, &s.full[slot], evict_first);
           }
       } else {
         const int kps = kps_of(u.R);
         for (int ch = 0; ch < u.nkb; ch += kps) {
-          const int n = min(kps, u.nkb - ch);
           uint32_t slot;
-          if (!take(slot, n * u.R * 128)) return;
-          if (first && lane == 0) trace_mark(a, p, 5);
+          if (!take(slot, kps * u.R * 128)) return;
+          if (first) trace_mark(a, p, 5);
           first = false;
-          if (type == P_QKV) {  // rows r0..r0+7 and their RoPE partners r0+64..r0+71: two boxes per k-block
-            if (lane < 2 * n) {
-              const int j = lane >> 1, hi = lane & 1;
-              tma_load_2d_hint(ring + slot * SLOT + j * u.R * 128 + hi * 8 * 128, u.map, (u.kb0 + ch + j) * 64,
-                               u.r0 + 64 * hi, &s.full[slot], evict_first);
-            }
-          } else if (lane < n) {
-            tma_load_2d_hint(ring + slot * SLOT + lane * u.R * 128, u.map, (u.kb0 + ch + lane) * 64, u.r0,
-                             &s.full[slot], evict_first);
-          }
+          if (type == P_QKV)  // rows r0..r0+7 and their RoPE partners r0+64..r0+71
+            tma_load_4d_hint(ring + slot * SLOT, u.map, 0, u.r0, 0, u.kb0 + ch, &s.full[slot], evict_first);
+          else
+            tma_load_3d_hint(ring + slot * SLOT, u.map, 0, u.r0, u.kb0 + ch, &s.full[slot], evict_first);
         }
       }
-      if (lane == 0) trace_mark(a, p, 6);
+      trace_mark(a, p, 6);
     }
   }
 }
 
 // ------------------------------------------------- compute-side helpers
-// Stage the phase's activation rows: nkb boxes of 64 columns x 32 rows from
-// k-block kb0 of the activation map into xs ([kb][32 rows][128 B], swizzled).
-// Issued by one warp right after the barrier (lane j issues boxes j, j + 32,
-// ...); the writers' data was released through the grid barrier, the proxy
-// fences order it ahead of the copies.
-__device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CUtensorMap *amap, int kb0, int nkb,
-                                            int lane) {
+// Stage the phase's activation rows: sbox k-blocks of 64 columns x 32 rows
+// from k-block kb0 of the activation map into xs ([kb][32 rows][128 B],
+// swizzled), one tensor copy issued right after the barrier. The writers' data
+// was released through the grid barrier; the proxy fences order it (and this
+// CTA's earlier generic accesses to xs) ahead of the copy.
+__device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CUtensorMap *amap, int kb0, int sbox) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  if (lane == 0) mbar_arrive_expect_tx(s.x_bar, nkb * MAXB * 128);
-  __syncwarp();
-  for (int j = lane; j < nkb; j += 32) tma_load_2d(xs + j * MAXB * 128, amap, (kb0 + j) * 64, 0, s.x_bar);
+  mbar_arrive_expect_tx(s.x_bar, sbox * MAXB * 128);
+  tma_load_3d(xs, amap, 0, 0, kb0, s.x_bar);
 }
 
-// 1/rms of each sequence's row from the per-CTA partial sums of squares of a
-// norm: units [0, nu) of ss[norm]. Eight threads per sequence load every
-// eighth partial (all loads first), combined in a fixed order.
-__device__ void load_inv(const StepArgs &a, const Smem &s, int norm, int nu, int e) {
-  const int b = e >> 3, q = e & 7;
-  const float *src = a.ss + (size_t)norm * a.grid * 32;
-  constexpr int NL = 20;  // nu <= grid <= 8 * NL
-  float v[NL];
+// 1/rms of each sequence's row from the staged bf16 row itself (the normed
+// phases stage the whole row, K = d): warp w sums the squares of k-blocks w,
+// w + 8, ... (lane = sequence), the warps' partials are added in warp order.
+__device__ void smem_inv(const StepArgs &a, const Smem &s, const uint8_t *xs, int nkb, int warp, int lane, int e) {
+  float acc = 0.f;
+  for (int kb = warp; kb < nkb; kb += NCW) {
+    const uint4 *row = reinterpret_cast<const uint4 *>(xs + kb * MAXB * 128 + lane * 128);
+    // the row's 16-byte chunks in column order (the swizzle permutes them by
+    // row), so every row sums in the same order and the lanes hit different banks
 #pragma unroll
-  for (int i = 0; i < NL; i++) {
-    const int u = q + 8 * i;
-    v[i] = u < nu ? __ldcg(src + (size_t)u * 32 + b) : 0.f;
+    for (int c = 0; c < 8; c++) {
+      const uint4 v = row[c ^ (lane & 7)];
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const float lo = __uint_as_float(w4[i] << 16), hi = __uint_as_float(w4[i] & 0xffff0000u);
+        acc = fmaf(lo, lo, acc);
+        acc = fmaf(hi, hi, acc);
+      }
+    }
   }
-  float sum = 0.f;
+  s.red_ss[warp * 32 + lane] = acc;
+  csync();
+  if (e < MAXB) {
+    float sum = 0.f;
 #pragma unroll
-  for (int i = 0; i < NL; i++) sum += v[i];
-  sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-  sum += __shfl_xor_sync(0xffffffffu, sum, 4);
-  if (q == 0) s.inv[b] = b < a.B ? rsqrtf(sum / a.d + a.eps) : 0.f;
+    for (int w = 0; w < NCW; w++) sum += s.red_ss[w * 32 + e];
+    s.inv[e] = e < a.B ? rsqrtf(sum / a.d + a.eps) : 0.f;
+  }
+  csync();
 }
 
 // The unit's product for every sequence, this warp's K part (k-blocks kb
@@ -523,17 +550,6 @@ __device__ float *reduce_warps(float *red, int R, int MT, int e) {
   }
   csync();
   return out;
-}
-
-// Per-sequence sum over the unit's rows of sq[b * R + r] (fixed order),
-// written as this CTA's partial of norm `norm`.
-__device__ void write_ss(const StepArgs &a, const float *sq, int R, int norm, int u, int e) {
-  if (e < MAXB) {
-    float sum = 0.f;
-    if (e < a.B)
-      for (int r = 0; r < R; r++) sum += sq[e * R + r];
-    a.ss[((size_t)norm * a.grid + u) * 32 + e] = sum;
-  }
 }
 
 // ------------------------------------------------------------ attention
@@ -814,23 +830,19 @@ __device__ __forceinline__ void load_resid(const StepArgs &a, const Unit &u, con
   }
 }
 
-__device__ void resid_epilogue(const StepArgs &a, float *sum, const Unit &u, const float (&xr)[XR], float *xout,
-                               bf16 *xbout, int norm, int e) {
+__device__ void resid_epilogue(const StepArgs &a, const float *sum, const Unit &u, const float (&xr)[XR],
+                               float *xout, bf16 *xbout, int e) {
 #pragma unroll
   for (int i = 0; i < XR; i++) {
     const int idx = e + 32 * NCW * i;
     if (idx >= MAXB * u.R) break;
     const int b = idx / u.R, r = idx % u.R, col = u.r0 + r;
-    float v = 0.f;
     if (b < a.B && col < u.N) {
-      v = xr[i] + sum[idx];
+      const float v = xr[i] + sum[idx];
       xout[(size_t)b * a.d + col] = v;
       xbout[(size_t)b * a.d + col] = __float2bfloat16_rn(v);
     }
-    sum[idx] = v * v;
   }
-  csync();
-  write_ss(a, sum, u.R, norm, u.u, e);
 }
 
 // lm_head rows [row0, row0 + 64): softcap, logits, and the running
@@ -956,8 +968,10 @@ __host__ __device__ constexpr int xreg_bytes(int d) {
               : (NCW + 1) * MAXB * MAX_R * 4);
 }
 
-// 9 warps of at most 200 registers: one CTA per SM with every warp resident
-__global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
+// 9 warps: registers are allocated to warps in groups of four (one per SM
+// sub-partition), so the block is charged for 12 warps and must stay within
+// 168 registers a thread
+__global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
@@ -973,7 +987,8 @@ __global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
     s.pos = s.abort_flag + 1;
     s.valid = s.pos + 32;
     s.inv = reinterpret_cast<float *>(s.valid + 32);
-    s.flag = reinterpret_cast<int *>(s.inv + 32);
+    s.red_ss = s.inv + 32;
+    s.flag = reinterpret_cast<int *>(s.red_ss + NCW * 32);
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1002,7 +1017,7 @@ __global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
   __syncthreads();
 
   if (warp == 0) {
-    producer(a, s, ring, lane);
+    if (lane == 0) producer(a, s, ring);
   } else {
     const int e = threadIdx.x - 32;
     const int cw = warp - 1;  // compute warp 0..7
@@ -1035,21 +1050,10 @@ __global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
           float tot = 0.f;
           for (int w = 0; w < NCW; w++) tot += red[w];
           const float inv = rsqrtf(tot / a.d + a.eps);
-          float sq2 = 0.f;
           for (int i = e; i < a.d; i += 32 * NCW) {
             const float v = __bfloat162float(row[i]) * inv;
             a.x0[(size_t)b * a.d + i] = v;
             a.xb0[(size_t)b * a.d + i] = __float2bfloat16_rn(v);
-            sq2 += v * v;
-          }
-          sq2 = warp_sum(sq2);
-          if (lane == 0) red[NCW + cw] = sq2;
-          csync();
-          // norm 0 (the first layer's pre-attention norm) has one partial
-          if (e == 0) {
-            float t2 = 0.f;
-            for (int w = 0; w < NCW; w++) t2 += red[NCW + w];
-            a.ss[b] = t2;
           }
           csync();
         }
@@ -1081,17 +1085,14 @@ __global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
         // linear layer
         const Unit u = unit_of(a, type, layer, blockIdx.x);
         if (u.active) {
-          if (cw == 0) stage_issue(s, xs, u.amap, u.kb0, u.nkb, lane);
+          if (e == 0) stage_issue(s, xs, u.amap, u.kb0, u.sbox);
           float xr[XR];  // residual inputs of the rows this thread finishes
           if (type == P_OPROJ) load_resid(a, u, a.x0, e, xr);
           else if (type == P_PROJ) load_resid(a, u, a.x1, e, xr);
-          // the row factors of a normed input, while the copies fly
-          if (type == P_QKV) load_inv(a, s, 2 * layer, layer == 0 ? 1 : a.n_p, e);
-          else if (type == P_FC) load_inv(a, s, 2 * layer + 1, a.n_o, e);
-          else if (type == P_HEAD) load_inv(a, s, 2 * a.L, a.L == 0 ? 1 : a.n_p, e);
           mbar_wait(s.x_bar, xph & 1, s.abort_flag, a.status);
           xph++;
-          csync();  // s.inv written
+          // the row factors of a normed input (QKV, MLP fc, lm_head)
+          if (type == P_QKV || type == P_FC || type == P_HEAD) smem_inv(a, s, xs, u.nkb, cw, lane, e);
           if (e == 0) trace_mark(a, p, 1);
           if (ok && type == P_HEAD) {
             ArgMax best[4];
@@ -1136,7 +1137,7 @@ __global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
               if (type == P_QKV) {
                 qkv_epilogue(a, s, sum, u, layer, e);
               } else if (type == P_OPROJ) {
-                resid_epilogue(a, sum, u, xr, a.x1, a.xb1, 2 * layer + 1, e);
+                resid_epilogue(a, sum, u, xr, a.x1, a.xb1, e);
               } else if (type == P_FC) {
                 for (int idx = e; idx < a.B * u.R; idx += 32 * NCW) {
                   const int b = idx / u.R, r = idx % u.R, col = u.r0 + r;
@@ -1177,7 +1178,7 @@ __global__ void __maxnreg__(200) decode_step_kernel(StepArgs a) {
                     sum[idx] = v;
                   }
                   csync();
-                  resid_epilogue(a, sum, u, xr, a.x0, a.xb0, 2 * layer + 2, e);
+                  resid_epilogue(a, sum, u, xr, a.x0, a.xb0, e);
                 }
                 csync();  // s.flag is rewritten by the next use
               }
@@ -1196,7 +1197,8 @@ int round8(int v) { return (v + 7) / 8 * 8; }
 
 }  // namespace
 
-bool make_map_bf16_k64(CUtensorMap *map, const void *ptr, int rows, int cols, int ld, int box_rows);
+bool make_map_bf16(CUtensorMap *map, const void *ptr, int rank, const uint64_t *dims, const uint64_t *strides,
+                   const uint32_t *box);
 
 bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *pl) {
   *pl = StepPlan{};
@@ -1247,7 +1249,6 @@ bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *pl) {
   p.off_y = take(2 * MAXB * d);
   p.off_f = take(2 * MAXB * (size_t)F);
   p.off_qk = take(sizeof(float) * MAXB * (H + 1) * 128);
-  p.off_ss = take(sizeof(float) * (2 * c.depth + 1) * (size_t)G * 32);
   p.off_cv = take(sizeof(float) * (size_t)G * 32);
   p.off_ci = take(sizeof(int) * (size_t)G * 32);
   p.off_ap = take(sizeof(float) * MAXB * MAX_SPLIT * 16 * AROW);
@@ -1262,44 +1263,76 @@ int decode_step_maps_count(const nc_config &c) { return 4 * c.depth + 1 + 4 + 4;
 
 int decode_step_prefix_map_index(const nc_config &c) { return 4 * c.depth + 3; }
 
+namespace {
+// [rows, K] bf16 weights (row pitch K) as (64 columns, rows, K / 64 k-blocks):
+// a box of (64, box_rows, box_kb) lands as [kb][row][128 B]
+bool weight_map(CUtensorMap *m, const void *w, int rows, int K, int box_rows, int box_kb) {
+  const uint64_t dims[3] = {64, (uint64_t)rows, (uint64_t)(K / 64)};
+  const uint64_t strides[2] = {(uint64_t)K * 2, 128};
+  const uint32_t box[3] = {64, (uint32_t)box_rows, (uint32_t)box_kb};
+  return make_map_bf16(m, w, 3, dims, strides, box);
+}
+
+// the K or V cache, [rows][128] bf16, as (64 dims, rows, 2 halves): a box of
+// (64, 64 keys, 2) lands as [half][key][128 B]
+bool cache_map(CUtensorMap *m, const void *cache, int rows) {
+  const uint64_t dims[3] = {64, (uint64_t)rows, 2};
+  const uint64_t strides[2] = {256, 128};
+  const uint32_t box[3] = {64, (uint32_t)KT, 2};
+  return make_map_bf16(m, cache, 3, dims, strides, box);
+}
+}  // namespace
+
 // The two maps through which the step kernel reads shared-prefix rows: the
 // prefix cache's K and V viewed as [depth * max_batch * max_seq, 128].
 bool decode_step_prefix_maps(const void *kcache, const void *vcache, const nc_config &c, int max_batch, int max_seq,
                              CUtensorMap *out) {
   const int rows = c.depth * max_batch * max_seq;
-  return make_map_bf16_k64(&out[0], kcache, rows, 128, 128, KT) && make_map_bf16_k64(&out[1], vcache, rows, 128, 128, KT);
+  return cache_map(&out[0], kcache, rows) && cache_map(&out[1], vcache, rows);
 }
 
 // Tensor maps of the step kernel, written to host memory `out` (to be copied
-// to the device): per layer QKV (8-row boxes: a unit is two RoPE-paired
-// half blocks), O, fc, proj weights (boxes of the unit's rows), the lm_head
-// (64-row boxes); the K and V caches viewed as [depth * max_batch * max_seq,
-// 128]; the activations the linear phases stage (bf16(x0), y, bf16(x1), f)
-// as [32, K] with 32-row boxes.
+// to the device): per layer the QKV weights as (64 columns, rows, 2 RoPE
+// halves 64 rows apart, k-blocks) so that a unit's 8 + 8 paired rows arrive
+// in one copy, then the O, fc, proj weights (boxes of the unit's rows and a
+// slot's k-blocks), the lm_head (64 rows x 2 k-blocks); the K and V caches
+// (this cache, then the prefix cache, initially this one); the activations
+// the linear phases stage (bf16(x0), y, bf16(x1), f) as (64 columns, 32 rows,
+// k-blocks) with a box of the phase's k-blocks.
 bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *vcache, int max_batch, int max_seq,
                             const StepPlan &p, void *ws, CUtensorMap *out) {
   const nc_config &c = m->cfg;
   const int d = c.d_model, F = c.mlp_hidden, H = c.n_head;
   for (int l = 0; l < c.depth; l++) {
     const nc_layer_w &w = m->layers[l];
-    if (!make_map_bf16_k64(&out[4 * l + 0], w.wqkv, (H + 2) * 128, d, d, 8)) return false;
-    if (!make_map_bf16_k64(&out[4 * l + 1], w.wo, d, H * 128, H * 128, p.r_o)) return false;
-    if (!make_map_bf16_k64(&out[4 * l + 2], w.wfc, F, d, d, p.r_f)) return false;
-    if (!make_map_bf16_k64(&out[4 * l + 3], w.wproj, d, F, F, p.r_p)) return false;
+    {
+      const uint64_t dims[4] = {64, (uint64_t)((H + 2) * 128 - 64), 2, (uint64_t)(d / 64)};
+      const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)64 * d * 2, 128};
+      const uint32_t box[4] = {64, 8, 2, (uint32_t)kps_of(16)};
+      if (!make_map_bf16(&out[4 * l + 0], w.wqkv, 4, dims, strides, box)) return false;
+    }
+    if (!weight_map(&out[4 * l + 1], w.wo, d, H * 128, p.r_o, kps_of(p.r_o))) return false;
+    if (!weight_map(&out[4 * l + 2], w.wfc, F, d, p.r_f, kps_of(p.r_f))) return false;
+    if (!weight_map(&out[4 * l + 3], w.wproj, d, F, p.r_p, kps_of(p.r_p))) return false;
   }
-  if (!make_map_bf16_k64(&out[4 * c.depth], m->wlm, c.vocab, d, d, HG)) return false;
+  if (!weight_map(&out[4 * c.depth], m->wlm, c.vocab, d, HG, 2)) return false;
   const int rows = c.depth * max_batch * max_seq;
-  if (!make_map_bf16_k64(&out[4 * c.depth + 1], kcache, rows, 128, 128, KT)) return false;
-  if (!make_map_bf16_k64(&out[4 * c.depth + 2], vcache, rows, 128, 128, KT)) return false;
+  if (!cache_map(&out[4 * c.depth + 1], kcache, rows) || !cache_map(&out[4 * c.depth + 2], vcache, rows)) return false;
   // no shared prefixes yet: the prefix maps view this cache
   out[4 * c.depth + 3] = out[4 * c.depth + 1];
   out[4 * c.depth + 4] = out[4 * c.depth + 2];
   uint8_t *base = static_cast<uint8_t *>(ws);
   CUtensorMap *am = out + 4 * c.depth + 5;
-  if (!make_map_bf16_k64(&am[0], base + p.off_xb0, MAXB, d, d, MAXB)) return false;
-  if (!make_map_bf16_k64(&am[1], base + p.off_y, MAXB, d, d, MAXB)) return false;
-  if (!make_map_bf16_k64(&am[2], base + p.off_xb1, MAXB, d, d, MAXB)) return false;
-  if (!make_map_bf16_k64(&am[3], base + p.off_f, MAXB, F, F, MAXB)) return false;
+  auto act_map = [&](CUtensorMap *mp, size_t off, int K, int box_kb) {
+    const uint64_t dims[3] = {64, (uint64_t)MAXB, (uint64_t)(K / 64)};
+    const uint64_t strides[2] = {(uint64_t)K * 2, 128};
+    const uint32_t box[3] = {64, (uint32_t)MAXB, (uint32_t)box_kb};
+    return make_map_bf16(mp, base + off, 3, dims, strides, box);
+  };
+  const int kbs = (F / 64 + p.s_p - 1) / p.s_p;
+  if (!act_map(&am[0], p.off_xb0, d, d / 64) || !act_map(&am[1], p.off_y, d, d / 64) ||
+      !act_map(&am[2], p.off_xb1, d, d / 64) || !act_map(&am[3], p.off_f, F, kbs))
+    return false;
   return true;
 }
 
@@ -1374,7 +1407,6 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
   a.y = reinterpret_cast<bf16 *>(base + pl.off_y);
   a.f = reinterpret_cast<bf16 *>(base + pl.off_f);
   a.qk = reinterpret_cast<float *>(base + pl.off_qk);
-  a.ss = reinterpret_cast<float *>(base + pl.off_ss);
   a.kc = (bf16 *)kc;
   a.vc = (bf16 *)vc;
   a.rope = rope;
