@@ -68,14 +68,21 @@ extern "C" {
 #define NC_BF16 1
 
 /* Model shape. Fields follow the feature list above; n_kv_head = 1 is the
- * page's multi-query attention. Constants the pages leave open are inputs:
+ * page's multi-query attention. n_kv_head > 1 groups the query heads: head h
+ * reads KV head h / (n_head / n_kv_head) (grouped-query attention; n_kv_head
+ * = n_head is multi-head attention, the reading under which the lineage
+ * article "Karpathy 的 nano 諧系" pretraining bullet's d20 of about 560M
+ * parameters comes out). Constants the pages leave open are inputs:
  * rope_base (10000), softcap (15), norm_eps (1e-6, inside the sqrt of every
  * RMSNorm). */
 typedef struct {
   int depth;       /* number of Transformer blocks (>= 0) */
   int d_model;     /* residual width d */
   int n_head;      /* query heads H; n_head * head_dim == d_model */
-  int n_kv_head;   /* KV heads; must divide n_head (this build: 1) */
+  int n_kv_head;   /* KV heads; must divide n_head. The sm_100a decode step takes
+                      up to 16 query heads per KV head, the tensor-core prefill
+                      attention a group size dividing 128 (or one KV head);
+                      other shapes run the generic kernels */
   int head_dim;    /* hd, even */
   int mlp_hidden;  /* F (4*d in the presets) */
   int vocab;       /* V */
@@ -112,7 +119,8 @@ int nc_device_status(nc_model *model, uint32_t *out_bits);
  * 0. A bf16 decode step of up to 32 sequences runs as one persistent kernel
  * (NC_K_STEP); with the environment variable NC_DECODE_STEP_KERNEL=0 set
  * when the cache is created, it runs as one launch per layer step instead
- * (a diagnostic switch: same results within the stated tolerances).
+ * (one KV head) or on the generic kernels (several KV heads): a diagnostic
+ * switch, same results within the stated tolerances.
  * Errors: NC_EINVAL, NC_ENOMEM, NC_ECUDA. */
 int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out);
 

@@ -178,7 +178,7 @@ cudaError_t norm_rows(nc_model *m, nc_kv *kv, int M, cudaStream_t s) {
 // RoPE + QK norm of the M rows of kv->qkv, q out, K/V appended to the cache.
 cudaError_t rope_append(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (!rm.pos && !rm.off && nc::rowops_supported(c))
+  if (!rm.pos && !rm.off && c.n_kv_head == 1 && nc::rowops_supported(c))
     return nc::k_rope_qk_bf16(kv->qkv, M, rm.T, c.n_head, kv->rope, kv->q, kc, vc, kv->max_seq, c.norm_eps, s);
   nc::k_rope_qknorm_append(c.dtype, kv->qkv, rm, M, c.n_head, c.n_kv_head, c.head_dim, kv->rope, kv->q, kc, vc,
                            kv->max_seq, kv->valid, c.norm_eps, s);
@@ -190,12 +190,13 @@ int layer_of(const nc_kv *kv, const void *kc) {
   return (int)(((const char *)kc - (const char *)kv->k) / (ptrdiff_t)(kv->layer_elems * kv->model->elem));
 }
 
-// Causal MQA attention of the M rows in kv->q against layer cache kc/vc.
+// Causal attention of the M rows in kv->q (H query heads in groups of H/Hkv
+// per KV head) against layer cache kc/vc.
 cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
   if (m->fast && !rm.pos && !rm.off && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
-    return nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, kv->max_batch, kv->max_seq, kv->y,
-                                 m->status, s);
+    return nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, c.n_kv_head, kv->max_batch, kv->max_seq,
+                                 kv->y, m->status, s);
   // decode rows and appended chunks may read shared-prefix rows; prefill rows
   // replace their sequences
   const nc::KvPrefix pre = (rm.pos || rm.off) ? prefix_view(kv, layer_of(kv, kc)) : nc::KvPrefix{};
@@ -215,15 +216,15 @@ cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::Row
 //          except in the last layer
 bool fused_layers_ok(const nc_model *m, const nc_kv *kv, int M, nc::RowMap rm) {
   const nc_config &c = m->cfg;
-  const int d = c.d_model, q = c.n_head * 128, F = c.mlp_hidden;
+  const int d = c.d_model, q = c.n_head * 128, F = c.mlp_hidden, qkv = q + 256 * c.n_kv_head;
   return m->fast && !rm.pos && !rm.off && M >= 128 && kv->row_ss && nc::rowops_supported(c) &&
-         nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim) && nc::gemm_tc_supported(M, q + 256, d, d) &&
+         nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim) && nc::gemm_tc_supported(M, qkv, d, d) &&
          nc::gemm_tc_supported(M, d, q, q) && nc::gemm_tc_supported(M, F, d, d) && nc::gemm_tc_supported(M, d, F, F);
 }
 
 int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  const int d = c.d_model, H = c.n_head, F = c.mlp_hidden, q = H * 128;
+  const int d = c.d_model, H = c.n_head, F = c.mlp_hidden, q = H * 128, qkv = q + 256 * c.n_kv_head;
   nc::GemmFuse fz;
   fz.eps = c.norm_eps;
   fz.xb = kv->h;
@@ -232,6 +233,7 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
   fz.q = kv->q;
   fz.T = rm.T;
   fz.H = H;
+  fz.Hkv = c.n_kv_head;
   fz.max_seq = kv->max_seq;
   const int nss = (d + 127) / 128;
   cudaError_t e = cudaSuccess;
@@ -251,7 +253,7 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
       ProfScope p(m, NC_K_GEMM, s);
       fz.ss_in = kv->row_ss;
       fz.nss = l == 0 ? 0 : nss;
-      gemm(nc::EPI_QKV, kv->h, d, w.wqkv, q + 256, d, nullptr);
+      gemm(nc::EPI_QKV, kv->h, d, w.wqkv, qkv, d, nullptr);
     }
     if (e == cudaSuccess) {
       ProfScope p(m, NC_K_ATTN, s);
@@ -473,7 +475,7 @@ int prefill_tail(nc_model *m, nc_kv *kv, int B, int T, int logits_mode, float *d
     }
   } else {
     logits = d_logits ? d_logits : kv->logits;
-    if (kv->dec_fast && nc::decode_fast_supported(c, B)) {
+    if (kv->dec_fast && B <= 32) {
       // last rows -> fused norm + lm_head + softcap + argmax (the decode head kernel)
       ProfScope p(m, NC_K_HEAD, s);
       cudaError_t e = nc::k_gather_rows_ss(kv->x, B, c.d_model, T, T - 1, kv->xl, kv->ss, 32, s);
@@ -637,7 +639,7 @@ int nc_kv_create(const nc_model *model, int max_batch, int max_seq, nc_kv **out)
   kv->link_seq.assign(max_batch, -1);
   kv->dep_count.assign(max_batch, 0);
   if (model->fast && nc::rowops_supported(c)) alloc((void **)&kv->row_ss, sizeof(float) * ((d + 127) / 128) * rows);
-  kv->dec_fast = nc::decode_fast_supported(c, 1);
+  kv->dec_fast = nc::decode_head_supported(c);
   if (kv->dec_fast) {
     int nb = max_batch < 32 ? max_batch : 32;
     kv->part_floats = nc::decode_part_floats(c, nb, max_seq, model->num_sms, &kv->attn_splits, &kv->attn_chunk);
@@ -777,7 +779,7 @@ int nc_decode_step(nc_model *m, nc_kv *kv, const int32_t *d_tokens, const int32_
   const nc_config &c = m->cfg;
   cudaStream_t s = as_stream(stream);
   float *logits = d_logits ? d_logits : kv->logits;
-  if (kv->dec_fast && nc::decode_fast_supported(c, B))
+  if (kv->dec_fast && ((kv->step_grid > 0 && nc::decode_step_supported(c, B)) || nc::decode_fast_supported(c, B)))
     return decode_fast(m, kv, d_tokens, d_positions, B, d_noise, logits, d_next, s);
   if (!d_positions) {
     // positions default to the current lengths
@@ -959,7 +961,7 @@ int nc_attention_prefill_bf16(const void *d_q, const void *d_k, const void *d_v,
   if (rc) return rc;
   cudaStream_t s = as_stream(stream);
   if (nc::attn_prefill_tc_supported(H, 1, hd)) {
-    const cudaError_t e = nc::k_attn_prefill_tc(d_q, d_k, d_v, B, T, H, B, max_seq, d_y, status, s);
+    const cudaError_t e = nc::k_attn_prefill_tc(d_q, d_k, d_v, B, T, H, 1, B, max_seq, d_y, status, s);
     if (e != cudaSuccess) return fail(NC_ECUDA, "attention launch failed: %s", cudaGetErrorString(e));
     return NC_OK;
   }

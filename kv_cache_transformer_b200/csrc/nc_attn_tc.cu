@@ -1,10 +1,13 @@
-// nc_attn_tc.cu — causal multi-query prefill attention on tcgen05.
+// nc_attn_tc.cu — causal multi-query / grouped-query prefill attention on
+// tcgen05.
 //
-// With one KV head, the H query heads of a position all read the same keys
-// and values (the feature list's multi-query attention). The queries of a
-// sequence, stored [T, H, hd], are therefore one [T*H, hd] matrix whose row
-// r = t*H + h belongs to position t. A work item is 256 consecutive rows of
-// one sequence, two 128-row Q tiles (A and B) that share every K/V tile:
+// The H query heads form Hkv groups of G = H/Hkv heads, and the G heads of a
+// group read the same keys and values (one KV head: the feature list's
+// multi-query attention, Hkv = 1; multi-head attention, G = 1). For one
+// sequence and KV head j, the queries of group j at positions 0..T-1 are one
+// [T*G, hd] matrix whose row r = t*G + g is head j*G + g at position t. A
+// work item is 256 consecutive rows of one (sequence, KV head), two 128-row Q
+// tiles (A and B) that share every K/V tile:
 //   S_t  = Q_t K_j^T       (tcgen05, M=128 rows, N=128 keys, K=hd) -> TMEM
 //   P_t  = 2^(S_t*scale*log2e - m) with the causal mask key <= t(row), online
 //          max/sum, bf16 pairs written back into the upper half of S_t's
@@ -55,7 +58,8 @@ constexpr uint32_t TMEM_COLS = 512;
 
 struct AttnArgs {
   int T, H, B, max_seq;
-  int rows_per_seq;  // T*H
+  int Hkv, G;        // KV heads, query heads per KV head
+  int rows_per_seq;  // T*G rows of one (sequence, KV head)
   float scale_log2;  // log2(e) / sqrt(hd)
   bf16 *y;           // [B*T*H, 128]
   uint32_t *status;
@@ -148,16 +152,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_pairs = (a.rows_per_seq + ITEM - 1) / ITEM;
-  const int n_items = n_pairs * a.B;
+  const int nvs = a.B * a.Hkv;  // (sequence, KV head) pairs
+  const int n_items = n_pairs * nvs;
   const int G = gridDim.x, c = blockIdx.x;
 
-  // item i: rows 256*pp .. of sequence b, pp heaviest first; n_kv key tiles
-  auto item_of = [&](int i, int &b, int &row0, int &n_kv) {
-    const int pp = n_pairs - 1 - i / a.B;
-    b = i % a.B;
+  // item i: rows 256*pp .. of sequence b and KV head j, pp heaviest first;
+  // n_kv key tiles
+  auto item_of = [&](int i, int &b, int &j, int &row0, int &n_kv) {
+    const int pp = n_pairs - 1 - i / nvs;
+    b = (i % nvs) / a.Hkv;
+    j = i % a.Hkv;
     row0 = pp * ITEM;
     const int last = min(row0 + ITEM, a.rows_per_seq) - 1;
-    n_kv = (last / a.H) / BKV + 1;
+    n_kv = (last / a.G) / BKV + 1;
   };
 
   if (threadIdx.x == 0) {
@@ -196,24 +203,28 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int r = 0, it = 0; ok; r++, it++) {
         const int i = item_at(r, c, G);
         if (i >= n_items) break;
-        int b, row0, n_kv;
-        item_of(i, b, row0, n_kv);
+        int b, j, row0, n_kv;
+        item_of(i, b, j, row0, n_kv);
         if (!mbar_wait(q_empty, (it & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(q_full, 2 * TILE);
-        const int qrow = b * a.rows_per_seq + row0;
-        tma_load_2d(smem + OFF_Q, &mapQ, 0, qrow, q_full);
-        tma_load_2d(smem + OFF_Q + SUB, &mapQ, 64, qrow, q_full);
-        tma_load_2d(smem + OFF_Q + TILE, &mapQ, 0, qrow + BR, q_full);
-        tma_load_2d(smem + OFF_Q + TILE + SUB, &mapQ, 64, qrow + BR, q_full);
-        const int krow = b * a.max_seq;
-        for (int j = 0; j < n_kv && ok; j++)
+        // Q map (128 dims, G heads, Hkv groups, rows): with one KV head the
+        // rows are (position, head) pairs, else positions with G heads each
+        const int qz = a.Hkv == 1 ? 0 : j;
+        const int qw = a.Hkv == 1 ? b * a.rows_per_seq + row0 : b * a.T + row0 / a.G;
+        const int qstep = a.Hkv == 1 ? BR : BR / a.G;
+        tma_load_4d(smem + OFF_Q, &mapQ, 0, 0, qz, qw, q_full);
+        tma_load_4d(smem + OFF_Q + SUB, &mapQ, 64, 0, qz, qw, q_full);
+        tma_load_4d(smem + OFF_Q + TILE, &mapQ, 0, 0, qz, qw + qstep, q_full);
+        tma_load_4d(smem + OFF_Q + TILE + SUB, &mapQ, 64, 0, qz, qw + qstep, q_full);
+        const int krow = b * a.max_seq, kx = j * HD;
+        for (int kt = 0; kt < n_kv && ok; kt++)
           for (int w = 0; w < 2; w++, n++) {
             const int s = n % NSLOT;
             if (!mbar_wait(&kv_empty[s], ((n / NSLOT) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
             mbar_arrive_expect_tx(&kv_full[s], TILE);
             const CUtensorMap *map = w ? &mapV : &mapK;
-            tma_load_2d(smem + OFF_KV + s * TILE, map, 0, krow + j * BKV, &kv_full[s]);
-            tma_load_2d(smem + OFF_KV + s * TILE + SUB, map, 64, krow + j * BKV, &kv_full[s]);
+            tma_load_2d(smem + OFF_KV + s * TILE, map, kx, krow + kt * BKV, &kv_full[s]);
+            tma_load_2d(smem + OFF_KV + s * TILE + SUB, map, kx + 64, krow + kt * BKV, &kv_full[s]);
           }
       }
     }
@@ -245,8 +256,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int r = 0, it = 0; ok; r++, it++) {
         const int i = item_at(r, c, G);
         if (i >= n_items) break;
-        int b, row0, n_kv;
-        item_of(i, b, row0, n_kv);
+        int b, j_kv, row0, n_kv;
+        item_of(i, b, j_kv, row0, n_kv);
         if (!mbar_wait(q_full, it & 1, abort_flag, a.status)) break;
         uint32_t kaddr, vaddr;
         int kslot, vslot;
@@ -292,10 +303,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int rr = 0;; rr++) {
       const int i = item_at(rr, c, G);
       if (i >= n_items) break;
-      int b, row0, n_kv;
-      item_of(i, b, row0, n_kv);
-      const int row = row0 + t * BR + r;  // row inside the sequence
-      const int t_row = row < a.rows_per_seq ? row / a.H : 0x3fffffff;
+      int b, j_kv, row0, n_kv;
+      item_of(i, b, j_kv, row0, n_kv);
+      const int row = row0 + t * BR + r;  // row inside the (sequence, KV head)
+      const int t_row = row < a.rows_per_seq ? row / a.G : 0x3fffffff;
       float m = -INFINITY, l = 0.f;  // running max (scaled, log2 units) and sum
       for (int j = 0; j < n_kv; j++, g++) {
         ok = ok && mbar_wait(&s_full[t], g & 1, abort_flag, a.status);
@@ -395,7 +406,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = ok && mbar_wait(&o_done[t], (g - 1) & 1, abort_flag, a.status);
       tc_fence_after();
       const float inv = 1.f / l;
-      bf16 *dst = a.y + ((size_t)b * a.rows_per_seq + row) * HD;
+      // y row of (position t_row, head j*G + g) in [B*T, H, 128]
+      bf16 *dst = a.y + (((size_t)b * a.T + (row < a.rows_per_seq ? t_row : 0)) * a.H + j_kv * a.G + row % a.G) * HD;
 #pragma unroll 1
       for (int cc = 0; cc < HD; cc += 32) {
         uint32_t o[32];
@@ -425,17 +437,36 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 }  // namespace
 
-bool attn_prefill_tc_supported(int H, int Hkv, int hd) { return hd == HD && Hkv == 1 && H >= 1; }
+// A Q tile of 128 rows holds whole positions of one group unless there is a
+// single KV head (then it holds (position, head) rows in order).
+bool attn_prefill_tc_supported(int H, int Hkv, int hd) {
+  return hd == HD && H >= 1 && Hkv >= 1 && H % Hkv == 0 && (Hkv == 1 || BR % (H / Hkv) == 0);
+}
 
-// q: [B*T*H, 128] bf16 (rotated + normed), kc/vc: layer cache [max_batch*max_seq, 128],
-// y: [B*T*H, 128] bf16.
-cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int max_batch,
-                              int max_seq, void *y, uint32_t *status, cudaStream_t s) {
+bool make_map_bf16(CUtensorMap *map, const void *ptr, int rank, const uint64_t *dims, const uint64_t *strides,
+                   const uint32_t *box);
+
+// q: [B*T, H, 128] bf16 (rotated + normed), kc/vc: layer cache
+// [max_batch*max_seq, Hkv*128], y: [B*T, H, 128] bf16.
+cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int Hkv,
+                              int max_batch, int max_seq, void *y, uint32_t *status, cudaStream_t s) {
+  if (!attn_prefill_tc_supported(H, Hkv, HD)) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
-  const int rows = T * H;
-  if (!make_map_bf16_k64(&mq, q, B * rows, HD, HD, BR) ||
-      !make_map_bf16_k64(&mk, kc, max_batch * max_seq, HD, HD, BKV) ||
-      !make_map_bf16_k64(&mv, vc, max_batch * max_seq, HD, HD, BKV))
+  const int G = H / Hkv, rows = T * G;
+  bool ok;
+  if (Hkv == 1) {  // rows (position, head) in order: (128 dims, 1, 1, B*T*H rows)
+    const uint64_t dims[4] = {HD, 1, 1, (uint64_t)B * T * H};
+    const uint64_t strides[3] = {HD * 2, HD * 2, HD * 2};
+    const uint32_t box[4] = {64, 1, 1, BR};
+    ok = make_map_bf16(&mq, q, 4, dims, strides, box);
+  } else {  // (128 dims, G heads, Hkv groups, B*T positions), a box of 128/G positions
+    const uint64_t dims[4] = {HD, (uint64_t)G, (uint64_t)Hkv, (uint64_t)B * T};
+    const uint64_t strides[3] = {HD * 2, (uint64_t)G * HD * 2, (uint64_t)H * HD * 2};
+    const uint32_t box[4] = {64, (uint32_t)G, 1, (uint32_t)(BR / G)};
+    ok = make_map_bf16(&mq, q, 4, dims, strides, box);
+  }
+  if (!ok || !make_map_bf16_k64(&mk, kc, max_batch * max_seq, Hkv * HD, Hkv * HD, BKV) ||
+      !make_map_bf16_k64(&mv, vc, max_batch * max_seq, Hkv * HD, Hkv * HD, BKV))
     return cudaErrorInvalidValue;
   {
     const cudaError_t e = ensure_smem_attr((const void *)attn_prefill_tc_kernel, SMEM_BYTES);
@@ -446,6 +477,8 @@ cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int
   a.H = H;
   a.B = B;
   a.max_seq = max_seq;
+  a.Hkv = Hkv;
+  a.G = G;
   a.rows_per_seq = rows;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   a.y = (bf16 *)y;
@@ -456,7 +489,7 @@ cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   }
-  const int items = ((rows + ITEM - 1) / ITEM) * B;
+  const int items = ((rows + ITEM - 1) / ITEM) * B * Hkv;
   dim3 grid(items < sms ? items : sms);
   count_launch();
   attn_prefill_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(mq, mk, mv, a);

@@ -744,9 +744,13 @@ cudaError_t launch_dec_linear_nb(int src, int epi, const CUtensorMap &map, DecLi
 
 }  // namespace
 
+bool decode_head_supported(const nc_config &c) {
+  return c.dtype == NC_BF16 && c.head_dim == 128 && c.d_model % 128 == 0 && c.mlp_hidden % 128 == 0 &&
+         c.vocab % 128 == 0 && c.d_model / 128 <= 64;
+}
+
 bool decode_fast_supported(const nc_config &c, int B) {
-  return c.dtype == NC_BF16 && c.head_dim == 128 && c.n_kv_head == 1 && c.n_head <= 16 && B >= 1 && B <= 32 &&
-         c.d_model % 128 == 0 && c.mlp_hidden % 128 == 0 && c.vocab % 128 == 0 && c.d_model / 128 <= 64;
+  return decode_head_supported(c) && c.n_kv_head == 1 && c.n_head <= 16 && B >= 1 && B <= 32;
 }
 
 // Scratch sizes for a cache of max_batch sequences (see DecodeScratch).
@@ -754,7 +758,7 @@ size_t decode_part_floats(const nc_config &c, int max_batch, int max_seq, int nu
                           int *attn_chunk) {
   (void)max_batch;
   size_t need = 0;
-  const int N[5] = {(c.n_head + 2) * 128, c.d_model, c.mlp_hidden, c.d_model, c.vocab};
+  const int N[5] = {(c.n_head + 2 * c.n_kv_head) * 128, c.d_model, c.mlp_hidden, c.d_model, c.vocab};
   const int K[5] = {c.d_model, c.n_head * 128, c.d_model, c.mlp_hidden, c.d_model};
   for (int i = 0; i < 5; i++) {
     int splits, kbs;

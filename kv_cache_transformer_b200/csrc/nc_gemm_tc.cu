@@ -117,7 +117,9 @@ __device__ __forceinline__ void transpose_chunk(uint32_t taddr, float *ebuf, int
 
 // EPI_QKV for one 128-column head of the warp's 32 rows (rbase + lane); the
 // head's accumulator columns start at TMEM address tcol, `scale` is the RMS
-// factor of this lane's row. Heads 0..H-1 are q, head H is k, head H+1 is v.
+// factor of this lane's row. Heads 0..H-1 are q, heads H..H+Hkv-1 the keys
+// and H+Hkv..H+2Hkv-1 the values of the Hkv KV heads; KV head j occupies
+// elements [128j, 128j + 128) of a cache row.
 // RoPE pairs element e with element e+64 and rotates by the angle of
 // (e, position); q and k are then RMS normed over their 128 elements. A
 // rotation keeps each pair's sum of squares, so the norm factor is taken from
@@ -126,7 +128,8 @@ __device__ __forceinline__ void transpose_chunk(uint32_t taddr, float *ebuf, int
 __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane, int head, uint32_t tcol, float scale,
                                          float *ebuf) {
   const GemmFuse &f = g.fz;
-  const bool isv = head > f.H;
+  const bool isv = head >= f.H + f.Hkv;
+  const int kvh = head < f.H ? 0 : (isv ? head - f.H - f.Hkv : head - f.H);  // KV head of a k or v head
   float fac = scale;
   if (!isv) {
     float ss = 0.f;
@@ -154,7 +157,7 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
   auto dst_of = [&](int i) -> bf16 * {
     const int row = rbase + 4 * i + rsub;
     return (head < f.H ? reinterpret_cast<bf16 *>(f.q) + ((size_t)row * f.H + head) * 128
-                       : reinterpret_cast<bf16 *>(head == f.H ? f.kc : f.vc) + (size_t)crow[i] * 128) +
+                       : reinterpret_cast<bf16 *>(isv ? f.vc : f.kc) + ((size_t)crow[i] * f.Hkv + kvh) * 128) +
            4 * q;
   };
   if (isv) {
@@ -390,7 +393,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         if constexpr (EPI == EPI_QKV) {
           const int head = nh / 128;  // one head per half
-          if (head < g.fz.H + 2) qkv_head(g, m0 + quarter * 32, lane, head, tbase, scale, ebuf);
+          if (head < g.fz.H + 2 * g.fz.Hkv) qkv_head(g, m0 + quarter * 32, lane, head, tbase, scale, ebuf);
         } else {
           float ss = 0.f;
 #pragma unroll 1
@@ -490,7 +493,7 @@ cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int
                       float cap, uint32_t *status, int num_sms, cudaStream_t s, const GemmFuse *fz) {
   if (!gemm_tc_supported(M, N, K, lda)) return cudaErrorInvalidValue;
   if ((epi == EPI_QKV || epi == EPI_RESID_X) && !fz) return cudaErrorInvalidValue;
-  if (epi == EPI_QKV && N != (fz->H + 2) * 128) return cudaErrorInvalidValue;
+  if (epi == EPI_QKV && N != (fz->H + 2 * fz->Hkv) * 128) return cudaErrorInvalidValue;
   CUtensorMap ma, mw;
   if (!make_map_bf16_k64(&ma, A, M, K, lda, BM) || !make_map_bf16_k64(&mw, W, N, K, K, BN))
     return cudaErrorInvalidValue;

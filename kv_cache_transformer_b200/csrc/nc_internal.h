@@ -57,7 +57,7 @@ struct KvPrefix {
 // of its device workspace.
 struct StepPlan {
   int grid = 0;                      // CTAs, one per SM (0 = no plan)
-  int n_qkv = 0;                     // QKV units of 16 rows (8 RoPE pairs)
+  int n_qkv = 0, r_q = 0;            // QKV units of r_q rows (r_q / 2 RoPE pairs of one head)
   int r_o = 0, r_f = 0, r_p = 0;     // rows per CTA: O projection, MLP fc, MLP projection
   int s_p = 0;                       // K splits of the MLP projection
   int r_h = 0;                       // lm_head rows per CTA
@@ -170,7 +170,7 @@ struct GemmFuse {
   float *ss_out = nullptr;
   const float2 *rope = nullptr;
   void *q = nullptr, *kc = nullptr, *vc = nullptr;
-  int T = 1, H = 0, max_seq = 0;
+  int T = 1, H = 0, Hkv = 1, max_seq = 0;  // query heads, KV heads (the cache row holds Hkv heads)
 };
 
 // ---- generic kernels (any even head_dim; fp32 or bf16 storage) ----
@@ -213,10 +213,10 @@ cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int
                       float cap, uint32_t *status, int num_sms, cudaStream_t s, const GemmFuse *fz = nullptr);
 
 
-// ---- sm_100a causal MQA prefill attention (nc_attn_tc.cu) ----
+// ---- sm_100a causal MQA / GQA prefill attention (nc_attn_tc.cu) ----
 bool attn_prefill_tc_supported(int H, int Hkv, int hd);
-cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int max_batch,
-                              int max_seq, void *y, uint32_t *status, cudaStream_t s);
+cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int Hkv,
+                              int max_batch, int max_seq, void *y, uint32_t *status, cudaStream_t s);
 
 
 // ---- row-wise prefill kernels for bf16 head_dim-128 models (nc_rowops.cu) ----
@@ -228,7 +228,10 @@ cudaError_t k_gather_rows_ss(const float *x, int rows, int d, int stride, int of
                              cudaStream_t s);
 
 // ---- decode step kernels (nc_decode.cu) ----
+// the per-kernel decode launches (one KV head)
 bool decode_fast_supported(const nc_config &c, int B);
+// the decode scratch and the fused last-row lm_head + argmax kernel (any KV heads)
+bool decode_head_supported(const nc_config &c);
 size_t decode_part_floats(const nc_config &c, int max_batch, int max_seq, int num_sms, int *attn_splits,
                           int *attn_chunk);
 cudaError_t k_dec_embed(const int32_t *tokens, const int32_t *positions, int32_t *len, int32_t *pos_ws,

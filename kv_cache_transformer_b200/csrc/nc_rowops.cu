@@ -105,8 +105,8 @@ __global__ void gather_rows_ss_kernel(const float *x, int d, int stride, int off
 }  // namespace
 
 bool rowops_supported(const nc_config &c) {
-  return c.dtype == NC_BF16 && c.head_dim == 128 && c.n_kv_head == 1 && c.d_model % 128 == 0 &&
-         c.d_model / 128 <= 16 && c.n_head <= 16;
+  return c.dtype == NC_BF16 && c.head_dim == 128 && c.d_model % 128 == 0 && c.d_model / 128 <= 16 &&
+         c.n_head <= 16;
 }
 
 cudaError_t k_rows_norm_bf16(const float *x, int rows, int d, float eps, void *h, cudaStream_t s) {

@@ -19,13 +19,16 @@
 //  * linear layers split their output rows over all CTAs and keep the whole
 //    K in each CTA, so no CTA waits for another's partial sums. A phase's
 //    activation rows (bf16, [32][K]) arrive with one bulk tensor copy right
-//    after the barrier; four compute warps split K, multiply with mma.sync
+//    after the barrier; eight compute warps split K, multiply with mma.sync
 //    m16n8k16 (M = the sequences, N = 8 weight rows) out of shared memory and
-//    add their partials in a fixed order. The MLP projection (K = 4d) splits
-//    K four ways instead; the last of the four CTAs of a row block to arrive
-//    adds the partials in split order;
-//  * attention splits each sequence's keys over 4-8 CTAs (flash decoding
-//    with mma.sync, rows = query heads); the last split to arrive merges the
+//    add their partials in a fixed order. A normed input's 1/rms per row is
+//    computed from the staged bf16 rows themselves. The MLP projection
+//    (K = 4d) splits K four ways instead; the last of the four CTAs of a row
+//    block to arrive adds the partials in split order;
+//  * attention runs per (sequence, KV head): the G = H/Hkv query heads of a
+//    KV head are the rows of its MMAs (flash decoding with mma.sync); each
+//    pair's keys are split over up to 8 CTAs, or CTAs take several pairs when
+//    there are more pairs than CTAs; the last split to arrive merges the
 //    softmax states in split order.
 // Every reduction has a fixed order, so results do not depend on timing.
 //
@@ -38,14 +41,14 @@
 // full K cost nothing extra.
 //
 // Phases: EMBED | depth x [QKV | ATTN | OPROJ | FC | PROJ] | HEAD | MERGE.
-//   EMBED  validate positions, x0 = rmsnorm(wte[token]), bf16(x0), sum of squares
+//   EMBED  validate positions, x0 = rmsnorm(wte[token]), bf16(x0)
 //   QKV    (bf16(x0) . [Wq;Wk;Wv]^T) / rms(x0); RoPE on q and k (fp32 out);
 //          v appended to the cache
-//   ATTN   QK norm of q and of the new key (appended to the cache), flash
+//   ATTN   QK norm of q and of the new keys (appended to the cache), flash
 //          decoding over the cache, merge of the key splits -> y
-//   OPROJ  x1 = x0 + y . Wo^T, bf16(x1), sums of squares of x1
+//   OPROJ  x1 = x0 + y . Wo^T, bf16(x1)
 //   FC     f = relu((bf16(x1) . Wfc^T) / rms(x1))^2
-//   PROJ   x0 = x1 + f . Wproj^T (four K splits), bf16(x0), sums of squares
+//   PROJ   x0 = x1 + f . Wproj^T (four K splits), bf16(x0)
 //   HEAD   logits = cap * tanh((bf16(x0) . Wlm^T) / rms(x0) / cap) (+ noise),
 //          per-CTA argmax winners
 //   MERGE  next token per sequence, lengths advanced
@@ -69,7 +72,9 @@ constexpr int MAX_R = 64;               // weight rows per CTA in the K-split li
 constexpr int HG = 64;                  // lm_head rows per pass (16 per warp of each warp group)
 constexpr int SMEM_CAP = 227 * 1024;
 constexpr int MISC = 2048;              // barriers and per-sequence tables
-constexpr int CTR_BYTES = 2048;         // counters zeroed before each launch
+constexpr int CTR_BYTES = 4096;         // counters zeroed before each launch
+constexpr int MAX_HKV = 16;             // KV heads (attention arrival counters per sequence)
+static_assert(64 + 4 * 32 * MAX_HKV + 4 * 256 <= CTR_BYTES, "counter region: barrier, attention, projection");
 constexpr int AROW = 132;               // floats per attention state row: m, l, O[128], padding
 // attention scratch: the warps' softmax states, q and the new key in bf16,
 // per-row merge factors
@@ -79,13 +84,14 @@ enum Phase { P_EMBED = 0, P_QKV, P_ATTN, P_OPROJ, P_FC, P_PROJ, P_HEAD, P_MERGE 
 
 struct StepArgs {
   int L, d, H, F, V, B, max_batch, max_seq, grid;
-  int r_o, r_f, r_p, s_p, r_h, n_o, n_f, n_p, n_h, n_qkv;
+  int Hkv, G;                 // KV heads, query heads per KV head (G = H / Hkv <= 16)
+  int r_q, r_o, r_f, r_p, s_p, r_h, n_o, n_f, n_p, n_h, n_qkv;
   int slots, splits;
   float eps, cap, scale_log2;
   const bf16 *wte;
-  const CUtensorMap *wmaps;   // [4L + 1]: per layer qkv (8-row box), o, fc, proj; then lm_head
-  const CUtensorMap *kvmaps;  // [4]: K and V caches as [L * max_batch * max_seq][128], then the same
-                              // views of the prefix cache (shared rows, nc_kv_fork_shared)
+  const CUtensorMap *wmaps;   // [4L + 1]: per layer qkv (r_q/2-row box), o, fc, proj; then lm_head
+  const CUtensorMap *kvmaps;  // [4]: K and V caches as [L * max_batch * max_seq][Hkv][128], then the
+                              // same views of the prefix cache (shared rows, nc_kv_fork_shared)
   const CUtensorMap *amaps;   // [4]: xb0, y, xb1, f as [32][K] (32-row boxes)
   const int32_t *pre_seq, *pre_len;  // [max_batch]: shared rows of each sequence (0: none)
   int pmax_batch, pmax_seq;   // shape of the prefix cache
@@ -93,18 +99,18 @@ struct StepArgs {
   int32_t *len;
   float *x0, *x1;             // [32][d] fp32 residual: layer input, after attention
   bf16 *xb0, *xb1, *y, *f;    // [32][d], [32][d], [32][d], [32][F]
-  float *qk;                  // [32][H + 1][128]: q heads and k after RoPE, before QK norm
-  bf16 *kc, *vc;              // [L][max_batch][max_seq][128]
+  float *qk;                  // [32][H + Hkv][128]: q heads and k heads after RoPE, before QK norm
+  bf16 *kc, *vc;              // [L][max_batch][max_seq][Hkv][128]
   const float2 *rope;         // [max_seq][64]
   float *logits;              // [B][V]
   const float *noise;         // [B][V] or null
   int32_t *next;              // [B] or null
   float *cand_v;              // [grid][32]
   int *cand_i;
-  float *apart;               // [32][MAX_SPLIT][16][AROW]: attention softmax states (m, l, O)
+  float *apart;               // [32 * Hkv][MAX_SPLIT][G][AROW]: attention softmax states (m, l, O)
   float *ppart;               // [n_p][s_p][32][r_p]: MLP projection partial sums
   unsigned long long *bar;    // grid barrier counter
-  unsigned *acnt;             // [32] attention arrivals, cumulative over layers
+  unsigned *acnt;             // [32 * Hkv] attention arrivals, cumulative over layers
   unsigned *pcnt;             // [n_p] projection arrivals, cumulative over layers
   uint32_t *status;
   unsigned long long *trace;  // [grid][phases][8] phase timestamps (ns), or null
@@ -178,8 +184,9 @@ __device__ __forceinline__ void phase_of(const StepArgs &a, int p, int &type, in
 }
 
 // This CTA's share of a linear phase: weight rows [r0, r0 + R) (QKV: rows
-// r0 .. r0+7 and r0+64 .. r0+71 of one head), k-blocks [kb0, kb0 + nkb) of
-// 64 columns, the weight map and the activation map it stages.
+// r0 .. r0+R/2-1 and their RoPE partners 64 rows on, of one head), k-blocks
+// [kb0, kb0 + nkb) of 64 columns, the weight map and the activation map it
+// stages.
 struct Unit {
   bool active;
   int u, split;   // unit index, K split (MLP projection)
@@ -196,11 +203,12 @@ __device__ __forceinline__ Unit unit_of(const StepArgs &a, int type, int layer, 
   u.kb0 = 0;
   u.sbox = a.d / 64;
   if (type == P_QKV) {
-    u.N = (a.H + 2) * 128;
-    u.R = 16;
+    u.N = (a.H + 2 * a.Hkv) * 128;
+    u.R = a.r_q;
     u.u = c;
     u.active = c < a.n_qkv;
-    u.r0 = (c >> 3) * 128 + (c & 7) * 8;
+    const int uph = 128 / a.r_q;  // units per head
+    u.r0 = (c / uph) * 128 + (c % uph) * (a.r_q / 2);
     u.nkb = a.d / 64;
     u.map = a.wmaps + 4 * layer;
     u.amap = a.amaps + 0;
@@ -364,26 +372,28 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
     phase_of(a, p, type, layer);
     bool first = true;
     if (type == P_ATTN) {
-      if (c >= a.B * a.splits) continue;
-      const int b = c / a.splits, sp = c % a.splits;
-      if (!s.valid[b]) continue;
-      int k0, k1;
-      key_range(s.pos[b] + 1, sp, a.splits, k0, k1);
-      const int row0 = (layer * a.max_batch + b) * a.max_seq;
-      // tiles below the shared length (a multiple of 64) come from the prefix cache
-      const int plen = a.pre_len[b];
-      const int prow0 = (layer * a.pmax_batch + a.pre_seq[b]) * a.pmax_seq;
-      for (int key = k0; key < k1; key += KT)
-        for (int which = 0; which < 2; which++) {
-          uint32_t slot;
-          if (!take(slot, SLOT)) return;
-          if (first) trace_mark(a, p, 5);
-          first = false;
-          const bool sh = key < plen;
-          tma_load_3d(ring + slot * SLOT, a.kvmaps + (sh ? 2 : 0) + which, 0, (sh ? prow0 : row0) + key, 0,
-                      &s.full[slot]);
-        }
-      trace_mark(a, p, 6);
+      // this CTA's units (sequence, KV head, split), in the consumers' order
+      for (int un = c; un < a.B * a.Hkv * a.splits; un += a.grid) {
+        const int b = un / (a.Hkv * a.splits), j = (un / a.splits) % a.Hkv, sp = un % a.splits;
+        if (!s.valid[b]) continue;
+        int k0, k1;
+        key_range(s.pos[b] + 1, sp, a.splits, k0, k1);
+        const int row0 = (layer * a.max_batch + b) * a.max_seq;
+        // tiles below the shared length (a multiple of 64) come from the prefix cache
+        const int plen = a.pre_len[b];
+        const int prow0 = (layer * a.pmax_batch + a.pre_seq[b]) * a.pmax_seq;
+        for (int key = k0; key < k1; key += KT)
+          for (int which = 0; which < 2; which++) {
+            uint32_t slot;
+            if (!take(slot, SLOT)) return;
+            if (first) trace_mark(a, p, 5);
+            first = false;
+            const bool sh = key < plen;
+            tma_load_4d(ring + slot * SLOT, a.kvmaps + (sh ? 2 : 0) + which, 0, (sh ? prow0 : row0) + key, 0, j,
+                        &s.full[slot]);
+          }
+      }
+      if (!first) trace_mark(a, p, 6);
     } else if (type == P_QKV || type == P_OPROJ || type == P_FC || type == P_PROJ || type == P_HEAD) {
       const Unit u = unit_of(a, type, layer, c);
       if (!u.active) continue;
@@ -560,35 +570,33 @@ __device__ float *reduce_warps(float *red, int R, int MT, int e) {
 // of parity g, each warp 16 keys of a tile. The eight warps' softmax states
 // are merged (per-row factors first), the split's state goes to apart, and
 // the last split to arrive merges all splits in split order into y.
-__device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
-                                uint32_t &t, uint32_t &xph, int p) {
-  const int c = blockIdx.x;
-  if (c >= a.B * a.splits) return true;
-  const int b = c / a.splits, sp = c % a.splits;
-  if (!s.valid[b]) return true;
+__device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
+                               uint32_t &t, uint32_t &xph, int p, int b, int j, int sp) {
   const int warp = e >> 5, lane = e & 31, g = lane >> 2, t4 = lane & 3;
   const int grp = warp >> 2, wq = warp & 3;
-  const size_t lay = (size_t)layer * a.max_batch * a.max_seq * 128;
+  const int G = a.G, vs = b * a.Hkv + j;  // query heads j*G .. j*G+G-1 read KV head j
+  const size_t lay = (size_t)layer * a.max_batch * a.max_seq * a.Hkv * 128;
+  const size_t crow = ((size_t)b * a.max_seq + s.pos[b]) * a.Hkv + j;  // cache row of the new key / value
   const int pos = s.pos[b], n_keys = pos + 1;
   int k0, k1;
   key_range(n_keys, sp, a.splits, k0, k1);
   float *cw = reinterpret_cast<float *>(xs);                                 // [8 warps][16 rows][AROW]
   bf16 *qs = reinterpret_cast<bf16 *>(xs + NCW * 16 * AROW * 4);             // [17][128]: q heads, the new key
   float *fac = reinterpret_cast<float *>(xs + NCW * 16 * AROW * 4 + 17 * 128 * 2);  // [NCW + 2][16]
-  // QK norm of the H query heads and of the new key, in fp32, to bf16 (the
+  // QK norm of the G query heads and of the new key, in fp32, to bf16 (the
   // warp's heads w, w+8, w+16 are loaded before any is used)
   {
     float4 qv[3];
 #pragma unroll
     for (int i = 0; i < 3; i++) {
-      const int h = warp + NCW * i;
-      qv[i] = h <= a.H ? __ldcg(reinterpret_cast<const float4 *>(a.qk + ((size_t)b * (a.H + 1) + h) * 128) + lane)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int h = warp + NCW * i, src = h < G ? j * G + h : a.H + j;
+      qv[i] = h <= G ? __ldcg(reinterpret_cast<const float4 *>(a.qk + ((size_t)b * (a.H + a.Hkv) + src) * 128) + lane)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int i = 0; i < 3; i++) {
       const int h = warp + NCW * i;
-      if (h > a.H) break;
+      if (h > G) break;
       const float4 v = qv[i];
       const float r = rsqrtf(warp_sum(v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w) * (1.0f / 128) + a.eps);
       *reinterpret_cast<uint2 *>(qs + h * 128 + 4 * lane) =
@@ -596,18 +604,17 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
     }
   }
   csync();
-  const bf16 *knew = qs + a.H * 128;
+  const bf16 *knew = qs + G * 128;
   if (pos >= k0 && pos < k1 && e < 16)  // this split holds the new key: append it to the cache
-    *reinterpret_cast<uint4 *>(a.kc + lay + ((size_t)b * a.max_seq + pos) * 128 + e * 8) =
-        *reinterpret_cast<const uint4 *>(knew + e * 8);
+    *reinterpret_cast<uint4 *>(a.kc + lay + crow * 128 + e * 8) = *reinterpret_cast<const uint4 *>(knew + e * 8);
   uint32_t qa[8][4];
 #pragma unroll
   for (int ks = 0; ks < 8; ks++) {
     const int c0 = ks * 16 + t4 * 2;
-    qa[ks][0] = g < a.H ? *reinterpret_cast<const uint32_t *>(qs + g * 128 + c0) : 0u;
-    qa[ks][1] = g + 8 < a.H ? *reinterpret_cast<const uint32_t *>(qs + (g + 8) * 128 + c0) : 0u;
-    qa[ks][2] = g < a.H ? *reinterpret_cast<const uint32_t *>(qs + g * 128 + c0 + 8) : 0u;
-    qa[ks][3] = g + 8 < a.H ? *reinterpret_cast<const uint32_t *>(qs + (g + 8) * 128 + c0 + 8) : 0u;
+    qa[ks][0] = g < G ? *reinterpret_cast<const uint32_t *>(qs + g * 128 + c0) : 0u;
+    qa[ks][1] = g + 8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g + 8) * 128 + c0) : 0u;
+    qa[ks][2] = g < G ? *reinterpret_cast<const uint32_t *>(qs + g * 128 + c0 + 8) : 0u;
+    qa[ks][3] = g + 8 < G ? *reinterpret_cast<const uint32_t *>(qs + (g + 8) * 128 + c0 + 8) : 0u;
   }
   float o[16][4];
 #pragma unroll
@@ -631,7 +638,7 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
       if (e < 32) {
         const int cc = e & 15;
         const uint4 v = e < 16 ? *reinterpret_cast<const uint4 *>(knew + cc * 8)
-                               : __ldcg(reinterpret_cast<const uint4 *>(a.vc + lay + ((size_t)b * a.max_seq + pos) * 128 + cc * 8));
+                               : __ldcg(reinterpret_cast<const uint4 *>(a.vc + lay + crow * 128 + cc * 8));
         *reinterpret_cast<uint4 *>((e < 16 ? K : V) + kv_tile_off(pr, cc)) = v;
       }
       csync();
@@ -724,8 +731,8 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
   }
   csync();
   // the eight warps' states merged: per-row factors, then the rows, to apart[b][sp]
-  float *dst = a.apart + ((size_t)b * MAX_SPLIT + sp) * 16 * AROW;
-  if (e < a.H) {
+  float *dst = a.apart + ((size_t)vs * MAX_SPLIT + sp) * G * AROW;
+  if (e < G) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < NCW; w++) M = fmaxf(M, cw[(w * 16 + e) * AROW]);
@@ -741,7 +748,7 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
     dst[e * AROW + 1] = Ls;
   }
   csync();
-  for (int idx = e; idx < a.H * 128; idx += 32 * NCW) {
+  for (int idx = e; idx < G * 128; idx += 32 * NCW) {
     const int row = idx >> 7, col = idx & 127;
     float O = 0.f;
 #pragma unroll
@@ -751,66 +758,77 @@ __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring,
   csync();
   if (e == 0) {
     unsigned old;
-    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.acnt + b) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.acnt + vs) : "memory");
     *s.flag = old == (unsigned)((layer + 1) * a.splits - 1) ? 1 : 0;
   }
   csync();
   if (*s.flag) {  // the last split: merge all splits in split order
-    // every split's H state rows in one bulk copy each, over the warp states
+    // every split's G state rows in one bulk copy each, over the warp states
     // (free now: this split's state is in apart)
-    float *st = cw;  // [splits][H][AROW]
-    const uint32_t rows_bytes = (uint32_t)(a.H * AROW * 4);
+    float *st = cw;  // [splits][G][AROW]
+    const uint32_t rows_bytes = (uint32_t)(G * AROW * 4);
     if (e == 0) {
       asm volatile("fence.proxy.async.global;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive_expect_tx(s.x_bar, rows_bytes * a.splits);
       for (int q = 0; q < a.splits; q++)
-        bulk_copy(st + q * a.H * AROW, a.apart + ((size_t)b * MAX_SPLIT + q) * 16 * AROW, rows_bytes, s.x_bar);
+        bulk_copy(st + q * G * AROW, a.apart + ((size_t)vs * MAX_SPLIT + q) * G * AROW, rows_bytes, s.x_bar);
     }
     mbar_wait(s.x_bar, xph & 1, s.abort_flag, a.status);
     xph++;
-    if (e < a.H) {
+    if (e < G) {
       float M = -INFINITY;
-      for (int q = 0; q < a.splits; q++) M = fmaxf(M, st[(q * a.H + e) * AROW]);
+      for (int q = 0; q < a.splits; q++) M = fmaxf(M, st[(q * G + e) * AROW]);
       float Ls = 0.f;
       for (int q = 0; q < a.splits; q++) {
-        const float mq = st[(q * a.H + e) * AROW];
+        const float mq = st[(q * G + e) * AROW];
         const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
         fac[q * 16 + e] = f;
-        Ls += f * st[(q * a.H + e) * AROW + 1];
+        Ls += f * st[(q * G + e) * AROW + 1];
       }
       fac[NCW * 16 + e] = Ls > 0.f ? 1.f / Ls : 0.f;
     }
     csync();
-    for (int idx = e; idx < a.H * 128; idx += 32 * NCW) {
+    for (int idx = e; idx < G * 128; idx += 32 * NCW) {
       const int row = idx >> 7, col = idx & 127;
       float O = 0.f;
-      for (int q = 0; q < a.splits; q++) O += fac[q * 16 + row] * st[(q * a.H + row) * AROW + 2 + col];
-      a.y[(size_t)b * a.d + row * 128 + col] = __float2bfloat16_rn(O * fac[NCW * 16 + row]);
+      for (int q = 0; q < a.splits; q++) O += fac[q * 16 + row] * st[(q * G + row) * AROW + 2 + col];
+      a.y[(size_t)b * a.d + (j * G + row) * 128 + col] = __float2bfloat16_rn(O * fac[NCW * 16 + row]);
     }
   }
   csync();  // s.flag and the scratch are rewritten by the next use
+}
+
+// This CTA's attention units (sequence, KV head, split), in the producer's order.
+__device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
+                                uint32_t &t, uint32_t &xph, int p) {
+  for (int un = blockIdx.x; un < a.B * a.Hkv * a.splits; un += a.grid) {
+    const int b = un / (a.Hkv * a.splits), j = (un / a.splits) % a.Hkv, sp = un % a.splits;
+    if (!s.valid[b]) continue;
+    attention_unit(a, s, ring, xs, layer, e, t, xph, p, b, j, sp);
+  }
   if (e == 0) trace_mark(a, p, 3);
   return true;
 }
 
 // ------------------------------------------------------------- epilogues
-// QKV: rows i (< 8) and 8 + i of the unit are head rows j0 + i and j0 + 64 + i
-// (a RoPE pair). q and k heads: scale by 1/rms(x0), rotate, to qk (fp32);
-// the v head: scale, bf16, appended to the value cache.
+// QKV: rows i and hq + i of the unit (hq = R / 2) are head rows j0 + i and
+// j0 + 64 + i (a RoPE pair). q and k heads: scale by 1/rms(x0), rotate, to
+// qk (fp32); a v head: scale, bf16, appended to its KV head's slot of the
+// value cache.
 __device__ void qkv_epilogue(const StepArgs &a, const Smem &s, const float *sum, const Unit &u, int layer, int e) {
-  const int head = u.r0 >> 7, j0 = u.r0 & 127;
-  const size_t lay = (size_t)layer * a.max_batch * a.max_seq * 128;
-  for (int idx = e; idx < a.B * 8; idx += 32 * NCW) {
-    const int b = idx >> 3, i = idx & 7;
-    const float lo = sum[b * 16 + i] * s.inv[b], hi = sum[b * 16 + 8 + i] * s.inv[b];
-    if (head <= a.H) {
+  const int head = u.r0 >> 7, j0 = u.r0 & 127, hq = u.R / 2;
+  const size_t lay = (size_t)layer * a.max_batch * a.max_seq * a.Hkv * 128;
+  for (int idx = e; idx < a.B * hq; idx += 32 * NCW) {
+    const int b = idx / hq, i = idx % hq;
+    const float lo = sum[b * u.R + i] * s.inv[b], hi = sum[b * u.R + hq + i] * s.inv[b];
+    if (head < a.H + a.Hkv) {
       const float2 cs = a.rope[(size_t)s.pos[b] * 64 + j0 + i];
-      float *dst = a.qk + ((size_t)b * (a.H + 1) + head) * 128;
+      float *dst = a.qk + ((size_t)b * (a.H + a.Hkv) + head) * 128;
       dst[j0 + i] = lo * cs.x - hi * cs.y;
       dst[j0 + 64 + i] = hi * cs.x + lo * cs.y;
     } else if (s.valid[b]) {
-      bf16 *dst = a.vc + lay + ((size_t)b * a.max_seq + s.pos[b]) * 128;
+      bf16 *dst = a.vc + lay + (((size_t)b * a.max_seq + s.pos[b]) * a.Hkv + (head - a.H - a.Hkv)) * 128;
       dst[j0 + i] = __float2bfloat16_rn(lo);
       dst[j0 + 64 + i] = __float2bfloat16_rn(hi);
     }
@@ -1202,14 +1220,16 @@ bool make_map_bf16(CUtensorMap *map, const void *ptr, int rank, const uint64_t *
 
 bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *pl) {
   *pl = StepPlan{};
-  if (!decode_fast_supported(c, 1) || c.n_head > 16 || c.d_model % 64 || c.mlp_hidden % 64 || c.vocab % 8 ||
-      num_sms < 8)
-    return false;
-  const int d = c.d_model, F = c.mlp_hidden, V = c.vocab, H = c.n_head;
+  if (!decode_step_supported(c, 1) || num_sms < 8) return false;
+  const int d = c.d_model, F = c.mlp_hidden, V = c.vocab, H = c.n_head, Hkv = c.n_kv_head, Gq = H / Hkv;
   const int G = num_sms;
   StepPlan p;
   p.grid = G;
-  p.n_qkv = (H + 2) * 8;
+  // QKV units: 8, 16 or 32 RoPE pairs of one head, the smallest that fits the grid
+  for (p.r_q = 16; p.r_q <= 64 && (H + 2 * Hkv) * (128 / p.r_q) > G; p.r_q *= 2) {
+  }
+  if (p.r_q > 64) return false;
+  p.n_qkv = (H + 2 * Hkv) * (128 / p.r_q);
   p.r_o = round8((d + G - 1) / G);
   p.r_f = round8((F + G - 1) / G);
   p.s_p = (F + d - 1) / d;  // K splits of the MLP projection: K per split <= d
@@ -1223,8 +1243,8 @@ bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *pl) {
   if (p.n_qkv > G || p.r_o > MAX_R || p.r_f > MAX_R || p.r_p > MAX_R || p.n_p * p.s_p > G || p.n_p > 256 ||
       p.n_o > G || p.n_f > G || p.n_h > G || p.s_p > NCW)
     return false;
-  // the attention merge stages every split's H state rows in the activation region
-  if (MAX_SPLIT * H * AROW * 4 > xreg_bytes(d)) return false;
+  // the attention merge stages every split's G state rows in the activation region
+  if (MAX_SPLIT * Gq * AROW * 4 > xreg_bytes(d)) return false;
   // the projection's K per split must fit the staged rows like the others
   const int kbt = F / 64, kbs = (kbt + p.s_p - 1) / p.s_p;
   if (kbs * 64 > d) return false;
@@ -1248,16 +1268,22 @@ bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *pl) {
   p.off_xb1 = take(2 * MAXB * d);
   p.off_y = take(2 * MAXB * d);
   p.off_f = take(2 * MAXB * (size_t)F);
-  p.off_qk = take(sizeof(float) * MAXB * (H + 1) * 128);
+  p.off_qk = take(sizeof(float) * MAXB * (H + Hkv) * 128);
   p.off_cv = take(sizeof(float) * (size_t)G * 32);
   p.off_ci = take(sizeof(int) * (size_t)G * 32);
-  p.off_ap = take(sizeof(float) * MAXB * MAX_SPLIT * 16 * AROW);
+  p.off_ap = take(sizeof(float) * MAXB * Hkv * MAX_SPLIT * Gq * AROW);
   p.off_pp = take(sizeof(float) * (size_t)p.n_p * p.s_p * MAXB * p.r_p);
   *pl = p;
   return true;
 }
 
-bool decode_step_supported(const nc_config &c, int B) { return decode_fast_supported(c, B) && B <= MAXB; }
+// bf16, head_dim 128, G = H / Hkv <= 16 query heads per KV head (the rows of
+// one attention unit's MMAs), H * 128 = d, at most 32 sequences
+bool decode_step_supported(const nc_config &c, int B) {
+  return decode_head_supported(c) && c.n_head % c.n_kv_head == 0 && c.n_head / c.n_kv_head <= 16 &&
+         c.n_kv_head <= MAX_HKV && c.n_head * 128 == c.d_model && c.mlp_hidden % 64 == 0 && c.vocab % 8 == 0 &&
+         B >= 1 && B <= MAXB;
+}
 
 int decode_step_maps_count(const nc_config &c) { return 4 * c.depth + 1 + 4 + 4; }
 
@@ -1273,28 +1299,28 @@ bool weight_map(CUtensorMap *m, const void *w, int rows, int K, int box_rows, in
   return make_map_bf16(m, w, 3, dims, strides, box);
 }
 
-// the K or V cache, [rows][128] bf16, as (64 dims, rows, 2 halves): a box of
-// (64, 64 keys, 2) lands as [half][key][128 B]
-bool cache_map(CUtensorMap *m, const void *cache, int rows) {
-  const uint64_t dims[3] = {64, (uint64_t)rows, 2};
-  const uint64_t strides[2] = {256, 128};
-  const uint32_t box[3] = {64, (uint32_t)KT, 2};
-  return make_map_bf16(m, cache, 3, dims, strides, box);
+// the K or V cache, [rows][Hkv][128] bf16, as (64 dims, rows, 2 halves, Hkv
+// heads): a box of (64, 64 keys, 2, 1) lands as [half][key][128 B]
+bool cache_map(CUtensorMap *m, const void *cache, int rows, int Hkv) {
+  const uint64_t dims[4] = {64, (uint64_t)rows, 2, (uint64_t)Hkv};
+  const uint64_t strides[3] = {(uint64_t)Hkv * 256, 128, 256};
+  const uint32_t box[4] = {64, (uint32_t)KT, 2, 1};
+  return make_map_bf16(m, cache, 4, dims, strides, box);
 }
 }  // namespace
 
 // The two maps through which the step kernel reads shared-prefix rows: the
-// prefix cache's K and V viewed as [depth * max_batch * max_seq, 128].
+// prefix cache's K and V viewed as [depth * max_batch * max_seq, Hkv, 128].
 bool decode_step_prefix_maps(const void *kcache, const void *vcache, const nc_config &c, int max_batch, int max_seq,
                              CUtensorMap *out) {
   const int rows = c.depth * max_batch * max_seq;
-  return cache_map(&out[0], kcache, rows) && cache_map(&out[1], vcache, rows);
+  return cache_map(&out[0], kcache, rows, c.n_kv_head) && cache_map(&out[1], vcache, rows, c.n_kv_head);
 }
 
 // Tensor maps of the step kernel, written to host memory `out` (to be copied
 // to the device): per layer the QKV weights as (64 columns, rows, 2 RoPE
-// halves 64 rows apart, k-blocks) so that a unit's 8 + 8 paired rows arrive
-// in one copy, then the O, fc, proj weights (boxes of the unit's rows and a
+// halves 64 rows apart, k-blocks) so that a unit's r_q/2 + r_q/2 paired rows
+// arrive in one copy, then the O, fc, proj weights (boxes of the unit's rows and a
 // slot's k-blocks), the lm_head (64 rows x 2 k-blocks); the K and V caches
 // (this cache, then the prefix cache, initially this one); the activations
 // the linear phases stage (bf16(x0), y, bf16(x1), f) as (64 columns, 32 rows,
@@ -1302,13 +1328,13 @@ bool decode_step_prefix_maps(const void *kcache, const void *vcache, const nc_co
 bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *vcache, int max_batch, int max_seq,
                             const StepPlan &p, void *ws, CUtensorMap *out) {
   const nc_config &c = m->cfg;
-  const int d = c.d_model, F = c.mlp_hidden, H = c.n_head;
+  const int d = c.d_model, F = c.mlp_hidden, H = c.n_head, Hkv = c.n_kv_head;
   for (int l = 0; l < c.depth; l++) {
     const nc_layer_w &w = m->layers[l];
     {
-      const uint64_t dims[4] = {64, (uint64_t)((H + 2) * 128 - 64), 2, (uint64_t)(d / 64)};
+      const uint64_t dims[4] = {64, (uint64_t)((H + 2 * Hkv) * 128 - 64), 2, (uint64_t)(d / 64)};
       const uint64_t strides[3] = {(uint64_t)d * 2, (uint64_t)64 * d * 2, 128};
-      const uint32_t box[4] = {64, 8, 2, (uint32_t)kps_of(16)};
+      const uint32_t box[4] = {64, (uint32_t)(p.r_q / 2), 2, (uint32_t)kps_of(p.r_q)};
       if (!make_map_bf16(&out[4 * l + 0], w.wqkv, 4, dims, strides, box)) return false;
     }
     if (!weight_map(&out[4 * l + 1], w.wo, d, H * 128, p.r_o, kps_of(p.r_o))) return false;
@@ -1317,7 +1343,8 @@ bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *v
   }
   if (!weight_map(&out[4 * c.depth], m->wlm, c.vocab, d, HG, 2)) return false;
   const int rows = c.depth * max_batch * max_seq;
-  if (!cache_map(&out[4 * c.depth + 1], kcache, rows) || !cache_map(&out[4 * c.depth + 2], vcache, rows)) return false;
+  if (!cache_map(&out[4 * c.depth + 1], kcache, rows, Hkv) || !cache_map(&out[4 * c.depth + 2], vcache, rows, Hkv))
+    return false;
   // no shared prefixes yet: the prefix maps view this cache
   out[4 * c.depth + 3] = out[4 * c.depth + 1];
   out[4 * c.depth + 4] = out[4 * c.depth + 2];
@@ -1363,6 +1390,9 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
   a.L = c.depth;
   a.d = c.d_model;
   a.H = c.n_head;
+  a.Hkv = c.n_kv_head;
+  a.G = c.n_head / c.n_kv_head;
+  a.r_q = pl.r_q;
   a.F = c.mlp_hidden;
   a.V = c.vocab;
   a.B = B;
@@ -1381,7 +1411,9 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
   a.n_qkv = pl.n_qkv;
   a.slots = pl.slots;
   {
-    int sp = pl.grid / B;
+    // key splits per (sequence, KV head): as many as the grid holds in one
+    // round; with more pairs than CTAs, one split and CTAs taking several pairs
+    int sp = pl.grid / (B * c.n_kv_head);
     if (sp > MAX_SPLIT) sp = MAX_SPLIT;
     if (sp < 1) sp = 1;
     a.splits = sp;
@@ -1419,7 +1451,7 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
   a.ppart = reinterpret_cast<float *>(base + pl.off_pp);
   a.bar = reinterpret_cast<unsigned long long *>(base + pl.off_ctr);
   a.acnt = reinterpret_cast<unsigned *>(base + pl.off_ctr + 64);
-  a.pcnt = reinterpret_cast<unsigned *>(base + pl.off_ctr + 64 + 4 * MAXB);
+  a.pcnt = reinterpret_cast<unsigned *>(base + pl.off_ctr + 64 + 4 * MAXB * MAX_HKV);
   a.status = m->status;
   a.trace = trace;
   a.valid_out = valid_out;

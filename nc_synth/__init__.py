@@ -104,6 +104,8 @@ TINY = ModelConfig(depth=2, d_model=128, n_head=2, n_kv_head=1, head_dim=64, mlp
 D20 = depth_config(20)
 D26 = depth_config(26)
 D30 = depth_config(30)
+# d20 with one KV head per query head (multi-head attention): the 560M count
+D20_MHA = depth_config(20, n_kv_head=10)
 
 
 @dataclasses.dataclass(frozen=True)
