@@ -374,6 +374,7 @@ def run_ours(args):
                                                                  shared=True)
         workloads["d20_extend"] = extend_workload(args, world, local, peaks, peaks_src)
         workloads["sample_topk"] = sample_kernel_us(args)
+        workloads["d20_mha"] = mha_workload(args, world, local, peaks, peaks_src)
 
     # ---------------- CPU oracle on a bounded sample (rank 0, N = 1)
     cpu = None
@@ -411,7 +412,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local):
+def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local, traffic="d20", desc=None):
     import torch
     import kv_cache_transformer_b200 as nc
     import nc_synth as syn
@@ -465,15 +466,75 @@ def run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local):
 
     return {
         "value": world * B * S / (t_ms / 1e3), "unit": "tok/s", "ms_per_step": ms_step, "steps": S,
-        "config": {"workload": "d20_decode: 32 sequences prefilled to 2048 Zipf tokens, 128 greedy steps "
-                               "(positions 2048..2175), CUDA-graph replay", "batch": B, "ctx": [T, T + S]},
+        "config": {"workload": desc or ("d20_decode: 32 sequences prefilled to 2048 Zipf tokens, 128 greedy steps "
+                                        "(positions 2048..2175), CUDA-graph replay"), "batch": B, "ctx": [T, T + S]},
         "roofline": {"bound": "hbm", "kernel": "whole decode step (one persistent kernel per step)",
                      "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                     "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "traffic": DECODE_STEP_DRAM_BYTES,
+                     "frac_of_nominal": gbs / NOMINAL_HBM_GBS,
+                     "traffic": DECODE_STEP_DRAM_BYTES if traffic == "d20" else traffic,
                      "bytes_per_step": by["total"], "bytes": by, "peak_source": f"{peaks_src} hbm_gbs"},
         "phase_trace": trace,
         "gpu_launches": int(launches), "clocks": clk,
     }
+
+
+def mha_workload(args, world: int, local: int, peaks, peaks_src) -> dict:
+    """The d20 shapes with multi-head attention (n_kv_head = 10, the 560M
+    model): prefill 8 x 2048 (tensor-core roofline of the GEMMs and of the
+    whole step) and decode at batch 32, context 2048..2175 (HBM roofline;
+    the KV cache is 10x the MQA model's, 6.9 of the 8.1 GB a step reads)."""
+    import torch
+    import kv_cache_transformer_b200 as nc
+    import nc_synth as syn
+    wp, wd = syn.WORKLOADS["d20_mha_prefill"], syn.WORKLOADS["d20_mha_decode"]
+    cfg = wp.model
+    model = nc.Model(cfg, syn.make_blob(cfg, wp.weight_seed))
+    kv = model.kv(max(wp.batch, wd.batch), wd.prompt_len + args.decode_steps)
+    B, T = wp.batch, wp.prompt_len
+    tokens = torch.from_numpy(syn.prompt_tokens(wp)).cuda()
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    nxt = torch.empty((B,), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        model.prefill(kv, tokens, 0, logits, nxt)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    steps = max(1, min(args.steps, 10))
+    barrier(world)
+    model.profile(True)
+    model.profile_read()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        model.prefill(kv, tokens, 0, logits, nxt)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    kms, kn = model.profile_read()
+    model.profile(False)
+    barrier(world)
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    fl = prefill_flops(cfg, B, T)
+    ms_step = t_ms / steps
+    gemm_ms = kms[nc.NC_K_GEMM] / steps
+    attn_ms = kms[nc.NC_K_ATTN] / steps
+    peak = peaks["bf16_tflops"]
+    prefill = {
+        "value": replica_throughput(steps * B * T, t_ms, world), "unit": "tok/s", "ms_per_step": ms_step,
+        "steps": steps, "config": {"workload": "d20_mha_prefill: 8 x 2048 Zipf(1.1) tokens, d20 MHA bf16",
+                                   "batch": B, "seq_len": T},
+        "gemm_tflops": fl["gemm"] / (gemm_ms / 1e3) / 1e12,
+        "gemm_frac": fl["gemm"] / (gemm_ms / 1e3) / 1e12 / peak,
+        "attn_tflops": fl["attn"] / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else None,
+        "step_tflops": fl["total"] / (ms_step / 1e3) / 1e12,
+        "step_frac_of_peak": fl["total"] / (ms_step / 1e3) / 1e12 / peak,
+        "peak_source": f"{peaks_src} bf16_tflops (burst)",
+    }
+    decode = run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local, traffic=None,
+                        desc="d20_mha_decode: d20 MHA, 32 sequences prefilled to 2048 Zipf tokens, greedy steps "
+                             "from position 2048, CUDA-graph replay")
+    kv.close()
+    model.close()
+    return {"prefill": prefill, "decode": decode}
 
 
 def decode_phase_trace(kv, step, depth: int):
@@ -711,14 +772,19 @@ def sample_kernel_us(args) -> dict:
 
 
 def run_decode_workload(args):
-    """One JSON line for --workload d26_latency | d30_rollout."""
+    """One JSON line for --workload d26_latency | d30_rollout | d20_mha | sample_topk."""
     import torch
     from kv_cache_transformer_b200 import build as ncbuild
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
     ncbuild.build()
     peaks, peaks_src = load_peaks()
-    line = decode_workload(args.workload, args, 1, local, peaks, peaks_src)
+    if args.workload == "d20_mha":
+        line = mha_workload(args, 1, local, peaks, peaks_src)
+    elif args.workload == "sample_topk":
+        line = sample_kernel_us(args)
+    else:
+        line = decode_workload(args.workload, args, 1, local, peaks, peaks_src)
     line["warmup"] = args.warmup
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -734,9 +800,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only", choices=("all", "decode"), default="all",
                     help="decode: skip the prefill timing (for profiling the decode kernels)")
-    ap.add_argument("--workload", choices=("d20", "d26_latency", "d30_rollout"), default="d20",
+    ap.add_argument("--workload", choices=("d20", "d26_latency", "d30_rollout", "d20_mha", "sample_topk"), default="d20",
                     help="d20: the headline prefill + decode line; d26_latency / d30_rollout: the other "
-                         "decode workloads, one JSON line each")
+                         "decode workloads, d20_mha: prefill and decode of the multi-head d20, one JSON line each")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the d26 latency and d30 rollout lines")
     ap.add_argument("--ref-tokens", type=int, default=128,

@@ -243,10 +243,10 @@ int nc_profile_read(nc_model *model, double *ms, long long *launches);
  * for each CTA c and phase p, eight %globaltimer readings (ns) to
  * d_buf[(c * phases + p) * 8 + slot]: slot 0 phase start (after the previous
  * grid barrier), 1 inputs staged (linear phases) or first cache tile in
- * (attention), 2 first accumulator complete (linear) or keys done
- * (attention), 3 cluster reduction / merge done, 4 phase work done (barrier
- * entry), 5 and 6 the TMA producer's first and last load of the phase, 7 the
- * MMA issuer's last commit of the phase. Slots a CTA does not reach in a
+ * (attention), 2 products done (linear) or keys done (attention), 3 the
+ * reduction over the compute warps or the merge of the key splits done, 4
+ * phase work done (barrier entry), 5 and 6 the TMA producer's first and last
+ * load of the phase, 7 unused. Slots a CTA does not reach in a
  * phase keep their old contents (clear the buffer first). Phases are EMBED,
  * then per layer QKV, ATTN, O-proj, MLP fc, MLP proj, then HEAD and MERGE.
  * d_buf = NULL turns tracing off. *grid and *phases (host, may be NULL)

@@ -11,6 +11,8 @@
 // norm, untied lm_head and softcap cap*tanh(z/cap).
 #include <math.h>
 
+#include <type_traits>
+
 #include "nc_internal.h"
 
 namespace nc {
@@ -94,10 +96,58 @@ __global__ void embed_norm_kernel(const int32_t *tokens, const T *wte, int d, in
   for (int i = threadIdx.x; i < d; i += blockDim.x) x[(size_t)m * d + i] = to_f32(row[i]) * inv;
 }
 
+// bf16 tables with d a multiple of 8: one warp per row, 16-byte loads of 8
+// elements, the row kept in registers between the sum of squares and the
+// scaled fp32 stores (d <= 8 * 32 * EC).
+template <int EC>
+__global__ void embed_norm_bf16_kernel(const int32_t *tokens, const bf16 *wte, int M, int d, int vocab, float eps,
+                                       float *x, uint32_t *status) {
+  const int lane = threadIdx.x & 31, m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (m >= M) return;
+  int tok = tokens[m];
+  if (tok < 0 || tok >= vocab) {
+    if (lane == 0) atomicOr(status, (unsigned)NC_DEV_BAD_TOKEN);
+    tok = tok < 0 ? 0 : vocab - 1;
+  }
+  const uint4 *row = reinterpret_cast<const uint4 *>(wte + (size_t)tok * d);
+  const int nc = d / 8;
+  float v[EC][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < EC; j++) {
+    const int c = lane + 32 * j;
+    uint4 u = c < nc ? __ldg(row + c) : make_uint4(0, 0, 0, 0);
+    const bf16 *h = reinterpret_cast<const bf16 *>(&u);
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+      v[j][q] = __bfloat162float(h[q]);
+      ss = fmaf(v[j][q], v[j][q], ss);
+    }
+  }
+  const float inv = rsqrtf(warp_sum(ss) / d + eps);
+  float4 *dst = reinterpret_cast<float4 *>(x + (size_t)m * d);
+#pragma unroll
+  for (int j = 0; j < EC; j++) {
+    const int c = lane + 32 * j;
+    if (c < nc) {
+      dst[2 * c] = make_float4(v[j][0] * inv, v[j][1] * inv, v[j][2] * inv, v[j][3] * inv);
+      dst[2 * c + 1] = make_float4(v[j][4] * inv, v[j][5] * inv, v[j][6] * inv, v[j][7] * inv);
+    }
+  }
+}
+
 void k_embed_norm(int dtype, const int32_t *tokens, int M, const void *wte, int d, int vocab, float eps,
                   float *x, uint32_t *status, cudaStream_t s) {
   if (M <= 0) return;
   count_launch();
+  if (dtype == NC_BF16 && d % 8 == 0 && d <= 8 * 32 * 8) {
+    const int grid = (M + 7) / 8;
+    if (d <= 8 * 32 * 4)
+      embed_norm_bf16_kernel<4><<<grid, 256, 0, s>>>(tokens, (const bf16 *)wte, M, d, vocab, eps, x, status);
+    else
+      embed_norm_bf16_kernel<8><<<grid, 256, 0, s>>>(tokens, (const bf16 *)wte, M, d, vocab, eps, x, status);
+    return;
+  }
   if (dtype == NC_F32)
     embed_norm_kernel<float><<<M, 256, 0, s>>>(tokens, (const float *)wte, d, vocab, eps, x, status);
   else
@@ -385,8 +435,11 @@ struct ForkArgs {
 
 // One (layer, K or V, destination) per blockIdx.(y, z): copy the rows the
 // destination owns; the source's rows below its own shared length come from
-// its prefix cache. Lengths and prefix tables are read on the device.
+// its prefix cache. Lengths and prefix tables are read on the device. Words
+// are W x 32 bits (W = 4: 16-byte copies when every row offset allows it).
+template <int W>
 __global__ void kv_fork_kernel(ForkArgs f) {
+  using Vec = typename std::conditional<W == 4, uint4, uint32_t>::type;
   const int layer = blockIdx.y >> 1, which = blockIdx.y & 1, i = blockIdx.z;
   int len = *f.src_len;
   if (len > f.dst_max_seq) {
@@ -401,9 +454,12 @@ __global__ void kv_fork_kernel(ForkArgs f) {
                                       (size_t)*f.src_pre_seq * f.pre_seq_words
                                 : own;
   uint32_t *dst = (which ? f.dst_v : f.dst_k) + layer * f.dst_layer_words + (size_t)(f.dst_first + i) * f.dst_seq_words;
-  const size_t w0 = (size_t)first * f.row_words, total = (size_t)len * f.row_words, wsh = (size_t)spl * f.row_words;
+  const size_t w0 = (size_t)first * f.row_words / W, total = (size_t)len * f.row_words / W,
+               wsh = (size_t)spl * f.row_words / W;
+  const Vec *ownv = reinterpret_cast<const Vec *>(own), *prev = reinterpret_cast<const Vec *>(pre);
+  Vec *dstv = reinterpret_cast<Vec *>(dst);
   for (size_t w = w0 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (size_t)gridDim.x * blockDim.x)
-    dst[w] = w < wsh ? pre[w] : own[w];
+    dstv[w] = w < wsh ? prev[w] : ownv[w];
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
     f.dst_len[f.dst_first + i] = len;
     f.dst_pre_len[f.dst_first + i] = first;
@@ -445,9 +501,18 @@ void k_kv_fork(int elem_bytes, const void *src_k, const void *src_v, size_t src_
   f.dst_pre_len = dst_pre_len;
   f.shared = shared ? 1 : 0;
   f.status = status;
-  dim3 grid(32, (unsigned)(depth > 0 ? depth * 2 : 1), (unsigned)n);
+  // 16-byte copies when rows, sequences, layers and the bases are 16-byte aligned
+  const bool vec = row_words % 4 == 0 && ((uintptr_t)src_k | (uintptr_t)src_v | (uintptr_t)dst_k |
+                                          (uintptr_t)dst_v | (uintptr_t)(src_pre.k ? src_pre.k : src_k) |
+                                          (uintptr_t)(src_pre.v ? src_pre.v : src_v)) % 16 == 0;
+  // blocks along the rows: about four vectors per thread at the longest length
+  const size_t words = (size_t)dst_max_seq * row_words / (vec ? 4 : 1);
+  unsigned bx = (unsigned)((words + 4 * 256 - 1) / (4 * 256));
+  bx = bx < 1 ? 1 : (bx > 64 ? 64 : bx);
+  dim3 grid(bx, (unsigned)(depth > 0 ? depth * 2 : 1), (unsigned)n);
   count_launch();
-  kv_fork_kernel<<<grid, 256, 0, s>>>(f);
+  if (vec) kv_fork_kernel<4><<<grid, 256, 0, s>>>(f);
+  else kv_fork_kernel<1><<<grid, 256, 0, s>>>(f);
 }
 
 }  // namespace nc

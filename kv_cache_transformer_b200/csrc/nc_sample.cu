@@ -8,9 +8,11 @@
 // the same convention as the engine's argmax(logits + noise) pick;
 // temperature 0 is the greedy pick.
 //
-// One CTA of 1024 threads per row. Each thread owns a contiguous slice of
-// the row (so the lowest-index rule on the cut is a block prefix sum), the
-// row is re-read from L2 on every pass (it was just written by the lm_head):
+// One CTA of 1024 threads per row. Each warp owns a contiguous slice of the
+// row and reads it 32 consecutive logits at a time (coalesced), so the
+// lowest-index rule on the cut is a prefix sum over the warps plus a ballot
+// within each read; the row is re-read from L2 on every pass (it was just
+// written by the lm_head):
 //   select   the top_k-th largest logit by radix select on an order-preserving
 //            32-bit key, 11 + 11 + 10 bits, histograms in shared memory with
 //            warp-aggregated increments;
@@ -71,9 +73,10 @@ __global__ void __launch_bounds__(ST, 1)
   __shared__ ArgMax s_best[ST / 32];
   const float *z = logits + (size_t)row * (size_t)stride;
   const float *g = noise ? noise + (size_t)row * (size_t)V : nullptr;
-  const int t = threadIdx.x, lane = t & 31;
-  const int per = (V + ST - 1) / ST;
-  const int i0 = min(V, t * per), i1 = min(V, i0 + per);
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  // warp w reads [w0, w1) in rounds of 32 consecutive logits
+  const int per_w = ((V + ST / 32 - 1) / (ST / 32) + 31) / 32 * 32;
+  const int w0 = min(V, w * per_w), w1 = min(V, w0 + per_w);
   const bool greedy = temperature == 0.f;
   const int K = (top_k <= 0 || top_k >= V) ? V : top_k;
 
@@ -91,8 +94,8 @@ __global__ void __launch_bounds__(ST, 1)
       const int hi_sh = sh + widths[pass];  // bits above this digit, fixed by earlier passes
       for (int i = t; i < NBIN; i += ST) hist[i] = 0;
       __syncthreads();
-      for (int i = i0; i < i0 + per; i++) {
-        const bool in = i < i1;
+      for (int i = w0 + lane; i < w0 + per_w; i += 32) {
+        const bool in = i < w1;
         const uint32_t key = in ? order_key(__ldg(z + i)) : 0u;
         const bool take = in && (pass == 0 || (key >> hi_sh) == prefix);
         const uint32_t digit = (key >> sh) & (uint32_t)(nb - 1);
@@ -130,22 +133,33 @@ __global__ void __launch_bounds__(ST, 1)
   }
 
   // ---- pick
-  int eq_base = 0;
-  if (cut && need < n_eq) {  // a tie on the cut: rank the equal keys by index
+  const bool tie = cut && need < n_eq;
+  int eq_base = 0;  // keys equal to tau in the warps before this one
+  if (tie) {        // a tie on the cut: rank the equal keys by index
     int mine = 0;
-    for (int i = i0; i < i1; i++) mine += order_key(__ldg(z + i)) == tau;
+    for (int i = w0 + lane; i < w0 + per_w; i += 32)
+      mine += __popc(__ballot_sync(0xffffffffu, i < w1 && order_key(__ldg(z + i)) == tau));
     int tot;
-    eq_base = block_excl_scan(mine, wsum, &tot);
+    eq_base = block_excl_scan(lane == 0 ? mine : 0, wsum, &tot);
+    eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   }
   ArgMax best{-INFINITY, 0x7fffffff};
-  int eq_seen = 0;
-  for (int i = i0; i < i1; i++) {
-    const float zi = __ldg(z + i);
-    bool member = true;
+  int eq_seen = 0;  // equal keys in this warp's earlier rounds
+  for (int i = w0 + lane; i < w0 + per_w; i += 32) {
+    const bool in = i < w1;
+    const float zi = in ? __ldg(z + i) : 0.f;
+    bool member = in;
     if (cut) {
       const uint32_t key = order_key(zi);
-      if (key == tau) member = eq_base + eq_seen++ < need;
-      else member = key > tau;
+      const bool eq = in && key == tau;
+      if (tie) {
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const int rank = eq_base + eq_seen + __popc(eqm & ((1u << lane) - 1u));
+        eq_seen += __popc(eqm);
+        member = in && (eq ? rank < need : key > tau);
+      } else {
+        member = in && (eq || key > tau);
+      }
     }
     if (!member) continue;
     const float s = greedy ? zi : __fadd_rn(__fdiv_rn(zi, temperature), g ? __ldg(g + i) : 0.f);

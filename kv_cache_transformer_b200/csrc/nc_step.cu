@@ -571,7 +571,7 @@ __device__ float *reduce_warps(float *red, int R, int MT, int e) {
 // are merged (per-row factors first), the split's state goes to apart, and
 // the last split to arrive merges all splits in split order into y.
 __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
-                               uint32_t &t, uint32_t &xph, int p, int b, int j, int sp) {
+                               uint32_t &t, uint32_t &xph, int p, int b, int j, int sp, bool first) {
   const int warp = e >> 5, lane = e & 31, g = lane >> 2, t4 = lane & 3;
   const int grp = warp >> 2, wq = warp & 3;
   const int G = a.G, vs = b * a.Hkv + j;  // query heads j*G .. j*G+G-1 read KV head j
@@ -629,7 +629,7 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
     // every warp waits for every tile (its arrival on the slot must follow the fill)
     mbar_wait(&s.full[ks_], kph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
     mbar_wait(&s.full[vs_], vph, s.abort_flag, a.status);
-    if (e == 0 && key0 == k0) trace_mark(a, p, 1);
+    if (first && e == 0 && key0 == k0) trace_mark(a, p, 1);
     uint8_t *K = ring + ks_ * SLOT, *V = ring + vs_ * SLOT;
     // the new key (normed here) and value (written in the QKV phase) may
     // postdate the prefetch of their tile: patch that row
@@ -802,10 +802,12 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
 // This CTA's attention units (sequence, KV head, split), in the producer's order.
 __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
                                 uint32_t &t, uint32_t &xph, int p) {
+  bool first = true;
   for (int un = blockIdx.x; un < a.B * a.Hkv * a.splits; un += a.grid) {
     const int b = un / (a.Hkv * a.splits), j = (un / a.splits) % a.Hkv, sp = un % a.splits;
     if (!s.valid[b]) continue;
-    attention_unit(a, s, ring, xs, layer, e, t, xph, p, b, j, sp);
+    attention_unit(a, s, ring, xs, layer, e, t, xph, p, b, j, sp, first);
+    first = false;
   }
   if (e == 0) trace_mark(a, p, 3);
   return true;
@@ -1411,12 +1413,24 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
   a.n_qkv = pl.n_qkv;
   a.slots = pl.slots;
   {
-    // key splits per (sequence, KV head): as many as the grid holds in one
-    // round; with more pairs than CTAs, one split and CTAs taking several pairs
-    int sp = pl.grid / (B * c.n_kv_head);
-    if (sp > MAX_SPLIT) sp = MAX_SPLIT;
-    if (sp < 1) sp = 1;
-    a.splits = sp;
+    // key splits per (sequence, KV head): the units (pair, split) are dealt
+    // to the CTAs in rounds, so a CTA streams ceil(units / grid) splits of
+    // 1/s of a pair's keys and pays a unit's fixed cost (QK norm, merges:
+    // measured at about a third of streaming a whole 2048-key pair) per
+    // round. B = 32 with one KV head: 4 splits in one round; with ten KV
+    // heads: one split, 3 rounds
+    const int pairs = B * c.n_kv_head;
+    int best = 1;
+    double best_cost = 1e30;
+    for (int sp = 1; sp <= MAX_SPLIT; sp++) {
+      const int rounds = (pairs * sp + pl.grid - 1) / pl.grid;
+      const double cost = (double)rounds / sp + 0.35 * rounds;
+      if (cost < best_cost - 1e-9) {
+        best_cost = cost;
+        best = sp;
+      }
+    }
+    a.splits = best;
   }
   a.eps = c.norm_eps;
   a.cap = c.softcap;

@@ -134,6 +134,11 @@ WORKLOADS = {
                             token_dist="zipf", token_seed=3),
     "d30_rollout": Workload("d30_rollout", D30, batch=1, prompt_len=256, decode_steps=256,
                             token_dist="zipf", token_seed=4, fork=16, noise_seed=5),
+    # the d20 shapes with multi-head attention (10 KV heads: the 560M model)
+    "d20_mha_prefill": Workload("d20_mha_prefill", D20_MHA, batch=8, prompt_len=2048, decode_steps=0,
+                                token_dist="zipf", token_seed=1),
+    "d20_mha_decode": Workload("d20_mha_decode", D20_MHA, batch=32, prompt_len=2048, decode_steps=128,
+                               token_dist="zipf", token_seed=2),
 }
 
 
