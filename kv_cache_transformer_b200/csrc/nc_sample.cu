@@ -9,13 +9,15 @@
 // temperature 0 is the greedy pick.
 //
 // One CTA of 1024 threads per row. Each warp owns a contiguous slice of the
-// row and reads it 32 consecutive logits at a time (coalesced), so the
-// lowest-index rule on the cut is a prefix sum over the warps plus a ballot
-// within each read; the row is re-read from L2 on every pass (it was just
-// written by the lm_head):
+// row and reads it 32 consecutive logits at a time (coalesced), eight such
+// rounds in flight before any is used, so the lowest-index rule on the cut is
+// a prefix sum over the warps plus a ballot within each round; the row is
+// re-read from L2 on every pass (it was just written by the lm_head):
 //   select   the top_k-th largest logit by radix select on an order-preserving
-//            32-bit key, 11 + 11 + 10 bits, histograms in shared memory with
-//            warp-aggregated increments;
+//            32-bit key, four 8-bit digits; each warp counts into its own
+//            histogram in shared memory (increments aggregated over the warp's
+//            lanes with equal digits), and the 32 histograms are added before
+//            the digit is chosen, so no two warps contend for a bin;
 //   pick     among keys above the cut (and the first `need` keys equal to it),
 //            the largest fl(fl(z / T) + g), lowest index on ties.
 #include "nc_internal.h"
@@ -25,7 +27,8 @@ namespace nc {
 namespace {
 
 constexpr int ST = 1024;   // threads per row
-constexpr int NBIN = 2048;  // histogram bins (11-bit digits)
+constexpr int NBIN = 256;   // histogram bins (8-bit digits)
+constexpr int NBAT = 8;     // rounds of 32 logits a warp loads before using them
 
 // Order-preserving key of a logit: larger z, larger key; -0 is keyed as +0 so
 // that equal logits have equal keys.
@@ -66,7 +69,8 @@ __global__ void __launch_bounds__(ST, 1)
                        float temperature, int top_k, const uint8_t *__restrict__ valid, int32_t *__restrict__ next) {
   const int row = blockIdx.x;
   if (valid && !valid[row]) return;
-  __shared__ int hist[NBIN];
+  __shared__ int whist[ST / 32][NBIN];  // one histogram per warp
+  __shared__ int part[4][NBIN];         // sums over warps 8q .. 8q+7
   __shared__ int wsum[32];
   __shared__ uint32_t s_digit;
   __shared__ int s_above, s_count;
@@ -74,8 +78,8 @@ __global__ void __launch_bounds__(ST, 1)
   const float *z = logits + (size_t)row * (size_t)stride;
   const float *g = noise ? noise + (size_t)row * (size_t)V : nullptr;
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  // warp w reads [w0, w1) in rounds of 32 consecutive logits
-  const int per_w = ((V + ST / 32 - 1) / (ST / 32) + 31) / 32 * 32;
+  // warp w reads [w0, w1) in rounds of 32 consecutive logits, NBAT rounds a batch
+  const int per_w = ((V + ST / 32 - 1) / (ST / 32) + 32 * NBAT - 1) / (32 * NBAT) * (32 * NBAT);
   const int w0 = min(V, w * per_w), w1 = min(V, w0 + per_w);
   const bool greedy = temperature == 0.f;
   const int K = (top_k <= 0 || top_k >= V) ? V : top_k;
@@ -88,42 +92,51 @@ __global__ void __launch_bounds__(ST, 1)
   if (cut) {
     uint32_t prefix = 0;
     int rem = K;
-    const int shifts[3] = {21, 10, 0}, widths[3] = {11, 11, 10};
-    for (int pass = 0; pass < 3; pass++) {
-      const int sh = shifts[pass], nb = 1 << widths[pass];
-      const int hi_sh = sh + widths[pass];  // bits above this digit, fixed by earlier passes
-      for (int i = t; i < NBIN; i += ST) hist[i] = 0;
-      __syncthreads();
-      for (int i = w0 + lane; i < w0 + per_w; i += 32) {
-        const bool in = i < w1;
-        const uint32_t key = in ? order_key(__ldg(z + i)) : 0u;
-        const bool take = in && (pass == 0 || (key >> hi_sh) == prefix);
-        const uint32_t digit = (key >> sh) & (uint32_t)(nb - 1);
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        if (take) {
-          const unsigned peers = __match_any_sync(m, digit);
-          if (lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+    for (int pass = 0; pass < 4; pass++) {
+      const int sh = 24 - 8 * pass;
+      const int hi_sh = sh + 8;  // bits above this digit, fixed by earlier passes (pass >= 1)
+#pragma unroll
+      for (int i = lane; i < NBIN; i += 32) whist[w][i] = 0;
+      __syncwarp();
+      for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
+        uint32_t key[NBAT];
+#pragma unroll
+        for (int r = 0; r < NBAT; r++) {
+          const int i = base + 32 * r + lane;
+          key[r] = i < w1 ? order_key(__ldg(z + i)) : 0u;
+        }
+#pragma unroll
+        for (int r = 0; r < NBAT; r++) {
+          const bool take = base + 32 * r + lane < w1 && (pass == 0 ? true : (key[r] >> hi_sh) == prefix);
+          const uint32_t digit = (key[r] >> sh) & (uint32_t)(NBIN - 1);
+          const unsigned m = __ballot_sync(0xffffffffu, take);
+          if (take) {
+            const unsigned peers = __match_any_sync(m, digit);
+            if (lane == __ffs(peers) - 1) atomicAdd(&whist[w][digit], __popc(peers));
+          }
         }
       }
       __syncthreads();
-      // bins from the top: thread t owns bins nb-1-2t and nb-2-2t
-      int c0 = 0, c1 = 0;
-      const int b0 = nb - 1 - 2 * t, b1 = nb - 2 - 2 * t;
-      if (b0 >= 0) c0 = hist[b0];
-      if (b1 >= 0) c1 = hist[b1];
+      {  // the warps' histograms added: thread t sums bin t % 256 over 8 warps
+        const int bin = t & (NBIN - 1), q = t / NBIN;
+        int c = 0;
+#pragma unroll
+        for (int v = 0; v < 8; v++) c += whist[8 * q + v][bin];
+        part[q][bin] = c;
+      }
+      __syncthreads();
+      // bins from the top: thread t < 256 owns bin 255 - t
+      const int b0 = NBIN - 1 - t;
+      const int c0 = t < NBIN ? part[0][b0] + part[1][b0] + part[2][b0] + part[3][b0] : 0;
       int tot;
-      const int above = block_excl_scan(c0 + c1, wsum, &tot);
-      if (b0 >= 0 && above < rem && rem <= above + c0) {
+      const int above = block_excl_scan(c0, wsum, &tot);
+      if (t < NBIN && above < rem && rem <= above + c0) {
         s_digit = (uint32_t)b0;
         s_above = above;
         s_count = c0;
-      } else if (b1 >= 0 && above + c0 < rem && rem <= above + c0 + c1) {
-        s_digit = (uint32_t)b1;
-        s_above = above + c0;
-        s_count = c1;
       }
       __syncthreads();
-      prefix = (prefix << widths[pass]) | s_digit;
+      prefix = (prefix << 8) | s_digit;
       rem -= s_above;
       n_eq = s_count;
       __syncthreads();
@@ -137,33 +150,52 @@ __global__ void __launch_bounds__(ST, 1)
   int eq_base = 0;  // keys equal to tau in the warps before this one
   if (tie) {        // a tie on the cut: rank the equal keys by index
     int mine = 0;
-    for (int i = w0 + lane; i < w0 + per_w; i += 32)
-      mine += __popc(__ballot_sync(0xffffffffu, i < w1 && order_key(__ldg(z + i)) == tau));
+    for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
+      uint32_t key[NBAT];
+#pragma unroll
+      for (int r = 0; r < NBAT; r++) {
+        const int i = base + 32 * r + lane;
+        key[r] = i < w1 ? order_key(__ldg(z + i)) : ~tau;
+      }
+#pragma unroll
+      for (int r = 0; r < NBAT; r++) mine += __popc(__ballot_sync(0xffffffffu, key[r] == tau));
+    }
     int tot;
     eq_base = block_excl_scan(lane == 0 ? mine : 0, wsum, &tot);
     eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   }
   ArgMax best{-INFINITY, 0x7fffffff};
   int eq_seen = 0;  // equal keys in this warp's earlier rounds
-  for (int i = w0 + lane; i < w0 + per_w; i += 32) {
-    const bool in = i < w1;
-    const float zi = in ? __ldg(z + i) : 0.f;
-    bool member = in;
-    if (cut) {
-      const uint32_t key = order_key(zi);
-      const bool eq = in && key == tau;
-      if (tie) {
-        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-        const int rank = eq_base + eq_seen + __popc(eqm & ((1u << lane) - 1u));
-        eq_seen += __popc(eqm);
-        member = in && (eq ? rank < need : key > tau);
-      } else {
-        member = in && (eq || key > tau);
+  for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
+    float zv[NBAT], gv[NBAT];
+#pragma unroll
+    for (int r = 0; r < NBAT; r++) {
+      const int i = base + 32 * r + lane;
+      zv[r] = i < w1 ? __ldg(z + i) : 0.f;
+      gv[r] = (g && i < w1) ? __ldg(g + i) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < NBAT; r++) {
+      const int i = base + 32 * r + lane;
+      const bool in = i < w1;
+      bool member = in;
+      if (cut) {
+        const uint32_t key = order_key(zv[r]);
+        const bool eq = in && key == tau;
+        if (tie) {
+          const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+          const int rank = eq_base + eq_seen + __popc(eqm & ((1u << lane) - 1u));
+          eq_seen += __popc(eqm);
+          member = in && (eq ? rank < need : key > tau);
+        } else {
+          member = in && (eq || key > tau);
+        }
+      }
+      if (member) {
+        const float sc = greedy ? zv[r] : __fadd_rn(__fdiv_rn(zv[r], temperature), gv[r]);
+        best = argmax_merge(best, ArgMax{sc, i});
       }
     }
-    if (!member) continue;
-    const float s = greedy ? zi : __fadd_rn(__fdiv_rn(zi, temperature), g ? __ldg(g + i) : 0.f);
-    best = argmax_merge(best, ArgMax{s, i});
   }
   best = warp_argmax(best);
   if (lane == 0) s_best[t >> 5] = best;

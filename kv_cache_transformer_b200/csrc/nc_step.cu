@@ -353,15 +353,24 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint3
 // behind prefetched weights.
 __host__ __device__ __forceinline__ int kps_of(int R) { return SLOT / (R * 128); }
 
+// Ring position of the producer and of each consumer: the slot in the low 16
+// bits, the parity of the slot's current fill in bit 16 (advanced without a
+// division by the runtime slot count).
+__device__ __forceinline__ uint32_t ring_slot(uint32_t t) { return t & 0xffffu; }
+__device__ __forceinline__ uint32_t ring_ph(uint32_t t) { return t >> 16; }
+__device__ __forceinline__ uint32_t ring_next(uint32_t t, int slots) {
+  return (int)(t & 0xffffu) + 1 == slots ? ((t & 0x10000u) ^ 0x10000u) : t + 1;
+}
+
 __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
   uint64_t evict_first;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(evict_first));
   uint32_t t = 0;
   // the next slot, armed for `bytes`; false once the pipeline has aborted
   auto take = [&](uint32_t &slot, uint32_t bytes) -> bool {
-    slot = t % a.slots;
-    const uint32_t ph = (t / a.slots) & 1;
-    t++;
+    slot = ring_slot(t);
+    const uint32_t ph = ring_ph(t);
+    t = ring_next(t, a.slots);
     if (!mbar_wait(&s.empty[slot], ph ^ 1, s.abort_flag, a.status)) return false;
     mbar_arrive_expect_tx(&s.full[slot], bytes);
     return true;
@@ -486,8 +495,8 @@ __device__ bool gemv_t(const StepArgs &a, const Smem &s, uint8_t *ring, const ui
     for (int n = 0; n < NT; n++) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.f;
   constexpr int kps = SLOT / (R * 128);
   for (int ch = 0; ch < u.nkb; ch += kps) {
-    const uint32_t slot = t % a.slots, ph = (t / a.slots) & 1;
-    t++;
+    const uint32_t slot = ring_slot(t), ph = ring_ph(t);
+    t = ring_next(t, a.slots);
     mbar_wait(&s.full[slot], ph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
     const int n = min(kps, u.nkb - ch);
     const uint8_t *wslot = ring + slot * SLOT;
@@ -622,10 +631,10 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   int tile = 0;
   for (int key0 = k0; key0 < k1; key0 += KT, tile++) {
-    const uint32_t ks_ = t % a.slots, kph = (t / a.slots) & 1;
-    t++;
-    const uint32_t vs_ = t % a.slots, vph = (t / a.slots) & 1;
-    t++;
+    const uint32_t ks_ = ring_slot(t), kph = ring_ph(t);
+    t = ring_next(t, a.slots);
+    const uint32_t vs_ = ring_slot(t), vph = ring_ph(t);
+    t = ring_next(t, a.slots);
     // every warp waits for every tile (its arrival on the slot must follow the fill)
     mbar_wait(&s.full[ks_], kph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
     mbar_wait(&s.full[vs_], vph, s.abort_flag, a.status);
@@ -916,8 +925,8 @@ __device__ void head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
       for (int n = 0; n < 2; n++) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.f;
     uint32_t last_slot = 0;
     for (int kb2 = 0; kb2 < u.nkb; kb2 += 2) {
-      const uint32_t slot = t % a.slots, ph = (t / a.slots) & 1;
-      t++;
+      const uint32_t slot = ring_slot(t), ph = ring_ph(t);
+      t = ring_next(t, a.slots);
       mbar_wait(&s.full[slot], ph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
       const int n = min(2, u.nkb - kb2);
       if (grp < n) {
@@ -1042,7 +1051,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
     const int e = threadIdx.x - 32;
     const int cw = warp - 1;  // compute warp 0..7
     const int MT = a.B > 16 ? 2 : 1;
-    uint32_t t = 0;           // ring slots consumed, in the producer's order
+    uint32_t t = 0;           // ring position (slot, parity), in the producer's order
     uint32_t xph = 0;         // staging barrier phase
     const int P = n_phases(a);
     bool ok = true;
