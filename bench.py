@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -39,6 +40,21 @@ METRIC = "d20 bf16 prefill tok/s & decode tok/s (B=32); % of HBM / tensor-core r
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16, the vendor's figure
 NOMINAL_HBM_GBS = 8000.0
+
+
+def finite(v):
+    """v with every non-finite float replaced by None (strict JSON)."""
+    if isinstance(v, float):
+        return v if math.isfinite(v) else None
+    if isinstance(v, dict):
+        return {k: finite(x) for k, x in v.items()}
+    if isinstance(v, (list, tuple)):
+        return [finite(x) for x in v]
+    return v
+
+
+def emit(line: dict):
+    print(json.dumps(finite(line), allow_nan=False), flush=True)
 
 
 # ------------------------------------------------------------ accounting
@@ -92,10 +108,11 @@ GEMM_DRAM_BYTES_PER_LAUNCH = (54_963_200 + 196_754_176 + 166_150_400 + 388_773_6
 
 
 # DRAM bytes of one whole-step decode launch (d20, 32 sequences at context
-# 2051): dram__bytes_read.sum + dram__bytes_write.sum from an ncu capture of
-# `python bench.py --only decode --decode-steps 4 --warmup 3` with
-# -k regex:decode_step -s 3 -c 1. To be re-taken whenever nc_step.cu changes.
-DECODE_STEP_DRAM_BYTES = None  # re-taken from an ncu capture of the current kernel
+# 2051): dram__bytes_read.sum + dram__bytes_write.sum (1.543507 GB + 3.828 MB)
+# from an ncu capture of `python bench.py --only decode --decode-steps 8
+# --warmup 3` with -k regex:decode_step_kernel -s 6 -c 1. To be re-taken
+# whenever nc_step.cu changes.
+DECODE_STEP_DRAM_BYTES = 1_543_507_000 + 3_828_224
 
 
 class ClockSampler:
@@ -239,7 +256,7 @@ def run_reference(args):
                          "sample": sample},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(line)
 
 
 # --------------------------------------------------------------- our arm
@@ -282,7 +299,7 @@ def run_ours(args):
     if args.only == "decode":
         dec = run_decode(args, model, kv, wd, cfg, peaks, peaks_src, world, local)
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "only": "decode", "decode": dec}), flush=True)
+            emit({"metric": METRIC, "only": "decode", "decode": dec})
         kv.close()
         model.close()
         return
@@ -404,7 +421,7 @@ def run_ours(args):
         "decode": decode, "workloads": workloads,
     }
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        emit(line)
     kv.close()
     model.close()
     if world > 1:
@@ -619,8 +636,15 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src, s
 
         fork = src.fork_shared_to if shared else src.fork_to
 
+        prefilled = []
+
         def start():
-            model.prefill(src, prompts, 0, None, tok1)
+            # a source whose rows samples read cannot be replaced while they do:
+            # with shared forks it is prefilled once, and each later fork into
+            # dst replaces the samples (and their links)
+            if not (shared and prefilled):
+                model.prefill(src, prompts, 0, None, tok1)
+                prefilled.append(True)
             fork(0, dst, 0, n)
             tok.copy_(tok1.expand(n))
 
@@ -634,7 +658,8 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src, s
                 step(s_)
         torch.cuda.synchronize()
         e0.record(stream)
-        model.prefill(src, prompts, 0, None, tok1)
+        if not shared:
+            model.prefill(src, prompts, 0, None, tok1)
         e1.record(stream)
         ef = torch.cuda.Event(enable_timing=True)
         fork(0, dst, 0, n)
@@ -642,7 +667,7 @@ def decode_workload(name: str, args, world: int, local: int, peaks, peaks_src, s
         tok.copy_(tok1.expand(n))
         torch.cuda.synchronize()
         shared_rows = T // 64 * 64 if shared else 0
-        extra = {"prefill_ms": e0.elapsed_time(e1), "fork_ms": e1.elapsed_time(ef),
+        extra = {"prefill_ms": None if shared else e0.elapsed_time(e1), "fork_ms": e1.elapsed_time(ef),
                  "fork_bytes": cfg.depth * 2 * (T - shared_rows) * cfg.head_dim * 2 * n,
                  "fork_kind": "nc_kv_fork_shared (prefix rows read from the source)" if shared
                  else "nc_kv_fork (copy)"}
@@ -772,7 +797,7 @@ def sample_kernel_us(args) -> dict:
 
 
 def run_decode_workload(args):
-    """One JSON line for --workload d26_latency | d30_rollout | d20_mha | sample_topk."""
+    """One JSON line for --workload d26_latency | d30_rollout | d20_mha | d20_extend | sample_topk."""
     import torch
     from kv_cache_transformer_b200 import build as ncbuild
     world, rank, local = dist_env()
@@ -783,11 +808,13 @@ def run_decode_workload(args):
         line = mha_workload(args, 1, local, peaks, peaks_src)
     elif args.workload == "sample_topk":
         line = sample_kernel_us(args)
+    elif args.workload == "d20_extend":
+        line = extend_workload(args, 1, local, peaks, peaks_src)
     else:
         line = decode_workload(args.workload, args, 1, local, peaks, peaks_src)
     line["warmup"] = args.warmup
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        emit(line)
 
 
 def main():
@@ -800,7 +827,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--only", choices=("all", "decode"), default="all",
                     help="decode: skip the prefill timing (for profiling the decode kernels)")
-    ap.add_argument("--workload", choices=("d20", "d26_latency", "d30_rollout", "d20_mha", "sample_topk"), default="d20",
+    ap.add_argument("--workload", choices=("d20", "d26_latency", "d30_rollout", "d20_mha", "d20_extend", "sample_topk"), default="d20",
                     help="d20: the headline prefill + decode line; d26_latency / d30_rollout: the other "
                          "decode workloads, d20_mha: prefill and decode of the multi-head d20, one JSON line each")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -157,8 +157,12 @@ int nc_prefill(nc_model *model, nc_kv *kv, const int32_t *d_tokens, int B, int T
  * not fit (len + T > max_seq) is skipped: its cache and length stay
  * unchanged, NC_DEV_BAD_POSITION is raised, and its outputs are not
  * meaningful. A sequence reading a shared prefix (nc_kv_fork_shared) may be
- * extended. The linear layers run on the tensor-core GEMM; RoPE/QK norm and
- * attention over the cached prefix run on the shape-generic kernels.
+ * extended. On bf16 head_dim-128 models with at least 128 chunk rows, the
+ * chunk runs the same fused tensor-core layers as nc_prefill (RoPE, QK norm
+ * and the cache append in the QKV GEMM's epilogue, tcgen05 attention over the
+ * cached prefix and the chunk), unless the cache reads a shared prefix; then,
+ * and for smaller chunks, RoPE/QK norm and attention run on the shape-generic
+ * kernels.
  * Errors: as nc_prefill. */
 int nc_prefill_extend(nc_model *model, nc_kv *kv, const int32_t *d_tokens, int B, int T, int logits_mode,
                       float *d_logits, int32_t *d_next, const float *d_noise, void *stream);

@@ -194,9 +194,11 @@ int layer_of(const nc_kv *kv, const void *kc) {
 // per KV head) against layer cache kc/vc.
 cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::RowMap rm, cudaStream_t s) {
   const nc_config &c = m->cfg;
-  if (m->fast && !rm.pos && !rm.off && nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
+  // prefill rows, and appended chunks of a cache that reads no shared prefix
+  if (m->fast && !rm.pos && (!rm.off || !kv->prefix_src) &&
+      nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim))
     return nc::k_attn_prefill_tc(kv->q, kc, vc, M / rm.T, rm.T, c.n_head, c.n_kv_head, kv->max_batch, kv->max_seq,
-                                 kv->y, m->status, s);
+                                 kv->y, m->status, s, rm.off);
   // decode rows and appended chunks may read shared-prefix rows; prefill rows
   // replace their sequences
   const nc::KvPrefix pre = (rm.pos || rm.off) ? prefix_view(kv, layer_of(kv, kc)) : nc::KvPrefix{};
@@ -217,7 +219,8 @@ cudaError_t attention(nc_model *m, nc_kv *kv, void *kc, void *vc, int M, nc::Row
 bool fused_layers_ok(const nc_model *m, const nc_kv *kv, int M, nc::RowMap rm) {
   const nc_config &c = m->cfg;
   const int d = c.d_model, q = c.n_head * 128, F = c.mlp_hidden, qkv = q + 256 * c.n_kv_head;
-  return m->fast && !rm.pos && !rm.off && M >= 128 && kv->row_ss && nc::rowops_supported(c) &&
+  // appended chunks too, unless the cache reads rows of a shared prefix
+  return m->fast && !rm.pos && (!rm.off || !kv->prefix_src) && M >= 128 && kv->row_ss && nc::rowops_supported(c) &&
          nc::attn_prefill_tc_supported(c.n_head, c.n_kv_head, c.head_dim) && nc::gemm_tc_supported(M, qkv, d, d) &&
          nc::gemm_tc_supported(M, d, q, q) && nc::gemm_tc_supported(M, F, d, d) && nc::gemm_tc_supported(M, d, F, F);
 }
@@ -235,6 +238,8 @@ int run_blocks_fused(nc_model *m, nc_kv *kv, int M, nc::RowMap rm, cudaStream_t 
   fz.H = H;
   fz.Hkv = c.n_kv_head;
   fz.max_seq = kv->max_seq;
+  fz.off = rm.off;
+  fz.valid = rm.off ? kv->valid : nullptr;
   const int nss = (d + 127) / 128;
   cudaError_t e = cudaSuccess;
   auto gemm = [&](int epi, const void *A, int lda, const void *W, int N, int K, void *out) {

@@ -14,7 +14,9 @@
 //          TMEM columns
 //   O_t += P_t V_j         (tcgen05 with A read from TMEM, B = V read
 //                           MN-major straight from the cache layout) -> TMEM
-// and finally y = O_t / l in bf16.
+// and finally y = O_t / l in bf16. For a chunk appended to sequences that
+// already hold off[b] tokens, query t sits at position off[b] + t and its
+// keys are the cached rows 0 .. off[b] + t.
 // Warp roles (320 threads): warp 0 TMA (one thread: the Q tiles of each item,
 // then K_j and V_j alternately through a 4-slot ring), warp 1 TMEM
 // allocator + MMA issuer, warps 2-5 softmax of tile A and warps 6-9 of tile B,
@@ -60,6 +62,7 @@ struct AttnArgs {
   int T, H, B, max_seq;
   int Hkv, G;        // KV heads, query heads per KV head
   int rows_per_seq;  // T*G rows of one (sequence, KV head)
+  const int32_t *off;  // [B] position of row t = 0 of each sequence (appended chunks), or null
   float scale_log2;  // log2(e) / sqrt(hd)
   bf16 *y;           // [B*T*H, 128]
   uint32_t *status;
@@ -164,7 +167,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     j = i % a.Hkv;
     row0 = pp * ITEM;
     const int last = min(row0 + ITEM, a.rows_per_seq) - 1;
-    n_kv = (last / a.G) / BKV + 1;
+    n_kv = ((a.off ? a.off[b] : 0) + last / a.G) / BKV + 1;
   };
 
   if (threadIdx.x == 0) {
@@ -306,7 +309,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       int b, j_kv, row0, n_kv;
       item_of(i, b, j_kv, row0, n_kv);
       const int row = row0 + t * BR + r;  // row inside the (sequence, KV head)
-      const int t_row = row < a.rows_per_seq ? row / a.G : 0x3fffffff;
+      const int t_loc = row < a.rows_per_seq ? row / a.G : 0;  // its query among the T
+      // its position: the causal limit of its keys
+      const int t_row = row < a.rows_per_seq ? (a.off ? a.off[b] : 0) + t_loc : 0x3fffffff;
       float m = -INFINITY, l = 0.f;  // running max (scaled, log2 units) and sum
       for (int j = 0; j < n_kv; j++, g++) {
         ok = ok && mbar_wait(&s_full[t], g & 1, abort_flag, a.status);
@@ -407,7 +412,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const float inv = 1.f / l;
       // y row of (position t_row, head j*G + g) in [B*T, H, 128]
-      bf16 *dst = a.y + (((size_t)b * a.T + (row < a.rows_per_seq ? t_row : 0)) * a.H + j_kv * a.G + row % a.G) * HD;
+      bf16 *dst = a.y + (((size_t)b * a.T + t_loc) * a.H + j_kv * a.G + row % a.G) * HD;
 #pragma unroll 1
       for (int cc = 0; cc < HD; cc += 32) {
         uint32_t o[32];
@@ -449,7 +454,8 @@ bool make_map_bf16(CUtensorMap *map, const void *ptr, int rank, const uint64_t *
 // q: [B*T, H, 128] bf16 (rotated + normed), kc/vc: layer cache
 // [max_batch*max_seq, Hkv*128], y: [B*T, H, 128] bf16.
 cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int Hkv,
-                              int max_batch, int max_seq, void *y, uint32_t *status, cudaStream_t s) {
+                              int max_batch, int max_seq, void *y, uint32_t *status, cudaStream_t s,
+                              const int32_t *off) {
   if (!attn_prefill_tc_supported(H, Hkv, HD)) return cudaErrorInvalidValue;
   CUtensorMap mq, mk, mv;
   const int G = H / Hkv, rows = T * G;
@@ -480,6 +486,7 @@ cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int
   a.Hkv = Hkv;
   a.G = G;
   a.rows_per_seq = rows;
+  a.off = off;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   a.y = (bf16 *)y;
   a.status = status;

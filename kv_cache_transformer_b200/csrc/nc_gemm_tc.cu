@@ -145,14 +145,14 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
   }
   const int q = lane & 7, rsub = lane >> 3;
   float facr[8];
-  int pos[8], crow[8];  // position, and cache row b*max_seq + position
+  int pos[8], crow[8];  // position, and cache row b*max_seq + position (-1: no cache write)
 #pragma unroll
   for (int i = 0; i < 8; i++) {
     const int row = rbase + 4 * i + rsub;
     facr[i] = __shfl_sync(0xffffffffu, fac, 4 * i + rsub);
     const int b = row / f.T;
-    pos[i] = row < g.M ? row - b * f.T : 0;
-    crow[i] = row < g.M ? b * f.max_seq + pos[i] : 0;
+    pos[i] = row < g.M ? (f.off ? f.off[b] : 0) + row - b * f.T : 0;
+    crow[i] = row < g.M && (!f.valid || f.valid[b]) ? b * f.max_seq + pos[i] : -1;
   }
   auto dst_of = [&](int i) -> bf16 * {
     const int row = rbase + 4 * i + rsub;
@@ -167,7 +167,7 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
       transpose_chunk(tcol + 32 * c, ebuf, lane, v);
 #pragma unroll
       for (int i = 0; i < 8; i++)
-        if (rbase + 4 * i + rsub < g.M)
+        if (rbase + 4 * i + rsub < g.M && crow[i] >= 0)
           *reinterpret_cast<uint2 *>(dst_of(i) + 32 * c) =
               make_uint2(pack_bf16(v[i].x * facr[i], v[i].y * facr[i]), pack_bf16(v[i].z * facr[i], v[i].w * facr[i]));
     }
@@ -180,7 +180,7 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
     transpose_chunk(tcol + 64 + 32 * c, ebuf, lane, hi);
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-      if (rbase + 4 * i + rsub >= g.M) continue;
+      if (rbase + 4 * i + rsub >= g.M || (head >= f.H && crow[i] < 0)) continue;
       const float4 *cs = reinterpret_cast<const float4 *>(f.rope + (size_t)pos[i] * 64) + 16 * c + 2 * q;
       const float4 a = lo[i], h = hi[i], u = cs[0], w = cs[1];  // (cos, sin) of the 4 pairs
       const float F = facr[i];

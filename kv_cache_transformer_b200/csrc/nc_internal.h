@@ -171,6 +171,10 @@ struct GemmFuse {
   const float2 *rope = nullptr;
   void *q = nullptr, *kc = nullptr, *vc = nullptr;
   int T = 1, H = 0, Hkv = 1, max_seq = 0;  // query heads, KV heads (the cache row holds Hkv heads)
+  // appended chunks: row t of sequence b sits at position off[b] + t, and its
+  // keys and values are written only where valid[b] (null: from position 0, all)
+  const int32_t *off = nullptr;
+  const uint8_t *valid = nullptr;
 };
 
 // ---- generic kernels (any even head_dim; fp32 or bf16 storage) ----
@@ -216,7 +220,8 @@ cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int
 // ---- sm_100a causal MQA / GQA prefill attention (nc_attn_tc.cu) ----
 bool attn_prefill_tc_supported(int H, int Hkv, int hd);
 cudaError_t k_attn_prefill_tc(const void *q, const void *kc, const void *vc, int B, int T, int H, int Hkv,
-                              int max_batch, int max_seq, void *y, uint32_t *status, cudaStream_t s);
+                              int max_batch, int max_seq, void *y, uint32_t *status, cudaStream_t s,
+                              const int32_t *off = nullptr);
 
 
 // ---- row-wise prefill kernels for bf16 head_dim-128 models (nc_rowops.cu) ----

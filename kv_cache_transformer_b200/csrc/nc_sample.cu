@@ -15,9 +15,11 @@
 // re-read from L2 on every pass (it was just written by the lm_head):
 //   select   the top_k-th largest logit by radix select on an order-preserving
 //            32-bit key, four 8-bit digits; each warp counts into its own
-//            histogram in shared memory (increments aggregated over the warp's
-//            lanes with equal digits), and the 32 histograms are added before
-//            the digit is chosen, so no two warps contend for a bin;
+//            histogram in shared memory (plain shared atomics: lanes of one
+//            warp with equal digits are serialised by the hardware, which
+//            costs less than grouping them first), and the 32 histograms are
+//            added before the digit is chosen, so no two warps contend for a
+//            bin;
 //   pick     among keys above the cut (and the first `need` keys equal to it),
 //            the largest fl(fl(z / T) + g), lowest index on ties.
 #include "nc_internal.h"
@@ -109,11 +111,7 @@ __global__ void __launch_bounds__(ST, 1)
         for (int r = 0; r < NBAT; r++) {
           const bool take = base + 32 * r + lane < w1 && (pass == 0 ? true : (key[r] >> hi_sh) == prefix);
           const uint32_t digit = (key[r] >> sh) & (uint32_t)(NBIN - 1);
-          const unsigned m = __ballot_sync(0xffffffffu, take);
-          if (take) {
-            const unsigned peers = __match_any_sync(m, digit);
-            if (lane == __ffs(peers) - 1) atomicAdd(&whist[w][digit], __popc(peers));
-          }
+          if (take) atomicAdd(&whist[w][digit], 1);
         }
       }
       __syncthreads();

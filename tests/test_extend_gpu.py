@@ -113,3 +113,44 @@ def test_chunk_on_a_shared_prefix_sample():
             ref = seqs[b].step(int(chunk[b, t]))
             check_logits(lg[b, t], ref, tol_for(cfg), f"seq {b} position {t}")
     assert run.status() == 0
+
+
+def _misc_launches(run, fn):
+    import kv_cache_transformer_b200 as nc
+    run.model.profile(True)
+    run.model.profile_read()
+    out = fn()
+    _, launches = run.model.profile_read()
+    run.model.profile(False)
+    return out, launches[nc.NC_K_MISC]
+
+
+def test_fused_chunk_with_a_sequence_that_does_not_fit():
+    """180 chunk rows take the fused tensor-core layers (RoPE/QK norm and the
+    cache append in the QKV epilogue, the tcgen05 attention with per-sequence
+    offsets); sequence 0, one decode step ahead, does not fit and must keep
+    its cache and length."""
+    import kv_cache_transformer_b200 as nc
+    cfg, blob = SMALL, blob_for(SMALL)
+    B, T0, T1, max_seq = 3, 40, 60, 100
+    run = Run(cfg, blob, B, max_seq)
+    prompts = syn.tokens_zipf(88, (B, T0), cfg.vocab)
+    _, nxt = run.prefill(prompts)
+    om = orc.OracleModel(cfg, blob)
+    seqs = [om.new_seq(max_seq) for _ in range(B)]
+    for b in range(B):
+        seqs[b].prefill(prompts[b])
+    l, n = run.decode(nxt[:1], np.array([T0], np.int32))  # sequence 0 at 41: 41 + 60 > 100
+    check_logits(l[0], seqs[0].step(int(nxt[0])), tol_for(cfg), "decode before the chunk")
+    chunk = syn.tokens_zipf(89, (B, T1), cfg.vocab)
+    (lg, _), misc = _misc_launches(run, lambda: _extend(run, chunk, all_logits=True))
+    assert misc < 2 + 3 * cfg.depth, "the chunk did not take the fused layers"
+    assert list(run.kv.lengths(B)) == [T0 + 1, T0 + T1, T0 + T1]
+    assert run.status() == nc.NC_DEV_BAD_POSITION
+    for b in (1, 2):
+        for t in range(T1):
+            check_logits(lg[b, t], seqs[b].step(int(chunk[b, t])), tol_for(cfg), f"chunk seq {b} position {t}")
+    # the skipped sequence's cache is intact: its next decode step matches
+    l, _ = run.decode(n[:1], np.array([T0 + 1], np.int32))
+    check_logits(l[0], seqs[0].step(int(n[0])), tol_for(cfg), "sequence 0 after the skipped chunk")
+    assert run.status() == 0

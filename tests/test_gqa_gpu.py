@@ -185,3 +185,33 @@ def test_chunk_appended_to_gqa_cache():
     for b in range(B):
         check_logits(l[b], seqs[b].step(int(nx[b])), tol_for(cfg), f"decode after the chunk seq {b}")
     assert run.status() == 0
+
+
+def test_fused_chunk_on_gqa_cache():
+    """160 chunk rows on a grouped-query cache: the fused layers with per-sequence
+    offsets put each KV head of the chunk at its slot of the cache rows."""
+    import kv_cache_transformer_b200 as nc
+    import torch
+    cfg, blob = GQA2, blob_for(GQA2)
+    B, T0, T1 = 2, 33, 80
+    run = Run(cfg, blob, B, T0 + T1 + 2)
+    prompts = syn.tokens_zipf(96, (B, T0), cfg.vocab)
+    chunk = syn.tokens_zipf(97, (B, T1), cfg.vocab)
+    _, nxt = run.prefill(prompts)
+    om = orc.OracleModel(cfg, blob)
+    seqs = [om.new_seq(T0 + T1 + 2) for _ in range(B)]
+    for b in range(B):
+        seqs[b].prefill(prompts[b])
+    lg = torch.full((B, T1, cfg.vocab), float("nan"), dtype=torch.float32, device="cuda")
+    nx = torch.full((B,), -1, dtype=torch.int32, device="cuda")
+    (_, launches) = _launches(run, lambda: (run.model.extend(run.kv, torch.from_numpy(chunk).cuda(), 1, lg, nx),
+                                            torch.cuda.synchronize()))
+    assert launches[nc.NC_K_MISC] < 2 + 3 * cfg.depth, "the chunk did not take the fused layers"
+    lg = lg.cpu().numpy()
+    for b in range(B):
+        for t in range(T1):
+            check_logits(lg[b, t], seqs[b].step(int(chunk[b, t])), tol_for(cfg), f"chunk seq {b} position {t}")
+    l, _ = run.decode(nx.cpu().numpy(), np.full(B, T0 + T1, np.int32))
+    for b in range(B):
+        check_logits(l[b], seqs[b].step(int(nx[b])), tol_for(cfg), f"decode after the chunk seq {b}")
+    assert run.status() == 0
