@@ -102,9 +102,10 @@ def load_peaks():
 # prefill GEMMs, the mean over the QKV, O-proj, MLP fc and MLP proj launches of
 # one layer (one of each per layer, so also the mean over a step's 80 launches),
 # from an ncu capture (cold L2; writes still in L2 at kernel end not counted)
-# of `python bench.py --no-decode --no-cpu-baseline --steps 1 --warmup 3` with
-# -k regex:gemm_tc -s 240 -c 4. To be re-taken whenever nc_gemm_tc.cu changes.
-GEMM_DRAM_BYTES_PER_LAUNCH = (54_963_200 + 196_754_176 + 166_150_400 + 388_773_632) / 4
+# of `python bench.py --steps 1 --warmup 3 --no-decode --no-workloads
+# --no-cpu-baseline` with -k regex:gemm_tc -s 240 -c 4. To be re-taken
+# whenever nc_gemm_tc.cu changes.
+GEMM_DRAM_BYTES_PER_LAUNCH = (53_985_024 + 195_913_472 + 166_196_480 + 387_185_152) / 4
 
 
 # DRAM bytes of one whole-step decode launch (d20, 32 sequences at context
