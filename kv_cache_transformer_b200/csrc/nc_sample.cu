@@ -12,14 +12,16 @@
 // row and reads it 32 consecutive logits at a time (coalesced), eight such
 // rounds in flight before any is used, so the lowest-index rule on the cut is
 // a prefix sum over the warps plus a ballot within each round; the row is
-// re-read from L2 on every pass (it was just written by the lm_head):
+// re-read from L2 (it was just written by the lm_head):
 //   select   the top_k-th largest logit by radix select on an order-preserving
 //            32-bit key, four 8-bit digits; each warp counts into its own
-//            histogram in shared memory (plain shared atomics: lanes of one
-//            warp with equal digits are serialised by the hardware, which
-//            costs less than grouping them first), and the 32 histograms are
-//            added before the digit is chosen, so no two warps contend for a
-//            bin;
+//            histogram in shared memory (plain shared atomics), and the 32
+//            histograms are added before the digit is chosen, so no two
+//            warps contend for a bin. After the first digit, the keys whose
+//            top digit is at or above the chosen one (every candidate of the
+//            top_k) are compacted, in index order, into a list in shared
+//            memory when they fit, and the remaining digits and the pick run
+//            on that list; otherwise every pass re-reads the row;
 //   pick     among keys above the cut (and the first `need` keys equal to it),
 //            the largest fl(fl(z / T) + g), lowest index on ties.
 #include "nc_internal.h"
@@ -31,6 +33,8 @@ namespace {
 constexpr int ST = 1024;   // threads per row
 constexpr int NBIN = 256;   // histogram bins (8-bit digits)
 constexpr int NBAT = 8;     // rounds of 32 logits a warp loads before using them
+constexpr int LCAP = 6144;  // candidate list entries (key, index)
+constexpr size_t SMEM_BYTES = (size_t)LCAP * 8;  // the list, in dynamic shared memory
 
 // Order-preserving key of a logit: larger z, larger key; -0 is keyed as +0 so
 // that equal logits have equal keys.
@@ -77,6 +81,9 @@ __global__ void __launch_bounds__(ST, 1)
   __shared__ uint32_t s_digit;
   __shared__ int s_above, s_count;
   __shared__ ArgMax s_best[ST / 32];
+  extern __shared__ uint32_t lmem[];
+  uint32_t *lkey = lmem;                                 // [LCAP] candidate keys, in index order
+  int *lidx = reinterpret_cast<int *>(lmem + LCAP);      // [LCAP] their indices
   const float *z = logits + (size_t)row * (size_t)stride;
   const float *g = noise ? noise + (size_t)row * (size_t)V : nullptr;
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
@@ -91,6 +98,8 @@ __global__ void __launch_bounds__(ST, 1)
   uint32_t tau = 0;
   int need = 0, n_eq = 0;
   const bool cut = !greedy && K < V;
+  bool compact = false;  // the candidates are in the list
+  int n_list = 0;
   if (cut) {
     uint32_t prefix = 0;
     int rem = K;
@@ -100,6 +109,12 @@ __global__ void __launch_bounds__(ST, 1)
 #pragma unroll
       for (int i = lane; i < NBIN; i += 32) whist[w][i] = 0;
       __syncwarp();
+      if (compact) {
+        for (int e = t; e < n_list; e += ST) {
+          const uint32_t key = lkey[e];
+          if ((key >> hi_sh) == prefix) atomicAdd(&whist[w][(key >> sh) & (uint32_t)(NBIN - 1)], 1);
+        }
+      } else
       for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
         uint32_t key[NBAT];
 #pragma unroll
@@ -137,6 +152,41 @@ __global__ void __launch_bounds__(ST, 1)
       prefix = (prefix << 8) | s_digit;
       rem -= s_above;
       n_eq = s_count;
+      if (pass == 0 && s_above + s_count <= LCAP) {
+        // compact the keys with top digit >= d0, in index order: each warp's
+        // count from its own histogram, warp offsets by a block scan, then
+        // positions within a warp by ballot
+        const uint32_t d0 = s_digit;
+        int cw = 0;
+        for (int bin = (int)d0 + lane; bin < NBIN; bin += 32) cw += whist[w][bin];
+        cw = __reduce_add_sync(0xffffffffu, cw);
+        int tot;
+        int wbase = block_excl_scan(lane == 0 ? cw : 0, wsum, &tot);
+        wbase = __shfl_sync(0xffffffffu, wbase, 0);
+        int seen = 0;
+        for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
+          uint32_t key[NBAT];
+#pragma unroll
+          for (int r = 0; r < NBAT; r++) {
+            const int i = base + 32 * r + lane;
+            key[r] = i < w1 ? order_key(__ldg(z + i)) : 0u;
+          }
+#pragma unroll
+          for (int r = 0; r < NBAT; r++) {
+            const int i = base + 32 * r + lane;
+            const bool c = i < w1 && (key[r] >> 24) >= d0;
+            const unsigned m = __ballot_sync(0xffffffffu, c);
+            if (c) {
+              const int at = wbase + seen + __popc(m & ((1u << lane) - 1u));
+              lkey[at] = key[r];
+              lidx[at] = i;
+            }
+            seen += __popc(m);
+          }
+        }
+        n_list = tot;
+        compact = true;
+      }
       __syncthreads();
     }
     tau = prefix;
@@ -145,6 +195,28 @@ __global__ void __launch_bounds__(ST, 1)
 
   // ---- pick
   const bool tie = cut && need < n_eq;
+  ArgMax best{-INFINITY, 0x7fffffff};
+  if (compact) {
+    // thread t takes a contiguous run of the list (index order), so the rank of
+    // an equal key is a block prefix sum plus its place in the run
+    const int per = (n_list + ST - 1) / ST;
+    const int e0 = min(n_list, t * per), e1 = min(n_list, e0 + per);
+    int eq_rank = 0;
+    if (tie) {
+      int mine = 0;
+      for (int e = e0; e < e1; e++) mine += lkey[e] == tau;
+      int tot;
+      eq_rank = block_excl_scan(mine, wsum, &tot);
+    }
+    for (int e = e0; e < e1; e++) {
+      const uint32_t key = lkey[e];
+      const bool member = key == tau ? (!tie || eq_rank++ < need) : key > tau;
+      if (!member) continue;
+      const int i = lidx[e];
+      const float sc = __fadd_rn(__fdiv_rn(__ldg(z + i), temperature), g ? __ldg(g + i) : 0.f);
+      best = argmax_merge(best, ArgMax{sc, i});
+    }
+  } else {
   int eq_base = 0;  // keys equal to tau in the warps before this one
   if (tie) {        // a tie on the cut: rank the equal keys by index
     int mine = 0;
@@ -162,7 +234,6 @@ __global__ void __launch_bounds__(ST, 1)
     eq_base = block_excl_scan(lane == 0 ? mine : 0, wsum, &tot);
     eq_base = __shfl_sync(0xffffffffu, eq_base, 0);
   }
-  ArgMax best{-INFINITY, 0x7fffffff};
   int eq_seen = 0;  // equal keys in this warp's earlier rounds
   for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
     float zv[NBAT], gv[NBAT];
@@ -195,6 +266,7 @@ __global__ void __launch_bounds__(ST, 1)
       }
     }
   }
+  }
   best = warp_argmax(best);
   if (lane == 0) s_best[t >> 5] = best;
   __syncthreads();
@@ -209,8 +281,10 @@ __global__ void __launch_bounds__(ST, 1)
 
 cudaError_t k_sample_topk(const float *logits, int B, int V, long long stride, const float *noise, float temperature,
                           int top_k, const uint8_t *valid, int32_t *next, cudaStream_t s) {
+  const cudaError_t e = ensure_smem_attr((const void *)sample_topk_kernel, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   count_launch();
-  sample_topk_kernel<<<B, ST, 0, s>>>(logits, stride, V, noise, temperature, top_k, valid, next);
+  sample_topk_kernel<<<B, ST, SMEM_BYTES, s>>>(logits, stride, V, noise, temperature, top_k, valid, next);
   return cudaGetLastError();
 }
 
