@@ -110,6 +110,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 2^x (PTX ex2.approx.ftz: relative error ~2^-22, 2^-inf = 0)
@@ -316,34 +322,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int j = 0; j < n_kv; j++, g++) {
         ok = ok && mbar_wait(&s_full[t], g & 1, abort_flag, a.status);
         tc_fence_after();
-        // pass 1: raw row max (the scale is positive), 64 columns at a time;
-        // the causal mask only matters on a tile that reaches past the
-        // row's position
+        // the tile's 128 raw scores of this row, read from TMEM once; the
+        // causal mask only matters on a tile that reaches past the row's
+        // position (masked scores become -inf)
         const int kbase = j * BKV;
         const bool masked = kbase + BKV - 1 > t_row;
+        uint32_t v[BKV];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+        tmem_ld_wait();
+        if (masked) {  // a tile on the diagonal
+#pragma unroll
+          for (int q = 0; q < BKV; q++)
+            if (kbase + q > t_row) v[q] = __float_as_uint(-INFINITY);
+        }
+        // row max (the scale is positive)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int h = 0; h < 2; h++) {
-          uint32_t v[64];
-          tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-          tmem_ld_wait();
-          if (masked) {  // a tile on the diagonal
-            const int kh = kbase + h * 64;
 #pragma unroll
-            for (int q = 0; q < 64; q++) {
-              const float x = kh + q > t_row ? -INFINITY : __uint_as_float(v[q]);
-              mx[q & 3] = fmaxf(mx[q & 3], x);
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 64; q += 8) {
-              mx[0] = max3(mx[0], __uint_as_float(v[q]), __uint_as_float(v[q + 1]));
-              mx[1] = max3(mx[1], __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
-              mx[2] = max3(mx[2], __uint_as_float(v[q + 4]), __uint_as_float(v[q + 5]));
-              mx[3] = max3(mx[3], __uint_as_float(v[q + 6]), __uint_as_float(v[q + 7]));
-            }
-          }
+        for (int q = 0; q < BKV; q += 8) {
+          mx[0] = max3(mx[0], __uint_as_float(v[q]), __uint_as_float(v[q + 1]));
+          mx[1] = max3(mx[1], __uint_as_float(v[q + 2]), __uint_as_float(v[q + 3]));
+          mx[2] = max3(mx[2], __uint_as_float(v[q + 4]), __uint_as_float(v[q + 5]));
+          mx[3] = max3(mx[3], __uint_as_float(v[q + 6]), __uint_as_float(v[q + 7]));
         }
         const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.scale_log2;
         const bool need = (m == -INFINITY) ? (tmax != -INFINITY) : (tmax > m + RESCALE_LOG2);
@@ -363,43 +365,24 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_st32(tO + cc, o);
           }
         }
-        // pass 2: p = 2^(s*scale - m), one FMA and one ex2 per score (masked
-        // scores give 0), bf16 pairs into the P columns 64..127 of this S
-        // buffer. Keys 64..127 go first: their P lands on S columns 96..127,
-        // already read; keys 0..63 then land on columns 64..95.
+        // p = 2^(s*scale - m), one FMA and one ex2 per score (masked scores
+        // give 0), bf16 pairs into the P columns 64..127 of this S buffer
+        // (keys 0..63 on columns 64..95, keys 64..127 on 96..127: every score
+        // was read above)
         const float nm = -m_new;
         float sum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int hh = 0; hh < 2; hh++) {
-          const int h = 1 - hh;
-          uint32_t v[64];
-          tmem_ld32(tS + h * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld32(tS + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-          tmem_ld_wait();
-          uint32_t pk[32];
-          if (masked) {
-            const int kh = kbase + h * 64;
 #pragma unroll
-            for (int q = 0; q < 32; q++) {
-              const float s0 = kh + 2 * q > t_row ? -INFINITY : __uint_as_float(v[2 * q]);
-              const float s1 = kh + 2 * q + 1 > t_row ? -INFINITY : __uint_as_float(v[2 * q + 1]);
-              const float p0 = ex2(fmaf(s0, a.scale_log2, nm));
-              const float p1 = ex2(fmaf(s1, a.scale_log2, nm));
-              sum[(2 * q) & 3] += p0;
-              sum[(2 * q + 1) & 3] += p1;
-              pk[q] = pack2(p0, p1);
-            }
-          } else {
+        for (int c8 = 0; c8 < BKV / 16; c8++) {  // 16 keys -> 8 columns of bf16 pairs
+          uint32_t pk[8];
 #pragma unroll
-            for (int q = 0; q < 32; q++) {
-              const float p0 = ex2(fmaf(__uint_as_float(v[2 * q]), a.scale_log2, nm));
-              const float p1 = ex2(fmaf(__uint_as_float(v[2 * q + 1]), a.scale_log2, nm));
-              sum[(2 * q) & 3] += p0;
-              sum[(2 * q + 1) & 3] += p1;
-              pk[q] = pack2(p0, p1);
-            }
+          for (int q = 0; q < 8; q++) {
+            const float p0 = ex2(fmaf(__uint_as_float(v[c8 * 16 + 2 * q]), a.scale_log2, nm));
+            const float p1 = ex2(fmaf(__uint_as_float(v[c8 * 16 + 2 * q + 1]), a.scale_log2, nm));
+            sum[(2 * q) & 3] += p0;
+            sum[(2 * q + 1) & 3] += p1;
+            pk[q] = pack2(p0, p1);
           }
-          tmem_st32(tS + 64 + h * 32, pk);
+          tmem_st8(tS + 64 + c8 * 8, pk);
         }
         l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
         m = m_new;
