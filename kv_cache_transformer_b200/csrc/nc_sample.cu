@@ -70,6 +70,9 @@ __device__ __forceinline__ int block_excl_scan(int v, int *wsum, int *total) {
   return x - v + (w > 0 ? wsum[w - 1] : 0);
 }
 
+// VEC: rows start on 16-byte boundaries and V % 4 == 0, so the two full
+// reads (top-digit histogram, compaction) load four logits per lane per round.
+template <bool VEC>
 __global__ void __launch_bounds__(ST, 1)
     sample_topk_kernel(const float *__restrict__ logits, long long stride, int V, const float *__restrict__ noise,
                        float temperature, int top_k, const uint8_t *__restrict__ valid, int32_t *__restrict__ next) {
@@ -87,8 +90,9 @@ __global__ void __launch_bounds__(ST, 1)
   const float *z = logits + (size_t)row * (size_t)stride;
   const float *g = noise ? noise + (size_t)row * (size_t)V : nullptr;
   const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-  // warp w reads [w0, w1) in rounds of 32 consecutive logits, NBAT rounds a batch
-  const int per_w = ((V + ST / 32 - 1) / (ST / 32) + 32 * NBAT - 1) / (32 * NBAT) * (32 * NBAT);
+  // warp w reads [w0, w1) in rounds of 32 consecutive logits, NBAT rounds a
+  // batch (vector reads: rounds of 32 x 4, NBAT / 2 rounds a batch)
+  const int per_w = ((V + ST / 32 - 1) / (ST / 32) + 64 * NBAT - 1) / (64 * NBAT) * (64 * NBAT);
   const int w0 = min(V, w * per_w), w1 = min(V, w0 + per_w);
   const bool greedy = temperature == 0.f;
   const int K = (top_k <= 0 || top_k >= V) ? V : top_k;
@@ -113,6 +117,24 @@ __global__ void __launch_bounds__(ST, 1)
         for (int e = t; e < n_list; e += ST) {
           const uint32_t key = lkey[e];
           if ((key >> hi_sh) == prefix) atomicAdd(&whist[w][(key >> sh) & (uint32_t)(NBIN - 1)], 1);
+        }
+      } else if (VEC && pass == 0) {
+        constexpr int NB4 = NBAT / 2;
+        for (int base = w0; base < w0 + per_w; base += 128 * NB4) {
+          float4 zq[NB4];
+#pragma unroll
+          for (int r = 0; r < NB4; r++) {
+            const int i = base + 128 * r + 4 * lane;
+            zq[r] = i < w1 ? __ldg(reinterpret_cast<const float4 *>(z + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int r = 0; r < NB4; r++) {
+            if (base + 128 * r + 4 * lane >= w1) continue;
+            atomicAdd(&whist[w][order_key(zq[r].x) >> 24], 1);
+            atomicAdd(&whist[w][order_key(zq[r].y) >> 24], 1);
+            atomicAdd(&whist[w][order_key(zq[r].z) >> 24], 1);
+            atomicAdd(&whist[w][order_key(zq[r].w) >> 24], 1);
+          }
         }
       } else
       for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
@@ -164,6 +186,43 @@ __global__ void __launch_bounds__(ST, 1)
         int wbase = block_excl_scan(lane == 0 ? cw : 0, wsum, &tot);
         wbase = __shfl_sync(0xffffffffu, wbase, 0);
         int seen = 0;
+        if (VEC) {
+          // a round is 128 consecutive logits, 4 per lane: a key's place is
+          // the candidates of the lanes below plus those before it in its lane
+          constexpr int NB4 = NBAT / 2;
+          for (int base = w0; base < w0 + per_w; base += 128 * NB4) {
+            float4 zq[NB4];
+#pragma unroll
+            for (int r = 0; r < NB4; r++) {
+              const int i = base + 128 * r + 4 * lane;
+              zq[r] = i < w1 ? __ldg(reinterpret_cast<const float4 *>(z + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int r = 0; r < NB4; r++) {
+              const int i = base + 128 * r + 4 * lane;
+              const bool in = i < w1;
+              const uint32_t k4[4] = {order_key(zq[r].x), order_key(zq[r].y), order_key(zq[r].z), order_key(zq[r].w)};
+              int c = 0;
+#pragma unroll
+              for (int q = 0; q < 4; q++) c += in && (k4[q] >> 24) >= d0;
+              int incl = c;  // inclusive prefix over the lanes
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+              }
+              int at = wbase + seen + incl - c;
+#pragma unroll
+              for (int q = 0; q < 4; q++)
+                if (in && (k4[q] >> 24) >= d0) {
+                  lkey[at] = k4[q];
+                  lidx[at] = i + q;
+                  at++;
+                }
+              seen += __shfl_sync(0xffffffffu, incl, 31);
+            }
+          }
+        } else
         for (int base = w0; base < w0 + per_w; base += 32 * NBAT) {
           uint32_t key[NBAT];
 #pragma unroll
@@ -281,10 +340,13 @@ __global__ void __launch_bounds__(ST, 1)
 
 cudaError_t k_sample_topk(const float *logits, int B, int V, long long stride, const float *noise, float temperature,
                           int top_k, const uint8_t *valid, int32_t *next, cudaStream_t s) {
-  const cudaError_t e = ensure_smem_attr((const void *)sample_topk_kernel, SMEM_BYTES);
+  const bool vec = V % 4 == 0 && stride % 4 == 0 && (uintptr_t)logits % 16 == 0;
+  const void *fn = vec ? (const void *)sample_topk_kernel<true> : (const void *)sample_topk_kernel<false>;
+  const cudaError_t e = ensure_smem_attr(fn, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   count_launch();
-  sample_topk_kernel<<<B, ST, SMEM_BYTES, s>>>(logits, stride, V, noise, temperature, top_k, valid, next);
+  if (vec) sample_topk_kernel<true><<<B, ST, SMEM_BYTES, s>>>(logits, stride, V, noise, temperature, top_k, valid, next);
+  else sample_topk_kernel<false><<<B, ST, SMEM_BYTES, s>>>(logits, stride, V, noise, temperature, top_k, valid, next);
   return cudaGetLastError();
 }
 

@@ -114,8 +114,9 @@ def test_exact_ties_pick_the_lowest_index(cfg):
             assert run.status() == 0
 
 
-@pytest.mark.parametrize("temp,k", [(0.0, 0), (1.0, 0), (1.0, 50), (0.7, 1000), (1.3, 1), (0.9, 65535)])
-def test_sample_topk_kernel_matches_oracle(temp, k):
+@pytest.mark.parametrize("temp,k,pad", [(0.0, 0, 96), (1.0, 0, 96), (1.0, 50, 96), (0.7, 1000, 96), (1.3, 1, 96),
+                                         (0.9, 65535, 96), (1.0, 50, 3), (0.7, 1000, 3)])
+def test_sample_topk_kernel_matches_oracle(temp, k, pad):
     """nc_sample_topk against the oracle's pick on the same fp32 logits and
     noise: the decision is taken in fp32 on both sides, so it must agree
     exactly; rows carry exact ties, some of them on the top-k cut."""
@@ -130,7 +131,7 @@ def test_sample_topk_kernel_matches_oracle(temp, k):
     z[4, 5] = np.float32(-0.0)
     z[4, 6] = np.float32(0.0)
     noise = syn.gumbel(17, (B, V), stream=int(10 * temp) + k)
-    stride = V + 96                                # rows of a wider logits buffer
+    stride = V + pad                               # rows of a wider logits buffer (pad 3: rows not 16-byte aligned)
     buf = torch.zeros((B, stride), dtype=torch.float32)
     buf[:, :V] = torch.from_numpy(z)
     lg = buf.cuda()[:, :V]
