@@ -32,8 +32,9 @@
 //    softmax states in split order.
 // Every reduction has a fixed order, so results do not depend on timing.
 //
-// Measured costs behind the choice of mma.sync for the linear layers
-// (microbenchmarks on this GPU): a tcgen05.mma with N <= 128 takes ~72 cycles
+// Measured costs behind the choice of mma.sync for the linear layers (the
+// probes in kv_cache_transformer_b200/microbench, on a B200): a tcgen05.mma
+// with N <= 128 takes ~72 cycles
 // whatever its M and N, so at 32 sequences it consumes weights at ~57
 // B/cycle; mma.sync m16n8k16 runs at 8 cycles per warp instruction per SM
 // sub-partition (1024 MACs/cycle/SM), the same ~64 B/cycle of weights at 32
@@ -294,15 +295,6 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(addr));
-}
-
-__device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
-                                                 uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
-      : "memory");
 }
 
 // Tensor copies of rank 3 and 4 (one copy per ring slot, per cache tile, per
