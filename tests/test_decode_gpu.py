@@ -220,3 +220,51 @@ def test_decode_step_trace_fills_and_fits_the_event_time():
     event_us = 1e3 * e0.elapsed_time(e1)
     assert 0.5 * event_us <= span_us <= event_us, (span_us, event_us)
     assert a.status() == 0
+
+
+def test_d26_latency_workload_sampled():
+    """The d26 latency workload's shape (one sequence, 1024-token Zipf prompt,
+    greedy steps on the whole-step kernel), every logit against the oracle
+    for the first decode steps."""
+    w = syn.WORKLOADS["d26_latency"]
+    cfg = w.model
+    worst = greedy_session(cfg, blob_for(cfg), syn.prompt_tokens(w), 3, [0], max_seq=w.prompt_len + w.decode_steps)
+    assert worst <= TOL_BF16
+
+
+@pytest.mark.parametrize("shared", [False, True])
+def test_d30_rollout_workload_sampled(shared):
+    """The d30 rollout workload's shape: a 256-token prompt prefilled once,
+    forked to 16 samples (copied, or sharing the prompt's rows), decode steps
+    picking argmax(logits + Gumbel noise) with the workload's noise; samples 0
+    and 15 replayed by the oracle."""
+    import torch
+    w = syn.WORKLOADS["d30_rollout"]
+    cfg, blob = w.model, blob_for(w.model)
+    n, T, max_seq, steps = w.fork, w.prompt_len, w.prompt_len + w.decode_steps, 3
+    src = Run(cfg, blob, 1, max_seq)
+    _, nxt = src.prefill(syn.prompt_tokens(w))
+    dst = src.model.kv(n, max_seq)
+    (src.kv.fork_shared_to if shared else src.kv.fork_to)(0, dst, 0, n)
+    om = orc.OracleModel(cfg, blob)
+    base = om.new_seq(max_seq)
+    base.prefill(syn.prompt_tokens(w)[0])
+    refs = {i: om.new_seq(max_seq) for i in (0, n - 1)}
+    for r in refs.values():
+        r.copy_from(base)
+    cur = np.full(n, int(nxt[0]), np.int32)
+    for s in range(steps):
+        noise = syn.gumbel(w.noise_seed, (n, cfg.vocab), stream=s)
+        t = torch.from_numpy(cur).cuda()
+        lg = torch.full((n, cfg.vocab), float("nan"), dtype=torch.float32, device="cuda")
+        nx = torch.full((n,), -1, dtype=torch.int32, device="cuda")
+        src.model.decode_step(dst, t, None, torch.from_numpy(noise).cuda(), lg, nx)
+        torch.cuda.synchronize()
+        lg, nx = lg.cpu().numpy(), nx.cpu().numpy()
+        for i, r in refs.items():
+            ref = r.step(int(cur[i]))
+            check_logits(lg[i], ref, TOL_BF16, f"sample {i} step {s}")
+            check_token(int(nx[i]), ref, noise[i], f"sample {i} step {s}")
+        cur = nx.copy()
+    assert src.status() == 0
+    dst.close()
