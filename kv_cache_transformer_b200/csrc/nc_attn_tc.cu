@@ -166,14 +166,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int G = gridDim.x, c = blockIdx.x;
 
   // item i: rows 256*pp .. of sequence b and KV head j, pp heaviest first;
-  // n_kv key tiles
-  auto item_of = [&](int i, int &b, int &j, int &row0, int &n_kv) {
+  // n_kv key tiles, of which Q tile A needs the first n_kv_a (one fewer when
+  // its last position ends a key tile earlier than tile B's, as with one
+  // query head per KV head)
+  auto item_of = [&](int i, int &b, int &j, int &row0, int &n_kv, int &n_kv_a) {
     const int pp = n_pairs - 1 - i / nvs;
     b = (i % nvs) / a.Hkv;
     j = i % a.Hkv;
     row0 = pp * ITEM;
-    const int last = min(row0 + ITEM, a.rows_per_seq) - 1;
-    n_kv = ((a.off ? a.off[b] : 0) + last / a.G) / BKV + 1;
+    const int off = a.off ? a.off[b] : 0;
+    const int last = min(row0 + ITEM, a.rows_per_seq) - 1, last_a = min(row0 + BR, a.rows_per_seq) - 1;
+    n_kv = (off + last / a.G) / BKV + 1;
+    n_kv_a = (off + last_a / a.G) / BKV + 1;
   };
 
   if (threadIdx.x == 0) {
@@ -212,8 +216,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int r = 0, it = 0; ok; r++, it++) {
         const int i = item_at(r, c, G);
         if (i >= n_items) break;
-        int b, j, row0, n_kv;
-        item_of(i, b, j, row0, n_kv);
+        int b, j, row0, n_kv, n_kv_a;
+        item_of(i, b, j, row0, n_kv, n_kv_a);
         if (!mbar_wait(q_empty, (it & 1) ^ 1, abort_flag, a.status)) break;
         mbar_arrive_expect_tx(q_full, 2 * TILE);
         // Q map (128 dims, G heads, Hkv groups, rows): with one KV head the
@@ -242,8 +246,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t id_s = idesc_bf16_f32(BR, BKV);
       const uint32_t id_o = idesc_bf16_f32(BR, HD) | (1u << 16);  // B (V) is MN-major
       const uint32_t qlo = desc_lo_k(smem_u32(smem + OFF_Q));
-      uint32_t n = 0;  // K/V ring position
-      int g = 0;       // key tiles done so far, over all items
+      uint32_t n = 0;          // K/V ring position
+      int gt[2] = {0, 0};      // key tiles of each Q tile done so far, over all items
       bool ok = true;
       auto take = [&](uint32_t &addr, int &slot) -> bool {
         slot = n % NSLOT;
@@ -265,8 +269,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int r = 0, it = 0; ok; r++, it++) {
         const int i = item_at(r, c, G);
         if (i >= n_items) break;
-        int b, j_kv, row0, n_kv;
-        item_of(i, b, j_kv, row0, n_kv);
+        int b, j_kv, row0, n_kv, n_kv_a;
+        item_of(i, b, j_kv, row0, n_kv, n_kv_a);
+        const int nkt[2] = {n_kv_a, n_kv};
         if (!mbar_wait(q_full, it & 1, abort_flag, a.status)) break;
         uint32_t kaddr, vaddr;
         int kslot, vslot;
@@ -275,22 +280,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         issue_s(1, kaddr);
         mma_commit(&kv_empty[kslot]);
         if (n_kv == 1) mma_commit(q_empty);
-        for (int j = 0; j < n_kv && ok; j++, g++) {
+        for (int j = 0; j < n_kv && ok; j++) {
           if (!take(vaddr, vslot)) { ok = false; break; }
           for (int t = 0; t < 2 && ok; t++) {
-            if (!mbar_wait(&p_full[t], g & 1, abort_flag, a.status)) { ok = false; break; }
-            // the epilogue of the previous item must have read O_t
-            if (j == 0 && !mbar_wait(&o_free[t], (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t pa = tmem + t * 128 + 64, vb = desc_lo_mn(vaddr);
+            if (j < nkt[t]) {  // key tile j reaches some row of Q tile t
+              if (!mbar_wait(&p_full[t], gt[t] & 1, abort_flag, a.status)) { ok = false; break; }
+              gt[t]++;
+              // the epilogue of the previous item must have read O_t
+              if (j == 0 && !mbar_wait(&o_free[t], (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t pa = tmem + t * 128 + 64, vb = desc_lo_mn(vaddr);
 #pragma unroll
-            for (int k = 0; k < BKV / 16; k++)
-              mma_ts(tmem + 256 + t * 128, pa + k * 8, vb + ((k * 2048) >> 4), id_o, (j | k) != 0);
-            mma_commit(&o_done[t]);
+              for (int k = 0; k < BKV / 16; k++)
+                mma_ts(tmem + 256 + t * 128, pa + k * 8, vb + ((k * 2048) >> 4), id_o, (j | k) != 0);
+              mma_commit(&o_done[t]);
+            }
             if (t == 1) mma_commit(&kv_empty[vslot]);
             if (j + 1 < n_kv) {
               if (t == 0 && !take(kaddr, kslot)) { ok = false; break; }
-              issue_s(t, kaddr);
+              if (j + 1 < nkt[t]) issue_s(t, kaddr);
               if (t == 1) {
                 mma_commit(&kv_empty[kslot]);
                 if (j + 2 == n_kv) mma_commit(q_empty);  // the item's last S
@@ -312,14 +320,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int rr = 0;; rr++) {
       const int i = item_at(rr, c, G);
       if (i >= n_items) break;
-      int b, j_kv, row0, n_kv;
-      item_of(i, b, j_kv, row0, n_kv);
+      int b, j_kv, row0, n_kv, n_kv_a;
+      item_of(i, b, j_kv, row0, n_kv, n_kv_a);
+      const int nk = t == 0 ? n_kv_a : n_kv;  // key tiles this Q tile takes
       const int row = row0 + t * BR + r;  // row inside the (sequence, KV head)
       const int t_loc = row < a.rows_per_seq ? row / a.G : 0;  // its query among the T
       // its position: the causal limit of its keys
       const int t_row = row < a.rows_per_seq ? (a.off ? a.off[b] : 0) + t_loc : 0x3fffffff;
       float m = -INFINITY, l = 0.f;  // running max (scaled, log2 units) and sum
-      for (int j = 0; j < n_kv; j++, g++) {
+      for (int j = 0; j < nk; j++, g++) {
         ok = ok && mbar_wait(&s_full[t], g & 1, abort_flag, a.status);
         tc_fence_after();
         // the tile's 128 raw scores of this row, read from TMEM once; the
