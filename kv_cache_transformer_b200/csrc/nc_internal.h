@@ -62,7 +62,7 @@ struct StepPlan {
   int s_p = 0;                       // K splits of the MLP projection
   int r_h = 0;                       // lm_head rows per CTA
   int n_o = 0, n_f = 0, n_p = 0, n_h = 0;  // units of each phase
-  int slots = 0;                     // 16 KB ring slots
+  int slots = 0;                     // 32 KB ring slots
   size_t smem = 0;                   // dynamic shared memory per CTA
   size_t ws_bytes = 0;               // device workspace
   size_t off_ctr = 0, off_x0 = 0, off_x1 = 0, off_xb0 = 0, off_xb1 = 0, off_y = 0, off_f = 0, off_qk = 0,

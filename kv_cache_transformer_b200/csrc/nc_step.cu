@@ -12,7 +12,7 @@
 //
 //  * warp 0 is a TMA producer that walks the same phase program as everyone
 //    and streams every weight tile and KV-cache tile this CTA will need into
-//    a ring of 16 KB slots (as deep as shared memory allows), running ahead
+//    a ring of 32 KB slots (as deep as shared memory allows), running ahead
 //    across phase barriers: neither the weights nor the cached keys depend
 //    on the step's activations, so they are mostly resident when a phase
 //    starts;
@@ -65,7 +65,8 @@ namespace {
 
 constexpr int NCW = 8;                  // compute warps (two per SM sub-partition)
 constexpr int THREADS = 32 * (1 + NCW);  // warp 0: TMA producer
-constexpr int SLOT = 16384;             // ring slot bytes
+constexpr int SLOT = 32768;             // ring slot bytes: a 64-key K and V tile pair, or k-blocks of weights
+constexpr int HKB = SLOT / (64 * 128);  // lm_head k-blocks per slot (64 rows each)
 constexpr int KT = 64;                  // keys per attention tile
 constexpr int MAXB = 32;                // sequences per step: rows of every staged activation
 constexpr int MAX_SPLIT = 8;            // attention key splits per sequence
@@ -339,10 +340,9 @@ __device__ __forceinline__ void bulk_copy(void *smem_dst, const void *src, uint3
 // in a slot, [kb][R rows][128 B], as one tensor copy whose box spans the
 // k-blocks (the last slot of a unit may run past the unit's k-blocks: zero
 // fill past K, or a few bytes of the next split that nobody reads); the
-// lm_head puts 2 k-blocks of 64 rows; attention puts one K or V tile of 64
-// keys, [half][key][128 B]. Few, large copies keep the SM's queue of pending
-// tensor copies short, so the activations a phase stages are not queued
-// behind prefetched weights.
+// lm_head puts HKB k-blocks of 64 rows; attention puts the K tile and then
+// the V tile of 64 keys, each [half][key][128 B]. Few, large slots halve the
+// per-slot waits and releases of every phase.
 __host__ __device__ __forceinline__ int kps_of(int R) { return SLOT / (R * 128); }
 
 // Ring position of the producer and of each consumer: the slot in the low 16
@@ -383,16 +383,16 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
         // tiles below the shared length (a multiple of 64) come from the prefix cache
         const int plen = a.pre_len[b];
         const int prow0 = (layer * a.pmax_batch + a.pre_seq[b]) * a.pmax_seq;
-        for (int key = k0; key < k1; key += KT)
-          for (int which = 0; which < 2; which++) {
-            uint32_t slot;
-            if (!take(slot, SLOT)) return;
-            if (first) trace_mark(a, p, 5);
-            first = false;
-            const bool sh = key < plen;
-            tma_load_4d(ring + slot * SLOT, a.kvmaps + (sh ? 2 : 0) + which, 0, (sh ? prow0 : row0) + key, 0, j,
-                        &s.full[slot]);
-          }
+        for (int key = k0; key < k1; key += KT) {  // K at the slot's start, V 16 KB on
+          uint32_t slot;
+          if (!take(slot, SLOT)) return;
+          if (first) trace_mark(a, p, 5);
+          first = false;
+          const bool sh = key < plen;
+          for (int which = 0; which < 2; which++)
+            tma_load_4d(ring + slot * SLOT + which * (SLOT / 2), a.kvmaps + (sh ? 2 : 0) + which, 0,
+                        (sh ? prow0 : row0) + key, 0, j, &s.full[slot]);
+        }
       }
       if (!first) trace_mark(a, p, 6);
     } else if (type == P_QKV || type == P_OPROJ || type == P_FC || type == P_PROJ || type == P_HEAD) {
@@ -401,9 +401,9 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
       if (type == P_HEAD) {
         const int rows = min(u.R, a.V - u.r0);
         for (int g0 = 0; g0 < rows; g0 += HG)
-          for (int kb = 0; kb < u.nkb; kb += 2) {
+          for (int kb = 0; kb < u.nkb; kb += HKB) {
             uint32_t slot;
-            if (!take(slot, 2 * HG * 128)) return;
+            if (!take(slot, HKB * HG * 128)) return;
             if (first) trace_mark(a, p, 5);
             first = false;
             tma_load_3d_hint(ring + slot * SLOT, u.map, 0, u.r0 + g0, kb, &s.full[slot], evict_first);
@@ -625,13 +625,10 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
   for (int key0 = k0; key0 < k1; key0 += KT, tile++) {
     const uint32_t ks_ = ring_slot(t), kph = ring_ph(t);
     t = ring_next(t, a.slots);
-    const uint32_t vs_ = ring_slot(t), vph = ring_ph(t);
-    t = ring_next(t, a.slots);
     // every warp waits for every tile (its arrival on the slot must follow the fill)
     mbar_wait(&s.full[ks_], kph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
-    mbar_wait(&s.full[vs_], vph, s.abort_flag, a.status);
     if (first && e == 0 && key0 == k0) trace_mark(a, p, 1);
-    uint8_t *K = ring + ks_ * SLOT, *V = ring + vs_ * SLOT;
+    uint8_t *K = ring + ks_ * SLOT, *V = K + SLOT / 2;
     // the new key (normed here) and value (written in the QKV phase) may
     // postdate the prefetch of their tile: patch that row
     const int pr = pos - key0;
@@ -705,10 +702,7 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
       }
     }
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&s.empty[ks_]);
-      mbar_arrive(&s.empty[vs_]);
-    }
+    if (lane == 0) mbar_arrive(&s.empty[ks_]);
   }
   if (e == 0) trace_mark(a, p, 2);
   l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -916,14 +910,14 @@ __device__ void head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
 #pragma unroll
       for (int n = 0; n < 2; n++) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.f;
     uint32_t last_slot = 0;
-    for (int kb2 = 0; kb2 < u.nkb; kb2 += 2) {
+    for (int kb2 = 0; kb2 < u.nkb; kb2 += HKB) {
       const uint32_t slot = ring_slot(t), ph = ring_ph(t);
       t = ring_next(t, a.slots);
       mbar_wait(&s.full[slot], ph, s.abort_flag, a.status);  // a timeout is raised at the next grid barrier
-      const int n = min(2, u.nkb - kb2);
-      if (grp < n) {
-        const uint32_t wb = smem_u32(ring + slot * SLOT + grp * HG * 128);
-        const uint32_t xb = smem_u32(xs + (kb2 + grp) * MAXB * 128);
+      const int n = min(HKB, u.nkb - kb2);
+      for (int q = grp; q < n; q += 2) {  // warp group g takes the slot's k-blocks g, g + 2, ...
+        const uint32_t wb = smem_u32(ring + slot * SLOT + q * HG * 128);
+        const uint32_t xb = smem_u32(xs + (kb2 + q) * MAXB * 128);
         uint32_t af[4][MT][4], bf[4][4];
 #pragma unroll
         for (int ks = 0; ks < 4; ks++) {
@@ -942,7 +936,7 @@ __device__ void head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
             mma16816(acc[m][1], af[ks][m], bf[ks][2], bf[ks][3]);
           }
       }
-      if (kb2 + 2 < u.nkb) {
+      if (kb2 + HKB < u.nkb) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&s.empty[slot]);
       } else {
@@ -1255,7 +1249,7 @@ bool decode_step_plan(const nc_config &c, int num_sms, StepPlan *pl) {
   const int fixed = 1024 /*alignment*/ + xreg + MISC;
   p.slots = (SMEM_CAP - fixed) / SLOT;
   if (p.slots > 10) p.slots = 10;
-  if (p.slots < 4) return false;
+  if (p.slots < 3) return false;
   p.smem = (size_t)fixed + (size_t)p.slots * SLOT;
   // workspace layout
   auto take = [&](size_t bytes) {
@@ -1344,7 +1338,7 @@ bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *v
     if (!weight_map(&out[4 * l + 2], w.wfc, F, d, p.r_f, kps_of(p.r_f))) return false;
     if (!weight_map(&out[4 * l + 3], w.wproj, d, F, p.r_p, kps_of(p.r_p))) return false;
   }
-  if (!weight_map(&out[4 * c.depth], m->wlm, c.vocab, d, HG, 2)) return false;
+  if (!weight_map(&out[4 * c.depth], m->wlm, c.vocab, d, HG, HKB)) return false;
   const int rows = c.depth * max_batch * max_seq;
   if (!cache_map(&out[4 * c.depth + 1], kcache, rows, Hkv) || !cache_map(&out[4 * c.depth + 2], vcache, rows, Hkv))
     return false;

@@ -196,10 +196,14 @@ def test_decode_step_trace_fills_and_fits_the_event_time():
     blob = blob_for(cfg)
     B, T = 4, 16
     prompts = syn.tokens_zipf(66, (B, T), cfg.vocab)
-    a, b_ = Run(cfg, blob, B, T + 2), Run(cfg, blob, B, T + 2)
+    a, b_ = Run(cfg, blob, B, T + 3), Run(cfg, blob, B, T + 3)
     _, na = a.prefill(prompts)
     _, nb = b_.prefill(prompts)
     assert np.array_equal(na, nb)
+    # one untraced step first: the traced one is not the cache's first launch
+    _, na = a.decode(na, np.full(B, T, np.int32))
+    _, nb = b_.decode(nb, np.full(B, T, np.int32))
+    T += 1
     grid, P = a.kv.trace(None)
     assert grid > 0 and P == 3 + 5 * cfg.depth
     buf = torch.zeros(grid * P * 8, dtype=torch.int64, device="cuda")
