@@ -94,7 +94,8 @@ struct StepArgs {
   const CUtensorMap *wmaps;   // [4L + 1]: per layer qkv (r_q/2-row box), o, fc, proj; then lm_head
   const CUtensorMap *kvmaps;  // [4]: K and V caches as [L * max_batch * max_seq][Hkv][128], then the
                               // same views of the prefix cache (shared rows, nc_kv_fork_shared)
-  const CUtensorMap *amaps;   // [4]: xb0, y, xb1, f as [32][K] (32-row boxes)
+  const CUtensorMap *amaps;   // [4]: xb0, y, xb1, f as [32][K], boxes of rb rows
+  int rb;                     // activation rows staged: 16 for B <= 16, else 32
   const int32_t *pre_seq, *pre_len;  // [max_batch]: shared rows of each sequence (0: none)
   int pmax_batch, pmax_seq;   // shape of the prefix cache
   const int32_t *tokens, *positions;
@@ -427,15 +428,16 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
 }
 
 // ------------------------------------------------- compute-side helpers
-// Stage the phase's activation rows: sbox k-blocks of 64 columns x 32 rows
-// from k-block kb0 of the activation map into xs ([kb][32 rows][128 B],
+// Stage the phase's activation rows: sbox k-blocks of 64 columns x rb rows
+// from k-block kb0 of the activation map into xs ([kb][rb rows][128 B],
 // swizzled), one tensor copy issued right after the barrier. The writers' data
 // was released through the grid barrier; the proxy fences order it (and this
 // CTA's earlier generic accesses to xs) ahead of the copy.
-__device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CUtensorMap *amap, int kb0, int sbox) {
+__device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CUtensorMap *amap, int kb0, int sbox,
+                                            int rb) {
   asm volatile("fence.proxy.async.global;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  mbar_arrive_expect_tx(s.x_bar, sbox * MAXB * 128);
+  mbar_arrive_expect_tx(s.x_bar, sbox * rb * 128);
   tma_load_3d(xs, amap, 0, 0, kb0, s.x_bar);
 }
 
@@ -445,7 +447,9 @@ __device__ __forceinline__ void stage_issue(const Smem &s, uint8_t *xs, const CU
 __device__ void smem_inv(const StepArgs &a, const Smem &s, const uint8_t *xs, int nkb, int warp, int lane, int e) {
   float acc = 0.f;
   for (int kb = warp; kb < nkb; kb += NCW) {
-    const uint4 *row = reinterpret_cast<const uint4 *>(xs + kb * MAXB * 128 + lane * 128);
+    // rows past rb belong to the next k-block (or lie past the staging):
+    // their sums are not used
+    const uint4 *row = reinterpret_cast<const uint4 *>(xs + kb * a.rb * 128 + lane * 128);
     // the row's 16-byte chunks in column order (the swizzle permutes them by
     // row), so every row sums in the same order and the lanes hit different banks
 #pragma unroll
@@ -495,7 +499,7 @@ __device__ bool gemv_t(const StepArgs &a, const Smem &s, uint8_t *ring, const ui
     for (int j = 0; j < n; j++) {
       const int kb = ch + j;
       if (kb % NCW != warp) continue;
-      const uint32_t wb = smem_u32(wslot + j * R * 128), xb = smem_u32(xs + kb * MAXB * 128);
+      const uint32_t wb = smem_u32(wslot + j * R * 128), xb = smem_u32(xs + kb * a.rb * 128);
       uint32_t af[4][MT][4], bf[4][NT][2];
 #pragma unroll
       for (int ks = 0; ks < 4; ks++) {
@@ -917,7 +921,7 @@ __device__ void head_rows(const StepArgs &a, const Smem &s, uint8_t *ring, const
       const int n = min(HKB, u.nkb - kb2);
       for (int q = grp; q < n; q += 2) {  // warp group g takes the slot's k-blocks g, g + 2, ...
         const uint32_t wb = smem_u32(ring + slot * SLOT + q * HG * 128);
-        const uint32_t xb = smem_u32(xs + (kb2 + q) * MAXB * 128);
+        const uint32_t xb = smem_u32(xs + (kb2 + q) * a.rb * 128);
         uint32_t af[4][MT][4], bf[4][4];
 #pragma unroll
         for (int ks = 0; ks < 4; ks++) {
@@ -1100,7 +1104,7 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
         // linear layer
         const Unit u = unit_of(a, type, layer, blockIdx.x);
         if (u.active) {
-          if (e == 0) stage_issue(s, xs, u.amap, u.kb0, u.sbox);
+          if (e == 0) stage_issue(s, xs, u.amap, u.kb0, u.sbox, a.rb);
           float xr[XR];  // residual inputs of the rows this thread finishes
           if (type == P_OPROJ) load_resid(a, u, a.x0, e, xr);
           else if (type == P_PROJ) load_resid(a, u, a.x1, e, xr);
@@ -1282,7 +1286,7 @@ bool decode_step_supported(const nc_config &c, int B) {
          B >= 1 && B <= MAXB;
 }
 
-int decode_step_maps_count(const nc_config &c) { return 4 * c.depth + 1 + 4 + 4; }
+int decode_step_maps_count(const nc_config &c) { return 4 * c.depth + 1 + 4 + 8; }
 
 int decode_step_prefix_map_index(const nc_config &c) { return 4 * c.depth + 3; }
 
@@ -1318,10 +1322,11 @@ bool decode_step_prefix_maps(const void *kcache, const void *vcache, const nc_co
 // to the device): per layer the QKV weights as (64 columns, rows, 2 RoPE
 // halves 64 rows apart, k-blocks) so that a unit's r_q/2 + r_q/2 paired rows
 // arrive in one copy, then the O, fc, proj weights (boxes of the unit's rows and a
-// slot's k-blocks), the lm_head (64 rows x 2 k-blocks); the K and V caches
+// slot's k-blocks), the lm_head (64 rows x HKB k-blocks); the K and V caches
 // (this cache, then the prefix cache, initially this one); the activations
 // the linear phases stage (bf16(x0), y, bf16(x1), f) as (64 columns, 32 rows,
-// k-blocks) with a box of the phase's k-blocks.
+// k-blocks) with a box of the phase's k-blocks and 32 rows, then the same
+// four with boxes of 16 rows (batches of up to 16).
 bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *vcache, int max_batch, int max_seq,
                             const StepPlan &p, void *ws, CUtensorMap *out) {
   const nc_config &c = m->cfg;
@@ -1347,16 +1352,21 @@ bool decode_step_build_maps(const nc_model *m, const void *kcache, const void *v
   out[4 * c.depth + 4] = out[4 * c.depth + 2];
   uint8_t *base = static_cast<uint8_t *>(ws);
   CUtensorMap *am = out + 4 * c.depth + 5;
-  auto act_map = [&](CUtensorMap *mp, size_t off, int K, int box_kb) {
+  auto act_map = [&](CUtensorMap *mp, size_t off, int K, int box_kb, int rows) {
     const uint64_t dims[3] = {64, (uint64_t)MAXB, (uint64_t)(K / 64)};
     const uint64_t strides[2] = {(uint64_t)K * 2, 128};
-    const uint32_t box[3] = {64, (uint32_t)MAXB, (uint32_t)box_kb};
+    const uint32_t box[3] = {64, (uint32_t)rows, (uint32_t)box_kb};
     return make_map_bf16(mp, base + off, 3, dims, strides, box);
   };
   const int kbs = (F / 64 + p.s_p - 1) / p.s_p;
-  if (!act_map(&am[0], p.off_xb0, d, d / 64) || !act_map(&am[1], p.off_y, d, d / 64) ||
-      !act_map(&am[2], p.off_xb1, d, d / 64) || !act_map(&am[3], p.off_f, F, kbs))
-    return false;
+  // boxes of 32 rows (any batch), then of 16 rows (batches of up to 16)
+  for (int h = 0; h < 2; h++) {
+    const int rows = h ? 16 : MAXB;
+    CUtensorMap *m4 = am + 4 * h;
+    if (!act_map(&m4[0], p.off_xb0, d, d / 64, rows) || !act_map(&m4[1], p.off_y, d, d / 64, rows) ||
+        !act_map(&m4[2], p.off_xb1, d, d / 64, rows) || !act_map(&m4[3], p.off_f, F, kbs, rows))
+      return false;
+  }
   return true;
 }
 
@@ -1433,7 +1443,8 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
   a.wte = (const bf16 *)m->wte;
   a.wmaps = maps_dev;
   a.kvmaps = maps_dev + 4 * c.depth + 1;
-  a.amaps = maps_dev + 4 * c.depth + 5;
+  a.rb = B <= 16 ? 16 : MAXB;
+  a.amaps = maps_dev + 4 * c.depth + 5 + (B <= 16 ? 4 : 0);
   a.pre_seq = pre_seq;
   a.pre_len = pre_len;
   a.pmax_batch = pmax_batch;
