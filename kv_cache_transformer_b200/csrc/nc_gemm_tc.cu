@@ -4,23 +4,35 @@
 // contiguous (activations row-major, weights row-major [out, in]), fp32
 // accumulation in tensor memory (TMEM).
 //
-// Persistent kernel, one CTA per SM, 128 x 256 output tiles walked with a
-// static stride of gridDim.x. Warp roles (320 threads):
+// Persistent kernel, one CTA per SM. With more than 128 rows the CTAs run
+// as clusters of two on an SM pair: a pair walks 256 x 256 output tiles with
+// a static stride, its even CTA issues tcgen05.mma.cta_group::2 (M=256), and
+// each CTA loads its own 128 A rows and 128 of the 256 W rows of every
+// k-block (no multicast), so a stage is 32 KB and six fit. Otherwise one CTA
+// walks 128 x 256 tiles with 48 KB stages, four of them. Either way each CTA
+// finishes 128 x 256 outputs per tile. Warp roles (320 threads):
 //   warp 0      TMA producer: A and W tiles of 64 K-columns (128-byte
-//               swizzle) into a 4-stage shared-memory ring;
-//   warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma (M=128,
-//               N=256, K=16) per stage into one of two TMEM accumulators
-//               (2 x 256 fp32 columns), tcgen05.commit frees the stage;
+//               swizzle) into the shared-memory ring; in a pair both CTAs'
+//               bytes are counted on the even CTA's barrier;
+//   warp 1      TMEM allocator and MMA issuer: 4 x tcgen05.mma (K=16) per
+//               stage into one of two TMEM accumulators (2 x 256 fp32
+//               columns), tcgen05.commit frees the stage (in both CTAs of a
+//               pair);
 //   warps 2-9   epilogue: tcgen05.ld of the finished accumulator (each warp
 //               its 32-lane TMEM quarter = 32 rows, and one 128-column half),
 //               epilogue math, stores, then release the accumulator so the
-//               next tile's MMAs run while this one drains.
+//               next tile's MMAs run while this one drains (a pair's
+//               accumulator is free once all 16 epilogue warps released it).
+// The environment variable NC_GEMM_PAIR=0 selects the one-CTA kernel for
+// every shape.
 // Fused prefill epilogues (GemmFuse): the RMS factor of un-normed bf16(x)
 // rows applied to the accumulator; RoPE + QK norm + cache append of the qkv
 // projection; bf16(x) and per-tile sums of squares written beside the
 // residual update.
 // Every mbarrier wait is bounded (nc_sm100.cuh); a timeout sets
 // NC_DEV_TIMEOUT and all roles drain to the common exit, where TMEM is freed.
+#include <stdlib.h>
+
 #include "nc_internal.h"
 #include "nc_sm100.cuh"
 
@@ -29,16 +41,29 @@ using namespace sm100;
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-constexpr int B_BYTES = BN * BK * 2;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int EPI_WARPS = 8;   // two per TMEM lane quarter, one per 128-column half of the tile
 constexpr int HC = BN / 2;      // columns per epilogue warp
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr int EPI_BUF = EPI_WARPS * 32 * 32 * 4;  // per epilogue warp: a 32 x 32 fp32 transpose buffer
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BUF;
 constexpr uint32_t TMEM_COLS = 2 * BN;
+
+// Per-CTA tiling. A single CTA loads all BN = 256 W rows of a k-block into a
+// 4-stage ring (48 KB stages). A CTA pair (PAIR) computes a 256 x 256 tile
+// with tcgen05.mma.cta_group::2: each CTA loads its 128 A rows and 128 of the
+// 256 W rows, so a stage is 32 KB and the same shared memory holds 6 stages;
+// each CTA's TMEM still receives a 128 x 256 accumulator.
+template <bool PAIR>
+struct Tiling {
+  static constexpr int BNL = PAIR ? BN / 2 : BN;  // W rows this CTA loads per k-block
+  static constexpr int B_BYTES = BNL * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = PAIR ? 6 : 4;
+  static constexpr int TM = PAIR ? 2 * BM : BM;   // output rows per tile
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BUF;
+};
+static_assert(Tiling<false>::SMEM_BYTES <= 227 * 1024 && Tiling<true>::SMEM_BYTES <= 227 * 1024, "shared memory");
 
 struct GemmArgs {
   int M, N, K;
@@ -195,9 +220,11 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
   }
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapW, GemmArgs g) {
+  using TL = Tiling<PAIR>;
+  constexpr int STAGES = TL::STAGES, B_BYTES = TL::B_BYTES, STAGE_BYTES = TL::STAGE_BYTES, TM = TL::TM;
   extern __shared__ uint8_t smem_raw[];
   uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023) & ~1023u) - raw);
@@ -212,8 +239,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_n = (g.N + BN - 1) / BN;
-  const int tiles = ((g.M + BM - 1) / BM) * tiles_n;
+  const int tiles = ((g.M + TM - 1) / TM) * tiles_n;
   const int kblocks = g.K / BK;
+  // tiles are walked by CTA (or by pair) with a static stride
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const int walker = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int walkers = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; s++) {
@@ -222,16 +253,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; a++) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 32 * EPI_WARPS);
+      // a pair's accumulator is released by each epilogue warp of both CTAs
+      mbar_init(&tempty[a], PAIR ? 2 * EPI_WARPS : 32 * EPI_WARPS);
     }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&mapA);
     tma_prefetch_desc(&mapW);
   }
-  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    else tmem_alloc(tmem_slot, TMEM_COLS);
+  }
   tc_fence_before();
-  __syncthreads();
+  // a pair: the peer's barriers are initialised before any remote arrival
+  if constexpr (PAIR) cluster_sync();
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -240,16 +277,26 @@ __global__ void __launch_bounds__(THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+      for (int tile = walker; tile < tiles && ok; tile += walkers) {
+        // this CTA's A rows and W rows of the tile
+        const int m0 = (tile / tiles_n) * TM + (int)rank * BM, n0 = (tile % tiles_n) * BN + (int)rank * TL::BNL;
         for (int kb = 0; kb < kblocks; kb++) {
           if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, g.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sA + stage * A_BYTES, &mapA, kb * BK, m0, &full[stage]);
-          tma_load_2d(sW + stage * B_BYTES, &mapW, kb * BK, n0, &full[stage]);
+          if constexpr (PAIR) {
+            // both CTAs' bytes are counted on the rank-0 CTA's barrier, whose
+            // MMA thread reads both CTAs' stages
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+            const uint32_t fb = cluster_addr(smem_u32(&full[stage]), 0);
+            tma_load_2d_pair(sA + stage * A_BYTES, &mapA, kb * BK, m0, fb);
+            tma_load_2d_pair(sW + stage * B_BYTES, &mapW, kb * BK, n0, fb);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+            tma_load_2d(sA + stage * A_BYTES, &mapA, kb * BK, m0, &full[stage]);
+            tma_load_2d(sW + stage * B_BYTES, &mapW, kb * BK, n0, &full[stage]);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -258,15 +305,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN);
+    if (lane == 0 && rank == 0) {  // a pair's MMAs are issued by its rank-0 CTA
+      const uint32_t idesc = idesc_bf16_f32(TM, BN);
       int stage = 0, local = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, local++) {
+      for (int tile = walker; tile < tiles && ok; tile += walkers, local++) {
         const int acc = local & 1;
         const uint32_t accphase = (local >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], accphase ^ 1, abort_flag, g.status)) break;
+        if (PAIR ? !mbar_wait_cluster(&tempty[acc], accphase ^ 1, abort_flag, g.status)
+                 : !mbar_wait(&tempty[acc], accphase ^ 1, abort_flag, g.status))
+          break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
         // a wait's result takes ~160 cycles even when the stage is full, so
@@ -284,14 +333,21 @@ __global__ void __launch_bounds__(THREADS, 1)
           const bool next_ready = kb + 1 < kblocks && mbar_try_wait(smem_u32(&full[nstage]), nphase);
           const uint32_t a0 = smem_u32(sA + stage * A_BYTES), w0 = smem_u32(sW + stage * B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / 16; k++)
-            mma_bf16(d, desc_k_sw128(a0 + 32 * k), desc_k_sw128(w0 + 32 * k), idesc, (kb | k) != 0);
-          mma_commit(&empty[stage]);
+          for (int k = 0; k < BK / 16; k++) {
+            if constexpr (PAIR)
+              mma_bf16_pair(d, desc_k_sw128(a0 + 32 * k), desc_k_sw128(w0 + 32 * k), idesc, (kb | k) != 0);
+            else
+              mma_bf16(d, desc_k_sw128(a0 + 32 * k), desc_k_sw128(w0 + 32 * k), idesc, (kb | k) != 0);
+          }
+          // the stage is free in both CTAs of a pair once these MMAs are done
+          if constexpr (PAIR) mma_commit_pair(&empty[stage]);
+          else mma_commit(&empty[stage]);
           stage = nstage;
           phase = nphase;
           ready = next_ready;
         }
-        mma_commit(&tfull[acc]);
+        if constexpr (PAIR) mma_commit_pair(&tfull[acc]);
+        else mma_commit(&tfull[acc]);
       }
     }
   } else {
@@ -300,10 +356,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int half = ew >> 2;      // its 128-column half of the tile
     float *ebuf = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES + 256) + ew * 1024;
     int local = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, local++) {
+    for (int tile = walker; tile < tiles; tile += walkers, local++) {
       const int acc = local & 1;
       const uint32_t accphase = (local >> 1) & 1;
-      const int m0 = (tile / tiles_n) * BM, n0 = (tile % tiles_n) * BN;
+      // this CTA's 128 rows of the tile, all of its 256 columns
+      const int m0 = (tile / tiles_n) * TM + (int)rank * BM, n0 = (tile % tiles_n) * BN;
       const int nh = n0 + half * HC;  // first column of this warp's half
       const int row = m0 + quarter * 32 + lane;
       const bool rok = row < g.M;
@@ -406,13 +463,28 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if constexpr (PAIR) {
+        // one arrival per warp, on the rank-0 CTA's barrier
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(smem_u32(&tempty[acc]), 0));
+      } else {
+        mbar_arrive(&tempty[acc]);
+      }
     }
   }
-  __syncthreads();
+  __syncwarp();
+  if constexpr (PAIR) {
+    // neither CTA leaves while the other may still read its shared memory
+    // (the MMAs read both CTAs' stages) or arrive on its barriers
+    tc_fence_before();
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, TMEM_COLS);
+    else tmem_dealloc(tmem, TMEM_COLS);
   }
 }
 
@@ -477,16 +549,77 @@ bool gemm_tc_supported(int M, int N, int K, int lda) {
   return M > 0 && N > 0 && K > 0 && K % BK == 0 && N % 32 == 0 && lda % 8 == 0;
 }
 
-template <int EPI>
+template <int EPI, bool PAIR>
 static cudaError_t launch_tc(const CUtensorMap &ma, const CUtensorMap &mw, const GemmArgs &g, int grid,
                              cudaStream_t s) {
+  constexpr int SMEM = Tiling<PAIR>::SMEM_BYTES;
   {
-    const cudaError_t e = ensure_smem_attr((const void *)gemm_tc_kernel<EPI>, SMEM_BYTES);
+    const cudaError_t e = ensure_smem_attr((const void *)gemm_tc_kernel<EPI, PAIR>, SMEM);
     if (e != cudaSuccess) return e;
   }
   count_launch();
-  gemm_tc_kernel<EPI><<<grid, THREADS, SMEM_BYTES, s>>>(ma, mw, g);
-  return cudaGetLastError();
+  if constexpr (!PAIR) {
+    gemm_tc_kernel<EPI, false><<<grid, THREADS, SMEM, s>>>(ma, mw, g);
+    return cudaGetLastError();
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, true>, ma, mw, g);
+  }
+}
+
+// How many CTA pairs of the pair kernel can be resident at once on this
+// device (0 if none, or when the environment sets NC_GEMM_PAIR=0, which
+// selects the one-CTA kernel for every shape).
+static int pair_slots() {
+  static int slots = -1;
+  if (slots >= 0) return slots;
+  slots = 0;
+  const char *env = getenv("NC_GEMM_PAIR");
+  if (env && atoi(env) == 0) return slots;
+  const void *fn = (const void *)gemm_tc_kernel<EPI_STORE, true>;
+  if (ensure_smem_attr(fn, Tiling<true>::SMEM_BYTES) != cudaSuccess) return slots;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Tiling<true>::SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  slots = n;
+  return slots;
+}
+
+template <bool PAIR>
+static cudaError_t dispatch_tc(int epi, const CUtensorMap &ma, const CUtensorMap &mw, const GemmArgs &g, int grid,
+                               cudaStream_t s) {
+  switch (epi) {
+    case EPI_STORE: return launch_tc<EPI_STORE, PAIR>(ma, mw, g, grid, s);
+    case EPI_RELU2: return launch_tc<EPI_RELU2, PAIR>(ma, mw, g, grid, s);
+    case EPI_RESID: return launch_tc<EPI_RESID, PAIR>(ma, mw, g, grid, s);
+    case EPI_QKV: return launch_tc<EPI_QKV, PAIR>(ma, mw, g, grid, s);
+    case EPI_RESID_X: return launch_tc<EPI_RESID_X, PAIR>(ma, mw, g, grid, s);
+    default: return launch_tc<EPI_SOFTCAP, PAIR>(ma, mw, g, grid, s);
+  }
 }
 
 cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int N, int K, void *out, int ldo,
@@ -494,20 +627,19 @@ cudaError_t k_gemm_tc(int epi, const void *A, int lda, const void *W, int M, int
   if (!gemm_tc_supported(M, N, K, lda)) return cudaErrorInvalidValue;
   if ((epi == EPI_QKV || epi == EPI_RESID_X) && !fz) return cudaErrorInvalidValue;
   if (epi == EPI_QKV && N != (fz->H + 2 * fz->Hkv) * 128) return cudaErrorInvalidValue;
-  CUtensorMap ma, mw;
-  if (!make_map_bf16_k64(&ma, A, M, K, lda, BM) || !make_map_bf16_k64(&mw, W, N, K, K, BN))
-    return cudaErrorInvalidValue;
   GemmArgs g{M, N, K, out, ldo, cap, status, fz ? *fz : GemmFuse{}};
-  int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  int grid = tiles < num_sms ? tiles : num_sms;
-  switch (epi) {
-    case EPI_STORE: return launch_tc<EPI_STORE>(ma, mw, g, grid, s);
-    case EPI_RELU2: return launch_tc<EPI_RELU2>(ma, mw, g, grid, s);
-    case EPI_RESID: return launch_tc<EPI_RESID>(ma, mw, g, grid, s);
-    case EPI_QKV: return launch_tc<EPI_QKV>(ma, mw, g, grid, s);
-    case EPI_RESID_X: return launch_tc<EPI_RESID_X>(ma, mw, g, grid, s);
-    default: return launch_tc<EPI_SOFTCAP>(ma, mw, g, grid, s);
+  const int tiles_n = (N + BN - 1) / BN;
+  // CTA pairs once there are two 128-row blocks to pair up
+  const int pairs = M > BM ? pair_slots() : 0;
+  CUtensorMap ma, mw;
+  if (!make_map_bf16_k64(&ma, A, M, K, lda, BM) || !make_map_bf16_k64(&mw, W, N, K, K, pairs > 0 ? BN / 2 : BN))
+    return cudaErrorInvalidValue;
+  if (pairs > 0) {
+    const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * tiles_n;
+    return dispatch_tc<true>(epi, ma, mw, g, 2 * (tiles < pairs ? tiles : pairs), s);
   }
+  const int tiles = ((M + BM - 1) / BM) * tiles_n;
+  return dispatch_tc<false>(epi, ma, mw, g, tiles < num_sms ? tiles : num_sms, s);
 }
 
 }  // namespace nc

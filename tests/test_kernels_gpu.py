@@ -1,6 +1,7 @@
 """Kernel-level parity: the tcgen05 GEMM entry point (nc_gemm_bf16) against a
 float64 CPU matmul of the same bf16 operands, for every epilogue, ragged and
-full-size shapes; rows outside M must stay untouched."""
+full-size shapes, on CTA pairs and on the one-CTA kernel; rows outside M must
+stay untouched."""
 import numpy as np
 import pytest
 
@@ -59,6 +60,46 @@ def test_gemm_bf16_matches_float64(M, N, K, epi):
     err = np.abs(got[:M] - want)
     assert np.all(err <= _tol(epi, want, K)), f"max err {err.max():.3g}"
     assert torch.equal(out[M:].cpu(), prev[M:]), "rows beyond M were written"
+
+
+_ONE_CTA_CHECK = r"""
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import kv_cache_transformer_b200 as nc
+from tests.test_kernels_gpu import _ref, _apply, _tol
+bad = []
+for M, N, K in [(300, 1536, 1280), (257, 1920, 1664), (640, 1280, 5120)]:
+    for epi in (0, 1, 2, 3):
+        g = torch.Generator().manual_seed(M + N + K + epi)
+        A = torch.randn(M, K, generator=g).to(torch.bfloat16)
+        W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16)
+        dt = torch.bfloat16 if epi in (0, 1) else torch.float32
+        prev = torch.randn(M, N, generator=g).to(dt)
+        out = prev.clone().cuda()
+        nc.nc_gemm_bf16(A.cuda(), W.cuda(), out, epi)
+        torch.cuda.synchronize()
+        want = _apply(epi, _ref(A, W).numpy(), prev.double().numpy())
+        if not np.all(np.abs(out.cpu().double().numpy() - want) <= _tol(epi, want, K)):
+            bad.append((M, N, K, epi))
+print(bad)
+sys.exit(1 if bad else 0)
+"""
+
+
+def test_gemm_one_cta_kernel_on_pair_shapes():
+    """Shapes of more than 128 rows run on CTA pairs (tcgen05.mma.cta_group::2);
+    NC_GEMM_PAIR=0 selects the one-CTA kernel for every shape. Its results on
+    the same ragged shapes, in a process of its own."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, NC_GEMM_PAIR="0")
+    r = subprocess.run([sys.executable, "-c", _ONE_CTA_CHECK, root], env=env, cwd=root,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
 
 
 def test_gemm_bf16_full_size_sampled_rows():
