@@ -140,18 +140,34 @@ __device__ __forceinline__ void transpose_chunk(uint32_t taddr, float *ebuf, int
   __syncwarp();
 }
 
+// Per-row metadata of EPI_QKV for the lane's 8 transposed rows rbase + 4i +
+// (lane >> 3): the position, and the cache row b*max_seq + position (-1: no
+// cache write). It reads only kernel inputs, so it runs before the
+// accumulator is ready.
+__device__ __forceinline__ void qkv_rows(const GemmArgs &g, int rbase, int lane, int (&pos)[8], int (&crow)[8]) {
+  const GemmFuse &f = g.fz;
+  const int rsub = lane >> 3;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const int row = rbase + 4 * i + rsub;
+    const int b = row / f.T;
+    pos[i] = row < g.M ? (f.off ? f.off[b] : 0) + row - b * f.T : 0;
+    crow[i] = row < g.M && (!f.valid || f.valid[b]) ? b * f.max_seq + pos[i] : -1;
+  }
+}
+
 // EPI_QKV for one 128-column head of the warp's 32 rows (rbase + lane); the
 // head's accumulator columns start at TMEM address tcol, `scale` is the RMS
-// factor of this lane's row. Heads 0..H-1 are q, heads H..H+Hkv-1 the keys
-// and H+Hkv..H+2Hkv-1 the values of the Hkv KV heads; KV head j occupies
-// elements [128j, 128j + 128) of a cache row.
+// factor of this lane's row, pos / crow come from qkv_rows. Heads 0..H-1
+// are q, heads H..H+Hkv-1 the keys and H+Hkv..H+2Hkv-1 the values of the Hkv
+// KV heads; KV head j occupies elements [128j, 128j + 128) of a cache row.
 // RoPE pairs element e with element e+64 and rotates by the angle of
 // (e, position); q and k are then RMS normed over their 128 elements. A
 // rotation keeps each pair's sum of squares, so the norm factor is taken from
 // the unrotated accumulator row (lane = row); the rotation, scaling and
 // stores then run on transposed chunks, lane = (row group, 4 columns).
 __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane, int head, uint32_t tcol, float scale,
-                                         float *ebuf) {
+                                         float *ebuf, const int (&pos)[8], const int (&crow)[8]) {
   const GemmFuse &f = g.fz;
   const bool isv = head >= f.H + f.Hkv;
   const int kvh = head < f.H ? 0 : (isv ? head - f.H - f.Hkv : head - f.H);  // KV head of a k or v head
@@ -170,15 +186,8 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
   }
   const int q = lane & 7, rsub = lane >> 3;
   float facr[8];
-  int pos[8], crow[8];  // position, and cache row b*max_seq + position (-1: no cache write)
 #pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const int row = rbase + 4 * i + rsub;
-    facr[i] = __shfl_sync(0xffffffffu, fac, 4 * i + rsub);
-    const int b = row / f.T;
-    pos[i] = row < g.M ? (f.off ? f.off[b] : 0) + row - b * f.T : 0;
-    crow[i] = row < g.M && (!f.valid || f.valid[b]) ? b * f.max_seq + pos[i] : -1;
-  }
+  for (int i = 0; i < 8; i++) facr[i] = __shfl_sync(0xffffffffu, fac, 4 * i + rsub);
   auto dst_of = [&](int i) -> bf16 * {
     const int row = rbase + 4 * i + rsub;
     return (head < f.H ? reinterpret_cast<bf16 *>(f.q) + ((size_t)row * f.H + head) * 128
@@ -203,19 +212,31 @@ __device__ __forceinline__ void qkv_head(const GemmArgs &g, int rbase, int lane,
     float4 lo[8], hi[8];
     transpose_chunk(tcol + 32 * c, ebuf, lane, lo);
     transpose_chunk(tcol + 64 + 32 * c, ebuf, lane, hi);
+    // the (cos, sin) of 4 rows' 4 pairs at a time, requested before any of
+    // their stores, so the L2 round trips of a group overlap
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-      if (rbase + 4 * i + rsub >= g.M || (head >= f.H && crow[i] < 0)) continue;
-      const float4 *cs = reinterpret_cast<const float4 *>(f.rope + (size_t)pos[i] * 64) + 16 * c + 2 * q;
-      const float4 a = lo[i], h = hi[i], u = cs[0], w = cs[1];  // (cos, sin) of the 4 pairs
-      const float F = facr[i];
-      const float l0 = a.x * u.x - h.x * u.y, h0 = a.x * u.y + h.x * u.x;
-      const float l1 = a.y * u.z - h.y * u.w, h1 = a.y * u.w + h.y * u.z;
-      const float l2 = a.z * w.x - h.z * w.y, h2 = a.z * w.y + h.z * w.x;
-      const float l3 = a.w * w.z - h.w * w.w, h3 = a.w * w.w + h.w * w.z;
-      bf16 *d = dst_of(i);
-      *reinterpret_cast<uint2 *>(d + 32 * c) = make_uint2(pack_bf16(l0 * F, l1 * F), pack_bf16(l2 * F, l3 * F));
-      *reinterpret_cast<uint2 *>(d + 64 + 32 * c) = make_uint2(pack_bf16(h0 * F, h1 * F), pack_bf16(h2 * F, h3 * F));
+    for (int i0 = 0; i0 < 8; i0 += 4) {
+      float4 cu[4], cw[4];
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        const float4 *cs = reinterpret_cast<const float4 *>(f.rope + (size_t)pos[i0 + k] * 64) + 16 * c + 2 * q;
+        cu[k] = __ldg(cs);
+        cw[k] = __ldg(cs + 1);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; k++) {
+        const int i = i0 + k;
+        if (rbase + 4 * i + rsub >= g.M || (head >= f.H && crow[i] < 0)) continue;
+        const float4 a = lo[i], h = hi[i], u = cu[k], w = cw[k];  // (cos, sin) of the 4 pairs
+        const float F = facr[i];
+        const float l0 = a.x * u.x - h.x * u.y, h0 = a.x * u.y + h.x * u.x;
+        const float l1 = a.y * u.z - h.y * u.w, h1 = a.y * u.w + h.y * u.z;
+        const float l2 = a.z * w.x - h.z * w.y, h2 = a.z * w.y + h.z * w.x;
+        const float l3 = a.w * w.z - h.w * w.w, h3 = a.w * w.w + h.w * w.z;
+        bf16 *d = dst_of(i);
+        *reinterpret_cast<uint2 *>(d + 32 * c) = make_uint2(pack_bf16(l0 * F, l1 * F), pack_bf16(l2 * F, l3 * F));
+        *reinterpret_cast<uint2 *>(d + 64 + 32 * c) = make_uint2(pack_bf16(h0 * F, h1 * F), pack_bf16(h2 * F, h3 * F));
+      }
     }
   }
 }
@@ -446,11 +467,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             scale = rsqrtf(t / g.K + g.fz.eps);
           }
         }
+        int qpos[8], qcrow[8];
+        if constexpr (EPI == EPI_QKV) qkv_rows(g, m0 + quarter * 32, lane, qpos, qcrow);
         if (!mbar_wait(&tfull[acc], accphase, abort_flag, g.status)) break;
         tc_fence_after();
         if constexpr (EPI == EPI_QKV) {
           const int head = nh / 128;  // one head per half
-          if (head < g.fz.H + 2 * g.fz.Hkv) qkv_head(g, m0 + quarter * 32, lane, head, tbase, scale, ebuf);
+          if (head < g.fz.H + 2 * g.fz.Hkv)
+            qkv_head(g, m0 + quarter * 32, lane, head, tbase, scale, ebuf, qpos, qcrow);
         } else {
           float ss = 0.f;
 #pragma unroll 1
