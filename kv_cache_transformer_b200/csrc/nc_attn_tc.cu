@@ -24,7 +24,9 @@
 // PV_B(j), S_B(j+1): while one warpgroup exponentiates, the tensor core works
 // for the other. S_t(j+1) overwrites the TMEM columns PV_t(j) reads P from;
 // tcgen05.mma operations of one CTA run in issue order, so it is issued right
-// after PV_t(j) with no wait in between. O is rescaled only when a row's
+// after PV_t(j) with no wait in between. PV_t(j) goes in two halves: the
+// first 64 keys as soon as the softmax threads have stored their P, while
+// they exponentiate the other 64. O is rescaled only when a row's
 // running max grows by more than 2^8 (the probabilities of a tile are then at
 // most 256, exact in fp32 and bf16). Items are ordered heaviest first and dealt
 // to the CTAs in zig-zag rounds, which evens out the causal work per CTA.
@@ -156,7 +158,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *p_full = s_full + 2;        // 2 (128 arrivals)
   uint64_t *o_done = p_full + 2;        // 2: every P V of the tile so far is done
   uint64_t *o_free = o_done + 2;        // 2 (128 arrivals): the item's O has been read
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(o_free + 2);
+  uint64_t *p_half = o_free + 2;        // 2 (128 arrivals): P of the tile's first 64 keys is in TMEM
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(p_half + 2);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -192,6 +195,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&p_full[t], 128);
       mbar_init(&o_done[t], 1);
       mbar_init(&o_free[t], 128);
+      mbar_init(&p_half[t], 128);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -284,15 +288,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!take(vaddr, vslot)) { ok = false; break; }
           for (int t = 0; t < 2 && ok; t++) {
             if (j < nkt[t]) {  // key tile j reaches some row of Q tile t
-              if (!mbar_wait(&p_full[t], gt[t] & 1, abort_flag, a.status)) { ok = false; break; }
-              gt[t]++;
+              // P of keys 0..63 first: its MMAs run while the softmax
+              // threads exponentiate keys 64..127
+              if (!mbar_wait(&p_half[t], gt[t] & 1, abort_flag, a.status)) { ok = false; break; }
               // the epilogue of the previous item must have read O_t
               if (j == 0 && !mbar_wait(&o_free[t], (it & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
               tc_fence_after();
               const uint32_t pa = tmem + t * 128 + 64, vb = desc_lo_mn(vaddr);
 #pragma unroll
-              for (int k = 0; k < BKV / 16; k++)
+              for (int k = 0; k < BKV / 32; k++)
                 mma_ts(tmem + 256 + t * 128, pa + k * 8, vb + ((k * 2048) >> 4), id_o, (j | k) != 0);
+              if (!mbar_wait(&p_full[t], gt[t] & 1, abort_flag, a.status)) { ok = false; break; }
+              gt[t]++;
+              tc_fence_after();
+#pragma unroll
+              for (int k = BKV / 32; k < BKV / 16; k++)
+                mma_ts(tmem + 256 + t * 128, pa + k * 8, vb + ((k * 2048) >> 4), id_o, 1);
               mma_commit(&o_done[t]);
             }
             if (t == 1) mma_commit(&kv_empty[vslot]);
@@ -392,6 +403,11 @@ __global__ void __launch_bounds__(THREADS, 1)
             pk[q] = pack2(p0, p1);
           }
           tmem_st8(tS + 64 + c8 * 8, pk);
+          if (c8 == BKV / 32 - 1) {  // keys 0..63 are in TMEM: their P V can start
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_half[t]);
+          }
         }
         l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
         m = m_new;
