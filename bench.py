@@ -105,7 +105,7 @@ def load_peaks():
 # of `python bench.py --steps 1 --warmup 3 --no-decode --no-workloads
 # --no-cpu-baseline` with -k regex:gemm_tc -s 240 -c 4. To be re-taken
 # whenever nc_gemm_tc.cu changes.
-GEMM_DRAM_BYTES_PER_LAUNCH = (53_985_024 + 195_913_472 + 166_196_480 + 387_185_152) / 4
+GEMM_DRAM_BYTES_PER_LAUNCH = (56_577_792 + 196_133_632 + 169_057_280 + 400_016_384) / 4
 
 
 # DRAM bytes of one whole-step decode launch (d20, 32 sequences at context
