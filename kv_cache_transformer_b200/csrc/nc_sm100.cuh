@@ -1,5 +1,6 @@
 // nc_sm100.cuh — sm_100a building blocks: mbarriers with bounded waits, TMA
-// tile loads (no cluster multicast anywhere), tcgen05 MMA / TMEM helpers.
+// tile loads (none with cluster multicast: each CTA fetches its own tiles),
+// tcgen05 MMA / TMEM helpers, and the CTA-pair (cta_group::2) forms.
 #pragma once
 
 #include <cuda.h>  // CUtensorMap (type only; the encoder is fetched at run time)
