@@ -33,6 +33,9 @@
 // NC_DEV_TIMEOUT and all roles drain to the common exit, where TMEM is freed.
 #include <stdlib.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "nc_internal.h"
 #include "nc_sm100.cuh"
 
@@ -602,35 +605,43 @@ static cudaError_t launch_tc(const CUtensorMap &ma, const CUtensorMap &mw, const
   }
 }
 
-// How many CTA pairs of the pair kernel can be resident at once on this
-// device (0 if none, or when the environment sets NC_GEMM_PAIR=0, which
-// selects the one-CTA kernel for every shape).
+// How many CTA pairs of the pair kernel can be resident at once on the
+// current device (0 if none, or when the environment sets NC_GEMM_PAIR=0,
+// which selects the one-CTA kernel for every shape). Computed once per device.
 static int pair_slots() {
-  static int slots = -1;
-  if (slots >= 0) return slots;
-  slots = 0;
-  const char *env = getenv("NC_GEMM_PAIR");
-  if (env && atoi(env) == 0) return slots;
-  const void *fn = (const void *)gemm_tc_kernel<EPI_STORE, true>;
-  if (ensure_smem_attr(fn, Tiling<true>::SMEM_BYTES) != cudaSuccess) return slots;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2);
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = Tiling<true>::SMEM_BYTES;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  static std::atomic<int> cache[64];
+  static std::once_flag init;
+  std::call_once(init, [] {
+    for (auto &c : cache) c.store(-1);
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int have = cache[dev].load();
+  if (have >= 0) return have;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    n = 0;
+  const char *env = getenv("NC_GEMM_PAIR");
+  if (!(env && atoi(env) == 0)) {
+    const void *fn = (const void *)gemm_tc_kernel<EPI_STORE, true>;
+    if (ensure_smem_attr(fn, Tiling<true>::SMEM_BYTES) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2);
+      cfg.blockDim = dim3(THREADS);
+      cfg.dynamicSmemBytes = Tiling<true>::SMEM_BYTES;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+      }
+    }
   }
-  slots = n;
-  return slots;
+  cache[dev].store(n);
+  return n;
 }
 
 template <bool PAIR>
