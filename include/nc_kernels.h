@@ -27,9 +27,11 @@ extern "C" {
  * elements, W bf16 [N, K] row-major (a weight stored [out, in]), fp32
  * accumulation; the epilogue writes d_out. Runs on the tcgen05 tensor-core
  * kernel when M >= 128, K % 64 == 0, N % 32 == 0 and lda % 8 == 0 (16-byte
- * rows for TMA), otherwise on the generic kernel. Device pointers must be
- * 16-byte aligned. Errors: NC_EINVAL (null pointer, non-positive size,
- * lda < K, ldo < N, unknown epilogue), NC_ECUDA. */
+ * rows for TMA), otherwise on the generic kernel. Above 128 rows the tcgen05
+ * kernel runs on CTA pairs (clusters of two CTAs, tcgen05.mma.cta_group::2);
+ * the environment variable NC_GEMM_PAIR=0 keeps it on single CTAs. Device
+ * pointers must be 16-byte aligned. Errors: NC_EINVAL (null pointer,
+ * non-positive size, lda < K, ldo < N, unknown epilogue), NC_ECUDA. */
 int nc_gemm_bf16(const void *d_A, int lda, const void *d_W, int M, int N, int K, int epi, void *d_out, int ldo,
                  float cap, void *stream);
 
