@@ -211,6 +211,35 @@ def test_mqa_equals_mha_with_replicated_kv_head():
     assert np.max(np.abs(a - b)) < 1e-12
 
 
+def test_gqa_equals_mha_with_each_kv_head_repeated_for_its_group():
+    # four query heads in two groups: heads 0, 1 read KV head 0, heads 2, 3
+    # read KV head 1 (head h reads KV head h // (H / Hkv)); the MHA model
+    # with each KV head's Wk, Wv rows repeated for its group computes the same
+    # function, while a model with the heads interleaved (h % Hkv) does not
+    gqa = syn.ModelConfig(depth=1, d_model=256, n_head=4, n_kv_head=2, head_dim=64, mlp_hidden=1024, vocab=512,
+                          dtype="f32")
+    blob = syn.make_blob(gqa, 31)
+    H, Hkv, hd = gqa.n_head, gqa.n_kv_head, gqa.head_dim
+    G = H // Hkv
+    mha = dataclasses.replace(gqa, n_kv_head=H)
+    grouped, interleaved = [], []
+    for name, r, c in syn.tensor_list(gqa):
+        t = _tensor(blob, gqa, name)
+        if name.endswith(".wk") or name.endswith(".wv"):
+            heads = t.reshape(Hkv, hd, c)
+            grouped.append(np.repeat(heads, G, axis=0).ravel())
+            interleaved.append(np.tile(heads, (G, 1, 1)).ravel())
+        else:
+            grouped.append(t.ravel())
+            interleaved.append(t.ravel())
+    toks = syn.tokens_uniform(11, (10,), gqa.vocab)
+    a = orc.OracleModel(gqa, blob).forward_full(toks)
+    b = orc.OracleModel(mha, np.concatenate(grouped)).forward_full(toks)
+    wrong = orc.OracleModel(mha, np.concatenate(interleaved)).forward_full(toks)
+    assert np.max(np.abs(a - b)) < 1e-12
+    assert np.max(np.abs(a - wrong)) > 1e-6
+
+
 def _edited(edits):
     blob = BLOB.copy()
     for name, fn in edits.items():
