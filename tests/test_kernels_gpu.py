@@ -35,6 +35,8 @@ def _tol(epi, want, K):
 
 @pytest.mark.parametrize("M,N,K", [
     (128, 256, 64),      # one tile, one k-block
+    (129, 256, 64),      # one CTA pair: the second CTA holds a single valid row
+    (256, 512, 128),     # exactly one 256-row pair tile per column block
     (300, 1536, 1280),   # ragged M, d20 QKV width
     (257, 1920, 1664),   # ragged M and N (d26 QKV), K not a multiple of 128
     (1000, 5120, 1280),  # d20 MLP fc
