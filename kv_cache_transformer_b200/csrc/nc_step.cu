@@ -27,9 +27,11 @@
 //    block to arrive adds the partials in split order;
 //  * attention runs per (sequence, KV head): the G = H/Hkv query heads of a
 //    KV head are the rows of its MMAs (flash decoding with mma.sync); each
-//    pair's keys are split over up to 8 CTAs, or CTAs take several pairs when
-//    there are more pairs than CTAs; the last split to arrive merges the
-//    softmax states in split order.
+//    pair's keys are split over up to 8 CTAs. When there are more pairs than
+//    CTAs, the pairs' 64-key tiles are dealt evenly instead (tile_deal): each
+//    CTA takes a contiguous run of them, which may span several pairs. The
+//    last split or segment of a pair to arrive merges the softmax states in
+//    order.
 // Every reduction has a fixed order, so results do not depend on timing.
 //
 // Measured costs behind the choice of mma.sync for the linear layers (the
@@ -55,6 +57,8 @@
 //   MERGE  next token per sequence, lengths advanced
 // Every wait is bounded (~2 s): a timeout raises NC_DEV_TIMEOUT and all
 // roles drain to the exit.
+#include <stdlib.h>
+
 #include "nc_internal.h"
 #include "nc_sm100.cuh"
 
@@ -70,6 +74,7 @@ constexpr int HKB = SLOT / (64 * 128);  // lm_head k-blocks per slot (64 rows ea
 constexpr int KT = 64;                  // keys per attention tile
 constexpr int MAXB = 32;                // sequences per step: rows of every staged activation
 constexpr int MAX_SPLIT = 8;            // attention key splits per sequence
+constexpr int SEGMAX = 8;               // attention segments of one CTA under the tile deal
 constexpr int MAX_R = 64;               // weight rows per CTA in the K-split linears
 constexpr int HG = 64;                  // lm_head rows per pass (16 per warp of each warp group)
 constexpr int SMEM_CAP = 227 * 1024;
@@ -89,6 +94,7 @@ struct StepArgs {
   int Hkv, G;                 // KV heads, query heads per KV head (G = H / Hkv <= 16)
   int r_q, r_o, r_f, r_p, s_p, r_h, n_o, n_f, n_p, n_h, n_qkv;
   int slots, splits;
+  int stream;                 // attention units outnumber the CTAs: deal their key tiles evenly
   float eps, cap, scale_log2;
   const bf16 *wte;
   const CUtensorMap *wmaps;   // [4L + 1]: per layer qkv (r_q/2-row box), o, fc, proj; then lm_head
@@ -137,6 +143,8 @@ struct Smem {
   float *inv;              // [32] per-sequence 1/rms of the phase's normed input
   float *red_ss;           // [NCW][32] per-warp sums of squares of the staged rows
   int *flag;
+  int *nseg;               // this CTA's attention segments under the tile deal; -1: units dealt in rounds
+  int *seg;                // [SEGMAX][6]: sequence, KV head, first key, end key, segment, segments of the unit
 };
 
 __device__ __forceinline__ void csync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -374,12 +382,25 @@ __device__ void producer(const StepArgs &a, const Smem &s, uint8_t *ring) {
     phase_of(a, p, type, layer);
     bool first = true;
     if (type == P_ATTN) {
-      // this CTA's units (sequence, KV head, split), in the consumers' order
-      for (int un = c; un < a.B * a.Hkv * a.splits; un += a.grid) {
-        const int b = un / (a.Hkv * a.splits), j = (un / a.splits) % a.Hkv, sp = un % a.splits;
-        if (!s.valid[b]) continue;
-        int k0, k1;
-        key_range(s.pos[b] + 1, sp, a.splits, k0, k1);
+      // this CTA's units (sequence, KV head, split) or segments of the tile
+      // deal, in the consumers' order
+      const int nseg = *s.nseg;
+      const int nun = nseg >= 0 ? nseg : (a.B * a.Hkv * a.splits + a.grid - 1 - c) / a.grid;
+      for (int iu = 0; iu < nun; iu++) {
+        int b, j, k0, k1;
+        if (nseg >= 0) {
+          const int *sg = s.seg + 6 * iu;
+          b = sg[0];
+          j = sg[1];
+          k0 = sg[2];
+          k1 = sg[3];
+        } else {
+          const int un = c + iu * a.grid;
+          b = un / (a.Hkv * a.splits);
+          j = (un / a.splits) % a.Hkv;
+          if (!s.valid[b]) continue;
+          key_range(s.pos[b] + 1, un % a.splits, a.splits, k0, k1);
+        }
         const int row0 = (layer * a.max_batch + b) * a.max_seq;
         // tiles below the shared length (a multiple of 64) come from the prefix cache
         const int plen = a.pre_len[b];
@@ -576,15 +597,14 @@ __device__ float *reduce_warps(float *red, int R, int MT, int e) {
 // are merged (per-row factors first), the split's state goes to apart, and
 // the last split to arrive merges all splits in split order into y.
 __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
-                               uint32_t &t, uint32_t &xph, int p, int b, int j, int sp, bool first) {
+                               uint32_t &t, uint32_t &xph, int p, int b, int j, int sp, int ns, int k0, int k1,
+                               bool first) {
   const int warp = e >> 5, lane = e & 31, g = lane >> 2, t4 = lane & 3;
   const int grp = warp >> 2, wq = warp & 3;
   const int G = a.G, vs = b * a.Hkv + j;  // query heads j*G .. j*G+G-1 read KV head j
   const size_t lay = (size_t)layer * a.max_batch * a.max_seq * a.Hkv * 128;
   const size_t crow = ((size_t)b * a.max_seq + s.pos[b]) * a.Hkv + j;  // cache row of the new key / value
-  const int pos = s.pos[b], n_keys = pos + 1;
-  int k0, k1;
-  key_range(n_keys, sp, a.splits, k0, k1);
+  const int pos = s.pos[b];
   float *cw = reinterpret_cast<float *>(xs);                                 // [8 warps][16 rows][AROW]
   bf16 *qs = reinterpret_cast<bf16 *>(xs + NCW * 16 * AROW * 4);             // [17][128]: q heads, the new key
   float *fac = reinterpret_cast<float *>(xs + NCW * 16 * AROW * 4 + 17 * 128 * 2);  // [NCW + 2][16]
@@ -758,7 +778,7 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
   if (e == 0) {
     unsigned old;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.acnt + vs) : "memory");
-    *s.flag = old == (unsigned)((layer + 1) * a.splits - 1) ? 1 : 0;
+    *s.flag = old == (unsigned)((layer + 1) * ns - 1) ? 1 : 0;
   }
   csync();
   if (*s.flag) {  // the last split: merge all splits in split order
@@ -769,17 +789,17 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
     if (e == 0) {
       asm volatile("fence.proxy.async.global;" ::: "memory");
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive_expect_tx(s.x_bar, rows_bytes * a.splits);
-      for (int q = 0; q < a.splits; q++)
+      mbar_arrive_expect_tx(s.x_bar, rows_bytes * ns);
+      for (int q = 0; q < ns; q++)
         bulk_copy(st + q * G * AROW, a.apart + ((size_t)vs * MAX_SPLIT + q) * G * AROW, rows_bytes, s.x_bar);
     }
     mbar_wait(s.x_bar, xph & 1, s.abort_flag, a.status);
     xph++;
     if (e < G) {
       float M = -INFINITY;
-      for (int q = 0; q < a.splits; q++) M = fmaxf(M, st[(q * G + e) * AROW]);
+      for (int q = 0; q < ns; q++) M = fmaxf(M, st[(q * G + e) * AROW]);
       float Ls = 0.f;
-      for (int q = 0; q < a.splits; q++) {
+      for (int q = 0; q < ns; q++) {
         const float mq = st[(q * G + e) * AROW];
         const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
         fac[q * 16 + e] = f;
@@ -791,22 +811,108 @@ __device__ void attention_unit(const StepArgs &a, const Smem &s, uint8_t *ring, 
     for (int idx = e; idx < G * 128; idx += 32 * NCW) {
       const int row = idx >> 7, col = idx & 127;
       float O = 0.f;
-      for (int q = 0; q < a.splits; q++) O += fac[q * 16 + row] * st[(q * G + row) * AROW + 2 + col];
+      for (int q = 0; q < ns; q++) O += fac[q * 16 + row] * st[(q * G + row) * AROW + 2 + col];
       a.y[(size_t)b * a.d + (j * G + row) * 128 + col] = __float2bfloat16_rn(O * fac[NCW * 16 + row]);
     }
   }
   csync();  // s.flag and the scratch are rewritten by the next use
 }
 
-// This CTA's attention units (sequence, KV head, split), in the producer's order.
+// The tile deal of the attention phases (one warp; positions are fixed for
+// the whole step, so it holds for every layer). The units (sequence b, KV
+// head j), in that order, hold n(u) = ceil((pos[b] + 1) / 64) key tiles, T in
+// all; CTA c takes the tiles [c*T/grid, (c+1)*T/grid) of the concatenation,
+// which cut the units into segments. A unit's segments are numbered by CTA
+// (tile t belongs to CTA (t*grid + grid - 1) / T, so with T >= grid every CTA
+// has tiles and a unit's CTAs are consecutive); the last one to finish merges
+// them in that order. The deal is kept only when T >= grid, every unit has at
+// most MAX_SPLIT segments and no CTA can have more than SEGMAX (conditions
+// every CTA evaluates alike); otherwise nseg = -1 and the units are dealt in
+// rounds of key splits.
+__device__ void tile_deal(const StepArgs &a, const Smem &s, int lane) {
+  const int units = a.B * a.Hkv;
+  const long long G = a.grid, c = blockIdx.x;
+  auto tiles_of = [&](int u) -> long long {
+    const int b = u / a.Hkv;
+    return s.valid[b] ? (s.pos[b] + 1 + KT - 1) / KT : 0;
+  };
+  long long T = 0, n_min = 1LL << 40;  // all tiles; fewest tiles of a unit that has any
+  for (int u = lane; u < units; u += 32) {
+    const long long n = tiles_of(u);
+    T += n;
+    if (n > 0 && n < n_min) n_min = n;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    T += __shfl_xor_sync(0xffffffffu, T, o);
+    n_min = min(n_min, __shfl_xor_sync(0xffffffffu, n_min, o));
+  }
+  // every CTA takes the same decision: a range of at most ceil(T / grid)
+  // tiles meets at most ceil(T / grid) / n_min + 2 units
+  bool ok = a.stream && T >= G && ((T + G - 1) / G) / n_min + 2 <= SEGMAX;
+  const long long lo = c * T / G, hi = (c + 1) * T / G;
+  int count = 0, max_ns = 0;
+  long long base = 0;  // tiles of the units before this chunk of 32
+  for (int u0 = 0; ok && u0 < units; u0 += 32) {
+    const int u = u0 + lane;
+    const long long n = u < units ? tiles_of(u) : 0;
+    long long incl = n;  // inclusive scan over the lanes
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const long long U = base + incl - n;  // first tile of unit u
+    const long long o0 = n > 0 ? (U * G + G - 1) / T : 0;
+    const int ns = n > 0 ? (int)(((U + n - 1) * G + G - 1) / T - o0 + 1) : 0;
+    const bool mine = n > 0 && U < hi && U + n > lo;
+    const unsigned mask = __ballot_sync(0xffffffffu, mine);
+    if (mine) {
+      const int slot = count + __popc(mask & ((1u << lane) - 1));
+      if (slot < SEGMAX) {
+        const int b = u / a.Hkv, n_keys = s.pos[b] + 1;
+        const long long t0 = (U > lo ? U : lo) - U, t1 = (U + n < hi ? U + n : hi) - U;
+        int *sg = s.seg + 6 * slot;
+        sg[0] = b;
+        sg[1] = u % a.Hkv;
+        sg[2] = (int)(t0 * KT);
+        sg[3] = (int)(t1 * KT < n_keys ? t1 * KT : n_keys);
+        sg[4] = (int)(c - o0);
+        sg[5] = ns;
+      }
+    }
+    count += __popc(mask);
+    int m = ns;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    max_ns = max(max_ns, m);
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  ok = ok && max_ns <= MAX_SPLIT;
+  if (lane == 0) *s.nseg = ok ? count : -1;
+}
+
+// This CTA's attention units (sequence, KV head, split) or segments of the
+// tile deal, in the producer's order.
 __device__ bool attention_phase(const StepArgs &a, const Smem &s, uint8_t *ring, uint8_t *xs, int layer, int e,
                                 uint32_t &t, uint32_t &xph, int p) {
   bool first = true;
-  for (int un = blockIdx.x; un < a.B * a.Hkv * a.splits; un += a.grid) {
-    const int b = un / (a.Hkv * a.splits), j = (un / a.splits) % a.Hkv, sp = un % a.splits;
-    if (!s.valid[b]) continue;
-    attention_unit(a, s, ring, xs, layer, e, t, xph, p, b, j, sp, first);
-    first = false;
+  const int nseg = *s.nseg;
+  if (nseg >= 0) {
+    for (int i = 0; i < nseg; i++) {
+      const int *sg = s.seg + 6 * i;
+      attention_unit(a, s, ring, xs, layer, e, t, xph, p, sg[0], sg[1], sg[4], sg[5], sg[2], sg[3], first);
+      first = false;
+    }
+  } else {
+    for (int un = blockIdx.x; un < a.B * a.Hkv * a.splits; un += a.grid) {
+      const int b = un / (a.Hkv * a.splits), j = (un / a.splits) % a.Hkv, sp = un % a.splits;
+      if (!s.valid[b]) continue;
+      int k0, k1;
+      key_range(s.pos[b] + 1, sp, a.splits, k0, k1);
+      attention_unit(a, s, ring, xs, layer, e, t, xph, p, b, j, sp, a.splits, k0, k1, first);
+      first = false;
+    }
   }
   if (e == 0) trace_mark(a, p, 3);
   return true;
@@ -1008,6 +1114,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
     s.inv = reinterpret_cast<float *>(s.valid + 32);
     s.red_ss = s.inv + 32;
     s.flag = reinterpret_cast<int *>(s.red_ss + NCW * 32);
+    s.nseg = s.flag + 1;
+    s.seg = s.nseg + 1;
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1033,6 +1141,8 @@ __global__ void __launch_bounds__(THREADS, 1) decode_step_kernel(StepArgs a) {
     s.valid[b] = ok;
     if (blockIdx.x == 0 && b < a.B) a.valid_out[b] = (uint8_t)ok;
   }
+  __syncthreads();
+  if (warp == 0) tile_deal(a, s, lane);
   __syncthreads();
 
   if (warp == 0) {
@@ -1436,6 +1546,14 @@ cudaError_t k_decode_step(const nc_model *m, const StepPlan &pl, int B, int max_
       }
     }
     a.splits = best;
+    // more units than CTAs: deal the key tiles evenly instead (the kernel
+    // falls back to the rounds when the deal does not fit its tables);
+    // NC_DECODE_TILE_DEAL=0 keeps the rounds
+    static const bool deal_on = [] {
+      const char *env = getenv("NC_DECODE_TILE_DEAL");
+      return !(env && atoi(env) == 0);
+    }();
+    a.stream = deal_on && pairs > pl.grid ? 1 : 0;
   }
   a.eps = c.norm_eps;
   a.cap = c.softcap;

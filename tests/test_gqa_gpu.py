@@ -108,6 +108,22 @@ def test_decode_with_more_attention_pairs_than_ctas_and_ragged_positions():
     assert run.status() == 0
 
 
+def test_more_pairs_than_ctas_dealt_in_rounds():
+    """With more (sequence, KV head) units than CTAs the decode step deals the
+    key tiles evenly; NC_DECODE_TILE_DEAL=0 keeps the rounds of key splits
+    that it falls back to when the deal does not fit. The test above, run in
+    a process of its own with the rounds."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, NC_DECODE_TILE_DEAL="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
+                        "tests/test_gqa_gpu.py::test_decode_with_more_attention_pairs_than_ctas_and_ragged_positions"],
+                       env=env, cwd=root, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
 def test_d20_mha_batch32_decode_sampled_sequences():
     """The d20 MHA model at batch 32: 320 (sequence, KV head) attention pairs
     over the CTAs; sequences 0, 13 and 31 replayed by the oracle."""
