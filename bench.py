@@ -109,11 +109,11 @@ GEMM_DRAM_BYTES_PER_LAUNCH = (56_577_792 + 196_133_632 + 169_057_280 + 400_016_3
 
 
 # DRAM bytes of one whole-step decode launch (d20, 32 sequences at context
-# 2051): dram__bytes_read.sum + dram__bytes_write.sum (1.551246 GB + 5.014 MB)
+# 2051): dram__bytes_read.sum + dram__bytes_write.sum (1.550685 GB + 8.508 MB)
 # from an ncu capture of `python bench.py --only decode --decode-steps 8
 # --warmup 3` with -k regex:decode_step_kernel -s 6 -c 1. To be re-taken
 # whenever nc_step.cu changes.
-DECODE_STEP_DRAM_BYTES = 1_551_246_000 + 5_014_272
+DECODE_STEP_DRAM_BYTES = 1_550_685_000 + 8_507_648
 
 
 class ClockSampler:
